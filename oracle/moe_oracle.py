@@ -1,0 +1,346 @@
+"""CPU oracle of the sparse Mixture-of-Experts FFN forward.
+
+TEST INFRASTRUCTURE ONLY. Nothing on the product path imports this module:
+only the test suite, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline /
+reference leg may call it. It shares no code with the CUDA library.
+
+It is written for a reader who checks it against the pages by eye: fp64 numpy,
+plain loops where the pages loop, a library matmul / sort / erf as single steps,
+no blocking, fusion or reordering. Inputs are the dtype-rounded values (bf16 or
+fp32) upcast exactly to fp64.
+
+Pages cited (by title and the listing or section that defines each step):
+
+* P1 — devtips.kr, "MoE (Mixture of Experts) 아키텍처 완전 정복: Mixtral부터
+  DeepSeek-MoE까지 구현 원리와 실전 최적화 기법": ``MoELayer``, ``DeepSeekMoE``, the
+  capacity snippet, ``load_balancing_loss``.
+* P2 — ricepunchb.github.io, "MoE" study note: §4 diagram (gate scores 0.8/0.2),
+  §5 formulas (garbled), §7 stabilisation list.
+* P3 — youngju.dev, "Mixture of Experts（MoE）架构深度解析：从 Switch Transformer 到
+  Mixtral 的演进与高效扩展策略": ``GatingNetwork``, ``MoELayer`` (GELU),
+  ``SwitchRouter``, ``load_balancing_loss``, ``MixtralMoELayer``, ``SwiGLUExpert``,
+  ``DeepSeekMoELayer``.
+* P4 — youngju.dev, "Sparse Mixture of Experts（MoE）アーキテクチャ深層分析：設計原理
+  からDeepSeek-V3・Qwen3まで": the gating equation, ``SwiGLUExpert``, ``TopKGating``,
+  ``compute_load_balancing_loss``, ``MoELayerWithAuxLoss``, ``router_z_loss``.
+* P5 — study-site lecture 03, "Mixture of Experts": "Token Routing" (gates 0.7/0.3,
+  unselected experts are not computed), "SiLU · SwiGLU · MoE" table.
+
+Readings taken where the pages are silent or disagree (each is also pinned by a
+test):
+
+* top-k is selected on the fp32 logits in every gate mode (softmax is monotone;
+  P4 selects on probabilities, P1/P3 on logits); slots are in descending value,
+  equal values go to the lower expert index first.
+* capacity = floor(cf * T * k / E) in double, T = every token of the call; no
+  minimum capacity; cf <= 0 means unlimited.
+* overflow is dropped in token-major, then slot, order; a dropped slot adds 0 and
+  the surviving gates are not renormalised.
+* f_i counts pre-drop assignments over T*k; P_i is the mean full softmax of the
+  router logits (router bias and logit bias included).
+* GELU is the exact erf form; dropout and routing noise are off (inference).
+* No intermediate rounding: everything after the fp32 logits is fp64.
+
+Parity status: every function below is pinned by the CPU test suite; none is
+"parity unpinned".
+"""
+from __future__ import annotations
+
+import math
+from typing import Optional, Sequence
+
+import numpy as np
+from scipy.special import erf as _erf
+
+ACTS = ("relu", "gelu", "swiglu")
+GATE_MODES = ("topk_softmax", "softmax_topk_renorm", "softmax_topk_raw")
+
+
+def _f64(a):
+    return None if a is None else np.asarray(a, dtype=np.float64)
+
+
+# --------------------------------------------------------------------------- router
+def router_logits(x, w_router, b_router=None, logit_bias=None) -> np.ndarray:
+    """z = x W_r^T (+ b_r) (+ logit_bias), exact in fp64, rounded once to fp32.
+
+    P1 ``MoELayer``: the gate is ``nn.Linear(hidden, E)`` with a bias.
+    P3 ``GatingNetwork`` / ``SwitchRouter`` / ``MixtralMoELayer``: bias-free gate.
+    ``logit_bias`` is the per-expert skew of the Switch workload, added to the logits.
+    """
+    z = _f64(x) @ _f64(w_router).T
+    if b_router is not None:
+        z = z + _f64(b_router)[None, :]
+    if logit_bias is not None:
+        z = z + _f64(logit_bias)[None, :]
+    return z.astype(np.float32)
+
+
+def softmax(z) -> np.ndarray:
+    """Row softmax over experts in fp64, max-subtracted (P3 ``SwitchRouter``, P4 ``TopKGating``)."""
+    z = _f64(z)
+    m = z.max(axis=-1, keepdims=True)
+    e = np.exp(z - m)
+    return e / e.sum(axis=-1, keepdims=True)
+
+
+def select_topk(logits32, k: int) -> np.ndarray:
+    """Indices [T, k] of the k largest fp32 logits per token, in descending order.
+
+    P1 ``MoELayer`` and P3 ``GatingNetwork``: ``torch.topk`` over the gate scores.
+    Ties: the lower expert index comes first (a stable sort of the negated values).
+    """
+    z = np.asarray(logits32, dtype=np.float32).astype(np.float64)
+    order = np.argsort(-z, axis=1, kind="stable")
+    return order[:, :k].astype(np.int32)
+
+
+def gate_values(logits32, idx, mode: str) -> np.ndarray:
+    """Gate weight per selected slot, fp64 [T, k].
+
+    * ``topk_softmax`` (P1 ``MoELayer``, P3 ``GatingNetwork``/``MixtralMoELayer``/
+      ``DeepSeekMoELayer``): softmax over the k selected logits only.
+    * ``softmax_topk_renorm`` (P4 ``TopKGating``): full softmax over E, keep the
+      selected probabilities, divide by their sum.
+    * ``softmax_topk_raw`` (P3 ``SwitchRouter``; P4 gating equation, where G is the
+      softmax inside the top-k and 0 elsewhere): the selected probabilities as they are.
+    """
+    z = np.asarray(logits32, dtype=np.float32).astype(np.float64)
+    idx = np.asarray(idx)
+    T, k = idx.shape
+    g = np.zeros((T, k), dtype=np.float64)
+    if mode == "topk_softmax":
+        for t in range(T):
+            sel = z[t, idx[t]]
+            e = np.exp(sel - sel.max())
+            g[t] = e / e.sum()
+    elif mode in ("softmax_topk_renorm", "softmax_topk_raw"):
+        p = softmax(z)
+        for t in range(T):
+            sel = p[t, idx[t]]
+            g[t] = sel / sel.sum() if mode == "softmax_topk_renorm" else sel
+    else:
+        raise ValueError(mode)
+    return g
+
+
+def topk_margin(logits32, k: int) -> np.ndarray:
+    """Smallest gap between consecutive values among the sorted top-(k+1) logits.
+
+    A token whose margin is tiny (below 1e-4) can legitimately be routed
+    differently by two correct fp32 implementations; such tokens are reported
+    apart from the parity failures.
+    """
+    z = np.sort(np.asarray(logits32, dtype=np.float32).astype(np.float64), axis=1)[:, ::-1]
+    m = min(k + 1, z.shape[1])
+    if m < 2:
+        return np.full(z.shape[0], np.inf)
+    gaps = z[:, :m - 1] - z[:, 1:m]
+    return gaps.min(axis=1)
+
+
+# ------------------------------------------------------------------- dispatch / drop
+def capacity(capacity_factor: float, T: int, k: int, E: int) -> Optional[int]:
+    """Per-expert row capacity, or None when unlimited.
+
+    P1 capacity snippet: (tokens * top_k / E) * capacity_factor.
+    P3 ``SwitchRouter``: ``int(capacity_factor * T / E)`` (top-1).
+    Taken as floor(cf * T * k / E) evaluated in double.
+    """
+    if capacity_factor is None or capacity_factor <= 0:
+        return None
+    return int(math.floor(float(capacity_factor) * T * k / E))
+
+
+def dispatch(idx, E: int, cap: Optional[int]):
+    """Walk (token, slot) pairs in token-major order and assign per-expert ranks.
+
+    P3 ``SwitchRouter``: for each expert, the positions routed to it are listed
+    in token order and those past ``capacity`` are dropped.
+
+    Returns ``counts`` [E] (before drops), ``rank`` [T, k] (the pair's position
+    inside its expert, before drops) and ``kept`` [T, k] bool.
+    """
+    idx = np.asarray(idx)
+    T, k = idx.shape
+    counts = np.zeros(E, dtype=np.int64)
+    rank = np.zeros((T, k), dtype=np.int64)
+    kept = np.zeros((T, k), dtype=bool)
+    for t in range(T):
+        for s in range(k):
+            e = int(idx[t, s])
+            rank[t, s] = counts[e]
+            counts[e] += 1
+            kept[t, s] = cap is None or rank[t, s] < cap
+    return counts, rank, kept
+
+
+def expert_layout(idx, rank, kept, E: int):
+    """Expert-contiguous row order of the kept pairs.
+
+    Rows of expert e occupy [offsets[e], offsets[e+1]) in token order;
+    ``perm[row]`` is the token of that row, ``inv[t, s]`` the row of pair (t, s)
+    or -1 when it was dropped.
+    """
+    idx = np.asarray(idx)
+    T, k = idx.shape
+    kept_counts = np.zeros(E, dtype=np.int64)
+    for t in range(T):
+        for s in range(k):
+            if kept[t, s]:
+                kept_counts[idx[t, s]] += 1
+    offsets = np.zeros(E + 1, dtype=np.int64)
+    offsets[1:] = np.cumsum(kept_counts)
+    perm = np.full(int(offsets[-1]), -1, dtype=np.int64)
+    inv = np.full((T, k), -1, dtype=np.int64)
+    for t in range(T):
+        for s in range(k):
+            if kept[t, s]:
+                row = offsets[idx[t, s]] + rank[t, s]
+                perm[row] = t
+                inv[t, s] = row
+    return offsets, perm, inv
+
+
+# -------------------------------------------------------------------------- experts
+def gelu(v):
+    """Exact GELU, 0.5 v (1 + erf(v / sqrt 2)) (``nn.GELU()`` default in P3 ``MoELayer``)."""
+    return 0.5 * v * (1.0 + _erf(v / math.sqrt(2.0)))
+
+
+def silu(v):
+    """SiLU(v) = v * sigmoid(v) (P5 table: scalar x sigma(x))."""
+    return v / (1.0 + np.exp(-v))
+
+
+def expert_ffn(x_rows, act: str, w1, w2, w3=None, b1=None, b2=None) -> np.ndarray:
+    """One expert on a block of rows, fp64.
+
+    * ``relu`` — P1 ``MoELayer`` experts: Linear(d, F) -> ReLU -> Linear(F, d), with bias.
+    * ``gelu`` — P3 ``MoELayer`` experts: Linear(d, F) -> GELU -> Linear(F, d), with bias.
+    * ``swiglu`` — P3/P4 ``SwiGLUExpert``, P5 table: w_down(silu(w_gate x) * w_up x),
+      no bias; ``w1`` is w_gate, ``w3`` is w_up, ``w2`` is w_down.
+    Weights use the nn.Linear [out, in] layout.
+    """
+    x = _f64(x_rows)
+    if act == "swiglu":
+        h = silu(x @ _f64(w1).T) * (x @ _f64(w3).T)
+    else:
+        v = x @ _f64(w1).T
+        if b1 is not None:
+            v = v + _f64(b1)[None, :]
+        h = np.maximum(v, 0.0) if act == "relu" else gelu(v)
+    o = h @ _f64(w2).T
+    if b2 is not None:
+        o = o + _f64(b2)[None, :]
+    return o
+
+
+def shared_experts(x, ws_gate, ws_up, ws_down, n_shared: int) -> np.ndarray:
+    """Sum of the always-on SwiGLU experts, unweighted (P3 ``DeepSeekMoELayer``;
+    P1 ``DeepSeekMoE``). The weights arrive concatenated along d_ff; each expert's
+    slice is applied separately and the outputs are added."""
+    Fs = ws_gate.shape[0] // n_shared
+    out = np.zeros((x.shape[0], ws_down.shape[0]), dtype=np.float64)
+    for j in range(n_shared):
+        sl = slice(j * Fs, (j + 1) * Fs)
+        out += expert_ffn(x, "swiglu", ws_gate[sl], ws_down[:, sl], w3=ws_up[sl])
+    return out
+
+
+# -------------------------------------------------------------------------- forward
+def route(x, params: dict, *, top_k: int, gate_mode: str, capacity_factor: float = 0.0,
+          logits=None) -> dict:
+    """Router, selection, gates, counts and capacity drops for all T tokens."""
+    if logits is None:
+        logits = router_logits(x, params["w_router"], params.get("b_router"),
+                               params.get("logit_bias"))
+    logits = np.asarray(logits, dtype=np.float32)
+    T, E = logits.shape
+    idx = select_topk(logits, top_k)
+    gates = gate_values(logits, idx, gate_mode)
+    cap = capacity(capacity_factor, T, top_k, E)
+    counts, rank, kept = dispatch(idx, E, cap)
+    offsets, perm, inv = expert_layout(idx, rank, kept, E)
+    return dict(logits=logits, idx=idx, gates=gates, capacity=cap, counts=counts,
+                rank=rank, kept=kept, offsets=offsets, perm=perm, inv=inv)
+
+
+def moe_forward(x, params: dict, *, top_k: int, act: str, gate_mode: str,
+                capacity_factor: float = 0.0, n_shared: int = 0,
+                logits=None, tokens: Optional[Sequence[int]] = None):
+    """y = sum_i G(x)_i E_i(x) (+ shared experts) for every token, or for ``tokens``.
+
+    P4 gating equation y = sum_i G(x)_i E_i(x); the loop form is P1 ``MoELayer`` /
+    P3 ``MixtralMoELayer`` / P4 ``MoELayerWithAuxLoss``: for every slot and every
+    expert, gather the rows routed there, run only that expert, and add the
+    gate-weighted result (P5 "Token Routing": unselected experts are not computed).
+    Capacity drops follow P3 ``SwitchRouter``; shared experts P3 ``DeepSeekMoELayer``.
+
+    Routing always covers all tokens (capacity depends on the global token
+    order); only the expert work is restricted to ``tokens``.
+    Returns (y [len(tokens) or T, d] fp64, routing dict).
+    """
+    x = _f64(x)
+    r = route(x, params, top_k=top_k, gate_mode=gate_mode,
+              capacity_factor=capacity_factor, logits=logits)
+    T = x.shape[0]
+    E = r["logits"].shape[1]
+    sel = np.arange(T) if tokens is None else np.asarray(tokens, dtype=np.int64)
+    in_sel = np.zeros(T, dtype=bool)
+    in_sel[sel] = True
+    pos = np.full(T, -1, dtype=np.int64)
+    pos[sel] = np.arange(len(sel))
+    y = np.zeros((len(sel), x.shape[1]), dtype=np.float64)
+    if n_shared > 0:
+        y += shared_experts(x[sel], params["ws_gate"], params["ws_up"], params["ws_down"],
+                            n_shared)
+    for s in range(top_k):
+        for e in range(E):
+            mask = (r["idx"][:, s] == e) & r["kept"][:, s] & in_sel
+            if not mask.any():
+                continue
+            w3 = params["w3"][e] if params.get("w3") is not None else None
+            b1 = params["b1"][e] if params.get("b1") is not None else None
+            b2 = params["b2"][e] if params.get("b2") is not None else None
+            out = expert_ffn(x[mask], act, params["w1"][e], params["w2"][e], w3, b1, b2)
+            y[pos[mask]] += r["gates"][mask, s][:, None] * out
+    return y, r
+
+
+# ---------------------------------------------------------------------- aux outputs
+def aux_stats(logits32, idx, E: int, top_k: int, alpha: float):
+    """Switch load-balancing statistics.
+
+    P3 ``load_balancing_loss`` and P4 ``compute_load_balancing_loss``:
+    f_i = (assignments to expert i) / (T * k), counted before capacity drops;
+    P_i = mean over tokens of the full softmax over experts;
+    aux = alpha * E * sum_i f_i P_i (alpha = ``aux_loss_weight``, 0.01 in
+    P4 ``MoEConfig`` and P3's default).
+    """
+    idx = np.asarray(idx)
+    T = idx.shape[0]
+    counts = np.zeros(E, dtype=np.int64)
+    for e in idx.ravel():
+        counts[int(e)] += 1
+    f = counts / float(T * top_k)
+    P = softmax(logits32).mean(axis=0)
+    aux = alpha * E * float((f * P).sum())
+    return f, P, aux
+
+
+def router_z_loss(logits32) -> float:
+    """P4 ``router_z_loss``: mean over tokens of logsumexp(logits)^2."""
+    z = _f64(logits32)
+    m = z.max(axis=1)
+    lse = m + np.log(np.exp(z - m[:, None]).sum(axis=1))
+    return float((lse ** 2).mean())
+
+
+def balance_sq_loss(idx, E: int) -> float:
+    """P1 ``load_balancing_loss``: sum_i (share_i - 1/E)^2, share_i = count_i / sum(counts)."""
+    counts = np.zeros(E, dtype=np.float64)
+    for e in np.asarray(idx).ravel():
+        counts[int(e)] += 1
+    share = counts / counts.sum()
+    return float(((share - 1.0 / E) ** 2).sum())

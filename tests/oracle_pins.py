@@ -1,0 +1,336 @@
+"""Checks that pin the CPU oracle to what the pages and the mathematics fix.
+
+Each ``check_*`` raises AssertionError on a mismatch. They take the oracle module
+as an argument so that the mutant tests can hand in a deliberately broken copy
+and confirm that at least one check catches every planted mistake.
+"""
+from __future__ import annotations
+
+import itertools
+import json
+import math
+import os
+
+import numpy as np
+import torch
+
+from sparse_mixture_experts_12_b200 import synth
+from tests import pages_torch_ref as ref
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+ACT = {synth.ACT_RELU: "relu", synth.ACT_GELU: "gelu", synth.ACT_SWIGLU: "swiglu"}
+MODE = {synth.GATE_TOPK_SOFTMAX: "topk_softmax",
+        synth.GATE_SOFTMAX_TOPK_RENORM: "softmax_topk_renorm",
+        synth.GATE_SOFTMAX_TOPK_RAW: "softmax_topk_raw"}
+
+
+def params_f64(inp: dict) -> dict:
+    return {k: synth.to_f64_numpy(v) for k, v in inp.items()}
+
+
+def _golden(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return json.load(f)
+
+
+# ------------------------------------------------------------------------ top-k
+def _brute_topk(zrow, k):
+    """All k-permutations; keep the one that is ordered by (value desc, index asc)
+    and that no unselected expert beats under the same order."""
+    E = len(zrow)
+    key = lambda e: (-float(zrow[e]), e)  # noqa: E731
+    found = []
+    for perm in itertools.permutations(range(E), k):
+        ordered = all(key(perm[j]) < key(perm[j + 1]) for j in range(k - 1))
+        rest = [e for e in range(E) if e not in perm]
+        dominated = all(key(perm[-1]) < key(e) for e in rest)
+        if ordered and dominated:
+            found.append(list(perm))
+    assert len(found) == 1
+    return found[0]
+
+
+def check_topk_bruteforce(O):
+    rng = np.random.default_rng(1)
+    for E in (1, 2, 3, 5, 6):
+        for k in range(1, E + 1):
+            z = rng.normal(size=(12, E)).astype(np.float32)
+            # constructed ties: a coarse grid makes many equal values
+            zt = (np.round(rng.normal(size=(12, E)) * 2) / 2).astype(np.float32)
+            for zz in (z, zt):
+                got = O.select_topk(zz, k)
+                for t in range(zz.shape[0]):
+                    assert list(got[t]) == _brute_topk(zz[t], k), (E, k, zz[t], got[t])
+
+
+# ------------------------------------------------------------------------ gates
+def check_gate_sums_and_ranges(O):
+    rng = np.random.default_rng(2)
+    for E, k in ((8, 2), (64, 6), (5, 5), (3, 1)):
+        z = (rng.normal(size=(40, E)) * 3).astype(np.float32)
+        idx = O.select_topk(z, k)
+        for mode in ("topk_softmax", "softmax_topk_renorm"):
+            g = O.gate_values(z, idx, mode)
+            assert np.all(np.abs(g.sum(axis=1) - 1.0) <= 4 * k * 2.0 ** -52)
+            assert np.all(g >= 0) and np.all(np.diff(g, axis=1) <= 1e-15)
+        graw = O.gate_values(z, idx, "softmax_topk_raw")
+        p = O.softmax(z)
+        assert np.all(graw[:, 0] >= 1.0 / E - 1e-15) and np.all(graw[:, 0] <= 1.0)
+        # the raw Switch gate of slot 0 is the largest probability
+        assert np.allclose(graw[:, 0], p.max(axis=1), rtol=0, atol=1e-15)
+        # modes A and B select the same set and give the same gates up to rounding
+        ga = O.gate_values(z, idx, "topk_softmax")
+        gb = O.gate_values(z, idx, "softmax_topk_renorm")
+        assert np.allclose(ga, gb, rtol=1e-12, atol=1e-15)
+
+
+def check_worked_gates(O):
+    for c in _golden("worked_gates.json")["cases"]:
+        z = np.array([c["logits"]], dtype=np.float32)
+        idx = O.select_topk(z, c["k"])
+        assert list(idx[0]) == c["expect_idx"], c["cite"]
+        for mode in ("topk_softmax", "softmax_topk_renorm"):
+            g = O.gate_values(z, idx, mode)[0]
+            assert np.allclose(g, c["expect_gates"], rtol=0, atol=2e-7), (c["cite"], mode, g)
+
+
+def check_softmax_closed_forms(O):
+    z = np.zeros((3, 7), dtype=np.float32)
+    assert np.allclose(O.softmax(z), 1.0 / 7, rtol=0, atol=1e-16)
+    z = np.array([[0.0, math.log(3.0)]], dtype=np.float64)
+    assert np.allclose(O.softmax(z), [[0.25, 0.75]], rtol=0, atol=1e-15)
+    # invariance to a per-row shift, and to huge logits (no overflow)
+    z = np.array([[1000.0, 999.0, 998.0]])
+    e = np.exp([0.0, -1.0, -2.0])
+    assert np.allclose(O.softmax(z), e / e.sum(), rtol=1e-14)
+
+
+# --------------------------------------------------------------------- logits
+def check_router_logits_exact(O):
+    rng = np.random.default_rng(3)
+    # small integers: every product and sum is exact in fp32 and fp64
+    x = rng.integers(-4, 5, size=(9, 16)).astype(np.float64)
+    w = rng.integers(-3, 4, size=(5, 16)).astype(np.float64)
+    b = rng.integers(-2, 3, size=(5,)).astype(np.float64)
+    lb = rng.integers(-2, 3, size=(5,)).astype(np.float64)
+    z = O.router_logits(x, w, b, lb)
+    want = np.zeros((9, 5))
+    for t in range(9):
+        for e in range(5):
+            want[t, e] = sum(x[t, j] * w[e, j] for j in range(16)) + b[e] + lb[e]
+    assert z.dtype == np.float32 and np.array_equal(z.astype(np.float64), want)
+    # non-integer inputs: the result is the fp32 rounding of the exact dot product
+    x = rng.normal(size=(4, 33))
+    w = rng.normal(size=(3, 33))
+    z = O.router_logits(x, w)
+    exact = np.array([[math.fsum(x[t] * w[e]) for e in range(3)] for t in range(4)])
+    assert np.array_equal(z, exact.astype(np.float32))
+
+
+# ------------------------------------------------------------ capacity / drops
+def check_capacity_golden(O):
+    for c in _golden("capacity.json")["cases"]:
+        assert O.capacity(c["cf"], c["T"], c["k"], c["E"]) == c["expect"], c["cite"]
+
+
+def check_counts_and_drop_order(O):
+    rng = np.random.default_rng(4)
+    for T, E, k, cap in ((50, 4, 1, 9), (64, 8, 2, 10), (33, 3, 3, 5), (20, 5, 2, None)):
+        z = rng.normal(size=(T, E)).astype(np.float32)
+        idx = O.select_topk(z, k)
+        counts, rank, kept = O.dispatch(idx, E, cap)
+        assert counts.sum() == T * k
+        for e in range(E):
+            # the pairs routed to e, listed token-major then slot
+            pairs = [(t, s) for t in range(T) for s in range(k) if idx[t, s] == e]
+            assert counts[e] == len(pairs)
+            for r, (t, s) in enumerate(pairs):
+                assert rank[t, s] == r
+                assert kept[t, s] == (cap is None or r < cap)
+            n_kept = sum(kept[t, s] for (t, s) in pairs)
+            assert n_kept == (len(pairs) if cap is None else min(len(pairs), cap))
+        n_drop = int((~kept).sum())
+        assert int(kept.sum()) == T * k - n_drop
+    # every token on one expert: exactly the first ``cap`` tokens survive
+    idx = np.zeros((30, 1), dtype=np.int32)
+    _, _, kept = O.dispatch(idx, 4, 7)
+    assert list(np.nonzero(kept[:, 0])[0]) == list(range(7))
+
+
+def check_layout(O):
+    rng = np.random.default_rng(5)
+    T, E, k, cap = 40, 6, 2, 11
+    idx = O.select_topk(rng.normal(size=(T, E)).astype(np.float32), k)
+    counts, rank, kept = O.dispatch(idx, E, cap)
+    offsets, perm, inv = O.expert_layout(idx, rank, kept, E)
+    assert offsets[0] == 0 and offsets[-1] == kept.sum()
+    for e in range(E):
+        rows = range(offsets[e], offsets[e + 1])
+        toks = [perm[r] for r in rows]
+        assert toks == sorted(toks)  # token order inside an expert
+        for r in rows:
+            t = perm[r]
+            s = [s for s in range(k) if idx[t, s] == e][0]
+            assert inv[t, s] == r
+    assert np.all((inv >= 0) == kept)
+
+
+# ------------------------------------------------------------------ forward
+def _small_inputs(wl, seed=0):
+    inp = synth.generate(wl, seed=seed)
+    return inp, params_f64(inp)
+
+
+def check_forward_vs_pages_torch(O):
+    """The numpy oracle and the torch restatement of the pages' listings agree."""
+    cases = [synth.SMALL["tiny"].replace(T=48),
+             synth.SMALL["mixtral_small"].replace(T=40, d_model=32, d_ff=48),
+             synth.SMALL["deepseek_small"].replace(T=30, d_model=32, d_ff=24, d_ff_shared=40),
+             synth.SMALL["switch_small"].replace(T=90, d_model=24, d_ff=40, n_experts=6),
+             synth.SMALL["fp32_gelu_cap"].replace(T=35, capacity_factor=0.0)]
+    for wl in cases:
+        inp, p = _small_inputs(wl, seed=7)
+        act, mode = ACT[wl.act], MODE[wl.gate_mode]
+        cap = O.capacity(wl.capacity_factor, wl.T, wl.top_k, wl.n_experts)
+        y, r = O.moe_forward(p["x"], p, top_k=wl.top_k, act=act, gate_mode=mode,
+                             capacity_factor=wl.capacity_factor, n_shared=wl.n_shared)
+        yt, zt, it, wt, pt = ref.moe_layer(p["x"], p, k=wl.top_k, act=act, mode=mode,
+                                           cap=cap, n_shared=wl.n_shared)
+        # the torch restatement keeps fp64 logits; both must pick the same experts
+        assert np.min(O.topk_margin(r["logits"], wl.top_k)) > 1e-5, wl.name
+        assert np.array_equal(r["idx"], it.numpy()), wl.name
+        assert np.allclose(r["logits"], zt.numpy(), rtol=1e-6, atol=1e-6), wl.name
+        assert np.allclose(r["gates"], wt.numpy(), rtol=1e-6, atol=1e-7), wl.name
+        scale = np.abs(yt.numpy()).max()
+        assert np.abs(y - yt.numpy()).max() <= 1e-6 * scale, wl.name
+        f, P, aux = O.aux_stats(r["logits"], r["idx"], wl.n_experts, wl.top_k, wl.aux_alpha)
+        ft, Pt, auxt = ref.load_balancing_loss(pt, it, wl.n_experts, wl.top_k, wl.aux_alpha)
+        assert np.allclose(f, ft.numpy(), rtol=0, atol=1e-15)
+        assert np.allclose(P, Pt.numpy(), rtol=1e-6, atol=1e-9)
+        assert abs(aux - float(auxt)) <= 1e-6 * abs(float(auxt)) + 1e-12
+
+
+def _dense_expert(p, e, act, x):
+    """One expert through torch.nn.functional in fp64 (a library restatement)."""
+    X = torch.as_tensor(x)
+    w1 = torch.as_tensor(p["w1"][e]); w2 = torch.as_tensor(p["w2"][e])
+    if act == "swiglu":
+        h = F.silu(F.linear(X, w1)) * F.linear(X, torch.as_tensor(p["w3"][e]))
+        return F.linear(h, w2).numpy()
+    b1 = None if p.get("b1") is None else torch.as_tensor(p["b1"][e])
+    b2 = None if p.get("b2") is None else torch.as_tensor(p["b2"][e])
+    v = F.linear(X, w1, b1)
+    h = F.relu(v) if act == "relu" else F.gelu(v)
+    return F.linear(h, w2, b2).numpy()
+
+
+import torch.nn.functional as F  # noqa: E402
+
+
+def check_sparse_equals_dense_masked(O):
+    """Computing every expert for every token and weighting by the full gate
+    matrix G (zero outside the kept top-k) gives the sparse result."""
+    for wl in (synth.SMALL["fp32_gelu_cap"].replace(T=60, capacity_factor=0.6),
+               synth.SMALL["deepseek_small"].replace(T=25, d_model=16, d_ff=24, d_ff_shared=8,
+                                                     n_experts=9, top_k=3),
+               synth.SMALL["tiny"].replace(T=20)):
+        inp, p = _small_inputs(wl, seed=11)
+        act, mode = ACT[wl.act], MODE[wl.gate_mode]
+        y, r = O.moe_forward(p["x"], p, top_k=wl.top_k, act=act, gate_mode=mode,
+                             capacity_factor=wl.capacity_factor, n_shared=wl.n_shared)
+        T, E = r["logits"].shape
+        G = np.zeros((T, E))
+        for t in range(T):
+            for s in range(wl.top_k):
+                if r["kept"][t, s]:
+                    G[t, r["idx"][t, s]] += r["gates"][t, s]
+        dense = np.zeros_like(y)
+        for e in range(E):
+            dense += G[:, e:e + 1] * _dense_expert(p, e, act, p["x"])
+        if wl.n_shared:
+            Fs = wl.d_ff_shared
+            for j in range(wl.n_shared):
+                sl = slice(j * Fs, (j + 1) * Fs)
+                X = torch.as_tensor(p["x"])
+                h = F.silu(F.linear(X, torch.as_tensor(p["ws_gate"][sl]))) * \
+                    F.linear(X, torch.as_tensor(p["ws_up"][sl]))
+                dense += F.linear(h, torch.as_tensor(p["ws_down"][:, sl])).numpy()
+        assert np.abs(y - dense).max() <= 1e-12 * max(1.0, np.abs(dense).max()), wl.name
+        if wl.capacity_factor > 0:
+            assert (~r["kept"]).any(), "the capped case must drop something"
+
+
+def check_special_cases(O):
+    # E = 1, k = 1, mode A: the layer is the plain expert FFN (gate 1)
+    for act_id in (synth.ACT_RELU, synth.ACT_GELU, synth.ACT_SWIGLU):
+        wl = synth.SMALL["tiny"].replace(T=10, d_model=8, d_ff=12, n_experts=1, top_k=1,
+                                         act=act_id, expert_bias=act_id != synth.ACT_SWIGLU)
+        inp, p = _small_inputs(wl, seed=3)
+        act = ACT[act_id]
+        y, r = O.moe_forward(p["x"], p, top_k=1, act=act, gate_mode="topk_softmax")
+        assert np.all(r["gates"] == 1.0)
+        assert np.allclose(y, _dense_expert(p, 0, act, p["x"]), rtol=1e-13, atol=1e-13)
+    # k = E, mode B: a dense soft mixture under the full softmax
+    wl = synth.SMALL["fp32_swiglu"].replace(T=12, d_model=8, d_ff=6, n_experts=4, top_k=4,
+                                            n_shared=0)
+    inp, p = _small_inputs(wl, seed=4)
+    y, r = O.moe_forward(p["x"], p, top_k=4, act="swiglu", gate_mode="softmax_topk_renorm")
+    probs = torch.softmax(torch.as_tensor(r["logits"], dtype=torch.float64), dim=-1).numpy()
+    dense = sum(probs[:, e:e + 1] * _dense_expert(p, e, "swiglu", p["x"]) for e in range(4))
+    assert np.allclose(y, dense, rtol=1e-12, atol=1e-13)
+    # SwiGLU with W_gate = 0: silu(0) = 0, so every routed output is 0
+    p0 = dict(p)
+    p0["w1"] = np.zeros_like(p["w1"])
+    y0, _ = O.moe_forward(p["x"], p0, top_k=2, act="swiglu", gate_mode="topk_softmax")
+    assert np.all(y0 == 0.0)
+    # two shared experts equal one expert with their weights concatenated along d_ff
+    wl = synth.SMALL["deepseek_small"].replace(T=9, d_model=16, d_ff=8, d_ff_shared=12)
+    inp, p = _small_inputs(wl, seed=5)
+    two = O.shared_experts(p["x"], p["ws_gate"], p["ws_up"], p["ws_down"], 2)
+    one = O.shared_experts(p["x"], p["ws_gate"], p["ws_up"], p["ws_down"], 1)
+    assert np.allclose(two, one, rtol=1e-12, atol=1e-13)
+    # the GELU and SiLU element functions against library routines
+    v = np.linspace(-6, 6, 101)
+    assert np.allclose(O.gelu(v), F.gelu(torch.as_tensor(v)).numpy(), rtol=1e-14, atol=1e-15)
+    assert np.allclose(O.silu(v), F.silu(torch.as_tensor(v)).numpy(), rtol=1e-14, atol=1e-15)
+
+
+# -------------------------------------------------------------------- aux stats
+def check_aux_closed_forms(O):
+    c = _golden("aux_small.json")
+    z = np.array(c["logits"], dtype=np.float32)
+    idx = O.select_topk(z, c["k"])
+    assert idx.tolist() == c["expect_idx"]
+    f, P, aux = O.aux_stats(z, idx, c["E"], c["k"], c["alpha"])
+    assert np.allclose(f, c["expect_f"], atol=1e-15)
+    assert np.allclose(P, c["expect_P"], atol=1e-7)
+    assert abs(aux - c["expect_aux"]) < 1e-8
+    a = 0.01
+    # uniform logits: P_i = 1/E, and with a balanced assignment f_i = 1/E -> aux = alpha
+    for E, k in ((8, 1), (8, 2), (4, 4)):
+        T = 4 * E
+        z = np.zeros((T, E), dtype=np.float32)
+        idx = np.array([[(t + s) % E for s in range(k)] for t in range(T)], dtype=np.int32)
+        f, P, aux = O.aux_stats(z, idx, E, k, a)
+        assert np.allclose(P, 1.0 / E, atol=1e-16) and np.allclose(f, 1.0 / E, atol=1e-16)
+        assert abs(aux - a) < 1e-15
+    # every token on expert 0 with a one-hot probability: aux -> alpha * E
+    E = 16
+    z = np.full((10, E), -200.0, dtype=np.float32)
+    z[:, 0] = 0.0
+    idx = O.select_topk(z, 1)
+    f, P, aux = O.aux_stats(z, idx, E, 1, a)
+    assert abs(aux - a * E) < 1e-12
+    # extra outputs: z-loss of zero logits is (log E)^2; squared balance loss
+    z = np.zeros((5, 8), dtype=np.float32)
+    assert abs(O.router_z_loss(z) - math.log(8) ** 2) < 1e-12
+    idx = np.zeros((6, 1), dtype=np.int32)
+    assert abs(O.balance_sq_loss(idx, 4) - ((1 - 0.25) ** 2 + 3 * 0.25 ** 2)) < 1e-15
+    idx = np.array([[0], [1], [2], [3]], dtype=np.int32)
+    assert O.balance_sq_loss(idx, 4) == 0.0
+
+
+ALL_CHECKS = [check_topk_bruteforce, check_gate_sums_and_ranges, check_worked_gates,
+              check_softmax_closed_forms, check_router_logits_exact, check_capacity_golden,
+              check_counts_and_drop_order, check_layout, check_forward_vs_pages_torch,
+              check_sparse_equals_dense_masked, check_special_cases, check_aux_closed_forms]

@@ -1,0 +1,125 @@
+"""Plant plausible mistakes in the CPU oracle and confirm the pins catch each one.
+
+Every mutant replaces one oracle function with a subtly wrong version (a dropped
+term, a wrong index, a swapped operand, a wrong normaliser). The pins must fail
+for every mutant; a mutant that survives means a pin is missing.
+"""
+import math
+
+import numpy as np
+import pytest
+
+from oracle import moe_oracle as O
+from tests import oracle_pins as pins
+
+_orig = {name: getattr(O, name) for name in dir(O) if callable(getattr(O, name))}
+
+
+def _topk_ties_high(logits32, k):
+    z = np.asarray(logits32, dtype=np.float32).astype(np.float64)
+    E = z.shape[1]
+    order = np.argsort(-z[:, ::-1], axis=1, kind="stable")
+    return (E - 1 - order[:, :k]).astype(np.int32)
+
+
+def _gates_no_renorm(logits32, idx, mode):
+    g = _orig["gate_values"](logits32, idx, "softmax_topk_raw")
+    return g if mode != "softmax_topk_raw" else g
+
+
+def _gates_modeA_full_softmax(logits32, idx, mode):
+    if mode == "topk_softmax":
+        return _orig["gate_values"](logits32, idx, "softmax_topk_raw")
+    return _orig["gate_values"](logits32, idx, mode)
+
+
+def _capacity_no_k(cf, T, k, E):
+    return _orig["capacity"](cf, T, 1, E)
+
+
+def _dispatch_keep_last(idx, E, cap):
+    counts, rank, kept = _orig["dispatch"](idx, E, None)
+    if cap is not None:
+        for e in range(E):
+            kept[idx == e] = rank[idx == e] >= counts[e] - cap
+    return counts, rank, kept
+
+
+def _gelu_tanh(v):
+    return 0.5 * v * (1 + np.tanh(math.sqrt(2 / math.pi) * (v + 0.044715 * v ** 3)))
+
+
+def _ffn_swapped_gate_up(x_rows, act, w1, w2, w3=None, b1=None, b2=None):
+    if act == "swiglu":
+        return _orig["expert_ffn"](x_rows, act, w3, w2, w1, b1, b2)
+    return _orig["expert_ffn"](x_rows, act, w1, w2, w3, b1, b2)
+
+
+def _ffn_no_b2(x_rows, act, w1, w2, w3=None, b1=None, b2=None):
+    return _orig["expert_ffn"](x_rows, act, w1, w2, w3, b1, None)
+
+
+def _ffn_transposed_down(x_rows, act, w1, w2, w3=None, b1=None, b2=None):
+    w2 = np.asarray(w2)
+    if w2.shape[0] == w2.shape[1]:
+        w2 = w2.T
+    else:
+        w2 = w2.T.reshape(w2.shape)
+    return _orig["expert_ffn"](x_rows, act, w1, w2, w3, b1, b2)
+
+
+def _logits_no_bias(x, w_router, b_router=None, logit_bias=None):
+    return _orig["router_logits"](x, w_router, None, logit_bias)
+
+
+def _aux_f_over_T(logits32, idx, E, top_k, alpha):
+    f, P, aux = _orig["aux_stats"](logits32, idx, E, top_k, alpha)
+    f = f * top_k
+    return f, P, alpha * E * float((f * P).sum())
+
+
+def _shared_dropped(x, ws_gate, ws_up, ws_down, n_shared):
+    return np.zeros((x.shape[0], ws_down.shape[0]))
+
+
+def _silu_sign(v):
+    return v / (1.0 + np.exp(v))
+
+
+def _layout_reverse(idx, rank, kept, E):
+    offsets, perm, inv = _orig["expert_layout"](idx, rank, kept, E)
+    for e in range(E):
+        a, b = offsets[e], offsets[e + 1]
+        perm[a:b] = perm[a:b][::-1].copy()
+    return offsets, perm, inv
+
+
+MUTANTS = {
+    "topk_ties_to_higher_index": ("select_topk", _topk_ties_high),
+    "gates_not_renormalised": ("gate_values", _gates_no_renorm),
+    "modeA_softmax_over_all_experts": ("gate_values", _gates_modeA_full_softmax),
+    "capacity_without_k": ("capacity", _capacity_no_k),
+    "drop_keeps_last_tokens": ("dispatch", _dispatch_keep_last),
+    "gelu_tanh_approximation": ("gelu", _gelu_tanh),
+    "swiglu_gate_up_swapped": ("expert_ffn", _ffn_swapped_gate_up),
+    "mlp_second_bias_dropped": ("expert_ffn", _ffn_no_b2),
+    "down_projection_transposed": ("expert_ffn", _ffn_transposed_down),
+    "router_bias_dropped": ("router_logits", _logits_no_bias),
+    "aux_f_normalised_by_T": ("aux_stats", _aux_f_over_T),
+    "shared_experts_not_added": ("shared_experts", _shared_dropped),
+    "silu_sign_flipped": ("silu", _silu_sign),
+    "layout_rows_reversed": ("expert_layout", _layout_reverse),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_mutant_is_caught(name, monkeypatch):
+    attr, fn = MUTANTS[name]
+    monkeypatch.setattr(O, attr, fn)
+    failed = []
+    for check in pins.ALL_CHECKS:
+        try:
+            check(O)
+        except Exception:  # an assertion, or a shape error from a transposed operand
+            failed.append(check.__name__)
+    assert failed, f"mutant {name} survived every pin"
