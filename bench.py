@@ -1,0 +1,425 @@
+#!/usr/bin/env python
+"""Throughput of the MoE FFN layer forward on B200.
+
+One step = one ``moe_forward`` over a batch of T tokens (router GEMM + softmax/
+top-k, histogram/scan/permute, grouped expert GEMMs, shared experts, combine),
+inputs already resident in HBM. Prints ONE JSON line on rank 0.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+Multi-GPU (torchrun, one rank per GPU): every rank runs the same layer on its
+own batch of T tokens (weak scaling, no data-path collective); the elapsed time
+is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from sparse_mixture_experts_12_b200 import synth  # noqa: E402
+
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+METRIC = "MoE-layer tokens/s"
+
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ------------------------------------------------------------------ clocks sampler
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+    REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+
+    def __init__(self, device: int):
+        self.lines: list[str] = []
+        self.proc = None
+        self.mark = None
+        try:
+            uuid = str(torch.cuda.get_device_properties(device).uuid)
+            sel = ["-i", uuid if uuid.startswith("GPU-") else "GPU-" + uuid]
+        except Exception:
+            sel = []
+        self.cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                    "-lms", "200", *sel]
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(self.cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
+                                         text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+        t0 = time.time()
+        while not self.lines and time.time() - t0 < 5:
+            time.sleep(0.05)
+
+    def _read(self):
+        for ln in self.proc.stdout:
+            self.lines.append((time.time(), ln.strip()))
+
+    def begin_load(self):
+        self.mark = time.time()
+
+    def stop(self):
+        end = time.time()
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = [ln for (t, ln) in self.lines if self.mark is None or self.mark <= t <= end + 0.2]
+        sm, mx, reasons = [], 0.0, set()
+        for ln in rows:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = max(mx, float(parts[1]))
+            except ValueError:
+                continue
+            for name, val in zip(self.REASONS, parts[3:7]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- oracle helpers
+class _F64View:
+    """Lazily upcast slices of a CPU tensor to fp64 numpy (input marshalling only)."""
+
+    def __init__(self, t):
+        self.t = t
+        self.shape = tuple(t.shape)
+
+    def __getitem__(self, i):
+        return self.t[i].to(torch.float64).numpy()
+
+
+def _oracle_params(inp):
+    out = {}
+    for k, v in inp.items():
+        if v is None:
+            out[k] = None
+        elif v.numel() > (1 << 22) and k not in ("x", "w_router"):
+            out[k] = _F64View(v)
+        else:
+            out[k] = v.to(torch.float64).numpy()
+    return out
+
+
+def _oracle_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+def oracle_sample_rate(wl, inp, n_tokens: int):
+    """Time the CPU oracle: routing of all T tokens plus the expert FFNs of
+    ``n_tokens`` strided tokens. Returns (tokens/s estimate for the full
+    workload, description)."""
+    from oracle import moe_oracle as O
+
+    acts = {0: "relu", 1: "gelu", 2: "swiglu"}
+    modes = {0: "topk_softmax", 1: "softmax_topk_renorm", 2: "softmax_topk_raw"}
+    P = _oracle_params(inp)
+    kw = dict(top_k=wl.top_k, act=acts[wl.act], gate_mode=modes[wl.gate_mode],
+              capacity_factor=wl.capacity_factor, n_shared=wl.n_shared)
+    t0 = time.perf_counter()
+    r = O.route(P["x"], P, top_k=wl.top_k, gate_mode=kw["gate_mode"],
+                capacity_factor=wl.capacity_factor)
+    t_route = time.perf_counter() - t0
+    toks = synth.token_sample(wl.T, n_tokens).numpy()
+    t0 = time.perf_counter()
+    O.moe_forward(P["x"], P, tokens=toks, logits=r["logits"], **kw)
+    t_all = time.perf_counter() - t0
+    # moe_forward re-runs the (cheap, given logits) selection/dispatch; count it once
+    t_ffn = max(t_all - 0.0, 1e-9)
+    per_token = t_route / wl.T + t_ffn / len(toks)
+    desc = (f"oracle (numpy fp64): routing of all {wl.T} tokens ({t_route:.2f} s) + expert "
+            f"FFNs of {len(toks)} strided tokens ({t_ffn:.2f} s); tokens/s = 1 / "
+            f"(t_route/T + t_ffn/n)")
+    return 1.0 / per_token, desc, t_route + t_ffn
+
+
+# ---------------------------------------------------------------- the reference arm
+def run_reference(args, wl, rank, world):
+    if rank != 0:
+        return
+    inp = synth.generate(wl, seed=0)
+    n = args.ref_sample
+    for _ in range(args.warmup):
+        oracle_sample_rate(wl, inp, n)
+    rates, secs = [], 0.0
+    desc = ""
+    for _ in range(args.steps):
+        r, desc, s = oracle_sample_rate(wl, inp, n)
+        rates.append(1.0 / r)
+        secs += s
+    value = len(rates) / sum(rates)
+    cores = _oracle_threads()
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1000.0 * secs / max(1, args.steps), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": _config(wl, world),
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                             "sample": desc},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def _config(wl, world):
+    return {"workload": wl.name, "T": wl.T, "d_model": wl.d_model, "n_experts": wl.n_experts,
+            "top_k": wl.top_k, "d_ff": wl.d_ff, "n_shared": wl.n_shared,
+            "d_ff_shared": wl.d_ff_shared, "capacity_factor": wl.capacity_factor,
+            "global_batch": wl.T * world, "seq_len": wl.T,
+            "parallelism": f"dp{world} (independent token batches, no data-path collective)",
+            "l2": "working set > L2 (weights >= 2.8 GB per step); no flush"}
+
+
+def _traffic(workload_name):
+    """DRAM bytes per launch of the expert-FFN kernels from the committed ncu summary,
+    valid only while the kernel source is unchanged since the capture."""
+    p = os.path.join(ROOT, "profiles", "ffn_tc_traffic.json")
+    src = os.path.join(ROOT, "sparse_mixture_experts_12_b200", "csrc", "ffn_tc.cu")
+    if not os.path.exists(p):
+        return None
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        sha = hashlib.sha256(open(src, "rb").read()).hexdigest()
+        ent = d.get(workload_name)
+        if ent is None or ent.get("ffn_tc_sha256") != sha:
+            return None
+        return ent.get("dram_bytes_per_call")
+    except Exception:
+        return None
+
+
+# ---------------------------------------------------------------------- our arm
+def run_ours(args, wl, rank, world, local_rank):
+    from sparse_mixture_experts_12_b200 import binding as B
+    from sparse_mixture_experts_12_b200 import build as BUILD
+
+    BUILD.build()
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    peaks, peaks_src = load_peaks()
+    t0 = time.time()
+    inp = synth.generate(wl, seed=0)
+    if rank > 0:  # same weights, an independent batch per rank
+        g = torch.Generator().manual_seed(1000 + rank)
+        inp["x"] = torch.empty((wl.T, wl.d_model)).normal_(0, 1, generator=g).to(wl.torch_dtype)
+    log(f"[rank {rank}] inputs drawn in {time.time() - t0:.1f} s")
+    layer = B.MoELayer(wl, inp, dev)
+    x = inp["x"].to(dev)
+    y = torch.empty_like(x)
+    want_aux = wl.capacity_factor > 0  # the Switch workload also emits f, P and the aux loss
+    aux = layer.new_aux() if want_aux else None
+    stream = torch.cuda.current_stream()
+    per_step_launches = 6 + (2 if wl.n_shared > 0 else 0)
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+
+    def max_over_ranks(v: float) -> float:
+        if world == 1:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        return float(t.item())
+
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    for _ in range(args.warmup):
+        layer.forward(x, y, aux)
+    torch.cuda.synchronize()
+    code, info = layer.last_device_error()
+    if code != 0:
+        raise RuntimeError(f"device error {code} ({info}) during warm-up")
+    barrier()
+    torch.cuda.synchronize()
+    clocks.begin_load()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        layer.forward(x, y, aux)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    ms = max_over_ranks(e0.elapsed_time(e1))
+    clk = clocks.stop()
+    code, info = layer.last_device_error()
+    if code != 0:
+        raise RuntimeError(f"device error {code} ({info}) in the timed region")
+    value = wl.T * world * args.steps / (ms / 1000.0)
+
+    # ---- expert FFN (grouped GEMMs) timed alone on the same stream, for the roofline
+    taps = layer.new_taps()
+    layer.forward(x, y, aux, taps=taps)
+    E, k = wl.n_experts, wl.top_k
+    xp = torch.empty((wl.T * k, wl.d_model), dtype=wl.torch_dtype, device=dev)
+    cnt = torch.empty(E, dtype=torch.int32, device=dev)
+    off = torch.empty(E + 1, dtype=torch.int32, device=dev)
+    perm = torch.empty(wl.T * k, dtype=torch.int32, device=dev)
+    inv = torch.empty(wl.T * k, dtype=torch.int32, device=dev)
+    layer.permute(x, taps["topk_idx"], cnt, off, perm, inv, xp)
+    yp = torch.empty_like(xp)
+    for _ in range(3):
+        layer.expert_ffn(xp, off, yp)
+    torch.cuda.synchronize()
+    n_ffn = max(args.steps, 10)
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    f0.record(stream)
+    for _ in range(n_ffn):
+        layer.expert_ffn(xp, off, yp)
+    f1.record(stream)
+    torch.cuda.synchronize()
+    ffn_ms = f0.elapsed_time(f1) / n_ffn
+    R = int(off[-1].item())
+    counts = taps["counts"].cpu().numpy()
+    kept = np.diff(off.cpu().numpy())
+    touched = int((kept > 0).sum())
+    F, d = wl.d_ff, wl.d_model
+    n_mats = 3 if wl.act == synth.ACT_SWIGLU else 2
+    flops = 2.0 * R * n_mats * d * F
+    w_bytes = touched * n_mats * d * F * wl.elem_bytes
+    alg_bytes = w_bytes + 2.0 * R * d * wl.elem_bytes  # weights + x_perm read + y_perm write
+    ridge = peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
+    if flops / alg_bytes >= ridge:
+        roof = {"bound": "tensor", "achieved": flops / (ffn_ms * 1e-3) / 1e12,
+                "peak": peaks["bf16_tflops"], "unit": "TFLOP/s"}
+        roof["frac_of_sustained"] = roof["achieved"] / peaks.get("bf16_tflops_sustained",
+                                                                 peaks["bf16_tflops"])
+    else:
+        roof = {"bound": "hbm", "achieved": alg_bytes / (ffn_ms * 1e-3) / 1e9,
+                "peak": peaks["hbm_gbs"], "unit": "GB/s"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["traffic"] = _traffic(wl.name)
+    roof["kernel"] = "grouped expert FFN (moe_expert_ffn: up-projection + down-projection tcgen05 GEMMs)"
+    roof["ms_per_launch"] = ffn_ms
+    roof["peak_source"] = f"{peaks_src} ({'burst' if roof['bound'] == 'tensor' else 'copy'})"
+    roof["algorithmic"] = {"flops": flops, "bytes": alg_bytes, "rows": R,
+                           "touched_experts": touched}
+
+    # ---- end to end through the public API with host buffers
+    xh = inp["x"].pin_memory()
+    yh = torch.empty(x.shape, dtype=x.dtype).pin_memory()
+    for _ in range(2):
+        x.copy_(xh, non_blocking=True)
+        layer.forward(x, y, aux)
+        yh.copy_(y, non_blocking=True)
+    torch.cuda.synchronize()
+    barrier()
+    g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    g0.record(stream)
+    for _ in range(args.steps):
+        x.copy_(xh, non_blocking=True)
+        layer.forward(x, y, aux)
+        yh.copy_(y, non_blocking=True)
+        if aux is not None:
+            aux.cpu()
+    g1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = max_over_ranks(g0.elapsed_time(g1))
+    e2e = {"value": wl.T * world * args.steps / (e2e_ms / 1000.0), "unit": "tokens/s",
+           "h2d_bytes_per_step": int(xh.numel() * xh.element_size()),
+           "d2h_bytes_per_step": int(yh.numel() * yh.element_size()) +
+           (int(aux.numel() * 4) if aux is not None else 0)}
+
+    if rank != 0:
+        return
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        rate, desc, _ = oracle_sample_rate(wl, inp, args.cpu_sample)
+        cpu = {"value": rate, "unit": "tokens/s", "cores": _oracle_threads(), "kind": "oracle",
+               "sample": desc}
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16"
+            if wl.dtype == synth.DT_BF16 else "f32",
+            "data": "synthetic (seeded N(0,1) activations, random-init weights)",
+            "config": _config(wl, world), "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": per_step_launches * args.steps, "clocks": clk,
+            "routing": {"rows_kept": R, "dropped": int(wl.T * k - R),
+                        "max_expert_load": int(counts.max()), "min_expert_load": int(counts.min())}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="mixtral_prefill", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-sample", type=int, default=8,
+                    help="tokens whose expert FFNs the CPU oracle computes")
+    ap.add_argument("--ref-sample", type=int, default=2,
+                    help="tokens per step of the reference (oracle) arm")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    wl = synth.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        run_reference(args, wl, rank, world)
+        return
+    if world > 1:
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                             device_id=torch.device("cuda", local_rank))
+    try:
+        run_ours(args, wl, rank, world, local_rank)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

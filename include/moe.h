@@ -1,0 +1,208 @@
+/*
+ * moe.h — C ABI of the B200 (sm_100a) sparse Mixture-of-Experts FFN forward.
+ *
+ * The layer computes, for every token x_t (pages cited by title and listing):
+ *
+ *   z_t   = W_r x_t (+ b_r) (+ logit_bias)                      router
+ *   S_t   = top-k experts of z_t (descending; ties -> lower index)
+ *   g_t,s = gate of slot s (three modes, see MOE_GATE_*)
+ *   y_t   = sum_{s kept} g_t,s * E_{S_t,s}(x_t) (+ sum_j Shared_j(x_t))
+ *
+ *   "MoE (Mixture of Experts) 아키텍처 완전 정복" (devtips.kr): MoELayer, DeepSeekMoE,
+ *       the capacity snippet.
+ *   "Mixture of Experts（MoE）架构深度解析" (youngju.dev, zh): GatingNetwork, MoELayer,
+ *       SwitchRouter, load_balancing_loss, MixtralMoELayer, SwiGLUExpert,
+ *       DeepSeekMoELayer.
+ *   "Sparse Mixture of Experts（MoE）アーキテクチャ深層分析" (youngju.dev, ja): the gating
+ *       equation y = sum_i G(x)_i E_i(x), SwiGLUExpert, TopKGating,
+ *       compute_load_balancing_loss, router_z_loss.
+ *   "Mixture of Experts" (study-site lecture 03): Token Routing, the SwiGLU table.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - Ownership: the caller allocates and owns every buffer (device memory unless
+ *   stated). The library never allocates, frees or keeps pointers after a call.
+ * - Asynchrony: every call only enqueues kernels on `stream` and returns; none
+ *   synchronises except moe_last_device_error().
+ * - Layout: row-major. Weights use the nn.Linear [out_features, in_features]
+ *   layout, stacked over experts. Activations, weights, x_perm, y_perm and y are
+ *   stored in cfg->dtype (fp32 or bf16); biases, logits, gates are fp32; index
+ *   arrays are int32.
+ * - Alignment: every pointer must be 16-byte aligned, the workspace 256-byte.
+ * - Validation: arguments are checked on the host before anything is launched;
+ *   a failed check returns an error status and enqueues nothing. No call aborts
+ *   or throws.
+ * - Device-side errors (an expert index out of range, offsets that are not a
+ *   valid partition, a bounded wait that gave up) are recorded in a sticky error
+ *   word at the start of the workspace; read and clear it with
+ *   moe_last_device_error(). A kernel that detects one skips the offending
+ *   access instead of faulting.
+ * - Workspace: one buffer of moe_workspace_size() bytes serves every entry point
+ *   of a configuration. Zero it once with moe_workspace_init() before first use.
+ *   Calls that share a workspace must not overlap on the GPU.
+ */
+#ifndef MOE_H_
+#define MOE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A cudaStream_t (NULL = the legacy default stream). */
+typedef struct CUstream_st *moe_stream_t;
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,  /* a size, mode or pointer is out of range / NULL */
+  MOE_ERR_UNSUPPORTED = 2,  /* valid, but outside what the kernels implement */
+  MOE_ERR_MISALIGNED = 3,   /* a pointer breaks the 16-byte (256 for ws) rule */
+  MOE_ERR_WORKSPACE = 4,    /* ws_bytes < moe_workspace_size() */
+  MOE_ERR_CUDA = 5,         /* a CUDA runtime call failed (launch, attribute) */
+  MOE_ERR_DEVICE = 6        /* moe_last_device_error() found a device-side error */
+} moe_status_t;
+
+/* Device error codes (the `code` of moe_last_device_error). */
+enum {
+  MOE_DEVERR_NONE = 0,
+  MOE_DEVERR_EXPERT_INDEX = 1,  /* topk_idx outside [0, E); info = token*k + slot */
+  MOE_DEVERR_OFFSETS = 2,       /* offsets not non-decreasing within [0, T*k]; info = expert */
+  MOE_DEVERR_ROW_INDEX = 3,     /* inv outside [-1, T*k); info = token*k + slot */
+  MOE_DEVERR_WAIT_TIMEOUT = 4   /* a pipeline wait exceeded its bound; info = site */
+};
+
+/* Expert FFN kinds. */
+enum {
+  MOE_ACT_RELU = 0,   /* Linear(d,F)+b1 -> ReLU -> Linear(F,d)+b2   (devtips.kr MoELayer)   */
+  MOE_ACT_GELU = 1,   /* Linear(d,F)+b1 -> GELU(erf) -> Linear(F,d)+b2 (youngju zh MoELayer) */
+  MOE_ACT_SWIGLU = 2  /* w_down(silu(w_gate x) * w_up x), no bias     (SwiGLUExpert)        */
+};
+
+/* Gate modes. Selection is always the top-k of the fp32 logits. */
+enum {
+  MOE_GATE_TOPK_SOFTMAX = 0,        /* softmax over the k selected logits (MoELayer, GatingNetwork) */
+  MOE_GATE_SOFTMAX_TOPK_RENORM = 1, /* full softmax, selected probs / their sum (TopKGating)     */
+  MOE_GATE_SOFTMAX_TOPK_RAW = 2     /* full softmax, selected probs as they are (SwitchRouter)   */
+};
+
+enum { MOE_DTYPE_F32 = 0, MOE_DTYPE_BF16 = 1 };
+
+/* Layer configuration (MoEConfig of the ja page, plus routing and storage fields).
+ * Limits: 1 <= E <= 256; 1 <= k <= min(E, 8); T >= 0 (T = 0 is a no-op);
+ * d_model, d_ff, d_ff_shared multiples of 64 for bf16 (tensor-core path) and of
+ * 4 for fp32; n_shared >= 0 (shared experts are SwiGLU). */
+typedef struct {
+  int32_t n_tokens;        /* T: tokens of the call (batch and sequence flattened) */
+  int32_t d_model;         /* d */
+  int32_t n_experts;       /* E routed experts */
+  int32_t top_k;           /* k */
+  int32_t d_ff;            /* F of each routed expert */
+  int32_t act;             /* MOE_ACT_* */
+  int32_t gate_mode;       /* MOE_GATE_* */
+  int32_t dtype;           /* MOE_DTYPE_*: storage of x, weights, x_perm, y_perm, y */
+  float capacity_factor;   /* > 0: capacity = floor(cf*T*k/E) rows per expert, overflow
+                              dropped in token-major then slot order; <= 0: unlimited */
+  float aux_alpha;         /* weight of the load-balancing loss (0.01 on the pages) */
+  int32_t n_shared;        /* always-on SwiGLU experts, added unweighted (0 = none) */
+  int32_t d_ff_shared;     /* F of each shared expert */
+} moe_cfg_t;
+
+/* Device pointers to the parameters. Unused entries must be NULL. */
+typedef struct {
+  const void *w_router;     /* [E, d]              dtype */
+  const float *b_router;    /* [E]  fp32 router bias, or NULL */
+  const float *logit_bias;  /* [E]  fp32 added to the logits, or NULL */
+  const void *w1;           /* [E, F, d]  dtype; SwiGLU: w_gate */
+  const void *w3;           /* [E, F, d]  dtype; SwiGLU: w_up (NULL for MLP experts) */
+  const void *w2;           /* [E, d, F]  dtype; w_down */
+  const float *b1;          /* [E, F] fp32 or NULL (MLP experts only) */
+  const float *b2;          /* [E, d] fp32 or NULL (MLP experts only) */
+  const void *ws_gate;      /* [n_shared*F_sh, d] dtype: shared experts' w_gate, concatenated */
+  const void *ws_up;        /* [n_shared*F_sh, d] dtype */
+  const void *ws_down;      /* [d, n_shared*F_sh] dtype */
+} moe_weights_t;
+
+/* Optional device buffers that moe_forward fills with its intermediates
+ * (any member may be NULL). Sizes as in moe_route / moe_permute. */
+typedef struct {
+  float *logits;       /* [T, E] */
+  int32_t *topk_idx;   /* [T, k] */
+  float *topk_gate;    /* [T, k] */
+  int32_t *counts;     /* [E]   assignments per expert before capacity drops */
+  int32_t *offsets;    /* [E+1] kept-row prefix: expert e owns rows [offsets[e], offsets[e+1]) */
+  int32_t *perm;       /* [T*k] row -> token (rows >= offsets[E] are left unspecified) */
+  int32_t *inv;        /* [T*k] (token, slot) -> row, -1 when dropped */
+} moe_taps_t;
+
+/* Bytes of workspace every entry point needs for `cfg`. */
+moe_status_t moe_workspace_size(const moe_cfg_t *cfg, size_t *bytes);
+
+/* Zero the workspace header (the sticky device error word). Call once after
+ * allocating a workspace. */
+moe_status_t moe_workspace_init(void *ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Router + selection + gates ("GatingNetwork"/"TopKGating"/"SwitchRouter").
+ * x [T, d] dtype, or NULL: then `logits` is an INPUT [T, E] and only selection
+ * and gates run. Otherwise logits [T, E] fp32 is an output (may be NULL).
+ * topk_idx [T, k] int32 and topk_gate [T, k] fp32 are outputs: slots in
+ * descending logit order, equal logits -> lower expert index first. */
+moe_status_t moe_route(const moe_cfg_t *cfg, const moe_weights_t *w, const void *x,
+                       float *logits, int32_t *topk_idx, float *topk_gate,
+                       void *ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Histogram, capacity, prefix sum and permutation ("SwitchRouter" drop rule).
+ * In: x [T, d] dtype, topk_idx [T, k]. Out: counts [E] (before drops), offsets
+ * [E+1] (kept-row prefix), perm [T*k] (row -> token), inv [T*k] ((t,s) -> row or
+ * -1), x_perm [T*k, d] dtype (row r holds x[perm[r]]; rows of expert e are in
+ * token order). Rows past offsets[E] are left unspecified. */
+moe_status_t moe_permute(const moe_cfg_t *cfg, const void *x, const int32_t *topk_idx,
+                         int32_t *counts, int32_t *offsets, int32_t *perm, int32_t *inv,
+                         void *x_perm, void *ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Expert FFNs on expert-contiguous rows ("SwiGLUExpert", MLP experts).
+ * Rows [offsets[e], offsets[e+1]) of x_perm [T*k, d] go through expert e and the
+ * result is written to the same rows of y_perm [T*k, d] (dtype). offsets is a
+ * device array [E+1]; it must be non-decreasing from 0 to at most T*k (checked on
+ * the device: MOE_DEVERR_OFFSETS, nothing computed). For the shared experts call
+ * it with n_experts = 1, d_ff = n_shared*F_sh, w1/w3/w2 = ws_gate/ws_up/ws_down. */
+moe_status_t moe_expert_ffn(const moe_cfg_t *cfg, const moe_weights_t *w, const void *x_perm,
+                            const int32_t *offsets, void *y_perm, void *ws, size_t ws_bytes,
+                            moe_stream_t stream);
+
+/* Gate-weighted combine (the gating equation; "MoELayer" scatter-add).
+ * y[t] = sum_{s: inv[t*k+s] >= 0} topk_gate[t*k+s] * y_perm[inv[t*k+s]]
+ *        (+ shared_y[t] when shared_y != NULL, fp32 [T, d]); y [T, d] dtype.
+ * Computed in fp32, rounded once. A token with every slot dropped gets 0 (+ shared). */
+moe_status_t moe_combine(const moe_cfg_t *cfg, const void *y_perm, const int32_t *inv,
+                         const float *topk_gate, const float *shared_y, void *y,
+                         void *ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Load-balancing statistics ("load_balancing_loss", "compute_load_balancing_loss",
+ * "router_z_loss", devtips.kr "load_balancing_loss").
+ * out [3 + 2E] fp32 = { aux, z_loss, balance_sq, f[0..E), P[0..E) } with
+ *   f_i = assignments to i (before drops) / (T*k), P_i = mean_t softmax(z_t)_i,
+ *   aux = alpha*E*sum_i f_i P_i, z_loss = mean_t logsumexp(z_t)^2,
+ *   balance_sq = sum_i (f_i - 1/E)^2. */
+moe_status_t moe_aux_stats(const moe_cfg_t *cfg, const float *logits, const int32_t *topk_idx,
+                           float *out, void *ws, size_t ws_bytes, moe_stream_t stream);
+
+/* The whole layer: route, permute, expert FFNs, shared experts, combine.
+ * x [T, d] and y [T, d] in dtype. aux_out (nullable) receives the moe_aux_stats
+ * vector [3 + 2E]. taps (nullable) receives intermediates. */
+moe_status_t moe_forward(const moe_cfg_t *cfg, const moe_weights_t *w, const void *x, void *y,
+                         float *aux_out, const moe_taps_t *taps, void *ws, size_t ws_bytes,
+                         moe_stream_t stream);
+
+/* Synchronise `stream`, read and clear the sticky device error word.
+ * Returns MOE_ERR_DEVICE when *code != 0, MOE_ERR_CUDA when the sync failed. */
+moe_status_t moe_last_device_error(void *ws, int32_t *code, int32_t *info, moe_stream_t stream);
+
+/* Human-readable name of a status. */
+const char *moe_status_string(moe_status_t s);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOE_H_ */

@@ -248,6 +248,24 @@ def shared_experts(x, ws_gate, ws_up, ws_down, n_shared: int) -> np.ndarray:
     return out
 
 
+def combine(y_rows, inv, gates, shared=None) -> np.ndarray:
+    """Gate-weighted combine of expert rows: y_t = sum_{s: inv[t,s] >= 0} g_{t,s} y_rows[inv[t,s]]
+    (+ shared_t). The gating equation of P4 with the pages' scatter-add written as a
+    gather; a dropped slot (inv = -1) contributes nothing (P3 ``SwitchRouter``)."""
+    y_rows = _f64(y_rows)
+    inv = np.asarray(inv).reshape(np.asarray(gates).shape)
+    gates = _f64(gates)
+    T, k = inv.shape
+    y = np.zeros((T, y_rows.shape[1]), dtype=np.float64)
+    if shared is not None:
+        y += _f64(shared)
+    for t in range(T):
+        for s in range(k):
+            if inv[t, s] >= 0:
+                y[t] += gates[t, s] * y_rows[inv[t, s]]
+    return y
+
+
 # -------------------------------------------------------------------------- forward
 def route(x, params: dict, *, top_k: int, gate_mode: str, capacity_factor: float = 0.0,
           logits=None) -> dict:

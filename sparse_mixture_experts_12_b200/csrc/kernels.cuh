@@ -1,0 +1,93 @@
+// Internal launch interface between the C-ABI layer and the kernel files.
+#pragma once
+
+#include "common.cuh"
+
+namespace moe {
+
+struct RouterArgs {
+  const void *x;            // [T, d] dtype, or nullptr when logits_in is given
+  const void *w;            // [E, d] dtype
+  const float *b_router;    // [E] or nullptr
+  const float *logit_bias;  // [E] or nullptr
+  const float *logits_in;   // [T, E] when x == nullptr
+  float *logits_out;        // [T, E] or nullptr
+  int32_t *topk_idx;        // [T, k]
+  float *topk_gate;         // [T, k]
+  int32_t *tile_counts;     // [E, NT] or nullptr
+  float *tile_p;            // [E, NT] or nullptr: per-tile sums of softmax probabilities
+  float *tile_z;            // [NT] or nullptr: per-tile sums of logsumexp^2
+  int T, d, E, k, gate_mode;
+};
+
+struct ScanArgs {
+  const int32_t *tile_counts;  // [E, NT]
+  int32_t *tile_base;          // [E, NT] exclusive prefix over tiles, per expert
+  int32_t *counts;             // [E]
+  int32_t *offsets;            // [E+1]
+  int32_t *mprefix;            // [E+1] prefix of ceil(kept_e / kRowTile)
+  int E, NT, cap;              // cap < 0: unlimited
+  // optional aux statistics
+  const float *tile_p;         // [E, NT]
+  const float *tile_z;         // [NT]
+  float *aux_out;              // [3 + 2E] or nullptr
+  int T, k;
+  float alpha;
+  int32_t *sh_tbl;             // [4] or nullptr: {0, T, 0, ceil(T/kRowTile)} for the shared experts
+};
+
+struct ScatterArgs {
+  const void *x;               // [T, d] dtype
+  const int32_t *topk_idx;     // [T, k]
+  const int32_t *tile_base;    // [E, NT]
+  const int32_t *offsets;      // [E+1]
+  int32_t *perm;               // [T*k]
+  int32_t *inv;                // [T*k]
+  void *x_perm;                // [T*k, d]
+  int T, d, E, k, cap, elem_bytes;
+  int32_t *err;
+};
+
+struct CombineArgs {
+  const void *y_perm;          // [R, d] dtype
+  const int32_t *inv;          // [T*k]
+  const float *gate;           // [T*k]
+  const float *shared_y;       // [T, d] fp32 or nullptr
+  void *y;                     // [T, d] dtype
+  int T, d, k, R;
+  int32_t *err;
+};
+
+// Grouped GEMM over expert-contiguous rows. Group g owns rows
+// [offsets[g], offsets[g+1]) of A and the weight rows of expert g.
+struct GroupedFfnArgs {
+  const void *a;          // [rows, d] dtype (x_perm, or x for the shared experts)
+  int a_rows;             // rows allocated in a/h/out (for the TMA bounds)
+  const int32_t *offsets; // [G+1]
+  const int32_t *mprefix; // [G+1]
+  int G;                  // groups (experts)
+  int m_tiles_ub;         // host upper bound on sum_g ceil(rows_g / kRowTile)
+  int d, F, act;
+  const void *w1, *w3, *w2;  // [G, F, d], [G, F, d] (SwiGLU), [G, d, F]
+  const float *b1, *b2;      // [G, F], [G, d] or nullptr
+  void *h;                // [a_rows, F] dtype (intermediate)
+  void *out;              // [a_rows, d]
+  int out_f32;            // 1: out is fp32 (shared experts), else dtype
+  int32_t *err;
+};
+
+cudaError_t launch_router(const RouterArgs &a, int dtype, cudaStream_t st);
+cudaError_t launch_tile_counts(const int32_t *topk_idx, int T, int k, int E, int32_t *tile_counts,
+                               int32_t *err, cudaStream_t st);
+cudaError_t launch_scan(const ScanArgs &a, cudaStream_t st);
+cudaError_t launch_scatter(const ScatterArgs &a, cudaStream_t st);
+cudaError_t launch_combine(const CombineArgs &a, int dtype, cudaStream_t st);
+// mprefix (and offset validation) from a caller-supplied offsets array
+cudaError_t launch_tile_table(const int32_t *offsets, int G, int max_rows, int32_t *mprefix,
+                              int32_t *err, cudaStream_t st);
+// fp32 SIMT path (any sizes)
+cudaError_t launch_ffn_simt(const GroupedFfnArgs &a, cudaStream_t st);
+// bf16 tcgen05 path
+cudaError_t launch_ffn_tc(const GroupedFfnArgs &a, cudaStream_t st);
+
+}  // namespace moe

@@ -1,0 +1,529 @@
+// C ABI of the MoE FFN forward: host-side validation, workspace layout and the
+// launch sequence. Every step of the layer runs in this library's kernels.
+#include <math.h>
+#include <string.h>
+
+#include <climits>
+
+#include "kernels.cuh"
+
+#define MOE_API extern "C" __attribute__((visibility("default")))
+
+namespace moe {
+namespace {
+
+enum Buf {
+  B_ERR, B_TILE_COUNTS, B_TILE_BASE, B_TILE_P, B_TILE_Z, B_COUNTS, B_OFFSETS, B_MPREFIX, B_SH_TBL,
+  B_LOGITS, B_IDX, B_GATE, B_PERM, B_INV, B_XPERM, B_H, B_YPERM, B_SH_H, B_SH_Y, B_NBUF
+};
+
+struct Layout {
+  size_t off[B_NBUF];
+  size_t total;
+};
+
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+Layout layout_for(const moe_cfg_t &c) {
+  const size_t T = (size_t)c.n_tokens, E = (size_t)c.n_experts, k = (size_t)c.top_k;
+  const size_t d = (size_t)c.d_model, F = (size_t)c.d_ff;
+  const size_t eb = c.dtype == MOE_DTYPE_F32 ? 4 : 2;
+  const size_t NT = (size_t)ceil_div(c.n_tokens > 0 ? c.n_tokens : 1, router_bm(c.n_experts));
+  const size_t Fs = (size_t)c.n_shared * (size_t)c.d_ff_shared;
+  size_t sz[B_NBUF];
+  sz[B_ERR] = 2 * sizeof(int32_t);
+  sz[B_TILE_COUNTS] = E * NT * 4;
+  sz[B_TILE_BASE] = E * NT * 4;
+  sz[B_TILE_P] = E * NT * 4;
+  sz[B_TILE_Z] = NT * 4;
+  sz[B_COUNTS] = E * 4;
+  sz[B_OFFSETS] = (E + 1) * 4;
+  sz[B_MPREFIX] = (E + 1) * 4;
+  sz[B_SH_TBL] = 4 * 4;
+  sz[B_LOGITS] = T * E * 4;
+  sz[B_IDX] = T * k * 4;
+  sz[B_GATE] = T * k * 4;
+  sz[B_PERM] = T * k * 4;
+  sz[B_INV] = T * k * 4;
+  sz[B_XPERM] = T * k * d * eb;
+  sz[B_H] = T * k * F * eb;
+  sz[B_YPERM] = T * k * d * eb;
+  sz[B_SH_H] = Fs ? T * Fs * eb : 0;
+  sz[B_SH_Y] = Fs ? T * d * 4 : 0;
+  Layout L;
+  size_t o = 0;
+  for (int i = 0; i < B_NBUF; ++i) {
+    L.off[i] = o;
+    o += align256(sz[i]);
+  }
+  L.total = o;
+  return L;
+}
+
+template <typename P>
+P *at(void *ws, const Layout &L, Buf b) {
+  return reinterpret_cast<P *>(static_cast<char *>(ws) + L.off[b]);
+}
+
+bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+moe_status_t check_cfg(const moe_cfg_t *c) {
+  if (c == nullptr) return MOE_ERR_INVALID_ARG;
+  if (c->n_tokens < 0 || c->d_model <= 0 || c->d_ff <= 0) return MOE_ERR_INVALID_ARG;
+  if (c->n_experts < 1 || c->n_experts > kMaxExperts) return MOE_ERR_INVALID_ARG;
+  if (c->top_k < 1 || c->top_k > c->n_experts || c->top_k > kMaxTopK) return MOE_ERR_INVALID_ARG;
+  if (c->act < MOE_ACT_RELU || c->act > MOE_ACT_SWIGLU) return MOE_ERR_INVALID_ARG;
+  if (c->gate_mode < MOE_GATE_TOPK_SOFTMAX || c->gate_mode > MOE_GATE_SOFTMAX_TOPK_RAW)
+    return MOE_ERR_INVALID_ARG;
+  if (c->dtype != MOE_DTYPE_F32 && c->dtype != MOE_DTYPE_BF16) return MOE_ERR_INVALID_ARG;
+  if (!isfinite(c->capacity_factor) || !isfinite(c->aux_alpha)) return MOE_ERR_INVALID_ARG;
+  if (c->n_shared < 0 || (c->n_shared > 0 && c->d_ff_shared <= 0)) return MOE_ERR_INVALID_ARG;
+  const long long rows = (long long)c->n_tokens * c->top_k;
+  if (rows > INT_MAX / 2) return MOE_ERR_UNSUPPORTED;
+  const long long fs = (long long)c->n_shared * c->d_ff_shared;
+  if (fs > INT_MAX / 2 || c->d_model > INT_MAX / 4 || c->d_ff > INT_MAX / 4)
+    return MOE_ERR_UNSUPPORTED;
+  if (c->dtype == MOE_DTYPE_BF16) {
+    if (c->d_model % 64 || c->d_ff % 64 || fs % 64) return MOE_ERR_UNSUPPORTED;
+    if ((long long)c->n_experts * c->d_ff > INT_MAX || (long long)c->n_experts * c->d_model > INT_MAX)
+      return MOE_ERR_UNSUPPORTED;
+  } else {
+    if (c->d_model % 4) return MOE_ERR_UNSUPPORTED;
+    // the fp32 path launches one CTA row per 128-row tile (grid.y limit)
+    if (rows / kRowTile + c->n_experts + 1 > 65535 || c->n_tokens / kRowTile + 2 > 65535)
+      return MOE_ERR_UNSUPPORTED;
+  }
+  return MOE_OK;
+}
+
+moe_status_t check_ws(const moe_cfg_t *c, const void *ws, size_t ws_bytes) {
+  if (ws == nullptr) return MOE_ERR_INVALID_ARG;
+  if (!aligned(ws, 256)) return MOE_ERR_MISALIGNED;
+  if (ws_bytes < layout_for(*c).total) return MOE_ERR_WORKSPACE;
+  return MOE_OK;
+}
+
+// every pointer in the list: non-null required unless allowed, 16-byte aligned
+moe_status_t check_ptrs(std::initializer_list<std::pair<const void *, bool>> ps) {
+  for (auto &p : ps) {
+    if (p.first == nullptr) {
+      if (p.second) return MOE_ERR_INVALID_ARG;
+      continue;
+    }
+    if (!aligned(p.first, 16)) return MOE_ERR_MISALIGNED;
+  }
+  return MOE_OK;
+}
+
+moe_status_t check_expert_weights(const moe_cfg_t *c, const moe_weights_t *w) {
+  if (w == nullptr) return MOE_ERR_INVALID_ARG;
+  const bool swiglu = c->act == MOE_ACT_SWIGLU;
+  if (swiglu && (w->b1 || w->b2)) return MOE_ERR_INVALID_ARG;  // SwiGLU experts have no bias
+  if (!swiglu && w->w3) return MOE_ERR_INVALID_ARG;
+  return check_ptrs({{w->w1, true}, {w->w2, true}, {w->w3, swiglu}, {w->b1, false},
+                     {w->b2, false}});
+}
+
+moe_status_t check_shared_weights(const moe_cfg_t *c, const moe_weights_t *w) {
+  const bool need = c->n_shared > 0;
+  if (!need) return MOE_OK;
+  return check_ptrs({{w->ws_gate, true}, {w->ws_up, true}, {w->ws_down, true}});
+}
+
+moe_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+#define MOE_TRY(expr)                        \
+  do {                                       \
+    moe_status_t s_ = (expr);                \
+    if (s_ != MOE_OK) return s_;             \
+  } while (0)
+#define MOE_CUDA(expr) MOE_TRY(cuda_status(expr))
+
+int capacity_of(const moe_cfg_t &c) {
+  if (!(c.capacity_factor > 0.f)) return -1;
+  const double cap = floor((double)c.capacity_factor * (double)c.n_tokens * (double)c.top_k /
+                           (double)c.n_experts);
+  return cap > (double)INT_MAX ? INT_MAX : (int)cap;
+}
+
+int m_tiles_ub(long long rows, int groups) {
+  long long ub = ceil_div((int)rows, kRowTile) + groups;
+  if (ub > rows) ub = rows;
+  return (int)ub;
+}
+
+cudaError_t run_ffn(const moe_cfg_t &c, const GroupedFfnArgs &a, cudaStream_t st) {
+  return c.dtype == MOE_DTYPE_F32 ? launch_ffn_simt(a, st) : launch_ffn_tc(a, st);
+}
+
+GroupedFfnArgs routed_ffn_args(const moe_cfg_t &c, const moe_weights_t &w, const void *x_perm,
+                               const int32_t *offsets, const int32_t *mprefix, void *h,
+                               void *y_perm, int32_t *err) {
+  GroupedFfnArgs a{};
+  a.a = x_perm;
+  a.a_rows = c.n_tokens * c.top_k;
+  a.offsets = offsets;
+  a.mprefix = mprefix;
+  a.G = c.n_experts;
+  a.m_tiles_ub = m_tiles_ub(a.a_rows, c.n_experts);
+  a.d = c.d_model;
+  a.F = c.d_ff;
+  a.act = c.act;
+  a.w1 = w.w1;
+  a.w3 = w.w3;
+  a.w2 = w.w2;
+  a.b1 = w.b1;
+  a.b2 = w.b2;
+  a.h = h;
+  a.out = y_perm;
+  a.out_f32 = 0;
+  a.err = err;
+  return a;
+}
+
+}  // namespace
+}  // namespace moe
+
+using namespace moe;
+
+MOE_API moe_status_t moe_workspace_size(const moe_cfg_t *cfg, size_t *bytes) {
+  MOE_TRY(check_cfg(cfg));
+  if (bytes == nullptr) return MOE_ERR_INVALID_ARG;
+  *bytes = layout_for(*cfg).total;
+  return MOE_OK;
+}
+
+MOE_API moe_status_t moe_workspace_init(void *ws, size_t ws_bytes, moe_stream_t stream) {
+  if (ws == nullptr || ws_bytes < 256) return MOE_ERR_INVALID_ARG;
+  if (!aligned(ws, 256)) return MOE_ERR_MISALIGNED;
+  MOE_CUDA(cudaMemsetAsync(ws, 0, 256, stream));
+  return MOE_OK;
+}
+
+MOE_API moe_status_t moe_route(const moe_cfg_t *cfg, const moe_weights_t *w, const void *x,
+                               float *logits, int32_t *topk_idx, float *topk_gate, void *ws,
+                               size_t ws_bytes, moe_stream_t stream) {
+  MOE_TRY(check_cfg(cfg));
+  MOE_TRY(check_ws(cfg, ws, ws_bytes));
+  if (cfg->n_tokens == 0) return MOE_OK;
+  if (w == nullptr) return MOE_ERR_INVALID_ARG;
+  if (x != nullptr) {
+    MOE_TRY(check_ptrs({{x, true}, {w->w_router, true}, {logits, false}}));
+  } else {
+    MOE_TRY(check_ptrs({{logits, true}}));
+  }
+  MOE_TRY(check_ptrs({{topk_idx, true}, {topk_gate, true}, {w->b_router, false},
+                      {w->logit_bias, false}}));
+  const moe_cfg_t &c = *cfg;
+  if (c.n_tokens == 0) return MOE_OK;
+  const Layout L = layout_for(c);
+  RouterArgs r{};
+  r.x = x;
+  r.w = w->w_router;
+  r.b_router = w->b_router;
+  r.logit_bias = w->logit_bias;
+  r.logits_in = x ? nullptr : logits;
+  r.logits_out = x ? logits : nullptr;
+  r.topk_idx = topk_idx;
+  r.topk_gate = topk_gate;
+  r.tile_counts = at<int32_t>(ws, L, B_TILE_COUNTS);
+  r.T = c.n_tokens;
+  r.d = c.d_model;
+  r.E = c.n_experts;
+  r.k = c.top_k;
+  r.gate_mode = c.gate_mode;
+  MOE_CUDA(launch_router(r, c.dtype, stream));
+  return MOE_OK;
+}
+
+MOE_API moe_status_t moe_permute(const moe_cfg_t *cfg, const void *x, const int32_t *topk_idx,
+                                 int32_t *counts, int32_t *offsets, int32_t *perm, int32_t *inv,
+                                 void *x_perm, void *ws, size_t ws_bytes, moe_stream_t stream) {
+  MOE_TRY(check_cfg(cfg));
+  MOE_TRY(check_ws(cfg, ws, ws_bytes));
+  MOE_TRY(check_ptrs({{x, true}, {topk_idx, true}, {counts, true}, {offsets, true}, {perm, true},
+                      {inv, true}, {x_perm, true}}));
+  const moe_cfg_t &c = *cfg;
+  if (c.n_tokens == 0) {
+    MOE_CUDA(cudaMemsetAsync(counts, 0, sizeof(int32_t) * c.n_experts, stream));
+    MOE_CUDA(cudaMemsetAsync(offsets, 0, sizeof(int32_t) * (c.n_experts + 1), stream));
+    return MOE_OK;
+  }
+  const Layout L = layout_for(c);
+  int32_t *err = at<int32_t>(ws, L, B_ERR);
+  int32_t *tile_counts = at<int32_t>(ws, L, B_TILE_COUNTS);
+  MOE_CUDA(launch_tile_counts(topk_idx, c.n_tokens, c.top_k, c.n_experts, tile_counts, err, stream));
+  ScanArgs s{};
+  s.tile_counts = tile_counts;
+  s.tile_base = at<int32_t>(ws, L, B_TILE_BASE);
+  s.counts = counts;
+  s.offsets = offsets;
+  s.mprefix = at<int32_t>(ws, L, B_MPREFIX);
+  s.E = c.n_experts;
+  s.NT = ceil_div(c.n_tokens, router_bm(c.n_experts));
+  s.cap = capacity_of(c);
+  s.T = c.n_tokens;
+  s.k = c.top_k;
+  MOE_CUDA(launch_scan(s, stream));
+  ScatterArgs p{};
+  p.x = x;
+  p.topk_idx = topk_idx;
+  p.tile_base = s.tile_base;
+  p.offsets = offsets;
+  p.perm = perm;
+  p.inv = inv;
+  p.x_perm = x_perm;
+  p.T = c.n_tokens;
+  p.d = c.d_model;
+  p.E = c.n_experts;
+  p.k = c.top_k;
+  p.cap = s.cap;
+  p.elem_bytes = c.dtype == MOE_DTYPE_F32 ? 4 : 2;
+  p.err = err;
+  MOE_CUDA(launch_scatter(p, stream));
+  return MOE_OK;
+}
+
+MOE_API moe_status_t moe_expert_ffn(const moe_cfg_t *cfg, const moe_weights_t *w,
+                                    const void *x_perm, const int32_t *offsets, void *y_perm,
+                                    void *ws, size_t ws_bytes, moe_stream_t stream) {
+  MOE_TRY(check_cfg(cfg));
+  MOE_TRY(check_ws(cfg, ws, ws_bytes));
+  if (cfg->n_tokens == 0) return MOE_OK;
+  MOE_TRY(check_expert_weights(cfg, w));
+  MOE_TRY(check_ptrs({{x_perm, true}, {offsets, true}, {y_perm, true}}));
+  const moe_cfg_t &c = *cfg;
+  if (c.n_tokens == 0) return MOE_OK;
+  const Layout L = layout_for(c);
+  int32_t *err = at<int32_t>(ws, L, B_ERR);
+  int32_t *mprefix = at<int32_t>(ws, L, B_MPREFIX);
+  MOE_CUDA(launch_tile_table(offsets, c.n_experts, c.n_tokens * c.top_k, mprefix, err, stream));
+  GroupedFfnArgs a = routed_ffn_args(c, *w, x_perm, offsets, mprefix, at<void>(ws, L, B_H),
+                                     y_perm, err);
+  MOE_CUDA(run_ffn(c, a, stream));
+  return MOE_OK;
+}
+
+MOE_API moe_status_t moe_combine(const moe_cfg_t *cfg, const void *y_perm, const int32_t *inv,
+                                 const float *topk_gate, const float *shared_y, void *y,
+                                 void *ws, size_t ws_bytes, moe_stream_t stream) {
+  MOE_TRY(check_cfg(cfg));
+  MOE_TRY(check_ws(cfg, ws, ws_bytes));
+  if (cfg->n_tokens == 0) return MOE_OK;
+  MOE_TRY(check_ptrs({{y_perm, true}, {inv, true}, {topk_gate, true}, {shared_y, false},
+                      {y, true}}));
+  const moe_cfg_t &c = *cfg;
+  if (c.n_tokens == 0) return MOE_OK;
+  const Layout L = layout_for(c);
+  CombineArgs a{};
+  a.y_perm = y_perm;
+  a.inv = inv;
+  a.gate = topk_gate;
+  a.shared_y = shared_y;
+  a.y = y;
+  a.T = c.n_tokens;
+  a.d = c.d_model;
+  a.k = c.top_k;
+  a.R = c.n_tokens * c.top_k;
+  a.err = at<int32_t>(ws, L, B_ERR);
+  MOE_CUDA(launch_combine(a, c.dtype, stream));
+  return MOE_OK;
+}
+
+MOE_API moe_status_t moe_aux_stats(const moe_cfg_t *cfg, const float *logits,
+                                   const int32_t *topk_idx, float *out, void *ws, size_t ws_bytes,
+                                   moe_stream_t stream) {
+  MOE_TRY(check_cfg(cfg));
+  MOE_TRY(check_ws(cfg, ws, ws_bytes));
+  MOE_TRY(check_ptrs({{logits, true}, {topk_idx, true}, {out, true}}));
+  const moe_cfg_t &c = *cfg;
+  if (c.n_tokens == 0) return MOE_ERR_INVALID_ARG;  // the statistics are means over tokens
+  const Layout L = layout_for(c);
+  int32_t *err = at<int32_t>(ws, L, B_ERR);
+  // softmax partial sums from the given logits (selection outputs go to scratch)
+  RouterArgs r{};
+  r.logits_in = logits;
+  r.topk_idx = at<int32_t>(ws, L, B_IDX);
+  r.topk_gate = at<float>(ws, L, B_GATE);
+  r.tile_p = at<float>(ws, L, B_TILE_P);
+  r.tile_z = at<float>(ws, L, B_TILE_Z);
+  r.T = c.n_tokens;
+  r.d = c.d_model;
+  r.E = c.n_experts;
+  r.k = c.top_k;
+  r.gate_mode = c.gate_mode;
+  MOE_CUDA(launch_router(r, c.dtype, stream));
+  int32_t *tile_counts = at<int32_t>(ws, L, B_TILE_COUNTS);
+  MOE_CUDA(launch_tile_counts(topk_idx, c.n_tokens, c.top_k, c.n_experts, tile_counts, err, stream));
+  ScanArgs s{};
+  s.tile_counts = tile_counts;
+  s.tile_base = at<int32_t>(ws, L, B_TILE_BASE);
+  s.counts = at<int32_t>(ws, L, B_COUNTS);
+  s.offsets = at<int32_t>(ws, L, B_OFFSETS);
+  s.mprefix = at<int32_t>(ws, L, B_MPREFIX);
+  s.E = c.n_experts;
+  s.NT = ceil_div(c.n_tokens, router_bm(c.n_experts));
+  s.cap = -1;
+  s.tile_p = r.tile_p;
+  s.tile_z = r.tile_z;
+  s.aux_out = out;
+  s.T = c.n_tokens;
+  s.k = c.top_k;
+  s.alpha = c.aux_alpha;
+  MOE_CUDA(launch_scan(s, stream));
+  return MOE_OK;
+}
+
+MOE_API moe_status_t moe_forward(const moe_cfg_t *cfg, const moe_weights_t *w, const void *x,
+                                 void *y, float *aux_out, const moe_taps_t *taps, void *ws,
+                                 size_t ws_bytes, moe_stream_t stream) {
+  MOE_TRY(check_cfg(cfg));
+  MOE_TRY(check_ws(cfg, ws, ws_bytes));
+  if (cfg->n_tokens == 0) return MOE_OK;  // nothing is read or written
+  if (w == nullptr) return MOE_ERR_INVALID_ARG;
+  MOE_TRY(check_ptrs({{x, true}, {y, true}, {aux_out, false}, {w->w_router, true},
+                      {w->b_router, false}, {w->logit_bias, false}}));
+  MOE_TRY(check_expert_weights(cfg, w));
+  MOE_TRY(check_shared_weights(cfg, w));
+  moe_taps_t tp{};
+  if (taps) {
+    tp = *taps;
+    MOE_TRY(check_ptrs({{tp.logits, false}, {tp.topk_idx, false}, {tp.topk_gate, false},
+                        {tp.counts, false}, {tp.offsets, false}, {tp.perm, false},
+                        {tp.inv, false}}));
+  }
+  const moe_cfg_t &c = *cfg;
+  const Layout L = layout_for(c);
+  int32_t *err = at<int32_t>(ws, L, B_ERR);
+  float *logits = tp.logits ? tp.logits : at<float>(ws, L, B_LOGITS);
+  int32_t *idx = tp.topk_idx ? tp.topk_idx : at<int32_t>(ws, L, B_IDX);
+  float *gate = tp.topk_gate ? tp.topk_gate : at<float>(ws, L, B_GATE);
+  int32_t *counts = tp.counts ? tp.counts : at<int32_t>(ws, L, B_COUNTS);
+  int32_t *offsets = tp.offsets ? tp.offsets : at<int32_t>(ws, L, B_OFFSETS);
+  int32_t *perm = tp.perm ? tp.perm : at<int32_t>(ws, L, B_PERM);
+  int32_t *inv = tp.inv ? tp.inv : at<int32_t>(ws, L, B_INV);
+  int32_t *mprefix = at<int32_t>(ws, L, B_MPREFIX);
+  int32_t *sh_tbl = at<int32_t>(ws, L, B_SH_TBL);
+  const bool want_aux = aux_out != nullptr;
+
+  // 1. router GEMM + softmax + top-k + gates + per-tile histogram
+  RouterArgs r{};
+  r.x = x;
+  r.w = w->w_router;
+  r.b_router = w->b_router;
+  r.logit_bias = w->logit_bias;
+  r.logits_out = (tp.logits || want_aux) ? logits : nullptr;
+  r.topk_idx = idx;
+  r.topk_gate = gate;
+  r.tile_counts = at<int32_t>(ws, L, B_TILE_COUNTS);
+  r.tile_p = want_aux ? at<float>(ws, L, B_TILE_P) : nullptr;
+  r.tile_z = want_aux ? at<float>(ws, L, B_TILE_Z) : nullptr;
+  r.T = c.n_tokens;
+  r.d = c.d_model;
+  r.E = c.n_experts;
+  r.k = c.top_k;
+  r.gate_mode = c.gate_mode;
+  MOE_CUDA(launch_router(r, c.dtype, stream));
+  // 2. scan: counts, capacity, offsets, GEMM tile table (+ aux statistics)
+  ScanArgs s{};
+  s.tile_counts = r.tile_counts;
+  s.tile_base = at<int32_t>(ws, L, B_TILE_BASE);
+  s.counts = counts;
+  s.offsets = offsets;
+  s.mprefix = mprefix;
+  s.E = c.n_experts;
+  s.NT = ceil_div(c.n_tokens, router_bm(c.n_experts));
+  s.cap = capacity_of(c);
+  s.tile_p = r.tile_p;
+  s.tile_z = r.tile_z;
+  s.aux_out = aux_out;
+  s.T = c.n_tokens;
+  s.k = c.top_k;
+  s.alpha = c.aux_alpha;
+  s.sh_tbl = c.n_shared > 0 ? sh_tbl : nullptr;
+  MOE_CUDA(launch_scan(s, stream));
+  // 3. stable permutation with capacity drops + row gather
+  ScatterArgs p{};
+  p.x = x;
+  p.topk_idx = idx;
+  p.tile_base = s.tile_base;
+  p.offsets = offsets;
+  p.perm = perm;
+  p.inv = inv;
+  p.x_perm = at<void>(ws, L, B_XPERM);
+  p.T = c.n_tokens;
+  p.d = c.d_model;
+  p.E = c.n_experts;
+  p.k = c.top_k;
+  p.cap = s.cap;
+  p.elem_bytes = c.dtype == MOE_DTYPE_F32 ? 4 : 2;
+  p.err = err;
+  MOE_CUDA(launch_scatter(p, stream));
+  // 4. always-on shared experts: one SwiGLU over all tokens, experts concatenated along F
+  float *sh_y = nullptr;
+  if (c.n_shared > 0) {
+    GroupedFfnArgs a{};
+    a.a = x;
+    a.a_rows = c.n_tokens;
+    a.offsets = sh_tbl;
+    a.mprefix = sh_tbl + 2;
+    a.G = 1;
+    a.m_tiles_ub = ceil_div(c.n_tokens, kRowTile);
+    a.d = c.d_model;
+    a.F = c.n_shared * c.d_ff_shared;
+    a.act = MOE_ACT_SWIGLU;
+    a.w1 = w->ws_gate;
+    a.w3 = w->ws_up;
+    a.w2 = w->ws_down;
+    a.h = at<void>(ws, L, B_SH_H);
+    sh_y = at<float>(ws, L, B_SH_Y);
+    a.out = sh_y;
+    a.out_f32 = 1;
+    a.err = err;
+    MOE_CUDA(run_ffn(c, a, stream));
+  }
+  // 5. routed experts on the expert-contiguous rows
+  GroupedFfnArgs a = routed_ffn_args(c, *w, p.x_perm, offsets, mprefix, at<void>(ws, L, B_H),
+                                     at<void>(ws, L, B_YPERM), err);
+  MOE_CUDA(run_ffn(c, a, stream));
+  // 6. gate-weighted combine (+ shared output)
+  CombineArgs cb{};
+  cb.y_perm = a.out;
+  cb.inv = inv;
+  cb.gate = gate;
+  cb.shared_y = sh_y;
+  cb.y = y;
+  cb.T = c.n_tokens;
+  cb.d = c.d_model;
+  cb.k = c.top_k;
+  cb.R = c.n_tokens * c.top_k;
+  cb.err = err;
+  MOE_CUDA(launch_combine(cb, c.dtype, stream));
+  return MOE_OK;
+}
+
+MOE_API moe_status_t moe_last_device_error(void *ws, int32_t *code, int32_t *info,
+                                           moe_stream_t stream) {
+  if (ws == nullptr || code == nullptr) return MOE_ERR_INVALID_ARG;
+  if (!aligned(ws, 256)) return MOE_ERR_MISALIGNED;
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return MOE_ERR_CUDA;
+  int32_t h[2] = {0, 0};
+  if (cudaMemcpy(h, ws, sizeof(h), cudaMemcpyDeviceToHost) != cudaSuccess) return MOE_ERR_CUDA;
+  if (cudaMemset(ws, 0, sizeof(h)) != cudaSuccess) return MOE_ERR_CUDA;
+  *code = h[0];
+  if (info) *info = h[1];
+  return h[0] != 0 ? MOE_ERR_DEVICE : MOE_OK;
+}
+
+MOE_API const char *moe_status_string(moe_status_t s) {
+  switch (s) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_INVALID_ARG: return "invalid argument";
+    case MOE_ERR_UNSUPPORTED: return "unsupported configuration";
+    case MOE_ERR_MISALIGNED: return "misaligned pointer";
+    case MOE_ERR_WORKSPACE: return "workspace too small";
+    case MOE_ERR_CUDA: return "CUDA runtime error";
+    case MOE_ERR_DEVICE: return "device-side error";
+  }
+  return "unknown status";
+}

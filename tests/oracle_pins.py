@@ -330,7 +330,32 @@ def check_aux_closed_forms(O):
     assert O.balance_sq_loss(idx, 4) == 0.0
 
 
-ALL_CHECKS = [check_topk_bruteforce, check_gate_sums_and_ranges, check_worked_gates,
+def check_combine(O):
+    """Layout -> per-row expert -> combine reproduces the masked loop; closed forms."""
+    wl = synth.SMALL["fp32_gelu_cap"].replace(T=40, capacity_factor=0.7)
+    inp, p = _small_inputs(wl, seed=13)
+    act, mode = ACT[wl.act], MODE[wl.gate_mode]
+    y, r = O.moe_forward(p["x"], p, top_k=wl.top_k, act=act, gate_mode=mode,
+                         capacity_factor=wl.capacity_factor)
+    rows = np.zeros((len(r["perm"]), wl.d_model))
+    for e in range(wl.n_experts):
+        a, b = r["offsets"][e], r["offsets"][e + 1]
+        if b > a:
+            rows[a:b] = _dense_expert(p, e, act, p["x"][r["perm"][a:b]])
+    assert np.allclose(O.combine(rows, r["inv"], r["gates"]), y, rtol=1e-12, atol=1e-13)
+    # one-hot gates pick the rows; all slots dropped gives the shared part only
+    rng = np.random.default_rng(14)
+    yr = rng.normal(size=(6, 5))
+    inv = np.array([[0, 3], [5, -1], [-1, -1]])
+    g = np.array([[1.0, 0.0], [0.0, 0.5], [0.3, 0.7]])
+    sh = rng.normal(size=(3, 5))
+    out = O.combine(yr, inv, g, sh)
+    assert np.allclose(out[0], yr[0] + sh[0], rtol=0, atol=1e-15)
+    assert np.allclose(out[1], sh[1], rtol=0, atol=1e-15)
+    assert np.allclose(out[2], sh[2], rtol=0, atol=1e-15)
+
+
+ALL_CHECKS = [check_combine, check_topk_bruteforce, check_gate_sums_and_ranges, check_worked_gates,
               check_softmax_closed_forms, check_router_logits_exact, check_capacity_golden,
               check_counts_and_drop_order, check_layout, check_forward_vs_pages_torch,
               check_sparse_equals_dense_masked, check_special_cases, check_aux_closed_forms]

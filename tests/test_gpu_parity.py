@@ -1,0 +1,410 @@
+"""Parity of the CUDA path (through the C ABI) against the CPU oracle.
+
+Every input is seeded and synthetic (sparse_mixture_experts_12_b200.synth); no
+expected value comes from the CUDA path. Integer outputs (indices, counts,
+offsets, permutation, drop decisions) must be bit-exact when both sides see the
+same logits / routing; floating outputs must be within the per-token max
+relative error of 1e-5 (fp32 layers) or 2e-2 (bf16 storage, fp32 accumulation).
+"""
+from __future__ import annotations
+
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import moe_oracle as O
+from sparse_mixture_experts_12_b200 import binding as B
+from sparse_mixture_experts_12_b200 import build as BUILD
+from sparse_mixture_experts_12_b200 import synth
+from tests import gpu_harness as H
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    if not torch.cuda.is_available():
+        pytest.fail("the GPU tests need a CUDA device")
+    BUILD.build()
+    B.load()
+
+
+def _raw_ws(cfg):
+    return B.new_workspace(cfg, DEV)
+
+
+def _s():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _p(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _devcheck(ws, expect=0):
+    code, info = ctypes.c_int32(0), ctypes.c_int32(0)
+    B.load().moe_last_device_error(_p(ws), ctypes.byref(code), ctypes.byref(info), _s())
+    assert code.value == expect, (code.value, info.value)
+    return info.value
+
+
+# =============================================================== routing (bit-exact)
+ROUTE_CASES = [(E, k, mode) for E in (1, 3, 8, 16, 20, 33, 64, 65, 128, 129, 256)
+               for k in sorted({1, 2, min(6, E), min(8, E)}) if k <= E
+               for mode in (0, 1, 2)]
+
+
+@pytest.mark.parametrize("E,k,mode", ROUTE_CASES)
+def test_route_given_logits_bitexact(E, k, mode):
+    T = 301
+    z = synth.random_logits(T, E, seed=E * 100 + k * 10 + mode, std=1.5, tie_fraction=0.3)
+    wl = synth.SMALL["mixtral_small"].replace(T=T, n_experts=E, top_k=k, gate_mode=mode)
+    cfg = B.make_cfg(wl)
+    ws = _raw_ws(cfg)
+    logits = z.to(DEV)
+    idx = torch.empty((T, k), dtype=torch.int32, device=DEV)
+    gate = torch.empty((T, k), dtype=torch.float32, device=DEV)
+    W = B.MoeWeights()
+    st = B.load().moe_route(ctypes.byref(cfg), ctypes.byref(W), None, _p(logits), _p(idx),
+                            _p(gate), _p(ws), ws.numel(), _s())
+    assert st == 0
+    torch.cuda.synchronize()
+    zn = z.numpy()
+    ref_idx = O.select_topk(zn, k)
+    assert np.array_equal(idx.cpu().numpy(), ref_idx)
+    ref_g = O.gate_values(zn, ref_idx, H.MODE[mode])
+    assert np.allclose(gate.cpu().numpy(), ref_g, rtol=4e-6, atol=1e-7)
+    _devcheck(ws)
+
+
+# ============================================================= permute (bit-exact)
+PERMUTE_CASES = [
+    # E, k, T, cf, dtype
+    (8, 2, 1000, 0.0, synth.DT_BF16),
+    (8, 2, 1000, 1.0, synth.DT_BF16),
+    (64, 6, 777, 0.0, synth.DT_BF16),
+    (128, 1, 3001, 1.25, synth.DT_BF16),
+    (256, 8, 513, 0.5, synth.DT_BF16),
+    (3, 3, 65, 0.8, synth.DT_F32),
+    (33, 4, 129, 0.0, synth.DT_F32),
+    (1, 1, 50, 0.3, synth.DT_BF16),
+]
+
+
+@pytest.mark.parametrize("E,k,T,cf,dt", PERMUTE_CASES)
+def test_permute_given_routing_bitexact(E, k, T, cf, dt):
+    d = 192 if dt == synth.DT_BF16 else 36
+    wl = synth.SMALL["mixtral_small"].replace(T=T, n_experts=E, top_k=k, capacity_factor=cf,
+                                              d_model=d, dtype=dt)
+    cfg = B.make_cfg(wl)
+    ws = _raw_ws(cfg)
+    z = synth.random_logits(T, E, seed=E + T, std=2.0)
+    if E >= 64:  # skew the load so that capacity bites
+        z = z + torch.linspace(3.0, -3.0, E)[None, :]
+    ref_idx = O.select_topk(z.numpy(), k)
+    x = synth.generate(wl, seed=T, with_weights=False)["x"]
+    xd = x.to(DEV)
+    idx = torch.from_numpy(ref_idx).to(DEV)
+    counts = torch.empty(E, dtype=torch.int32, device=DEV)
+    offsets = torch.empty(E + 1, dtype=torch.int32, device=DEV)
+    perm = torch.full((T * k,), -7, dtype=torch.int32, device=DEV)
+    inv = torch.empty(T * k, dtype=torch.int32, device=DEV)
+    x_perm = torch.zeros((T * k, d), dtype=x.dtype, device=DEV)
+    st = B.load().moe_permute(ctypes.byref(cfg), _p(xd), _p(idx), _p(counts), _p(offsets),
+                              _p(perm), _p(inv), _p(x_perm), _p(ws), ws.numel(), _s())
+    assert st == 0
+    torch.cuda.synchronize()
+    cap = O.capacity(cf, T, k, E)
+    rc, rank, kept = O.dispatch(ref_idx, E, cap)
+    roff, rperm, rinv = O.expert_layout(ref_idx, rank, kept, E)
+    R = int(roff[-1])
+    assert np.array_equal(counts.cpu().numpy(), rc)
+    assert np.array_equal(offsets.cpu().numpy(), roff)
+    assert np.array_equal(perm.cpu().numpy()[:R], rperm)
+    assert np.array_equal(inv.cpu().numpy().reshape(T, k), rinv)
+    xp = x_perm.cpu()
+    assert torch.equal(xp[:R], x[torch.from_numpy(rperm)])
+    if cap is not None:
+        assert (~kept).any() or E == 1
+    H.report("permute", E=E, k=k, T=T, cap=cap, dropped=int((~kept).sum()))
+    _devcheck(ws)
+
+
+def test_permute_reports_bad_expert_index():
+    """A corrupted routing index is reported through the device error word (no fault)."""
+    T, E, k = 100, 8, 2
+    wl = synth.SMALL["mixtral_small"].replace(T=T, n_experts=E, top_k=k, d_model=64)
+    cfg = B.make_cfg(wl)
+    ws = _raw_ws(cfg)
+    ref_idx = O.select_topk(synth.random_logits(T, E, seed=5).numpy(), k)
+    bad = ref_idx.copy()
+    bad[37, 1] = 99
+    x = synth.generate(wl, seed=1, with_weights=False)["x"].to(DEV)
+    outs = [torch.empty(E, dtype=torch.int32, device=DEV),
+            torch.empty(E + 1, dtype=torch.int32, device=DEV),
+            torch.empty(T * k, dtype=torch.int32, device=DEV),
+            torch.empty(T * k, dtype=torch.int32, device=DEV),
+            torch.empty((T * k, 64), dtype=torch.bfloat16, device=DEV)]
+    st = B.load().moe_permute(ctypes.byref(cfg), _p(x), _p(torch.from_numpy(bad).to(DEV)),
+                              *[_p(o) for o in outs], _p(ws), ws.numel(), _s())
+    assert st == 0
+    info = _devcheck(ws, expect=1)
+    assert info == 37 * k + 1
+    assert int(outs[3].cpu()[37 * k + 1]) == -1
+    _devcheck(ws, expect=0)  # the word is cleared after reading
+
+
+# ========================================================== expert FFN (tolerance)
+FFN_CASES = [
+    # name, act, dtype, d, F, E, rows per expert
+    ("swiglu_bf16", synth.ACT_SWIGLU, synth.DT_BF16, 256, 384, 5, [0, 1, 129, 300, 64]),
+    ("swiglu_bf16_ntail", synth.ACT_SWIGLU, synth.DT_BF16, 192, 192, 3, [200, 0, 17]),
+    ("gelu_bf16_bias", synth.ACT_GELU, synth.DT_BF16, 128, 320, 4, [5, 260, 0, 128]),
+    ("relu_bf16_bias", synth.ACT_RELU, synth.DT_BF16, 320, 256, 2, [131, 7]),
+    ("swiglu_f32", synth.ACT_SWIGLU, synth.DT_F32, 96, 160, 4, [3, 140, 0, 33]),
+    ("relu_f32_bias", synth.ACT_RELU, synth.DT_F32, 64, 256, 8, [16] * 8),
+    ("gelu_f32_odd", synth.ACT_GELU, synth.DT_F32, 36, 50, 3, [1, 2, 300]),
+]
+
+
+@pytest.mark.parametrize("name,act,dt,d,F,E,rows", FFN_CASES, ids=[c[0] for c in FFN_CASES])
+def test_expert_ffn_matches_oracle(name, act, dt, d, F, E, rows):
+    R = int(sum(rows))
+    k = 2
+    T = (R + k - 1) // k + 3  # x_perm holds T*k rows; the tail rows are unused
+    wl = synth.Workload(name, T=T, d_model=d, n_experts=E, top_k=k, d_ff=F, act=act,
+                        gate_mode=0, dtype=dt, expert_bias=act != synth.ACT_SWIGLU,
+                        bias_std=0.3)
+    inp = synth.generate(wl, seed=R)
+    layer = B.MoELayer(wl, inp, DEV)
+    g = torch.Generator().manual_seed(R + 1)
+    xp = torch.randn((T * k, d), generator=g).to(wl.torch_dtype)
+    offsets = torch.tensor(np.concatenate([[0], np.cumsum(rows)]), dtype=torch.int32)
+    y = torch.full((T * k, d), float("nan"), dtype=wl.torch_dtype, device=DEV)
+    layer.expert_ffn(xp.to(DEV), offsets.to(DEV), y)
+    torch.cuda.synchronize()
+    yc = y.cpu().to(torch.float64).numpy()
+    P = H.oracle_params(inp)
+    worst = 0.0
+    for e in range(E):
+        a, b = int(offsets[e]), int(offsets[e + 1])
+        if b == a:
+            continue
+        ref = O.expert_ffn(synth.to_f64_numpy(xp[a:b]), H.ACT[act], P["w1"][e], P["w2"][e],
+                           None if P["w3"] is None else P["w3"][e],
+                           None if P["b1"] is None else P["b1"][e],
+                           None if P["b2"] is None else P["b2"][e])
+        err = H.max_rel_err(yc[a:b], ref)
+        worst = max(worst, float(err.max()))
+    H.report("expert_ffn", case=name, worst_rel_err=worst)
+    assert worst <= H.TOL[dt], worst
+    # rows outside every expert's range are never written
+    assert np.isnan(yc[R:]).all()
+    _devcheck(layer.ws)
+
+
+def test_expert_ffn_rejects_bad_offsets():
+    wl = synth.SMALL["mixtral_small"].replace(T=64, d_model=128, d_ff=128)
+    layer = B.MoELayer(wl, synth.generate(wl, seed=2), DEV)
+    xp = torch.zeros((128, 128), dtype=torch.bfloat16, device=DEV)
+    y = torch.zeros_like(xp)
+    bad = torch.tensor([0, 10, 5, 20, 20, 30, 40, 50, 60], dtype=torch.int32, device=DEV)
+    layer.expert_ffn(xp, bad, y)
+    code, info = layer.last_device_error()
+    assert code == 2 and info == 1
+
+
+def test_shared_experts_through_expert_ffn():
+    wl = synth.SMALL["deepseek_small"]
+    inp = synth.generate(wl, seed=3)
+    layer = B.MoELayer(wl, inp, DEV)
+    cfg, wt = B.shared_as_experts(layer)
+    x = inp["x"].to(DEV)
+    y = torch.empty_like(x)
+    offsets = torch.tensor([0, wl.T], dtype=torch.int32, device=DEV)
+    layer.expert_ffn(x, offsets, y, cfg=cfg, weights=wt)
+    torch.cuda.synchronize()
+    P = H.oracle_params(inp)
+    ref = O.shared_experts(P["x"], P["ws_gate"], P["ws_up"], P["ws_down"], wl.n_shared)
+    err = H.max_rel_err(y.cpu().to(torch.float64).numpy(), ref)
+    assert err.max() <= H.TOL[wl.dtype], err.max()
+
+
+# =================================================================== combine
+@pytest.mark.parametrize("dt,with_shared", [(synth.DT_BF16, False), (synth.DT_BF16, True),
+                                            (synth.DT_F32, True)])
+def test_combine_matches_oracle(dt, with_shared):
+    T, k, d = 333, 3, 128
+    wl = synth.SMALL["mixtral_small"].replace(T=T, top_k=k, d_model=d, dtype=dt)
+    cfg = B.make_cfg(wl)
+    ws = _raw_ws(cfg)
+    g = torch.Generator().manual_seed(9)
+    R = T * k
+    y_rows = torch.randn((R, d), generator=g).to(wl.torch_dtype)
+    inv = torch.randperm(R, generator=g)[:T * k].reshape(T, k).to(torch.int32)
+    drop = torch.rand((T, k), generator=g) < 0.2
+    inv[drop] = -1
+    inv[5] = -1  # a token with every slot dropped
+    gates = torch.rand((T, k), generator=g)
+    shared = torch.randn((T, d), generator=g) if with_shared else None
+    y = torch.empty((T, d), dtype=wl.torch_dtype, device=DEV)
+    st = B.load().moe_combine(ctypes.byref(cfg), _p(y_rows.to(DEV)), _p(inv.to(DEV)),
+                              _p(gates.to(DEV)), _p(None if shared is None else shared.to(DEV)),
+                              _p(y), _p(ws), ws.numel(), _s())
+    assert st == 0
+    torch.cuda.synchronize()
+    ref = O.combine(synth.to_f64_numpy(y_rows), inv.numpy(), gates.numpy().astype(np.float64),
+                    None if shared is None else shared.numpy())
+    err = H.max_rel_err(y.cpu().to(torch.float64).numpy(), ref)
+    assert err.max() <= H.TOL[dt], err.max()
+    if not with_shared:
+        assert torch.all(y[5] == 0)
+    _devcheck(ws)
+
+
+# ================================================================= aux statistics
+@pytest.mark.parametrize("E,k", [(8, 2), (64, 6), (128, 1), (5, 5)])
+def test_aux_stats_matches_oracle(E, k):
+    T = 1237
+    wl = synth.SMALL["mixtral_small"].replace(T=T, n_experts=E, top_k=k)
+    cfg = B.make_cfg(wl)
+    ws = _raw_ws(cfg)
+    z = synth.random_logits(T, E, seed=E, std=2.0)
+    idx = O.select_topk(z.numpy(), k)
+    out = torch.zeros(3 + 2 * E, dtype=torch.float32, device=DEV)
+    st = B.load().moe_aux_stats(ctypes.byref(cfg), _p(z.to(DEV)),
+                                _p(torch.from_numpy(idx).to(DEV)), _p(out), _p(ws), ws.numel(),
+                                _s())
+    assert st == 0
+    torch.cuda.synchronize()
+    o = out.cpu().numpy().astype(np.float64)
+    f, P, aux = O.aux_stats(z.numpy(), idx, E, k, wl.aux_alpha)
+    assert np.allclose(o[3:3 + E], f, rtol=1e-6, atol=0)
+    assert np.allclose(o[3 + E:], P, rtol=2e-5, atol=1e-7)
+    assert abs(o[0] - aux) <= 2e-5 * aux
+    assert abs(o[1] - O.router_z_loss(z.numpy())) <= 2e-5 * O.router_z_loss(z.numpy())
+    assert abs(o[2] - O.balance_sq_loss(idx, E)) <= 1e-6 + 1e-5 * O.balance_sq_loss(idx, E)
+
+
+# ====================================================================== whole layer
+def _forward_and_compare(wl: synth.Workload, seed: int, n_sample=None, check_full_routing=True):
+    inp = synth.generate(wl, seed=seed)
+    layer = B.MoELayer(wl, inp, DEV)
+    x = inp["x"].to(DEV)
+    taps = layer.new_taps()
+    aux = layer.new_aux()
+    y = layer.forward(x, taps=taps, aux=aux)
+    torch.cuda.synchronize()
+    code, info = layer.last_device_error()
+    assert code == 0, (code, info)
+    P = H.oracle_params(inp)
+    T, E, k = wl.T, wl.n_experts, wl.top_k
+    tokens = None if n_sample is None else synth.token_sample(T, n_sample).numpy()
+    yref, r = O.moe_forward(P["x"], P, tokens=tokens, **H.oracle_kwargs(wl))
+    # logits against the fp32 accumulation bound
+    extra = np.zeros(E)
+    if P["b_router"] is not None:
+        extra += np.abs(P["b_router"])
+    if P["logit_bias"] is not None:
+        extra += np.abs(P["logit_bias"])
+    bound = H.logits_bound(P["x"], P["w_router"], extra)
+    zg = taps["logits"].cpu().numpy().astype(np.float64)
+    assert np.all(np.abs(zg - r["logits"]) <= bound)
+    # the forward's own routing: differences only on near-ties
+    gidx = taps["topk_idx"].cpu().numpy()
+    mism, affected, n_near = H.routing_compare(gidx, r["logits"], r["idx"], k, r["capacity"])
+    if len(mism) == 0:
+        assert np.array_equal(taps["counts"].cpu().numpy(), r["counts"])
+        assert np.array_equal(taps["offsets"].cpu().numpy(), r["offsets"])
+        R = int(r["offsets"][-1])
+        assert np.array_equal(taps["perm"].cpu().numpy()[:R], r["perm"])
+        assert np.array_equal(taps["inv"].cpu().numpy().reshape(T, k), r["inv"])
+        gg = taps["topk_gate"].cpu().numpy()
+        assert np.allclose(gg, r["gates"], rtol=2e-5, atol=1e-6)
+    # outputs on the compared tokens
+    sel = np.arange(T) if tokens is None else tokens
+    keep = np.array([t not in affected for t in sel])
+    yg = y.cpu().to(torch.float64).numpy()[sel]
+    err = H.max_rel_err(yg[keep], yref[keep])
+    # aux statistics (f from the forward's own routing)
+    a = aux.cpu().numpy().astype(np.float64)
+    f, Pm, auxv = O.aux_stats(r["logits"], r["idx"], E, k, wl.aux_alpha)
+    assert np.abs(a[3:3 + E] - f).max() <= len(mism) / (T * k) + 1e-7
+    assert np.allclose(a[3 + E:], Pm, rtol=1e-4, atol=1e-6)
+    assert abs(a[0] - auxv) <= 1e-4 * auxv + wl.aux_alpha * E * len(mism) / (T * k)
+    H.report("forward", workload=wl.name, T=T, compared=int(keep.sum()),
+             worst_rel_err=float(err.max()) if len(err) else 0.0,
+             p99_rel_err=float(np.quantile(err, 0.99)) if len(err) else 0.0,
+             routing_mismatch=len(mism), near_tie_tokens=n_near, excluded=len(affected),
+             dropped=int((~r["kept"]).sum()), R=int(r["offsets"][-1]))
+    assert err.max() <= H.TOL[wl.dtype], (wl.name, float(err.max()))
+    if check_full_routing:
+        _routing_on_oracle_logits(wl, layer, inp, r)
+    return layer, y
+
+
+def _routing_on_oracle_logits(wl, layer, inp, r):
+    """Feed the oracle's fp32 logits and routing to the GPU routing and permute
+    steps: everything integer must then be bit-exact at full size."""
+    T, E, k = wl.T, wl.n_experts, wl.top_k
+    logits = torch.from_numpy(r["logits"]).to(DEV)
+    idx = torch.empty((T, k), dtype=torch.int32, device=DEV)
+    gate = torch.empty((T, k), dtype=torch.float32, device=DEV)
+    layer.route(None, logits, idx, gate)
+    counts = torch.empty(E, dtype=torch.int32, device=DEV)
+    offsets = torch.empty(E + 1, dtype=torch.int32, device=DEV)
+    perm = torch.empty(T * k, dtype=torch.int32, device=DEV)
+    inv = torch.empty(T * k, dtype=torch.int32, device=DEV)
+    xp = torch.empty((T * k, wl.d_model), dtype=wl.torch_dtype, device=DEV)
+    layer.permute(inp["x"].to(DEV), torch.from_numpy(r["idx"]).to(DEV), counts, offsets, perm,
+                  inv, xp)
+    torch.cuda.synchronize()
+    assert np.array_equal(idx.cpu().numpy(), r["idx"])
+    assert np.allclose(gate.cpu().numpy(), r["gates"], rtol=4e-6, atol=1e-7)
+    assert np.array_equal(counts.cpu().numpy(), r["counts"])
+    assert np.array_equal(offsets.cpu().numpy(), r["offsets"])
+    R = int(r["offsets"][-1])
+    assert np.array_equal(perm.cpu().numpy()[:R], r["perm"])
+    assert np.array_equal(inv.cpu().numpy().reshape(T, k), r["inv"])
+    code, _ = layer.last_device_error()
+    assert code == 0
+
+
+@pytest.mark.parametrize("name", sorted(synth.SMALL))
+def test_forward_small_matches_oracle(name):
+    _forward_and_compare(synth.SMALL[name], seed=0)
+
+
+FULL = ["tiny", "mixtral_prefill", "deepseek", "switch", "decode32", "decode8", "decode1"]
+
+
+@pytest.mark.parametrize("name", FULL)
+def test_forward_full_size_sampled(name):
+    wl = synth.WORKLOADS[name]
+    n = None if wl.T <= 64 else 48
+    _forward_and_compare(wl, seed=0, n_sample=n)
+    torch.cuda.empty_cache()
+
+
+def test_forward_is_deterministic():
+    wl = synth.SMALL["switch_small"]
+    inp = synth.generate(wl, seed=4)
+    layer = B.MoELayer(wl, inp, DEV)
+    x = inp["x"].to(DEV)
+    y1 = layer.forward(x).clone()
+    y2 = layer.forward(x)
+    torch.cuda.synchronize()
+    assert torch.equal(y1, y2)
+
+
+def test_zero_tokens_is_a_noop():
+    wl = synth.SMALL["mixtral_small"].replace(T=0)
+    layer = B.MoELayer(wl, synth.generate(wl.replace(T=1), seed=0), DEV)
+    x = torch.empty((0, wl.d_model), dtype=torch.bfloat16, device=DEV)
+    y = layer.forward(x)
+    assert y.shape == (0, wl.d_model)
+    assert layer.last_device_error() == (0, 0)

@@ -94,7 +94,12 @@ def _layout_reverse(idx, rank, kept, E):
     return offsets, perm, inv
 
 
+def _combine_ignores_gates(y_rows, inv, gates, shared=None):
+    return _orig["combine"](y_rows, inv, np.ones_like(np.asarray(gates, dtype=float)), shared)
+
+
 MUTANTS = {
+    "combine_ignores_gates": ("combine", _combine_ignores_gates),
     "topk_ties_to_higher_index": ("select_topk", _topk_ties_high),
     "gates_not_renormalised": ("gate_values", _gates_no_renorm),
     "modeA_softmax_over_all_experts": ("gate_values", _gates_modeA_full_softmax),
