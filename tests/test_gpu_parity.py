@@ -149,8 +149,9 @@ def test_permute_reports_bad_expert_index():
             torch.empty(T * k, dtype=torch.int32, device=DEV),
             torch.empty(T * k, dtype=torch.int32, device=DEV),
             torch.empty((T * k, 64), dtype=torch.bfloat16, device=DEV)]
-    st = B.load().moe_permute(ctypes.byref(cfg), _p(x), _p(torch.from_numpy(bad).to(DEV)),
-                              *[_p(o) for o in outs], _p(ws), ws.numel(), _s())
+    bad_d = torch.from_numpy(bad).to(DEV)
+    st = B.load().moe_permute(ctypes.byref(cfg), _p(x), _p(bad_d), *[_p(o) for o in outs],
+                              _p(ws), ws.numel(), _s())
     assert st == 0
     info = _devcheck(ws, expect=1)
     assert info == 37 * k + 1
@@ -252,9 +253,11 @@ def test_combine_matches_oracle(dt, with_shared):
     gates = torch.rand((T, k), generator=g)
     shared = torch.randn((T, d), generator=g) if with_shared else None
     y = torch.empty((T, d), dtype=wl.torch_dtype, device=DEV)
-    st = B.load().moe_combine(ctypes.byref(cfg), _p(y_rows.to(DEV)), _p(inv.to(DEV)),
-                              _p(gates.to(DEV)), _p(None if shared is None else shared.to(DEV)),
-                              _p(y), _p(ws), ws.numel(), _s())
+    # keep every device tensor referenced until the kernels have run
+    yr_d, inv_d, g_d = y_rows.to(DEV), inv.to(DEV), gates.to(DEV)
+    sh_d = None if shared is None else shared.to(DEV)
+    st = B.load().moe_combine(ctypes.byref(cfg), _p(yr_d), _p(inv_d), _p(g_d), _p(sh_d), _p(y),
+                              _p(ws), ws.numel(), _s())
     assert st == 0
     torch.cuda.synchronize()
     ref = O.combine(synth.to_f64_numpy(y_rows), inv.numpy(), gates.numpy().astype(np.float64),
@@ -276,9 +279,9 @@ def test_aux_stats_matches_oracle(E, k):
     z = synth.random_logits(T, E, seed=E, std=2.0)
     idx = O.select_topk(z.numpy(), k)
     out = torch.zeros(3 + 2 * E, dtype=torch.float32, device=DEV)
-    st = B.load().moe_aux_stats(ctypes.byref(cfg), _p(z.to(DEV)),
-                                _p(torch.from_numpy(idx).to(DEV)), _p(out), _p(ws), ws.numel(),
-                                _s())
+    z_d, idx_d = z.to(DEV), torch.from_numpy(idx).to(DEV)
+    st = B.load().moe_aux_stats(ctypes.byref(cfg), _p(z_d), _p(idx_d), _p(out), _p(ws),
+                                ws.numel(), _s())
     assert st == 0
     torch.cuda.synchronize()
     o = out.cpu().numpy().astype(np.float64)
