@@ -19,7 +19,6 @@ import hashlib
 import json
 import os
 import statistics
-import subprocess
 import sys
 import threading
 import time
@@ -51,70 +50,67 @@ def load_peaks():
 
 # ------------------------------------------------------------------ clocks sampler
 class ClockSampler:
-    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
-              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
-              "clocks_event_reasons.sw_power_cap")
-    REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+    """Polls the GPU's SM clock and clock-event reasons through NVML every 20 ms
+    (read-only queries) while the timed region runs."""
+
+    # NVML clock-event reason bits (nvmlClocksEventReason*)
+    REASON_BITS = {"sw_power_cap": 0x4, "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20,
+                   "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80}
 
     def __init__(self, device: int):
-        self.lines: list[str] = []
-        self.proc = None
+        self.samples: list = []
+        self.nv = None
         self.mark = None
+        self.max_mhz = None
         try:
+            import pynvml as nv
+            nv.nvmlInit()
             uuid = str(torch.cuda.get_device_properties(device).uuid)
-            sel = ["-i", uuid if uuid.startswith("GPU-") else "GPU-" + uuid]
-        except Exception:
-            sel = []
-        self.cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                    "-lms", "200", *sel]
+            if not uuid.startswith("GPU-"):
+                uuid = "GPU-" + uuid
+            self.h = nv.nvmlDeviceGetHandleByUUID(uuid)
+            self.max_mhz = float(nv.nvmlDeviceGetMaxClockInfo(self.h, nv.NVML_CLOCK_SM))
+            self.nv = nv
+        except Exception as e:  # no NVML: clocks are reported as unknown
+            log(f"clock sampler unavailable: {e}")
+
+    def _reasons(self):
+        nv = self.nv
+        fn = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            getattr(nv, "nvmlDeviceGetCurrentClocksThrottleReasons")
+        return int(fn(self.h))
+
+    def _poll(self):
+        while not self.done.is_set():
+            try:
+                sm = float(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                self.samples.append((time.time(), sm, self._reasons()))
+            except Exception:
+                pass
+            time.sleep(0.02)
 
     def start(self):
-        try:
-            self.proc = subprocess.Popen(self.cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
-                                         text=True)
-        except OSError:
-            self.proc = None
+        if self.nv is None:
             return
-        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.done = threading.Event()
+        self.thread = threading.Thread(target=self._poll, daemon=True)
         self.thread.start()
-        t0 = time.time()
-        while not self.lines and time.time() - t0 < 5:
-            time.sleep(0.05)
-
-    def _read(self):
-        for ln in self.proc.stdout:
-            self.lines.append((time.time(), ln.strip()))
 
     def begin_load(self):
         self.mark = time.time()
 
     def stop(self):
         end = time.time()
-        if self.proc is None:
-            return None
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-        rows = [ln for (t, ln) in self.lines if self.mark is None or self.mark <= t <= end + 0.2]
-        sm, mx, reasons = [], 0.0, set()
-        for ln in rows:
-            parts = [p.strip() for p in ln.split(",")]
-            if len(parts) < 7:
-                continue
-            try:
-                sm.append(float(parts[0]))
-                mx = max(mx, float(parts[1]))
-            except ValueError:
-                continue
-            for name, val in zip(self.REASONS, parts[3:7]):
-                if val.lower().startswith("active"):
-                    reasons.add(name)
-        if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+        if self.nv is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0,
+                    "source": "unavailable"}
+        self.done.set()
+        self.thread.join(timeout=2)
+        rows = [(sm, r) for (t, sm, r) in self.samples if self.mark is None or self.mark <= t <= end]
+        reasons = sorted({n for (_, r) in rows for n, b in self.REASON_BITS.items() if r & b})
+        sm = [x for (x, _) in rows]
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(sm), "source": "NVML, 20 ms polling"}
 
 
 # ---------------------------------------------------------------- oracle helpers
@@ -170,9 +166,7 @@ def oracle_sample_rate(wl, inp, n_tokens: int):
     toks = synth.token_sample(wl.T, n_tokens).numpy()
     t0 = time.perf_counter()
     O.moe_forward(P["x"], P, tokens=toks, logits=r["logits"], **kw)
-    t_all = time.perf_counter() - t0
-    # moe_forward re-runs the (cheap, given logits) selection/dispatch; count it once
-    t_ffn = max(t_all - 0.0, 1e-9)
+    t_ffn = time.perf_counter() - t0  # includes the (cheap) re-selection from given logits
     per_token = t_route / wl.T + t_ffn / len(toks)
     desc = (f"oracle (numpy fp64): routing of all {wl.T} tokens ({t_route:.2f} s) + expert "
             f"FFNs of {len(toks)} strided tokens ({t_ffn:.2f} s); tokens/s = 1 / "
