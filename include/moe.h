@@ -161,6 +161,30 @@ moe_status_t moe_permute(const moe_cfg_t *cfg, const void *x, const int32_t *top
                          int32_t *counts, int32_t *offsets, int32_t *perm, int32_t *inv,
                          void *x_perm, void *ws, size_t ws_bytes, moe_stream_t stream);
 
+/* moe_permute for callers that cannot allocate device memory. (No counterpart on
+ * the pages: it is a deployment variant of the permute step above.)
+ * Some callers own no device memory beyond their inputs and outputs — a plugin
+ * or operator inside a framework that manages every other byte through its own
+ * arena, or a latency-critical loop where cudaMalloc (which may synchronise the
+ * device) is not allowed — so they cannot pass the workspace moe_permute needs.
+ * This variant takes the same inputs and outputs, with the same meaning, and
+ * keeps its scratch (per-tile expert counts and their prefix sums) in a fixed
+ * static device array of the library (about 0.5 MB, held on every GPU that uses
+ * the library until the process exits). It allocates nothing.
+ * Limit: n_experts * ceil(T / tile) <= 65536, with tile = 32 tokens for E <= 32,
+ * 64 for E <= 128 and 32 above (E = 8: T <= 262144; E = 128: T <= 32768);
+ * larger problems return MOE_ERR_WORKSPACE. d_model * element size must be a
+ * multiple of 16 bytes.
+ * All calls share the static array: calls that overlap on the GPU race, so the
+ * caller must serialise them (one stream, or explicit ordering). The first call on
+ * each device looks up the array's device address (cudaGetSymbolAddress); make
+ * that first call before any stream capture. Out-of-range expert indices are not
+ * reported (there is no workspace for the error word); such a pair is treated as
+ * dropped (inv = -1). */
+moe_status_t moe_permute_noalloc(const moe_cfg_t *cfg, const void *x, const int32_t *topk_idx,
+                                 int32_t *counts, int32_t *offsets, int32_t *perm, int32_t *inv,
+                                 void *x_perm, moe_stream_t stream);
+
 /* Expert FFNs on expert-contiguous rows ("SwiGLUExpert", MLP experts).
  * Rows [offsets[e], offsets[e+1]) of x_perm [T*k, d] go through expert e and the
  * result is written to the same rows of y_perm [T*k, d] (dtype). offsets is a

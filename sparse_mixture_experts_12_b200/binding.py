@@ -27,6 +27,7 @@ DEVERR_NAMES = {0: "none", 1: "expert index out of range", 2: "invalid offsets",
                 3: "row index out of range", 4: "pipeline wait timeout"}
 
 EXPORTED = ("moe_workspace_size", "moe_workspace_init", "moe_route", "moe_permute",
+            "moe_permute_noalloc",
             "moe_expert_ffn", "moe_combine", "moe_aux_stats", "moe_forward",
             "moe_last_device_error", "moe_status_string")
 
@@ -77,6 +78,7 @@ def load() -> ctypes.CDLL:
         "moe_workspace_init": [P, S, P],
         "moe_route": [cfgp, wp, P, P, P, P, P, S, P],
         "moe_permute": [cfgp, P, P, P, P, P, P, P, P, S, P],
+        "moe_permute_noalloc": [cfgp, P, P, P, P, P, P, P, P],
         "moe_expert_ffn": [cfgp, wp, P, P, P, P, S, P],
         "moe_combine": [cfgp, P, P, P, P, P, P, S, P],
         "moe_aux_stats": [cfgp, P, P, P, P, S, P],
