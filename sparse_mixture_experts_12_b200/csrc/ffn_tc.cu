@@ -7,44 +7,45 @@
 // an expert are multiplied by its weights ("Token Routing": unselected experts
 // are not computed at all).
 //
-// Design (one persistent CTA per SM, 256 threads, warp-specialised):
-//   warp 0      TMA producer: A tile [128 rows x 64 k] of the expert-contiguous
-//               activations and the B tile [256 rows x 64 k] of the expert's
-//               weights into a 4-stage shared-memory ring (128-byte swizzle).
-//               For SwiGLU the B tile is w_gate rows [n, n+128) stacked on w_up
-//               rows [n, n+128), so one N=256 MMA yields both halves.
-//   warp 1      MMA issuer: tcgen05.mma M=128 N=256 K=16, accumulator in TMEM,
-//               two 256-column accumulators so the epilogue of tile i overlaps
-//               the main loop of tile i+1.
+// Design (persistent, warp-specialised, 384 threads per CTA):
+//   warp 0      TMA producer: A rows of the expert-contiguous activations and the
+//               expert's weight rows, 64-element K slices with 128-byte swizzle,
+//               into a shared-memory ring.
+//   warp 1      MMA issuer: tcgen05.mma (kind::f16, fp32 accumulate in TMEM), two
+//               256-column accumulators so the epilogue of tile i overlaps the
+//               main loop of tile i+1.
 //   warp 2      TMEM allocator.
-//   warps 4..7  epilogue: tcgen05.ld, fused silu(g)*u / bias+ReLU / bias+GELU,
+//   warps 4..11 epilogue (two warps per TMEM lane quarter, half the columns
+//               each): tcgen05.ld, fused silu(g)*u / bias+ReLU / bias+GELU,
 //               bf16 (or fp32) stores masked to the expert's rows.
+// Two tile shapes: a CTA pair (cluster of 2, tcgen05.mma.cta_group::2, 256 rows x
+// 256 columns, 6 x 32 KB stages per CTA) by default, and a single CTA (128 rows x
+// 256 columns, 4 x 48 KB stages). For SwiGLU the 256 MMA columns are w_gate rows
+// [n, n+128) next to w_up rows [n, n+128), so one MMA yields both halves.
 // The tile list is built on the device (per-expert M-tile prefix), so no host
 // synchronisation sits between routing and the expert GEMMs. Every wait is
 // bounded; on a timeout the CTA records MOE_DEVERR_WAIT_TIMEOUT, drains its
 // in-flight copies and MMAs, frees TMEM and returns.
-#include <cuda.h>
-#include <cudaTypedefs.h>
-
 #include <algorithm>
 #include <mutex>
 
-#include "kernels.cuh"
+#include "tc_ptx.cuh"
 
 namespace moe {
 
 namespace {
 
+using namespace tc;
+
 constexpr int kStages = 4;
-constexpr int kBlockK = 64;  // 64 bf16 = one 128-byte swizzle row
 constexpr int kTileM = kRowTile;
 constexpr int kMmaN = 256;
 constexpr int kABytes = kTileM * kBlockK * 2;
 constexpr int kBBytes = kMmaN * kBlockK * 2;
 constexpr int kStageBytes = kABytes + kBBytes;
 constexpr int kTmemCols = 2 * kMmaN;
-constexpr int kThreads = 256;
-constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
+constexpr int kThreads = 384;  // warps 0-3: producer, MMA, TMEM, spare; 4-11: epilogue
+constexpr int kEpiWarps = 8;
 
 enum { EPI_SWIGLU = 0, EPI_ACT = 1, EPI_DOWN = 2 };
 
@@ -74,154 +75,96 @@ struct SmemCtl {
 
 constexpr size_t kSmemBytes = (size_t)kStages * kStageBytes + sizeof(SmemCtl) + 1024;
 
-// ------------------------------------------------------------------ PTX helpers
-__device__ __forceinline__ uint32_t smem_u32(const void *p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+
+__device__ __forceinline__ bool wait_bounded(uint64_t *bar, uint32_t parity, SmemCtl *ctl,
+                                             int32_t *err, int site, bool honour_abort = true) {
+  return wait_mbar(bar, parity, &ctl->abort_flag, 0u, err, site, honour_abort, kWaitLimitNs);
 }
-__device__ __forceinline__ uint64_t globaltimer_ns() {
-  uint64_t t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
-__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
-}
-__device__ __forceinline__ void fence_mbar_init() {
-  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-}
-__device__ __forceinline__ void mbar_expect_tx(uint64_t *bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
-               "r"(bytes)
-               : "memory");
-}
-__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
-__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}\n"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-// Wait for the phase of `parity` to complete. Gives up when another role has
-// aborted (honour_abort) or after kWaitLimitNs, recording the site.
-__device__ __noinline__ bool wait_bounded(uint64_t *bar, uint32_t parity, SmemCtl *ctl,
-                                          int32_t *err, int site, bool honour_abort = true) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = globaltimer_ns();
-  volatile int *abort_flag = &ctl->abort_flag;
-  while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if (honour_abort && *abort_flag) return false;
-    if (globaltimer_ns() - t0 > kWaitLimitNs) {
-      *abort_flag = 1;
-      report_error(err, MOE_DEVERR_WAIT_TIMEOUT, site);
-      return false;
+
+// ------------------------------------------------------------ shared epilogue
+// One accumulator tile (this thread's TMEM lane = one output row) -> global.
+// SwiGLU: columns [0,128) hold x.w_gate, [128,256) x.w_up; h = silu(g) * u.
+// ACT: bias + ReLU / GELU. DOWN: + bias. Stores are masked to the valid row and
+// to the N extent.
+template <int EPI>
+__device__ __forceinline__ void epilogue_tile(const TcArgs &a, uint32_t tbase, int g, int n,
+                                              bool valid, size_t orow, int half) {
+  // the two epilogue warps that share a TMEM lane quarter take half the columns each
+  if (EPI == EPI_SWIGLU) {
+    __nv_bfloat16 *out = static_cast<__nv_bfloat16 *>(a.out);
+#pragma unroll 1
+    for (int c = 2 * half; c < 2 * half + 2; ++c) {
+      uint32_t gv[32], uv[32];
+      tmem_ld32(tbase + c * 32, gv);
+      tmem_ld32(tbase + kMmaN / 2 + c * 32, uv);
+      tmem_ld_wait();
+      const int col0 = n * (kMmaN / 2) + c * 32;
+      if (valid && col0 < a.N) {
+        uint4 *dst = reinterpret_cast<uint4 *>(out + orow * a.N + col0);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          float h[8];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const float gt = __uint_as_float(gv[q * 8 + j]);
+            const float up = __uint_as_float(uv[q * 8 + j]);
+            h[j] = __fdividef(gt, 1.f + __expf(-gt)) * up;
+          }
+          dst[q] = pack16(h);
+        }
+      }
+    }
+  } else {
+#pragma unroll 1
+    for (int c = 4 * half; c < 4 * half + 4; ++c) {
+      uint32_t v[32];
+      tmem_ld32(tbase + c * 32, v);
+      tmem_ld_wait();
+      const int col0 = n * kMmaN + c * 32;
+      if (valid && col0 < a.N) {
+        float f[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) f[j] = __uint_as_float(v[j]);
+        if (a.bias) {  // the same 32 values for every lane: broadcast 16-byte loads
+          const float4 *b4 = reinterpret_cast<const float4 *>(a.bias + (size_t)g * a.N + col0);
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            const float4 b = __ldg(b4 + q);
+            f[4 * q] += b.x; f[4 * q + 1] += b.y; f[4 * q + 2] += b.z; f[4 * q + 3] += b.w;
+          }
+        }
+        if (EPI == EPI_ACT) {
+          if (a.act == MOE_ACT_RELU) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) f[j] = fmaxf(f[j], 0.f);
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) f[j] = gelu_erf(f[j]);
+          }
+        }
+        if (a.out_f32) {
+          float4 *dst =
+              reinterpret_cast<float4 *>(static_cast<float *>(a.out) + orow * a.N + col0);
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            dst[q] = make_float4(f[4 * q], f[4 * q + 1], f[4 * q + 2], f[4 * q + 3]);
+        } else {
+          uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(a.out) +
+                                                 orow * a.N + col0);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            float h[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) h[j] = f[q * 8 + j];
+            dst[q] = pack16(h);
+          }
+        }
+      }
     }
   }
 }
-__device__ __forceinline__ void tma_load_2d(const CUtensorMap *map, uint64_t *bar, void *dst,
-                                            int c0, int c1) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1)
-      : "memory");
-}
-__device__ __forceinline__ void prefetch_map(const CUtensorMap *map) {
-  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
-}
-__device__ __forceinline__ void tc_fence_before() {
-  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-}
-__device__ __forceinline__ void tc_fence_after() {
-  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-}
-__device__ __forceinline__ void tmem_alloc(uint32_t *dst, uint32_t ncols) {
-  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-                   smem_u32(dst)),
-               "r"(ncols)
-               : "memory");
-}
-__device__ __forceinline__ void tmem_relinquish() {
-  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
-  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
-               : "memory");
-}
-__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
-                                          uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
-      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-__device__ __forceinline__ void umma_commit(uint64_t *bar) {
-  asm volatile(
-      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-          smem_u32(bar))
-      : "memory");
-}
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
-        "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
-        "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
-        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
-        "=r"(r[31])
-      : "r"(taddr));
-}
-__device__ __forceinline__ void tmem_ld_wait() {
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-}
 
-// Shared-memory matrix descriptor: K-major operand, 128-byte swizzle, rows of
-// 128 bytes grouped in 8-row (1024-byte) swizzle atoms.
-__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
-  uint64_t d = 0;
-  d |= (uint64_t)((saddr >> 4) & 0x3FFFu);  // start address
-  d |= (uint64_t)1 << 16;                    // leading-dim byte offset (unused here)
-  d |= (uint64_t)(1024 >> 4) << 32;          // stride-dim byte offset: 8 rows x 128 B
-  d |= (uint64_t)1 << 46;                    // descriptor version (sm_100)
-  d |= (uint64_t)2 << 61;                    // SWIZZLE_128B
-  return d;
-}
-// Instruction descriptor, kind::f16: D fp32, A and B bf16, both K-major.
-__host__ __device__ constexpr uint32_t make_idesc(int M, int N) {
-  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) |
-         ((uint32_t)(M >> 4) << 24);
-}
-
-__device__ __forceinline__ void decode_tile(int tile, const int *mpre, int G, int n_tiles,
-                                            int &g, int &n, int &m) {
-  int lo = 0, hi = G - 1;  // last g with mpre[g] * n_tiles <= tile (never an empty group)
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (mpre[mid] * n_tiles <= tile) lo = mid; else hi = mid - 1;
-  }
-  g = lo;
-  const int mt = mpre[g + 1] - mpre[g];
-  const int local = tile - mpre[g] * n_tiles;
-  n = local / mt;
-  m = local % mt;
-}
-
-__device__ __forceinline__ float gelu_erf(float v) {
-  return 0.5f * v * (1.f + erff(v * 0.70710678118654752f));
-}
-
+// =========================================================== single-CTA kernel
 template <int EPI>
 __global__ void __launch_bounds__(kThreads, 1)
 k_ffn_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -245,7 +188,7 @@ k_ffn_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtens
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&ctl->tfull[s], 1);
-      mbar_init(&ctl->tempty[s], 4 * 32);
+      mbar_init(&ctl->tempty[s], kEpiWarps * 32);
     }
     mbar_init(&ctl->drain, 1);
     ctl->abort_flag = 0;
@@ -332,7 +275,8 @@ k_ffn_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtens
     }
   } else if (warp >= 4) {
     // ----------------------------------------------------------------- epilogue
-    const int ew = warp - 4;  // TMEM lanes [32*ew, 32*ew + 32)
+    const int ew = warp & 3;          // TMEM lanes [32*ew, 32*ew + 32) (warp % 4)
+    const int half = (warp - 4) >> 2;  // which half of the tile's columns
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
@@ -346,65 +290,7 @@ k_ffn_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtens
       const bool valid = grow < offs[g + 1] - offs[g];
       const size_t orow = (size_t)offs[g] + grow;
       const uint32_t tbase = tmem + ((uint32_t)(ew * 32) << 16) + (uint32_t)(acc * kMmaN);
-      if (EPI == EPI_SWIGLU) {
-        __nv_bfloat16 *out = static_cast<__nv_bfloat16 *>(a.out);
-#pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-          uint32_t gv[32], uv[32];
-          tmem_ld32(tbase + c * 32, gv);
-          tmem_ld32(tbase + kMmaN / 2 + c * 32, uv);
-          tmem_ld_wait();
-          const int col0 = n * (kMmaN / 2) + c * 32;
-          if (valid && col0 < a.N) {
-            uint4 *dst = reinterpret_cast<uint4 *>(out + orow * a.N + col0);
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              float h[8];
-#pragma unroll
-              for (int j = 0; j < 8; ++j) {
-                const float gt = __uint_as_float(gv[q * 8 + j]);
-                const float up = __uint_as_float(uv[q * 8 + j]);
-                h[j] = gt / (1.f + __expf(-gt)) * up;
-              }
-              dst[q] = pack16(h);
-            }
-          }
-        }
-      } else {
-#pragma unroll 1
-        for (int c = 0; c < kMmaN / 32; ++c) {
-          uint32_t v[32];
-          tmem_ld32(tbase + c * 32, v);
-          tmem_ld_wait();
-          const int col0 = n * kMmaN + c * 32;
-          if (valid && col0 < a.N) {
-            float f[32];
-#pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              float x = __uint_as_float(v[j]);
-              if (a.bias) x += __ldg(a.bias + (size_t)g * a.N + col0 + j);
-              if (EPI == EPI_ACT) x = (a.act == MOE_ACT_RELU) ? fmaxf(x, 0.f) : gelu_erf(x);
-              f[j] = x;
-            }
-            if (a.out_f32) {
-              float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(a.out) + orow * a.N + col0);
-#pragma unroll
-              for (int q = 0; q < 8; ++q)
-                dst[q] = make_float4(f[4 * q], f[4 * q + 1], f[4 * q + 2], f[4 * q + 3]);
-            } else {
-              uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(a.out) +
-                                                     orow * a.N + col0);
-#pragma unroll
-              for (int q = 0; q < 4; ++q) {
-                float h[8];
-#pragma unroll
-                for (int j = 0; j < 8; ++j) h[j] = f[q * 8 + j];
-                dst[q] = pack16(h);
-              }
-            }
-          }
-        }
-      }
+      epilogue_tile<EPI>(a, tbase, g, n, valid, orow, half);
       tc_fence_before();
       mbar_arrive(&ctl->tempty[acc]);
       if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
@@ -418,38 +304,218 @@ k_ffn_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtens
   }
 }
 
+// ============================================================= CTA-pair kernel
+// Two CTAs of a cluster share one 256-row tile: CTA r holds A rows [128r, 128r+128)
+// and B rows [128r, 128r+128) of the 256-row B tile (for SwiGLU: CTA 0 the w_gate
+// rows, CTA 1 the w_up rows). The leader (rank 0) issues tcgen05.mma.cta_group::2
+// M=256 N=256 K=16, which reads both CTAs' shared memory and writes both CTAs'
+// TMEM (rows 128r.. in CTA r). Each CTA's own TMA loads (no multicast) count on the
+// leader's `full` barrier; the MMA commits release `empty` and `tfull` in both
+// CTAs; both epilogues release the leader's `tempty`. Per CTA a stage is 32 KB
+// (vs 48 KB for the single-CTA tile), so six stages fit.
+constexpr int kStages2 = 6;
+constexpr int kPairM = 2 * kTileM;
+constexpr int kAHalf = kTileM * kBlockK * 2;
+constexpr int kBHalf = (kMmaN / 2) * kBlockK * 2;
+constexpr int kStage2Bytes = kAHalf + kBHalf;
+constexpr uint64_t kDrainNs = 50000000ull;  // 50 ms bound on end-of-kernel drains
+
+struct SmemCtl2 {
+  uint64_t full[kStages2];   // leader: both CTAs' copies of the stage landed
+  uint64_t empty[kStages2];  // each CTA: the pair's MMAs are done with the stage
+  uint64_t tfull[2];         // each CTA: accumulator ready for the epilogue
+  uint64_t tempty[2];        // leader: both epilogues have drained the accumulator
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort_flag;
+  int tbl[2 * (kMaxExperts + 1)];  // pair-tile prefix [G+1], offsets [G+1]
+};
+
+constexpr size_t kSmem2Bytes = (size_t)kStages2 * kStage2Bytes + sizeof(SmemCtl2) + 1024;
+
+// Bounded wait that, on its own timeout, also raises the peer CTA's abort flag.
+__device__ __forceinline__ bool wait_pair(uint64_t *bar, uint32_t parity, SmemCtl2 *ctl,
+                                          uint32_t peer_abort, int32_t *err, int site,
+                                          bool honour_abort = true,
+                                          uint64_t limit_ns = kWaitLimitNs) {
+  return wait_mbar(bar, parity, &ctl->abort_flag, peer_abort, err, site, honour_abort, limit_ns);
+}
+
+template <int EPI>
+__global__ void __launch_bounds__(kThreads, 1)
+k_ffn_tc2(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+          const __grid_constant__ CUtensorMap tmB3, TcArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  SmemCtl2 *ctl = reinterpret_cast<SmemCtl2 *>(smem + (size_t)kStages2 * kStage2Bytes);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int G = a.G;
+  int *ppre = ctl->tbl;
+  int *offs = ctl->tbl + (G + 1);
+  for (int i = tid; i <= G; i += kThreads) offs[i] = a.offsets[i];
+  if (tid == 0) {
+    for (int s = 0; s < kStages2; ++s) {
+      mbar_init(&ctl->full[s], 1);
+      mbar_init(&ctl->empty[s], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&ctl->tfull[s], 1);
+      mbar_init(&ctl->tempty[s], 2 * kEpiWarps * 32);
+    }
+    mbar_init(&ctl->drain, 1);
+    ctl->abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    // pair tiles per group = ceil(ceil(rows / 128) / 2) from the 128-row tile prefix
+    // (all zero when the offsets failed validation); warp scan over the groups
+    const int per = ceil_div(G, 32);
+    const int j0 = min(G, lane * per), j1 = min(G, j0 + per);
+    int sum = 0;
+    for (int j = j0; j < j1; ++j) sum += (a.mprefix[j + 1] - a.mprefix[j] + 1) >> 1;
+    int incl = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    int run = incl - sum;
+    for (int j = j0; j < j1; ++j) {
+      ppre[j] = run;
+      run += (a.mprefix[j + 1] - a.mprefix[j] + 1) >> 1;
+    }
+    if (lane == 31) ppre[G] = incl;
+  }
+  if (warp == 2) {
+    tmem_alloc_pair(&ctl->tmem_base, kTmemCols);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();  // both CTAs' barriers and TMEM exist before any cross-CTA use
+  tc_fence_after();
+  const uint32_t tmem = ctl->tmem_base;
+  const int total = ppre[G] * a.n_tiles;
+  const int nkb = ceil_div(a.K, kBlockK);
+  const uint32_t peer_abort = mapa_rank(smem_u32(&ctl->abort_flag), rank ^ 1u);
+  const int c0 = (int)cluster_index(), cstep = (int)cluster_count();
+
+  if (warp == 0 && lane == 0) {
+    // ------------------------------------------------------------ TMA producer
+    prefetch_map(&tmA);
+    prefetch_map(&tmB);
+    if (EPI == EPI_SWIGLU) prefetch_map(&tmB3);
+    const uint32_t full0 = mapa_rank(smem_u32(&ctl->full[0]), 0);  // the leader's barriers
+    const CUtensorMap *bmap = (EPI == EPI_SWIGLU && rank == 1) ? &tmB3 : &tmB;
+    int stage = 0;
+    uint32_t phase = 0, issued = 0, last_phase = 0;
+    bool ok = true;
+    for (int tile = c0; ok && tile < total; tile += cstep) {
+      int g, n, m;
+      decode_tile(tile, ppre, G, a.n_tiles, g, n, m);
+      const int arow = offs[g] + m * kPairM + (int)rank * kTileM;
+      const int brow = (EPI == EPI_SWIGLU) ? g * a.b_rows + n * (kMmaN / 2)
+                                           : g * a.b_rows + n * kMmaN + (int)rank * (kMmaN / 2);
+      for (int kb = 0; kb < nkb; ++kb) {
+        if (!wait_pair(&ctl->empty[stage], phase ^ 1u, ctl, peer_abort, a.err, 1)) {
+          ok = false;
+          break;
+        }
+        if (leader) mbar_expect_tx(&ctl->full[stage], 2 * kStage2Bytes);
+        uint8_t *sa = smem + (size_t)stage * kStage2Bytes;
+        const uint32_t fb = full0 + (uint32_t)(stage * sizeof(uint64_t));
+        tma_load_2d_pair(&tmA, fb, sa, kb * kBlockK, arow);
+        tma_load_2d_pair(bmap, fb, sa + kAHalf, kb * kBlockK, brow);
+        issued |= 1u << stage;
+        last_phase = (last_phase & ~(1u << stage)) | (phase << stage);
+        if (++stage == kStages2) { stage = 0; phase ^= 1u; }
+      }
+    }
+    // wait until the pair's MMAs have released every stage this CTA filled: the
+    // last reads of our shared memory and the commit arrivals on our barriers are done
+    for (int s = 0; s < kStages2; ++s)
+      if (issued & (1u << s))
+        wait_pair(&ctl->empty[s], (last_phase >> s) & 1u, ctl, peer_abort, nullptr, 0, false,
+                  ok ? kWaitLimitNs : kDrainNs);
+  } else if (warp == 1 && lane == 0 && leader) {
+    // --------------------------------------------------------------- MMA issuer
+    constexpr uint32_t idesc = make_idesc(kPairM, kMmaN);
+    int stage = 0, acc = 0;
+    uint32_t phase = 0, acc_phase = 0;
+    bool ok = true, any = false;
+    for (int tile = c0; ok && tile < total; tile += cstep) {
+      if (!wait_pair(&ctl->tempty[acc], acc_phase ^ 1u, ctl, peer_abort, a.err, 2)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t d_tmem = tmem + (uint32_t)(acc * kMmaN);
+      for (int kb = 0; kb < nkb; ++kb) {
+        if (!wait_pair(&ctl->full[stage], phase, ctl, peer_abort, a.err, 3)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t sa = smem_u32(smem + (size_t)stage * kStage2Bytes);
+        const uint64_t da = sw128_desc(sa);
+        const uint64_t db = sw128_desc(sa + kAHalf);
+#pragma unroll
+        for (int kk = 0; kk < kBlockK / 16; ++kk)
+          umma_bf16_pair(d_tmem, da + 2 * kk, db + 2 * kk, idesc, (kb | kk) != 0);
+        any = true;
+        umma_commit_pair_both(&ctl->empty[stage]);
+        if (++stage == kStages2) { stage = 0; phase ^= 1u; }
+      }
+      if (!ok) break;
+      umma_commit_pair_both(&ctl->tfull[acc]);
+      if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+    }
+    if (!ok && any) {  // retire the MMAs in flight before TMEM is released
+      umma_commit_pair_own(&ctl->drain);
+      wait_pair(&ctl->drain, 0, ctl, peer_abort, nullptr, 0, false, kDrainNs);
+    }
+  } else if (warp >= 4) {
+    // ----------------------------------------------------------------- epilogue
+    const int ew = warp & 3;
+    const int half = (warp - 4) >> 2;
+    const uint32_t tempty0 = mapa_rank(smem_u32(&ctl->tempty[0]), 0);
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int tile = c0; tile < total; tile += cstep) {
+      int g, n, m;
+      decode_tile(tile, ppre, G, a.n_tiles, g, n, m);
+      bool ok = wait_pair(&ctl->tfull[acc], acc_phase, ctl, peer_abort, a.err, 4);
+      __syncwarp();
+      if (!__all_sync(0xffffffffu, ok)) break;
+      tc_fence_after();
+      const int grow = m * kPairM + (int)rank * kTileM + ew * 32 + lane;
+      const bool valid = grow < offs[g + 1] - offs[g];
+      const size_t orow = (size_t)offs[g] + grow;
+      const uint32_t tbase = tmem + ((uint32_t)(ew * 32) << 16) + (uint32_t)(acc * kMmaN);
+      epilogue_tile<EPI>(a, tbase, g, n, valid, orow, half);
+      tc_fence_before();
+      mbar_arrive_cluster(tempty0 + (uint32_t)(acc * sizeof(uint64_t)));
+      if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+    }
+  }
+  if (*(volatile int *)&ctl->abort_flag) settle_ns(100000);  // copies in flight land
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();  // the peer's remote arrivals are done before either CTA exits
+  if (warp == 2) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem, kTmemCols);
+  }
+}
+
 // ------------------------------------------------------------------ host side
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void *p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  });
-  return fn;
-}
-
-// 2-D bf16 map over a row-major [rows, cols] matrix; box = [box_rows, 64 cols].
-bool make_map(CUtensorMap *map, const void *ptr, uint64_t rows, uint64_t cols, uint32_t box_rows) {
-  auto fn = encode_fn();
-  if (fn == nullptr) return false;
-  cuuint64_t dims[2] = {cols, rows};
-  cuuint64_t strides[1] = {cols * 2};
-  cuuint32_t box[2] = {(cuuint32_t)kBlockK, box_rows};
-  cuuint32_t estr[2] = {1, 1};
-  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(ptr), dims, strides,
-                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
-}
-
 struct DeviceInfo {
   int sms = 0;
-  bool attr_set[3] = {false, false, false};
+  bool attr_set[6] = {false, false, false, false, false, false};
+  int max_pairs[3] = {0, 0, 0};
 };
 
 DeviceInfo &device_info(int dev) {
@@ -457,16 +523,17 @@ DeviceInfo &device_info(int dev) {
   return infos[dev & 63];
 }
 
+std::mutex g_attr_mu;
+
 template <int EPI>
-cudaError_t launch_one(const CUtensorMap &ma, const CUtensorMap &mb, const CUtensorMap &mb3,
-                       const TcArgs &t, int grid, cudaStream_t st) {
+cudaError_t launch_single(const CUtensorMap &ma, const CUtensorMap &mb, const CUtensorMap &mb3,
+                          const TcArgs &t, long long tiles_ub, cudaStream_t st) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   DeviceInfo &info = device_info(dev);
-  static std::mutex mu;
   {
-    std::lock_guard<std::mutex> lock(mu);
+    std::lock_guard<std::mutex> lock(g_attr_mu);
     if (!info.attr_set[EPI]) {
       e = cudaFuncSetAttribute(k_ffn_tc<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                (int)kSmemBytes);
@@ -474,36 +541,82 @@ cudaError_t launch_one(const CUtensorMap &ma, const CUtensorMap &mb, const CUten
       info.attr_set[EPI] = true;
     }
   }
+  const int grid = (int)std::min<long long>(tiles_ub, sm_count());
   k_ffn_tc<EPI><<<grid, kThreads, kSmemBytes, st>>>(ma, mb, mb3, t);
   return cudaGetLastError();
 }
 
-int sm_count() {
+template <int EPI>
+cudaError_t launch_pair(const CUtensorMap &ma, const CUtensorMap &mb, const CUtensorMap &mb3,
+                        const TcArgs &t, long long tiles_ub, cudaStream_t st) {
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
   DeviceInfo &info = device_info(dev);
-  if (info.sms == 0) {
-    int n = 0;
-    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
-      n = 148;
-    info.sms = n;
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = kSmem2Bytes;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  {
+    std::lock_guard<std::mutex> lock(g_attr_mu);
+    if (!info.attr_set[3 + EPI]) {
+      e = cudaFuncSetAttribute(k_ffn_tc2<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)kSmem2Bytes);
+      if (e != cudaSuccess) return e;
+      cfg.gridDim = dim3(2 * (sm_count() / 2));
+      int n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, k_ffn_tc2<EPI>, &cfg) != cudaSuccess || n <= 0)
+        n = sm_count() / 2;
+      info.max_pairs[EPI] = n;
+      info.attr_set[3 + EPI] = true;
+    }
   }
-  return info.sms;
+  const long long pairs = std::min<long long>(tiles_ub, info.max_pairs[EPI]);
+  cfg.gridDim = dim3((unsigned)(2 * pairs));
+  e = cudaLaunchKernelEx(&cfg, k_ffn_tc2<EPI>, ma, mb, mb3, t);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+// Pair tiles (256 rows) halve the operand traffic per MMA; single-CTA tiles (128
+// rows) waste less work when experts hold few rows. Both compute the same result.
+#ifndef MOE_TC_SINGLE_CTA
+constexpr bool kUsePairs = true;
+#else
+constexpr bool kUsePairs = false;
+#endif
+
+template <int EPI>
+cudaError_t launch_gemm(const CUtensorMap &ma, const CUtensorMap &mb, const CUtensorMap &mb3,
+                        const TcArgs &t, int m_tiles_ub, int groups, cudaStream_t st) {
+  if (kUsePairs) {
+    const long long pairs_ub = (long long)(m_tiles_ub + groups + 1) / 2 * t.n_tiles;
+    return launch_pair<EPI>(ma, mb, mb3, t, std::max<long long>(pairs_ub, 1), st);
+  }
+  return launch_single<EPI>(ma, mb, mb3, t, (long long)m_tiles_ub * t.n_tiles, st);
 }
 
 }  // namespace
 
 cudaError_t launch_ffn_tc(const GroupedFfnArgs &a, cudaStream_t st) {
   if (a.m_tiles_ub <= 0) return cudaSuccess;
-  const int sms = sm_count();
   const bool swiglu = a.act == MOE_ACT_SWIGLU;
+  // single-CTA tiles load 256 B rows at once (SwiGLU: two 128-row halves); pair
+  // tiles load 128 B rows per CTA
+  const uint32_t b_box = (kUsePairs || swiglu) ? kMmaN / 2 : kMmaN;
   CUtensorMap ma, mb, mb3;
   // up projection: [rows, d] x [G*F, d]^T -> h [rows, F]
   if (!make_map(&ma, a.a, (uint64_t)a.a_rows, (uint64_t)a.d, kTileM)) return cudaErrorInvalidValue;
-  if (!make_map(&mb, a.w1, (uint64_t)a.G * a.F, (uint64_t)a.d, swiglu ? kMmaN / 2 : kMmaN))
-    return cudaErrorInvalidValue;
+  if (!make_map(&mb, a.w1, (uint64_t)a.G * a.F, (uint64_t)a.d, b_box)) return cudaErrorInvalidValue;
   if (swiglu) {
-    if (!make_map(&mb3, a.w3, (uint64_t)a.G * a.F, (uint64_t)a.d, kMmaN / 2))
+    if (!make_map(&mb3, a.w3, (uint64_t)a.G * a.F, (uint64_t)a.d, b_box))
       return cudaErrorInvalidValue;
   } else {
     mb3 = mb;
@@ -521,13 +634,13 @@ cudaError_t launch_ffn_tc(const GroupedFfnArgs &a, cudaStream_t st) {
   t.bias = a.b1;
   t.act = a.act;
   t.err = a.err;
-  int grid = (int)std::min<long long>((long long)a.m_tiles_ub * t.n_tiles, sms);
-  cudaError_t e = swiglu ? launch_one<EPI_SWIGLU>(ma, mb, mb3, t, grid, st)
-                         : launch_one<EPI_ACT>(ma, mb, mb3, t, grid, st);
+  cudaError_t e = swiglu ? launch_gemm<EPI_SWIGLU>(ma, mb, mb3, t, a.m_tiles_ub, a.G, st)
+                         : launch_gemm<EPI_ACT>(ma, mb, mb3, t, a.m_tiles_ub, a.G, st);
   if (e != cudaSuccess) return e;
   // down projection: h [rows, F] x [G*d, F]^T -> out [rows, d]
+  const uint32_t b_box2 = kUsePairs ? kMmaN / 2 : kMmaN;
   if (!make_map(&ma, a.h, (uint64_t)a.a_rows, (uint64_t)a.F, kTileM)) return cudaErrorInvalidValue;
-  if (!make_map(&mb, a.w2, (uint64_t)a.G * a.d, (uint64_t)a.F, kMmaN)) return cudaErrorInvalidValue;
+  if (!make_map(&mb, a.w2, (uint64_t)a.G * a.d, (uint64_t)a.F, b_box2)) return cudaErrorInvalidValue;
   t.N = a.d;
   t.K = a.F;
   t.n_tiles = ceil_div(a.d, kMmaN);
@@ -536,8 +649,7 @@ cudaError_t launch_ffn_tc(const GroupedFfnArgs &a, cudaStream_t st) {
   t.out_f32 = a.out_f32;
   t.bias = a.b2;
   t.act = -1;
-  grid = (int)std::min<long long>((long long)a.m_tiles_ub * t.n_tiles, sms);
-  return launch_one<EPI_DOWN>(ma, mb, mb, t, grid, st);
+  return launch_gemm<EPI_DOWN>(ma, mb, mb, t, a.m_tiles_ub, a.G, st);
 }
 
 }  // namespace moe

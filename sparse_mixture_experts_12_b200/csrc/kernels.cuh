@@ -73,6 +73,8 @@ struct GroupedFfnArgs {
   void *h;                // [a_rows, F] dtype (intermediate)
   void *out;              // [a_rows, d]
   int out_f32;            // 1: out is fp32 (shared experts), else dtype
+  int max_group_rows;     // host bound on the rows of any one group
+  float *part;            // fp32 split-K partials of the small-batch path, or nullptr
   int32_t *err;
 };
 
@@ -89,5 +91,9 @@ cudaError_t launch_tile_table(const int32_t *offsets, int G, int max_rows, int32
 cudaError_t launch_ffn_simt(const GroupedFfnArgs &a, cudaStream_t st);
 // bf16 tcgen05 path
 cudaError_t launch_ffn_tc(const GroupedFfnArgs &a, cudaStream_t st);
+// bf16 tcgen05 path for at most kDecodeMaxRows rows per group (weights on the M side)
+constexpr int kDecodeMaxRows = 32;
+cudaError_t launch_ffn_tc_decode(const GroupedFfnArgs &a, cudaStream_t st);
+size_t ffn_decode_partial_bytes(int max_rows, int d);
 
 }  // namespace moe

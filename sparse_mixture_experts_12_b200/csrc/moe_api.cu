@@ -14,7 +14,8 @@ namespace {
 
 enum Buf {
   B_ERR, B_TILE_COUNTS, B_TILE_BASE, B_TILE_P, B_TILE_Z, B_COUNTS, B_OFFSETS, B_MPREFIX, B_SH_TBL,
-  B_LOGITS, B_IDX, B_GATE, B_PERM, B_INV, B_XPERM, B_H, B_YPERM, B_SH_H, B_SH_Y, B_NBUF
+  B_LOGITS, B_IDX, B_GATE, B_PERM, B_INV, B_XPERM, B_H, B_YPERM, B_SH_H, B_SH_Y, B_YPART,
+  B_NBUF
 };
 
 struct Layout {
@@ -50,6 +51,10 @@ Layout layout_for(const moe_cfg_t &c) {
   sz[B_YPERM] = T * k * d * eb;
   sz[B_SH_H] = Fs ? T * Fs * eb : 0;
   sz[B_SH_Y] = Fs ? T * d * 4 : 0;
+  // split-K partials of the small-batch expert GEMM (bf16, at most 32 tokens)
+  sz[B_YPART] = (c.dtype == MOE_DTYPE_BF16 && T <= (size_t)kDecodeMaxRows)
+                    ? ffn_decode_partial_bytes((int)(T * k > T ? T * k : T), (int)d)
+                    : 0;
   Layout L;
   size_t o = 0;
   for (int i = 0; i < B_NBUF; ++i) {
@@ -58,6 +63,10 @@ Layout layout_for(const moe_cfg_t &c) {
   }
   L.total = o;
   return L;
+}
+
+size_t layout_size(const Layout &L, Buf b) {
+  return (b + 1 < B_NBUF ? L.off[b + 1] : L.total) - L.off[b];
 }
 
 template <typename P>
@@ -153,13 +162,18 @@ int m_tiles_ub(long long rows, int groups) {
 }
 
 cudaError_t run_ffn(const moe_cfg_t &c, const GroupedFfnArgs &a, cudaStream_t st) {
-  return c.dtype == MOE_DTYPE_F32 ? launch_ffn_simt(a, st) : launch_ffn_tc(a, st);
+  if (c.dtype == MOE_DTYPE_F32) return launch_ffn_simt(a, st);
+  // at most 32 rows in any group: stream the weights with the tokens on the MMA's N side
+  if (a.max_group_rows <= kDecodeMaxRows) return launch_ffn_tc_decode(a, st);
+  return launch_ffn_tc(a, st);
 }
 
 GroupedFfnArgs routed_ffn_args(const moe_cfg_t &c, const moe_weights_t &w, const void *x_perm,
                                const int32_t *offsets, const int32_t *mprefix, void *h,
-                               void *y_perm, int32_t *err) {
+                               void *y_perm, int32_t *err, int max_group_rows, float *part) {
   GroupedFfnArgs a{};
+  a.max_group_rows = max_group_rows;
+  a.part = part;
   a.a = x_perm;
   a.a_rows = c.n_tokens * c.top_k;
   a.offsets = offsets;
@@ -299,7 +313,8 @@ MOE_API moe_status_t moe_expert_ffn(const moe_cfg_t *cfg, const moe_weights_t *w
   int32_t *mprefix = at<int32_t>(ws, L, B_MPREFIX);
   MOE_CUDA(launch_tile_table(offsets, c.n_experts, c.n_tokens * c.top_k, mprefix, err, stream));
   GroupedFfnArgs a = routed_ffn_args(c, *w, x_perm, offsets, mprefix, at<void>(ws, L, B_H),
-                                     y_perm, err);
+                                     y_perm, err, c.n_tokens * c.top_k,
+                                     layout_size(L, B_YPART) > 0 ? at<float>(ws, L, B_YPART) : nullptr);
   MOE_CUDA(run_ffn(c, a, stream));
   return MOE_OK;
 }
@@ -461,6 +476,7 @@ MOE_API moe_status_t moe_forward(const moe_cfg_t *cfg, const moe_weights_t *w, c
   MOE_CUDA(launch_scatter(p, stream));
   // 4. always-on shared experts: one SwiGLU over all tokens, experts concatenated along F
   float *sh_y = nullptr;
+  float *part = layout_size(L, B_YPART) > 0 ? at<float>(ws, L, B_YPART) : nullptr;
   if (c.n_shared > 0) {
     GroupedFfnArgs a{};
     a.a = x;
@@ -479,12 +495,15 @@ MOE_API moe_status_t moe_forward(const moe_cfg_t *cfg, const moe_weights_t *w, c
     sh_y = at<float>(ws, L, B_SH_Y);
     a.out = sh_y;
     a.out_f32 = 1;
+    a.max_group_rows = c.n_tokens;
+    a.part = part;
     a.err = err;
     MOE_CUDA(run_ffn(c, a, stream));
   }
-  // 5. routed experts on the expert-contiguous rows
+  // 5. routed experts on the expert-contiguous rows (a token adds at most one row to
+  //    any expert, so no group holds more than T rows)
   GroupedFfnArgs a = routed_ffn_args(c, *w, p.x_perm, offsets, mprefix, at<void>(ws, L, B_H),
-                                     at<void>(ws, L, B_YPERM), err);
+                                     at<void>(ws, L, B_YPERM), err, c.n_tokens, part);
   MOE_CUDA(run_ffn(c, a, stream));
   // 6. gate-weighted combine (+ shared output)
   CombineArgs cb{};

@@ -17,76 +17,91 @@ namespace moe {
 
 namespace {
 
-// ----------------------------------------------------------------- block scan
-template <int NTHREADS>
-__device__ int block_inclusive_scan(int v, int *warp_buf) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+// ----------------------------------------------------------------- warp scan
+__device__ __forceinline__ int warp_incl_scan(int v) {
+  const int lane = threadIdx.x & 31;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
     const int n = __shfl_up_sync(0xffffffffu, v, o);
     if (lane >= o) v += n;
   }
-  if (lane == 31) warp_buf[warp] = v;
-  __syncthreads();
-  if (warp == 0) {
-    int w = (lane < NTHREADS / 32) ? warp_buf[lane] : 0;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int n = __shfl_up_sync(0xffffffffu, w, o);
-      if (lane >= o) w += n;
-    }
-    if (lane < NTHREADS / 32) warp_buf[lane] = w;
-  }
-  __syncthreads();
-  if (warp > 0) v += warp_buf[warp - 1];
   return v;
 }
 
 constexpr int kScanThreads = 1024;
+constexpr int kScanVPL = 8;  // tiles per lane per batch (loads issued together)
 
+// One CTA. Warp per expert: exclusive prefix of the expert's per-tile counts over
+// the token tiles (tile_counts is [E][NT], so a warp reads consecutive tiles).
+// Then one warp: counts, capacity, kept-row offsets and the 128-row tile prefix
+// over the experts. Optionally the load-balancing statistics (fixed-order sums).
 __global__ void __launch_bounds__(kScanThreads) k_scan(ScanArgs a) {
-  __shared__ int warp_buf[32];
-  __shared__ int seg_start[kMaxExperts + 1];
-  __shared__ int kept_s[kMaxExperts];
-  __shared__ float red[kScanThreads];
+  __shared__ int count_s[kMaxExperts];
+  __shared__ float P_s[kMaxExperts];
+  __shared__ float red[kScanThreads / 32];
   const int E = a.E, NT = a.NT;
-  const int N = E * NT;
-  const int tid = threadIdx.x;
-  const int chunk = ceil_div(N, kScanThreads);
-  const int i0 = min(N, tid * chunk), i1 = min(N, i0 + chunk);
-
-  int s = 0;
-  for (int i = i0; i < i1; ++i) s += a.tile_counts[i];
-  const int incl = block_inclusive_scan<kScanThreads>(s, warp_buf);
-  int run = incl - s;
-  for (int i = i0; i < i1; ++i) {
-    if (i % NT == 0) seg_start[i / NT] = run;
-    run += a.tile_counts[i];
-  }
-  if (tid == kScanThreads - 1) seg_start[E] = incl;
-  __syncthreads();
-  run = incl - s;
-  for (int i = i0; i < i1; ++i) {
-    a.tile_base[i] = run - seg_start[i / NT];
-    run += a.tile_counts[i];
-  }
-  if (tid < E) {
-    const int c = seg_start[tid + 1] - seg_start[tid];
-    a.counts[tid] = c;
-    kept_s[tid] = (a.cap < 0) ? c : min(c, a.cap);
-  }
-  __syncthreads();
-  if (tid == 0) {
-    int off = 0, mp = 0;
-    for (int e = 0; e < E; ++e) {
-      a.offsets[e] = off;
-      a.mprefix[e] = mp;
-      off += kept_s[e];
-      mp += ceil_div(kept_s[e], kRowTile);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  constexpr int nw = kScanThreads / 32;
+  for (int e = warp; e < E; e += nw) {
+    const int32_t *tc = a.tile_counts + (size_t)e * NT;
+    int32_t *tb = a.tile_base + (size_t)e * NT;
+    int run = 0;
+    for (int b0 = 0; b0 < NT; b0 += 32 * kScanVPL) {
+      int v[kScanVPL];
+#pragma unroll
+      for (int j = 0; j < kScanVPL; ++j) {
+        const int t = b0 + j * 32 + lane;
+        v[j] = t < NT ? tc[t] : 0;
+      }
+#pragma unroll
+      for (int j = 0; j < kScanVPL; ++j) {
+        const int incl = warp_incl_scan(v[j]);
+        const int t = b0 + j * 32 + lane;
+        if (t < NT) tb[t] = run + incl - v[j];
+        run += __shfl_sync(0xffffffffu, incl, 31);
+      }
     }
-    a.offsets[E] = off;
-    a.mprefix[E] = mp;
-    if (a.sh_tbl) {
+    if (lane == 0) count_s[e] = run;
+    if (a.aux_out) {
+      float p = 0.f;
+      for (int t = lane; t < NT; t += 32) p += a.tile_p[(size_t)e * NT + t];
+      p = warp_sum(p);
+      if (lane == 0) P_s[e] = p / (float)a.T;
+    }
+  }
+  __syncthreads();
+  if (warp == 0) {
+    // E <= 256: eight experts per lane
+    int cnt[8], kept[8], mt[8];
+    int sk = 0, sm = 0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int e = lane * 8 + j;
+      const int c = e < E ? count_s[e] : 0;
+      cnt[j] = c;
+      kept[j] = (a.cap < 0) ? c : min(c, a.cap);
+      mt[j] = ceil_div(kept[j], kRowTile);
+      sk += kept[j];
+      sm += mt[j];
+    }
+    const int ik = warp_incl_scan(sk), im = warp_incl_scan(sm);
+    int ok = ik - sk, om = im - sm;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int e = lane * 8 + j;
+      if (e < E) {
+        a.counts[e] = cnt[j];
+        a.offsets[e] = ok;
+        a.mprefix[e] = om;
+      }
+      ok += kept[j];
+      om += mt[j];
+    }
+    if (lane == 31) {
+      a.offsets[E] = ik;
+      a.mprefix[E] = im;
+    }
+    if (lane == 0 && a.sh_tbl) {
       a.sh_tbl[0] = 0;
       a.sh_tbl[1] = a.T;
       a.sh_tbl[2] = 0;
@@ -95,45 +110,26 @@ __global__ void __launch_bounds__(kScanThreads) k_scan(ScanArgs a) {
   }
   if (a.aux_out == nullptr) return;
 
-  // ---- load-balancing statistics (fixed-order reductions, deterministic)
-  int epow = 1;
-  while (epow < E) epow <<= 1;
-  const int G = kScanThreads / epow;  // threads per expert (>= 4)
-  {
-    const int e = tid / G, g = tid % G;
-    float p = 0.f;
-    if (e < E)
-      for (int tl = g; tl < NT; tl += G) p += a.tile_p[(size_t)e * NT + tl];
-    red[tid] = p;
-    __syncthreads();
-    for (int h = G / 2; h > 0; h >>= 1) {
-      if (g < h) red[tid] += red[tid + h];
-      __syncthreads();
-    }
-  }
-  __shared__ float P_s[kMaxExperts];
-  if (tid < E) P_s[tid] = red[tid * G] / (float)a.T;
-  __syncthreads();
+  // ---- load-balancing statistics
   float z = 0.f;
-  for (int tl = tid; tl < NT; tl += kScanThreads) z += a.tile_z[tl];
-  red[tid] = z;
+  for (int t = threadIdx.x; t < NT; t += kScanThreads) z += a.tile_z[t];
+  z = warp_sum(z);
+  if (lane == 0) red[warp] = z;
   __syncthreads();
-  for (int h = kScanThreads / 2; h > 0; h >>= 1) {
-    if (tid < h) red[tid] += red[tid + h];
-    __syncthreads();
-  }
-  if (tid == 0) {
+  if (threadIdx.x == 0) {
+    float zs = 0.f;
+    for (int w = 0; w < nw; ++w) zs += red[w];
     const double inv_tk = 1.0 / ((double)a.T * (double)a.k);
     double fp = 0.0, bsq = 0.0;
     for (int e = 0; e < E; ++e) {
-      const double f = (double)(seg_start[e + 1] - seg_start[e]) * inv_tk;
+      const double f = (double)count_s[e] * inv_tk;
       fp += f * (double)P_s[e];
       bsq += (f - 1.0 / E) * (f - 1.0 / E);
       a.aux_out[3 + e] = (float)f;
       a.aux_out[3 + E + e] = P_s[e];
     }
     a.aux_out[0] = (float)((double)a.alpha * E * fp);
-    a.aux_out[1] = red[0] / (float)a.T;
+    a.aux_out[1] = zs / (float)a.T;
     a.aux_out[2] = (float)bsq;
   }
 }
@@ -252,14 +248,21 @@ __global__ void __launch_bounds__(256) k_combine(CombineArgs a) {
   T *y = static_cast<T *>(a.y);
   const int nvec = a.d / VE;
   for (int v = lane; v < nvec; v += 32) {
+    // every slot's row is requested before any is used (a dropped slot reads nothing
+    // and contributes zero)
+    uint4 u[kMaxTopK];
+#pragma unroll
+    for (int s = 0; s < kMaxTopK; ++s)
+      u[s] = (row[s] >= 0) ? __ldg(reinterpret_cast<const uint4 *>(yp + (size_t)row[s] * a.d) + v)
+                           : make_uint4(0u, 0u, 0u, 0u);
     float acc[VE];
 #pragma unroll
     for (int i = 0; i < VE; ++i) acc[i] = 0.f;
 #pragma unroll
     for (int s = 0; s < kMaxTopK; ++s) {
-      if (row[s] < 0) continue;
+      if (s >= k) break;
       float f[VE];
-      unpack16(__ldg(reinterpret_cast<const uint4 *>(yp + (size_t)row[s] * a.d) + v), f);
+      unpack16(u[s], f);
 #pragma unroll
       for (int i = 0; i < VE; ++i) acc[i] = fmaf(g[s], f[i], acc[i]);
     }
@@ -276,21 +279,36 @@ __global__ void __launch_bounds__(256) k_combine(CombineArgs a) {
 }
 
 // ---------------------------------------------------------------- tile table
+// One warp: validate a caller-supplied offsets array and build the 128-row tile
+// prefix from it (all zero, so nothing is computed, when the offsets are invalid).
 __global__ void k_tile_table(const int32_t *offsets, int G, int max_rows, int32_t *mprefix,
                              int32_t *err) {
-  if (threadIdx.x != 0) return;
-  bool ok = offsets[0] >= 0;
-  int bad = 0;
-  for (int g = 0; g < G && ok; ++g) {
-    if (offsets[g + 1] < offsets[g] || offsets[g + 1] > max_rows) { ok = false; bad = g; }
+  const int lane = threadIdx.x;
+  int bad = G;
+  for (int g = lane; g < G; g += 32) {
+    const int a0 = offsets[g], a1 = offsets[g + 1];
+    if (a0 < 0 || a1 < a0 || a1 > max_rows) bad = min(bad, g);
   }
-  int mp = 0;
-  for (int g = 0; g < G; ++g) {
-    mprefix[g] = mp;
-    if (ok) mp += ceil_div(offsets[g + 1] - offsets[g], kRowTile);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) bad = min(bad, __shfl_xor_sync(0xffffffffu, bad, o));
+  const bool ok = bad == G;
+  int mt[8], sm = 0;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const int g = lane * 8 + j;
+    mt[j] = (ok && g < G) ? ceil_div(offsets[g + 1] - offsets[g], kRowTile) : 0;
+    sm += mt[j];
   }
-  mprefix[G] = mp;
-  if (!ok) report_error(err, MOE_DEVERR_OFFSETS, bad);
+  const int incl = warp_incl_scan(sm);
+  int run = incl - sm;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const int g = lane * 8 + j;
+    if (g < G) mprefix[g] = run;
+    run += mt[j];
+  }
+  if (lane == 31) mprefix[G] = incl;
+  if (!ok && lane == 0) report_error(err, MOE_DEVERR_OFFSETS, bad);
 }
 
 }  // namespace

@@ -169,6 +169,11 @@ FFN_CASES = [
     ("swiglu_f32", synth.ACT_SWIGLU, synth.DT_F32, 96, 160, 4, [3, 140, 0, 33]),
     ("relu_f32_bias", synth.ACT_RELU, synth.DT_F32, 64, 256, 8, [16] * 8),
     ("gelu_f32_odd", synth.ACT_GELU, synth.DT_F32, 36, 50, 3, [1, 2, 300]),
+    # at most 32 rows in all: the small-batch path (weights on the MMA's M side,
+    # split-K down projection)
+    ("swiglu_bf16_decode", synth.ACT_SWIGLU, synth.DT_BF16, 256, 384, 5, [0, 1, 3, 7, 2]),
+    ("gelu_bf16_decode_bias", synth.ACT_GELU, synth.DT_BF16, 128, 320, 4, [5, 0, 9, 2]),
+    ("relu_bf16_decode_ntail", synth.ACT_RELU, synth.DT_BF16, 192, 192, 2, [1, 12]),
 ]
 
 
