@@ -113,6 +113,32 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(sm), "source": "NVML, 20 ms polling"}
 
 
+# ----------------------------------------------------------- multi-rank plumbing
+def dist_env():
+    """(world, rank, local_rank) from the torchrun environment (1, 0, 0 when absent)."""
+    return (int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def barrier(world: int):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(v: float, world: int, device=None) -> float:
+    """The slowest rank's value: the job takes as long as its last rank."""
+    if world == 1:
+        return v
+    t = torch.tensor([v], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def tokens_per_second(T: int, world: int, steps: int, ms: float) -> float:
+    """Whole-job throughput: every rank processes its own batch of T tokens per step."""
+    return T * world * steps / (ms / 1000.0)
+
+
 # ---------------------------------------------------------------- oracle helpers
 class _F64View:
     """Lazily upcast slices of a CPU tensor to fp64 numpy (input marshalling only)."""
@@ -253,17 +279,6 @@ def run_ours(args, wl, rank, world, local_rank):
     stream = torch.cuda.current_stream()
     per_step_launches = 6 + (2 if wl.n_shared > 0 else 0)
 
-    def barrier():
-        if world > 1:
-            torch.distributed.barrier()
-
-    def max_over_ranks(v: float) -> float:
-        if world == 1:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        return float(t.item())
-
     clocks = ClockSampler(local_rank)
     clocks.start()
     for _ in range(args.warmup):
@@ -272,7 +287,7 @@ def run_ours(args, wl, rank, world, local_rank):
     code, info = layer.last_device_error()
     if code != 0:
         raise RuntimeError(f"device error {code} ({info}) during warm-up")
-    barrier()
+    barrier(world)
     torch.cuda.synchronize()
     clocks.begin_load()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -281,13 +296,13 @@ def run_ours(args, wl, rank, world, local_rank):
         layer.forward(x, y, aux)
     e1.record(stream)
     torch.cuda.synchronize()
-    barrier()
-    ms = max_over_ranks(e0.elapsed_time(e1))
+    barrier(world)
+    ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
     clk = clocks.stop()
     code, info = layer.last_device_error()
     if code != 0:
         raise RuntimeError(f"device error {code} ({info}) in the timed region")
-    value = wl.T * world * args.steps / (ms / 1000.0)
+    value = tokens_per_second(wl.T, world, args.steps, ms)
 
     # ---- expert FFN (grouped GEMMs) timed alone on the same stream, for the roofline
     taps = layer.new_taps()
@@ -345,7 +360,7 @@ def run_ours(args, wl, rank, world, local_rank):
         layer.forward(x, y, aux)
         yh.copy_(y, non_blocking=True)
     torch.cuda.synchronize()
-    barrier()
+    barrier(world)
     g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     g0.record(stream)
     for _ in range(args.steps):
@@ -356,9 +371,9 @@ def run_ours(args, wl, rank, world, local_rank):
             aux.cpu()
     g1.record(stream)
     torch.cuda.synchronize()
-    barrier()
-    e2e_ms = max_over_ranks(g0.elapsed_time(g1))
-    e2e = {"value": wl.T * world * args.steps / (e2e_ms / 1000.0), "unit": "tokens/s",
+    barrier(world)
+    e2e_ms = max_over_ranks(g0.elapsed_time(g1), world, dev)
+    e2e = {"value": tokens_per_second(wl.T, world, args.steps, e2e_ms), "unit": "tokens/s",
            "h2d_bytes_per_step": int(xh.numel() * xh.element_size()),
            "d2h_bytes_per_step": int(yh.numel() * yh.element_size()) +
            (int(aux.numel() * 4) if aux is not None else 0)}
@@ -397,9 +412,7 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    world, rank, local_rank = dist_env()
     wl = synth.WORKLOADS[args.workload]
     if args.impl == "reference":
         run_reference(args, wl, rank, world)
