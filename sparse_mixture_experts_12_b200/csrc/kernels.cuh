@@ -91,8 +91,9 @@ cudaError_t launch_tile_table(const int32_t *offsets, int G, int max_rows, int32
 cudaError_t launch_ffn_simt(const GroupedFfnArgs &a, cudaStream_t st);
 // bf16 tcgen05 path
 cudaError_t launch_ffn_tc(const GroupedFfnArgs &a, cudaStream_t st);
-// bf16 tcgen05 path for at most kDecodeMaxRows rows per group (weights on the M side)
-constexpr int kDecodeMaxRows = 32;
+// bf16 tcgen05 path for small groups (weights on the M side, tokens in 32-row
+// chunks); used when no group can hold more than kDecodeMaxRows rows
+constexpr int kDecodeMaxRows = 64;
 cudaError_t launch_ffn_tc_decode(const GroupedFfnArgs &a, cudaStream_t st);
 size_t ffn_decode_partial_bytes(int max_rows, int d);
 

@@ -51,7 +51,7 @@ Layout layout_for(const moe_cfg_t &c) {
   sz[B_YPERM] = T * k * d * eb;
   sz[B_SH_H] = Fs ? T * Fs * eb : 0;
   sz[B_SH_Y] = Fs ? T * d * 4 : 0;
-  // split-K partials of the small-batch expert GEMM (bf16, at most 32 tokens)
+  // split-K partials of the small-batch expert GEMM (bf16, few tokens)
   sz[B_YPART] = (c.dtype == MOE_DTYPE_BF16 && T <= (size_t)kDecodeMaxRows)
                     ? ffn_decode_partial_bytes((int)(T * k > T ? T * k : T), (int)d)
                     : 0;
@@ -163,7 +163,7 @@ int m_tiles_ub(long long rows, int groups) {
 
 cudaError_t run_ffn(const moe_cfg_t &c, const GroupedFfnArgs &a, cudaStream_t st) {
   if (c.dtype == MOE_DTYPE_F32) return launch_ffn_simt(a, st);
-  // at most 32 rows in any group: stream the weights with the tokens on the MMA's N side
+  // few rows in any group: stream the weights with the tokens on the MMA's N side
   if (a.max_group_rows <= kDecodeMaxRows) return launch_ffn_tc_decode(a, st);
   return launch_ffn_tc(a, st);
 }

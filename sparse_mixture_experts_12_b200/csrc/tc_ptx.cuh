@@ -244,6 +244,23 @@ __device__ __forceinline__ void settle_ns(uint64_t ns) {
   }
 }
 
+// As mbar_try_wait, but the thread may sleep in hardware (no issue slots) for up to
+// `suspend_ns` before giving up; it wakes as soon as the phase completes.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t *bar, uint32_t parity,
+                                                    uint32_t suspend_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(suspend_ns)
+      : "memory");
+  return ok != 0;
+}
+
+constexpr uint32_t kSuspendNs = 200000;  // re-check the abort flag and the bound every 0.2 ms
+
 // Wait for the phase of `parity` of `bar` to complete. Gives up when the CTA's
 // abort flag is raised (honour_abort) or after `limit_ns`; on its own timeout it
 // raises the abort flag (and the peer CTA's, when `peer_abort` is a cluster
@@ -255,7 +272,7 @@ static __device__ __noinline__ bool wait_mbar(uint64_t *bar, uint32_t parity, in
   const uint64_t t0 = globaltimer_ns();
   volatile int *abort_flag = abort_flag_ptr;
   while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait_sleep(bar, parity, kSuspendNs)) return true;
     if (honour_abort && *abort_flag) return false;
     if (globaltimer_ns() - t0 > limit_ns) {
       if (honour_abort) {

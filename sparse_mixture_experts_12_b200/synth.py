@@ -118,6 +118,8 @@ SMALL = {
     "decode_small": MIXTRAL_PREFILL.replace(name="decode_small", T=5, d_model=256, d_ff=384),
     "deepseek_decode": DEEPSEEK_FINE.replace(name="deepseek_decode", T=20, d_model=256, d_ff=256,
                                              d_ff_shared=384),
+    "decode_chunks": MIXTRAL_PREFILL.replace(name="decode_chunks", T=64, d_model=256, d_ff=384,
+                                             n_experts=2, top_k=1),
     "fp32_swiglu": DEEPSEEK_FINE.replace(name="fp32_swiglu", T=150, d_model=96, d_ff=160,
                                          n_experts=16, top_k=3, dtype=DT_F32,
                                          d_ff_shared=64),

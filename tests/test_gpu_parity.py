@@ -174,6 +174,9 @@ FFN_CASES = [
     ("swiglu_bf16_decode", synth.ACT_SWIGLU, synth.DT_BF16, 256, 384, 5, [0, 1, 3, 7, 2]),
     ("gelu_bf16_decode_bias", synth.ACT_GELU, synth.DT_BF16, 128, 320, 4, [5, 0, 9, 2]),
     ("relu_bf16_decode_ntail", synth.ACT_RELU, synth.DT_BF16, 192, 192, 2, [1, 12]),
+    # still the small-batch path, with an expert spanning two 32-row chunks
+    ("swiglu_bf16_decode_chunks", synth.ACT_SWIGLU, synth.DT_BF16, 256, 384, 2, [33, 20]),
+    ("gelu_bf16_decode_chunks", synth.ACT_GELU, synth.DT_BF16, 128, 256, 2, [45, 10]),
 ]
 
 
