@@ -238,21 +238,23 @@ def _config(wl, world):
 
 
 def _traffic(workload_name):
-    """DRAM bytes per launch of the expert-FFN kernels from the committed ncu summary,
-    valid only while the kernel source is unchanged since the capture."""
-    p = os.path.join(ROOT, "profiles", "ffn_tc_traffic.json")
-    src = os.path.join(ROOT, "sparse_mixture_experts_12_b200", "csrc", "ffn_tc.cu")
+    """DRAM bytes per expert-FFN call (all its kernel launches) from the committed ncu
+    summary, valid only while every kernel source it lists is unchanged since the
+    capture; None otherwise."""
+    p = os.path.join(ROOT, "profiles", "ffn_traffic.json")
     if not os.path.exists(p):
         return None
     try:
         with open(p) as f:
-            d = json.load(f)
-        sha = hashlib.sha256(open(src, "rb").read()).hexdigest()
-        ent = d.get(workload_name)
-        if ent is None or ent.get("ffn_tc_sha256") != sha:
+            ent = json.load(f).get(workload_name)
+        if ent is None:
             return None
-        return ent.get("dram_bytes_per_call")
-    except Exception:
+        for rel, sha in ent["sources"].items():
+            with open(os.path.join(ROOT, rel), "rb") as f:
+                if hashlib.sha256(f.read()).hexdigest() != sha:
+                    return None
+        return ent["dram_bytes_per_call"]
+    except (OSError, ValueError, KeyError, TypeError):
         return None
 
 

@@ -86,19 +86,22 @@ __device__ __forceinline__ bool wait_bounded(uint64_t *bar, uint32_t parity, Sme
 // SwiGLU: columns [0,128) hold x.w_gate, [128,256) x.w_up; h = silu(g) * u.
 // ACT: bias + ReLU / GELU. DOWN: + bias. Stores are masked to the valid row and
 // to the N extent.
+// Columns go in 32-wide chunks c in [c0, c1). SwiGLU: the gate value of chunk c
+// sits at accumulator column acc_off + 32c and the up value 128 columns further;
+// other tiles: accumulator column acc_off + 32c. Output column = out_base + 32c.
 template <int EPI>
-__device__ __forceinline__ void epilogue_tile(const TcArgs &a, uint32_t tbase, int g, int n,
-                                              bool valid, size_t orow, int half) {
-  // the two epilogue warps that share a TMEM lane quarter take half the columns each
+__device__ __forceinline__ void epilogue_tile(const TcArgs &a, uint32_t tbase, int g, int acc_off,
+                                              int out_base, int c0, int c1, bool valid,
+                                              size_t orow) {
   if (EPI == EPI_SWIGLU) {
     __nv_bfloat16 *out = static_cast<__nv_bfloat16 *>(a.out);
 #pragma unroll 1
-    for (int c = 2 * half; c < 2 * half + 2; ++c) {
+    for (int c = c0; c < c1; ++c) {
       uint32_t gv[32], uv[32];
-      tmem_ld32(tbase + c * 32, gv);
-      tmem_ld32(tbase + kMmaN / 2 + c * 32, uv);
+      tmem_ld32(tbase + acc_off + c * 32, gv);
+      tmem_ld32(tbase + acc_off + kMmaN / 2 + c * 32, uv);
       tmem_ld_wait();
-      const int col0 = n * (kMmaN / 2) + c * 32;
+      const int col0 = out_base + c * 32;
       if (valid && col0 < a.N) {
         uint4 *dst = reinterpret_cast<uint4 *>(out + orow * a.N + col0);
 #pragma unroll
@@ -116,11 +119,11 @@ __device__ __forceinline__ void epilogue_tile(const TcArgs &a, uint32_t tbase, i
     }
   } else {
 #pragma unroll 1
-    for (int c = 4 * half; c < 4 * half + 4; ++c) {
+    for (int c = c0; c < c1; ++c) {
       uint32_t v[32];
-      tmem_ld32(tbase + c * 32, v);
+      tmem_ld32(tbase + acc_off + c * 32, v);
       tmem_ld_wait();
-      const int col0 = n * kMmaN + c * 32;
+      const int col0 = out_base + c * 32;
       if (valid && col0 < a.N) {
         float f[32];
 #pragma unroll
@@ -290,7 +293,11 @@ k_ffn_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtens
       const bool valid = grow < offs[g + 1] - offs[g];
       const size_t orow = (size_t)offs[g] + grow;
       const uint32_t tbase = tmem + ((uint32_t)(ew * 32) << 16) + (uint32_t)(acc * kMmaN);
-      epilogue_tile<EPI>(a, tbase, g, n, valid, orow, half);
+      // the two warps sharing a TMEM lane quarter take half the columns each
+      if (EPI == EPI_SWIGLU)
+        epilogue_tile<EPI>(a, tbase, g, 0, n * (kMmaN / 2), 2 * half, 2 * half + 2, valid, orow);
+      else
+        epilogue_tile<EPI>(a, tbase, g, 0, n * kMmaN, 4 * half, 4 * half + 4, valid, orow);
       tc_fence_before();
       mbar_arrive(&ctl->tempty[acc]);
       if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
@@ -313,11 +320,21 @@ k_ffn_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtens
 // leader's `full` barrier; the MMA commits release `empty` and `tfull` in both
 // CTAs; both epilogues release the leader's `tempty`. Per CTA a stage is 32 KB
 // (vs 48 KB for the single-CTA tile), so six stages fit.
-constexpr int kStages2 = 6;
+constexpr int kStages2 = 6;  // ring depth of the 256-column pair tile
 constexpr int kPairM = 2 * kTileM;
 constexpr int kAHalf = kTileM * kBlockK * 2;
 constexpr int kBHalf = (kMmaN / 2) * kBlockK * 2;
-constexpr int kStage2Bytes = kAHalf + kBHalf;
+// NH = N halves per pair tile. NH = 1: 256 MMA columns, six 32 KB stages, two
+// TMEM accumulators. NH = 2: 512 columns (two MMAs per K step), four 48 KB
+// stages, one 512-column accumulator: twice the MMA work per stage and 25% fewer
+// operand bytes per flop, but the epilogue no longer overlaps the next tile's
+// main loop, so it pays off for long K.
+template <int NH> struct PairCfg {
+  static constexpr int kStages = NH == 1 ? kStages2 : 4;
+  static constexpr int kStageBytes = kAHalf + NH * kBHalf;
+  static constexpr int kAccBufs = NH == 1 ? 2 : 1;
+  static constexpr size_t kRing = (size_t)kStages * kStageBytes;
+};
 constexpr uint64_t kDrainNs = 50000000ull;  // 50 ms bound on end-of-kernel drains
 
 struct SmemCtl2 {
@@ -331,7 +348,32 @@ struct SmemCtl2 {
   int tbl[2 * (kMaxExperts + 1)];  // pair-tile prefix [G+1], offsets [G+1]
 };
 
-constexpr size_t kSmem2Bytes = (size_t)kStages2 * kStage2Bytes + sizeof(SmemCtl2) + 1024;
+template <int NH>
+constexpr size_t pair_smem_bytes() { return PairCfg<NH>::kRing + sizeof(SmemCtl2) + 1024; }
+
+// Work items of the persistent pair kernel. With NH = 2, when the last round of
+// tiles would leave at least half of the CTA pairs idle (r = total % pairs tiles,
+// 0 < 2r <= pairs), those r tiles are issued as 2r half tiles of one N half each,
+// so the last round takes half as long. Item -> (tile, sel): sel = -1 for a whole
+// tile, else the single N half it covers.
+struct PairItems {
+  int full, items;
+  __device__ PairItems(int total, int pairs, int nh) : full(total), items(total) {
+    const int r = total % pairs;
+    if (nh == 2 && r > 0 && 2 * r <= pairs) {
+      full = total - r;
+      items = total + r;
+    }
+  }
+  __device__ int tile(int it, int &sel) const {
+    if (it < full) {
+      sel = -1;
+      return it;
+    }
+    sel = (it - full) & 1;
+    return full + ((it - full) >> 1);
+  }
+};
 
 // Bounded wait that, on its own timeout, also raises the peer CTA's abort flag.
 __device__ __forceinline__ bool wait_pair(uint64_t *bar, uint32_t parity, SmemCtl2 *ctl,
@@ -341,14 +383,17 @@ __device__ __forceinline__ bool wait_pair(uint64_t *bar, uint32_t parity, SmemCt
   return wait_mbar(bar, parity, &ctl->abort_flag, peer_abort, err, site, honour_abort, limit_ns);
 }
 
-template <int EPI>
+template <int EPI, int NH>
 __global__ void __launch_bounds__(kThreads, 1)
 k_ffn_tc2(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
           const __grid_constant__ CUtensorMap tmB3, TcArgs a) {
+  using PC = PairCfg<NH>;
+  constexpr int kS = PC::kStages;
+  constexpr int kSB = PC::kStageBytes;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  SmemCtl2 *ctl = reinterpret_cast<SmemCtl2 *>(smem + (size_t)kStages2 * kStage2Bytes);
+  SmemCtl2 *ctl = reinterpret_cast<SmemCtl2 *>(smem + PC::kRing);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const uint32_t rank = cluster_ctarank();
   const bool leader = rank == 0;
@@ -357,11 +402,11 @@ k_ffn_tc2(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
   int *offs = ctl->tbl + (G + 1);
   for (int i = tid; i <= G; i += kThreads) offs[i] = a.offsets[i];
   if (tid == 0) {
-    for (int s = 0; s < kStages2; ++s) {
+    for (int s = 0; s < kS; ++s) {
       mbar_init(&ctl->full[s], 1);
       mbar_init(&ctl->empty[s], 1);
     }
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < PC::kAccBufs; ++s) {
       mbar_init(&ctl->tfull[s], 1);
       mbar_init(&ctl->tempty[s], 2 * kEpiWarps * 32);
     }
@@ -398,10 +443,10 @@ k_ffn_tc2(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
   cluster_sync_all();  // both CTAs' barriers and TMEM exist before any cross-CTA use
   tc_fence_after();
   const uint32_t tmem = ctl->tmem_base;
-  const int total = ppre[G] * a.n_tiles;
   const int nkb = ceil_div(a.K, kBlockK);
   const uint32_t peer_abort = mapa_rank(smem_u32(&ctl->abort_flag), rank ^ 1u);
   const int c0 = (int)cluster_index(), cstep = (int)cluster_count();
+  const PairItems work(ppre[G] * a.n_tiles, cstep, NH);
 
   if (warp == 0 && lane == 0) {
     // ------------------------------------------------------------ TMA producer
@@ -413,30 +458,37 @@ k_ffn_tc2(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
     int stage = 0;
     uint32_t phase = 0, issued = 0, last_phase = 0;
     bool ok = true;
-    for (int tile = c0; ok && tile < total; tile += cstep) {
-      int g, n, m;
-      decode_tile(tile, ppre, G, a.n_tiles, g, n, m);
+    for (int it = c0; ok && it < work.items; it += cstep) {
+      int sel, g, n, m;
+      decode_tile(work.tile(it, sel), ppre, G, a.n_tiles, g, n, m);
+      const int h0 = sel < 0 ? 0 : sel, h1 = sel < 0 ? NH : sel + 1;
       const int arow = offs[g] + m * kPairM + (int)rank * kTileM;
-      const int brow = (EPI == EPI_SWIGLU) ? g * a.b_rows + n * (kMmaN / 2)
-                                           : g * a.b_rows + n * kMmaN + (int)rank * (kMmaN / 2);
+      // this CTA's weight rows of N half h (SwiGLU: CTA 0 w_gate rows, CTA 1 w_up rows)
+      constexpr int kHStep = (EPI == EPI_SWIGLU) ? kMmaN / 2 : kMmaN;
+      const int brow0 = (EPI == EPI_SWIGLU)
+                            ? g * a.b_rows + n * NH * (kMmaN / 2)
+                            : g * a.b_rows + n * NH * kMmaN + (int)rank * (kMmaN / 2);
       for (int kb = 0; kb < nkb; ++kb) {
         if (!wait_pair(&ctl->empty[stage], phase ^ 1u, ctl, peer_abort, a.err, 1)) {
           ok = false;
           break;
         }
-        if (leader) mbar_expect_tx(&ctl->full[stage], 2 * kStage2Bytes);
-        uint8_t *sa = smem + (size_t)stage * kStage2Bytes;
+        if (leader) mbar_expect_tx(&ctl->full[stage], 2 * (kAHalf + (h1 - h0) * kBHalf));
+        uint8_t *sa = smem + (size_t)stage * kSB;
         const uint32_t fb = full0 + (uint32_t)(stage * sizeof(uint64_t));
         tma_load_2d_pair(&tmA, fb, sa, kb * kBlockK, arow);
-        tma_load_2d_pair(bmap, fb, sa + kAHalf, kb * kBlockK, brow);
+#pragma unroll
+        for (int h = 0; h < NH; ++h)
+          if (h >= h0 && h < h1)
+            tma_load_2d_pair(bmap, fb, sa + kAHalf + h * kBHalf, kb * kBlockK, brow0 + h * kHStep);
         issued |= 1u << stage;
         last_phase = (last_phase & ~(1u << stage)) | (phase << stage);
-        if (++stage == kStages2) { stage = 0; phase ^= 1u; }
+        if (++stage == kS) { stage = 0; phase ^= 1u; }
       }
     }
     // wait until the pair's MMAs have released every stage this CTA filled: the
     // last reads of our shared memory and the commit arrivals on our barriers are done
-    for (int s = 0; s < kStages2; ++s)
+    for (int s = 0; s < kS; ++s)
       if (issued & (1u << s))
         wait_pair(&ctl->empty[s], (last_phase >> s) & 1u, ctl, peer_abort, nullptr, 0, false,
                   ok ? kWaitLimitNs : kDrainNs);
@@ -446,7 +498,10 @@ k_ffn_tc2(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
     int stage = 0, acc = 0;
     uint32_t phase = 0, acc_phase = 0;
     bool ok = true, any = false;
-    for (int tile = c0; ok && tile < total; tile += cstep) {
+    for (int it = c0; ok && it < work.items; it += cstep) {
+      int sel;
+      work.tile(it, sel);
+      const int h0 = sel < 0 ? 0 : sel, h1 = sel < 0 ? NH : sel + 1;
       if (!wait_pair(&ctl->tempty[acc], acc_phase ^ 1u, ctl, peer_abort, a.err, 2)) {
         ok = false;
         break;
@@ -459,19 +514,23 @@ k_ffn_tc2(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
           break;
         }
         tc_fence_after();
-        const uint32_t sa = smem_u32(smem + (size_t)stage * kStage2Bytes);
+        const uint32_t sa = smem_u32(smem + (size_t)stage * kSB);
         const uint64_t da = sw128_desc(sa);
-        const uint64_t db = sw128_desc(sa + kAHalf);
 #pragma unroll
         for (int kk = 0; kk < kBlockK / 16; ++kk)
-          umma_bf16_pair(d_tmem, da + 2 * kk, db + 2 * kk, idesc, (kb | kk) != 0);
+#pragma unroll
+          for (int h = 0; h < NH; ++h)  // unrolled and predicated: a runtime loop here
+            if (h >= h0 && h < h1)      // measured ~7% slower
+              umma_bf16_pair(d_tmem + (uint32_t)(h * kMmaN), da + 2 * kk,
+                             sw128_desc(sa + kAHalf + h * kBHalf) + 2 * kk, idesc,
+                             (kb | kk) != 0);
         any = true;
         umma_commit_pair_both(&ctl->empty[stage]);
-        if (++stage == kStages2) { stage = 0; phase ^= 1u; }
+        if (++stage == kS) { stage = 0; phase ^= 1u; }
       }
       if (!ok) break;
       umma_commit_pair_both(&ctl->tfull[acc]);
-      if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+      if (++acc == PC::kAccBufs) { acc = 0; acc_phase ^= 1u; }
     }
     if (!ok && any) {  // retire the MMAs in flight before TMEM is released
       umma_commit_pair_own(&ctl->drain);
@@ -484,9 +543,9 @@ k_ffn_tc2(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
     const uint32_t tempty0 = mapa_rank(smem_u32(&ctl->tempty[0]), 0);
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int tile = c0; tile < total; tile += cstep) {
-      int g, n, m;
-      decode_tile(tile, ppre, G, a.n_tiles, g, n, m);
+    for (int it = c0; it < work.items; it += cstep) {
+      int sel, g, n, m;
+      decode_tile(work.tile(it, sel), ppre, G, a.n_tiles, g, n, m);
       bool ok = wait_pair(&ctl->tfull[acc], acc_phase, ctl, peer_abort, a.err, 4);
       __syncwarp();
       if (!__all_sync(0xffffffffu, ok)) break;
@@ -495,10 +554,22 @@ k_ffn_tc2(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
       const bool valid = grow < offs[g + 1] - offs[g];
       const size_t orow = (size_t)offs[g] + grow;
       const uint32_t tbase = tmem + ((uint32_t)(ew * 32) << 16) + (uint32_t)(acc * kMmaN);
-      epilogue_tile<EPI>(a, tbase, g, n, valid, orow, half);
+      if (NH == 1) {  // the two warps sharing a lane quarter take half the columns each
+        if (EPI == EPI_SWIGLU)
+          epilogue_tile<EPI>(a, tbase, g, 0, n * (kMmaN / 2), 2 * half, 2 * half + 2, valid, orow);
+        else
+          epilogue_tile<EPI>(a, tbase, g, 0, n * kMmaN, 4 * half, 4 * half + 4, valid, orow);
+      } else if (sel < 0 || sel == half) {  // ... or one N half (256 columns) each
+        if (EPI == EPI_SWIGLU)
+          epilogue_tile<EPI>(a, tbase, g, half * kMmaN, n * kMmaN + half * (kMmaN / 2), 0, 4,
+                             valid, orow);
+        else
+          epilogue_tile<EPI>(a, tbase, g, half * kMmaN, (2 * n + half) * kMmaN, 0, 8, valid,
+                             orow);
+      }
       tc_fence_before();
       mbar_arrive_cluster(tempty0 + (uint32_t)(acc * sizeof(uint64_t)));
-      if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+      if (++acc == PC::kAccBufs) { acc = 0; acc_phase ^= 1u; }
     }
   }
   if (*(volatile int *)&ctl->abort_flag) settle_ns(100000);  // copies in flight land
@@ -513,9 +584,8 @@ k_ffn_tc2(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
 
 // ------------------------------------------------------------------ host side
 struct DeviceInfo {
-  int sms = 0;
-  bool attr_set[6] = {false, false, false, false, false, false};
-  int max_pairs[3] = {0, 0, 0};
+  bool attr_set[9] = {};  // [EPI]: single-CTA kernel; [3 + slot]: pair kernel
+  int max_pairs[6] = {};  // [slot], slot = 3 * (NH - 1) + EPI
 };
 
 DeviceInfo &device_info(int dev) {
@@ -546,13 +616,15 @@ cudaError_t launch_single(const CUtensorMap &ma, const CUtensorMap &mb, const CU
   return cudaGetLastError();
 }
 
-template <int EPI>
+template <int EPI, int NH>
 cudaError_t launch_pair(const CUtensorMap &ma, const CUtensorMap &mb, const CUtensorMap &mb3,
                         const TcArgs &t, long long tiles_ub, cudaStream_t st) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   DeviceInfo &info = device_info(dev);
+  constexpr int slot = 3 * (NH - 1) + EPI;
+  constexpr size_t smem = pair_smem_bytes<NH>();
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -560,47 +632,62 @@ cudaError_t launch_pair(const CUtensorMap &ma, const CUtensorMap &mb, const CUte
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
   cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = kSmem2Bytes;
+  cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   {
     std::lock_guard<std::mutex> lock(g_attr_mu);
-    if (!info.attr_set[3 + EPI]) {
-      e = cudaFuncSetAttribute(k_ffn_tc2<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               (int)kSmem2Bytes);
+    if (!info.attr_set[3 + slot]) {
+      e = cudaFuncSetAttribute(k_ffn_tc2<EPI, NH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)smem);
       if (e != cudaSuccess) return e;
       cfg.gridDim = dim3(2 * (sm_count() / 2));
       int n = 0;
-      if (cudaOccupancyMaxActiveClusters(&n, k_ffn_tc2<EPI>, &cfg) != cudaSuccess || n <= 0)
+      if (cudaOccupancyMaxActiveClusters(&n, k_ffn_tc2<EPI, NH>, &cfg) != cudaSuccess || n <= 0)
         n = sm_count() / 2;
-      info.max_pairs[EPI] = n;
-      info.attr_set[3 + EPI] = true;
+      info.max_pairs[slot] = n;
+      info.attr_set[3 + slot] = true;
     }
   }
-  const long long pairs = std::min<long long>(tiles_ub, info.max_pairs[EPI]);
+  const long long pairs = std::min<long long>(tiles_ub, info.max_pairs[slot]);
   cfg.gridDim = dim3((unsigned)(2 * pairs));
-  e = cudaLaunchKernelEx(&cfg, k_ffn_tc2<EPI>, ma, mb, mb3, t);
+  e = cudaLaunchKernelEx(&cfg, k_ffn_tc2<EPI, NH>, ma, mb, mb3, t);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
-// Single-CTA tiles (128 rows) by default: measured 2-4% faster than pair tiles
-// (256 rows) on every workload here, and they waste less work when experts hold
-// few rows. MOE_TC_PAIR selects the CTA-pair kernel; both compute the same result.
+// Tile choice. A reduction of K >= kWideMinK takes the wide 256 x 512 CTA-pair
+// tile: twice the MMA work per pipeline stage hides the operand-load latency
+// that bounds the 128 x 256 single-CTA tile on long K. Short reductions keep the
+// single-CTA tile, whose double-buffered accumulator hides the epilogue (a large
+// share of a short tile). Building with MOE_TC_PAIR uses the 256 x 256 pair tile
+// everywhere instead. All three compute the same result.
+constexpr int kWideMinK = 2048;
+
 #ifdef MOE_TC_PAIR
 constexpr bool kUsePairs = true;
 #else
 constexpr bool kUsePairs = false;
 #endif
 
+inline bool uses_pairs(int K) { return kUsePairs || K >= kWideMinK; }
+
 template <int EPI>
 cudaError_t launch_gemm(const CUtensorMap &ma, const CUtensorMap &mb, const CUtensorMap &mb3,
-                        const TcArgs &t, int m_tiles_ub, int groups, cudaStream_t st) {
+                        TcArgs t, int m_tiles_ub, int groups, int n_cols, cudaStream_t st) {
+  // output columns per 256 accumulator columns
+  const int per_n = (EPI == EPI_SWIGLU) ? kMmaN / 2 : kMmaN;
+  const long long pair_m_ub = (long long)(m_tiles_ub + groups + 1) / 2;
   if (kUsePairs) {
-    const long long pairs_ub = (long long)(m_tiles_ub + groups + 1) / 2 * t.n_tiles;
-    return launch_pair<EPI>(ma, mb, mb3, t, std::max<long long>(pairs_ub, 1), st);
+    t.n_tiles = ceil_div(n_cols, per_n);
+    return launch_pair<EPI, 1>(ma, mb, mb3, t, std::max<long long>(pair_m_ub * t.n_tiles, 1), st);
   }
+  if (t.K >= kWideMinK) {
+    t.n_tiles = ceil_div(n_cols, 2 * per_n);
+    return launch_pair<EPI, 2>(ma, mb, mb3, t, std::max<long long>(pair_m_ub * t.n_tiles, 1), st);
+  }
+  t.n_tiles = ceil_div(n_cols, per_n);
   return launch_single<EPI>(ma, mb, mb3, t, (long long)m_tiles_ub * t.n_tiles, st);
 }
 
@@ -610,8 +697,8 @@ cudaError_t launch_ffn_tc(const GroupedFfnArgs &a, cudaStream_t st) {
   if (a.m_tiles_ub <= 0) return cudaSuccess;
   const bool swiglu = a.act == MOE_ACT_SWIGLU;
   // single-CTA tiles load 256 B rows at once (SwiGLU: two 128-row halves); pair
-  // tiles load 128 B rows per CTA
-  const uint32_t b_box = (kUsePairs || swiglu) ? kMmaN / 2 : kMmaN;
+  // tiles load 128 B rows per CTA and N half
+  const uint32_t b_box = (uses_pairs(a.d) || swiglu) ? kMmaN / 2 : kMmaN;
   CUtensorMap ma, mb, mb3;
   // up projection: [rows, d] x [G*F, d]^T -> h [rows, F]
   if (!make_map(&ma, a.a, (uint64_t)a.a_rows, (uint64_t)a.d, kTileM)) return cudaErrorInvalidValue;
@@ -628,29 +715,27 @@ cudaError_t launch_ffn_tc(const GroupedFfnArgs &a, cudaStream_t st) {
   t.G = a.G;
   t.N = a.F;
   t.K = a.d;
-  t.n_tiles = ceil_div(a.F, swiglu ? kMmaN / 2 : kMmaN);
   t.b_rows = a.F;
   t.out = a.h;
   t.out_f32 = 0;
   t.bias = a.b1;
   t.act = a.act;
   t.err = a.err;
-  cudaError_t e = swiglu ? launch_gemm<EPI_SWIGLU>(ma, mb, mb3, t, a.m_tiles_ub, a.G, st)
-                         : launch_gemm<EPI_ACT>(ma, mb, mb3, t, a.m_tiles_ub, a.G, st);
+  cudaError_t e = swiglu ? launch_gemm<EPI_SWIGLU>(ma, mb, mb3, t, a.m_tiles_ub, a.G, a.F, st)
+                         : launch_gemm<EPI_ACT>(ma, mb, mb3, t, a.m_tiles_ub, a.G, a.F, st);
   if (e != cudaSuccess) return e;
   // down projection: h [rows, F] x [G*d, F]^T -> out [rows, d]
-  const uint32_t b_box2 = kUsePairs ? kMmaN / 2 : kMmaN;
+  const uint32_t b_box2 = uses_pairs(a.F) ? kMmaN / 2 : kMmaN;
   if (!make_map(&ma, a.h, (uint64_t)a.a_rows, (uint64_t)a.F, kTileM)) return cudaErrorInvalidValue;
   if (!make_map(&mb, a.w2, (uint64_t)a.G * a.d, (uint64_t)a.F, b_box2)) return cudaErrorInvalidValue;
   t.N = a.d;
   t.K = a.F;
-  t.n_tiles = ceil_div(a.d, kMmaN);
   t.b_rows = a.d;
   t.out = a.out;
   t.out_f32 = a.out_f32;
   t.bias = a.b2;
   t.act = -1;
-  return launch_gemm<EPI_DOWN>(ma, mb, mb, t, a.m_tiles_ub, a.G, st);
+  return launch_gemm<EPI_DOWN>(ma, mb, mb, t, a.m_tiles_ub, a.G, a.d, st);
 }
 
 }  // namespace moe

@@ -177,6 +177,16 @@ FFN_CASES = [
     # still the small-batch path, with an expert spanning two 32-row chunks
     ("swiglu_bf16_decode_chunks", synth.ACT_SWIGLU, synth.DT_BF16, 256, 384, 2, [33, 20]),
     ("gelu_bf16_decode_chunks", synth.ACT_GELU, synth.DT_BF16, 128, 256, 2, [45, 10]),
+    # reductions of 2048 and more: the 256 x 512 CTA-pair tile (ragged N, a pair
+    # tile whose second CTA holds one row)
+    ("swiglu_bf16_wide_up", synth.ACT_SWIGLU, synth.DT_BF16, 2112, 320, 3, [300, 0, 200]),
+    ("gelu_bf16_wide_down_bias", synth.ACT_GELU, synth.DT_BF16, 192, 2112, 3, [260, 5, 0]),
+    ("relu_bf16_wide_both", synth.ACT_RELU, synth.DT_BF16, 2048, 2048, 2, [129, 257]),
+    # 80 wide tiles over the 74 CTA pairs of a B200: the last round runs as half tiles
+    ("relu_bf16_wide_tail", synth.ACT_RELU, synth.DT_BF16, 2048, 2048, 4,
+     [1300, 1300, 1000, 1000]),
+    ("swiglu_bf16_wide_tail", synth.ACT_SWIGLU, synth.DT_BF16, 2048, 1024, 4,
+     [1300, 1300, 1000, 1000]),
 ]
 
 
