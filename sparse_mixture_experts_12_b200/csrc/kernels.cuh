@@ -18,6 +18,7 @@ struct RouterArgs {
   float *tile_p;            // [E, NT] or nullptr: per-tile sums of softmax probabilities
   float *tile_z;            // [NT] or nullptr: per-tile sums of logsumexp^2
   int T, d, E, k, gate_mode;
+  int32_t *err;             // device error word (pipeline timeouts) or nullptr
 };
 
 struct ScanArgs {
@@ -79,6 +80,8 @@ struct GroupedFfnArgs {
 };
 
 cudaError_t launch_router(const RouterArgs &a, int dtype, cudaStream_t st);
+// bf16 router on the tensor cores (x given, 16 <= E <= 256)
+cudaError_t launch_router_tc(const RouterArgs &a, cudaStream_t st);
 cudaError_t launch_tile_counts(const int32_t *topk_idx, int T, int k, int E, int32_t *tile_counts,
                                int32_t *err, cudaStream_t st);
 cudaError_t launch_scan(const ScanArgs &a, cudaStream_t st);

@@ -246,6 +246,7 @@ MOE_API moe_status_t moe_route(const moe_cfg_t *cfg, const moe_weights_t *w, con
   r.E = c.n_experts;
   r.k = c.top_k;
   r.gate_mode = c.gate_mode;
+  r.err = at<int32_t>(ws, L, B_ERR);
   MOE_CUDA(launch_router(r, c.dtype, stream));
   return MOE_OK;
 }
@@ -367,6 +368,7 @@ MOE_API moe_status_t moe_aux_stats(const moe_cfg_t *cfg, const float *logits,
   r.E = c.n_experts;
   r.k = c.top_k;
   r.gate_mode = c.gate_mode;
+  r.err = err;
   MOE_CUDA(launch_router(r, c.dtype, stream));
   int32_t *tile_counts = at<int32_t>(ws, L, B_TILE_COUNTS);
   MOE_CUDA(launch_tile_counts(topk_idx, c.n_tokens, c.top_k, c.n_experts, tile_counts, err, stream));
@@ -438,6 +440,7 @@ MOE_API moe_status_t moe_forward(const moe_cfg_t *cfg, const moe_weights_t *w, c
   r.E = c.n_experts;
   r.k = c.top_k;
   r.gate_mode = c.gate_mode;
+  r.err = err;
   MOE_CUDA(launch_router(r, c.dtype, stream));
   // 2. scan: counts, capacity, offsets, GEMM tile table (+ aux statistics)
   ScanArgs s{};

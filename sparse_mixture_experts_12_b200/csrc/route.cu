@@ -16,6 +16,7 @@ namespace {
 constexpr int kRouterThreads = 256;
 constexpr int kBK = 32;  // K elements per slice per iteration
 constexpr int kRouterStages = 3;  // cp.async ring depth
+constexpr int kRouterTcMinTokens = 256;
 
 template <int EPAD> struct RouterShape;
 template <> struct RouterShape<8>   { static constexpr int BM = 32, TM = 1, TN = 8, KS = 8; };
@@ -576,6 +577,10 @@ cudaError_t launch_router(const RouterArgs &a, int dtype, cudaStream_t st) {
       8LL * a.d * (dtype == MOE_DTYPE_F32 ? 4 : 2) <= 96LL * 1024)
     return dtype == MOE_DTYPE_F32 ? launch_router_gemv<float>(a, st)
                                   : launch_router_gemv<__nv_bfloat16>(a, st);
+  // bf16 with many experts and enough tokens: the tensor-core router (the
+  // CUDA-core GEMM below is FMA-bound there)
+  if (dtype == MOE_DTYPE_BF16 && a.x != nullptr && E >= 16 && a.T >= kRouterTcMinTokens)
+    return launch_router_tc(a, st);
   if (E <= 8) return launch_router_e<8>(a, dtype, st);
   if (E <= 16) return launch_router_e<16>(a, dtype, st);
   if (E <= 32) return launch_router_e<32>(a, dtype, st);

@@ -120,6 +120,14 @@ SMALL = {
                                              d_ff_shared=384),
     "decode_chunks": MIXTRAL_PREFILL.replace(name="decode_chunks", T=64, d_model=256, d_ff=384,
                                              n_experts=2, top_k=1),
+    # bf16 routers with 20 and 256 experts (expert counts that pad to the MMA's N),
+    # router and logit biases, ragged token tiles
+    "router_e20": DEEPSEEK_FINE.replace(name="router_e20", T=700, d_model=256, d_ff=128,
+                                        n_experts=20, top_k=3, n_shared=0, d_ff_shared=0,
+                                        router_bias=True, bias_std=0.1, logit_bias_std=0.5),
+    "router_e256": SWITCH_CAPACITY.replace(name="router_e256", T=300, d_model=128, d_ff=64,
+                                           n_experts=256, top_k=8, capacity_factor=0.0,
+                                           bias_std=0.1),
     "fp32_swiglu": DEEPSEEK_FINE.replace(name="fp32_swiglu", T=150, d_model=96, d_ff=160,
                                          n_experts=16, top_k=3, dtype=DT_F32,
                                          d_ff_shared=64),
