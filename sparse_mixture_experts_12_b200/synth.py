@@ -120,6 +120,9 @@ SMALL = {
                                              d_ff_shared=384),
     "decode_chunks": MIXTRAL_PREFILL.replace(name="decode_chunks", T=64, d_model=256, d_ff=384,
                                              n_experts=2, top_k=1),
+    # SwiGLU experts with a capacity of 112 rows each
+    "mixtral_cap": MIXTRAL_PREFILL.replace(name="mixtral_cap", T=900, d_model=256, d_ff=384,
+                                           capacity_factor=0.5),
     # bf16 routers with 20 and 256 experts (expert counts that pad to the MMA's N),
     # router and logit biases, ragged token tiles
     "router_e20": DEEPSEEK_FINE.replace(name="router_e20", T=700, d_model=256, d_ff=128,

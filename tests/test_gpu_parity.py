@@ -177,6 +177,10 @@ FFN_CASES = [
     # still the small-batch path, with an expert spanning two 32-row chunks
     ("swiglu_bf16_decode_chunks", synth.ACT_SWIGLU, synth.DT_BF16, 256, 384, 2, [33, 20]),
     ("gelu_bf16_decode_chunks", synth.ACT_GELU, synth.DT_BF16, 128, 256, 2, [45, 10]),
+    # 190..256 rows in all: one or two 128-row tiles per expert
+    ("swiglu_bf16_medium", synth.ACT_SWIGLU, synth.DT_BF16, 256, 384, 5, [0, 1, 129, 60, 30]),
+    ("gelu_bf16_medium_bias", synth.ACT_GELU, synth.DT_BF16, 128, 320, 4, [200, 0, 17, 33]),
+    ("relu_bf16_medium_ntail", synth.ACT_RELU, synth.DT_BF16, 192, 192, 2, [100, 90]),
     # reductions of 2048 and more: the 256 x 512 CTA-pair tile (ragged N, a pair
     # tile whose second CTA holds one row)
     ("swiglu_bf16_wide_up", synth.ACT_SWIGLU, synth.DT_BF16, 2112, 320, 3, [300, 0, 200]),
