@@ -77,8 +77,8 @@ __device__ __forceinline__ bool rt_better(float v, int i, float bv, int bi) {
 // One token per thread (TMEM lane = token row). Pass 1 reads the logits from
 // TMEM in 32-column chunks, adds the biases, writes them out, keeps the running
 // max and parks z (NaN -> -inf) in the thread's row of the shared-memory tile.
-// Pass 2 takes the top-k from that row, pass 3 sums exp(z - max) and leaves the
-// probabilities in the row for the per-tile sums.
+// Then k argmax rounds over that row give the top-k, and a last pass sums
+// exp(z - max) and leaves the probabilities in the row for the per-tile sums.
 template <int EPAD>
 __device__ __forceinline__ void epilogue_rows(const RouterArgs &a, RtCtl *ctl, float *prob,
                                               uint32_t tmem, int t0, int NT, int BM, int warp,
@@ -132,37 +132,40 @@ __device__ __forceinline__ void epilogue_rows(const RouterArgs &a, RtCtl *ctl, f
     }
   }
 
-  // top-k in expert order; a candidate enters when it ranks above the current k-th
+  // top-k as k argmax rounds over the row, each taking the best entry ranked below
+  // the previous pick (value descending, ties to the lower index): no marks, no
+  // divergence; four interleaved partial argmaxes per round for ILP
   float tv[kMaxTopK];
   int ti[kMaxTopK];
+  float pv = INFINITY;
+  int pi = -1;
 #pragma unroll
-  for (int s = 0; s < kMaxTopK; ++s) { tv[s] = -INFINITY; ti[s] = 0x7fffffff; }
-  float kth_v = -INFINITY;
-  int kth_i = 0x7fffffff;
-#pragma unroll 1
-  for (int e = 0; e < E; ++e) {
-    const float z = row[e];
-    if (rt_better(z, e, kth_v, kth_i)) {
-      // sorted insertion from the tail: entries ranking below z move down one slot
+  for (int s = 0; s < kMaxTopK; ++s) {
+    tv[s] = -INFINITY;
+    ti[s] = 0x7fffffff;
+    if (s < k) {
+      float bv[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+      int bi[4] = {0x7fffffff, 0x7fffffff, 0x7fffffff, 0x7fffffff};
+      int e = 0;
+#pragma unroll 2
+      for (; e + 4 <= E; e += 4) {
 #pragma unroll
-      for (int s = kMaxTopK - 1; s >= 1; --s) {
-        if (s < k) {
-          if (rt_better(z, e, tv[s - 1], ti[s - 1])) {
-            tv[s] = tv[s - 1]; ti[s] = ti[s - 1];
-          } else if (rt_better(z, e, tv[s], ti[s])) {
-            tv[s] = z; ti[s] = e;
-          }
+        for (int q = 0; q < 4; ++q) {
+          const float z = row[e + q];
+          const bool below = z < pv || (z == pv && e + q > pi);
+          if (below && rt_better(z, e + q, bv[q], bi[q])) { bv[q] = z; bi[q] = e + q; }
         }
       }
-      if (rt_better(z, e, tv[0], ti[0])) { tv[0] = z; ti[0] = e; }
-      // the new k-th entry, as a select chain (an indexed read would go to local memory)
-      kth_v = tv[0];
-      kth_i = ti[0];
-#pragma unroll
-      for (int s = 1; s < kMaxTopK; ++s) {
-        kth_v = s < k ? tv[s] : kth_v;
-        kth_i = s < k ? ti[s] : kth_i;
+      for (; e < E; ++e) {
+        const float z = row[e];
+        const bool below = z < pv || (z == pv && e > pi);
+        if (below && rt_better(z, e, bv[0], bi[0])) { bv[0] = z; bi[0] = e; }
       }
+#pragma unroll
+      for (int q = 1; q < 4; ++q)
+        if (rt_better(bv[q], bi[q], bv[0], bi[0])) { bv[0] = bv[q]; bi[0] = bi[q]; }
+      tv[s] = pv = bv[0];
+      ti[s] = pi = bi[0];
     }
   }
 
