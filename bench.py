@@ -50,7 +50,7 @@ def load_peaks():
 
 # ------------------------------------------------------------------ clocks sampler
 class ClockSampler:
-    """Polls the GPU's SM clock and clock-event reasons through NVML every 20 ms
+    """Polls the GPU's SM clock and clock-event reasons through NVML every 5 ms
     (read-only queries) while the timed region runs."""
 
     # NVML clock-event reason bits (nvmlClocksEventReason*)
@@ -87,7 +87,7 @@ class ClockSampler:
                 self.samples.append((time.time(), sm, self._reasons()))
             except Exception:
                 pass
-            time.sleep(0.02)
+            time.sleep(0.005)
 
     def start(self):
         if self.nv is None:
@@ -107,10 +107,12 @@ class ClockSampler:
         self.done.set()
         self.thread.join(timeout=2)
         rows = [(sm, r) for (t, sm, r) in self.samples if self.mark is None or self.mark <= t <= end]
+        if not rows:  # a region shorter than the poll period: the first sample after it began
+            rows = [(sm, r) for (t, sm, r) in self.samples if self.mark is None or t >= self.mark][:1]
         reasons = sorted({n for (_, r) in rows for n, b in self.REASON_BITS.items() if r & b})
         sm = [x for (x, _) in rows]
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": self.max_mhz,
-                "reasons": reasons, "samples": len(sm), "source": "NVML, 20 ms polling"}
+                "reasons": reasons, "samples": len(sm), "source": "NVML, 5 ms polling"}
 
 
 # ----------------------------------------------------------- multi-rank plumbing
