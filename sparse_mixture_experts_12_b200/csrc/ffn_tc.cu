@@ -11,17 +11,20 @@
 //   warp 0      TMA producer: A rows of the expert-contiguous activations and the
 //               expert's weight rows, 64-element K slices with 128-byte swizzle,
 //               into a shared-memory ring.
-//   warp 1      MMA issuer: tcgen05.mma (kind::f16, fp32 accumulate in TMEM), two
-//               256-column accumulators so the epilogue of tile i overlaps the
-//               main loop of tile i+1.
+//   warp 1      MMA issuer: tcgen05.mma (kind::f16, fp32 accumulate in TMEM).
 //   warp 2      TMEM allocator.
 //   warps 4..11 epilogue (two warps per TMEM lane quarter, half the columns
 //               each): tcgen05.ld, fused silu(g)*u / bias+ReLU / bias+GELU,
 //               bf16 (or fp32) stores masked to the expert's rows.
-// Two tile shapes: a CTA pair (cluster of 2, tcgen05.mma.cta_group::2, 256 rows x
-// 256 columns, 6 x 32 KB stages per CTA) by default, and a single CTA (128 rows x
-// 256 columns, 4 x 48 KB stages). For SwiGLU the 256 MMA columns are w_gate rows
-// [n, n+128) next to w_up rows [n, n+128), so one MMA yields both halves.
+// Tile shapes, chosen per projection by its reduction length K:
+//   K >= 2048  a CTA pair (cluster of 2, tcgen05.mma.cta_group::2): 256 rows x 512
+//              columns, two M256 N256 MMAs per K step into one 512-column
+//              accumulator, 4 x 48 KB stages per CTA;
+//   K <  2048  a single CTA: 128 rows x 256 columns, two 256-column accumulators
+//              (the epilogue overlaps the next tile), 4 x 48 KB stages.
+// A 256 x 256 pair tile (6 x 32 KB stages) is built with -DMOE_TC_PAIR.
+// For SwiGLU each 256 MMA columns are w_gate rows next to the same w_up rows, so
+// one MMA yields both halves of silu(g) * u.
 // The tile list is built on the device (per-expert M-tile prefix), so no host
 // synchronisation sits between routing and the expert GEMMs. Every wait is
 // bounded; on a timeout the CTA records MOE_DEVERR_WAIT_TIMEOUT, drains its

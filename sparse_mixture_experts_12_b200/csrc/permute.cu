@@ -45,13 +45,18 @@ __global__ void __launch_bounds__(kScanThreads) k_scan(ScanArgs a) {
   for (int e = warp; e < E; e += nw) {
     const int32_t *tc = a.tile_counts + (size_t)e * NT;
     int32_t *tb = a.tile_base + (size_t)e * NT;
+    const float *tp = a.aux_out ? a.tile_p + (size_t)e * NT : nullptr;
     int run = 0;
+    float p = 0.f;  // this lane's tiles t = lane, lane + 32, ... in order
     for (int b0 = 0; b0 < NT; b0 += 32 * kScanVPL) {
+      // the counts and the probability sums of this block, all requested at once
       int v[kScanVPL];
+      float pv[kScanVPL];
 #pragma unroll
       for (int j = 0; j < kScanVPL; ++j) {
         const int t = b0 + j * 32 + lane;
         v[j] = t < NT ? tc[t] : 0;
+        pv[j] = (tp != nullptr && t < NT) ? tp[t] : 0.f;
       }
 #pragma unroll
       for (int j = 0; j < kScanVPL; ++j) {
@@ -59,12 +64,11 @@ __global__ void __launch_bounds__(kScanThreads) k_scan(ScanArgs a) {
         const int t = b0 + j * 32 + lane;
         if (t < NT) tb[t] = run + incl - v[j];
         run += __shfl_sync(0xffffffffu, incl, 31);
+        p += pv[j];
       }
     }
     if (lane == 0) count_s[e] = run;
-    if (a.aux_out) {
-      float p = 0.f;
-      for (int t = lane; t < NT; t += 32) p += a.tile_p[(size_t)e * NT + t];
+    if (tp != nullptr) {
       p = warp_sum(p);
       if (lane == 0) P_s[e] = p / (float)a.T;
     }
@@ -116,21 +120,30 @@ __global__ void __launch_bounds__(kScanThreads) k_scan(ScanArgs a) {
   z = warp_sum(z);
   if (lane == 0) red[warp] = z;
   __syncthreads();
-  if (threadIdx.x == 0) {
-    float zs = 0.f;
-    for (int w = 0; w < nw; ++w) zs += red[w];
+  if (warp == 0) {
+    // fp64 sums over the experts: lane l takes experts l, l + 32, ..., then a
+    // fixed shuffle tree
     const double inv_tk = 1.0 / ((double)a.T * (double)a.k);
     double fp = 0.0, bsq = 0.0;
-    for (int e = 0; e < E; ++e) {
+    for (int e = lane; e < E; e += 32) {
       const double f = (double)count_s[e] * inv_tk;
       fp += f * (double)P_s[e];
       bsq += (f - 1.0 / E) * (f - 1.0 / E);
       a.aux_out[3 + e] = (float)f;
       a.aux_out[3 + E + e] = P_s[e];
     }
-    a.aux_out[0] = (float)((double)a.alpha * E * fp);
-    a.aux_out[1] = zs / (float)a.T;
-    a.aux_out[2] = (float)bsq;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      fp += __shfl_xor_sync(0xffffffffu, fp, o);
+      bsq += __shfl_xor_sync(0xffffffffu, bsq, o);
+    }
+    if (lane == 0) {
+      float zs = 0.f;
+      for (int w = 0; w < nw; ++w) zs += red[w];
+      a.aux_out[0] = (float)((double)a.alpha * E * fp);
+      a.aux_out[1] = zs / (float)a.T;
+      a.aux_out[2] = (float)bsq;
+    }
   }
 }
 
