@@ -660,12 +660,15 @@ cudaError_t launch_pair(const CUtensorMap &ma, const CUtensorMap &mb, const CUte
   return cudaGetLastError();
 }
 
-// Tile choice. A reduction of K >= kWideMinK takes the wide 256 x 512 CTA-pair
-// tile: twice the MMA work per pipeline stage hides the operand-load latency
-// that bounds the 128 x 256 single-CTA tile on long K. Short reductions keep the
-// single-CTA tile, whose double-buffered accumulator hides the epilogue (a large
-// share of a short tile). Building with MOE_TC_PAIR uses the 256 x 256 pair tile
-// everywhere instead. All three compute the same result.
+// Tile choice. A reduction of K >= kWideMinK over experts that average at least
+// one 256-row pair tile takes the wide 256 x 512 CTA-pair tile: twice the MMA
+// work per pipeline stage hides the operand-load latency that bounds the
+// 128 x 256 single-CTA tile on long K. Short reductions keep the single-CTA tile,
+// whose double-buffered accumulator hides the epilogue (a large share of a short
+// tile), and so do experts with few rows (capacity-limited layers), where
+// 128-row tiles waste less and give every SM a tile of its own. Building with
+// MOE_TC_PAIR uses the 256 x 256 pair tile everywhere instead. All three compute
+// the same result.
 constexpr int kWideMinK = 2048;
 
 #ifdef MOE_TC_PAIR
@@ -674,11 +677,15 @@ constexpr bool kUsePairs = true;
 constexpr bool kUsePairs = false;
 #endif
 
-inline bool uses_pairs(int K) { return kUsePairs || K >= kWideMinK; }
+inline bool use_wide(int K, long long rows, int groups) {
+  return !kUsePairs && K >= kWideMinK && rows >= (long long)kPairM * groups;
+}
+inline bool uses_pairs(bool wide) { return kUsePairs || wide; }
 
 template <int EPI>
 cudaError_t launch_gemm(const CUtensorMap &ma, const CUtensorMap &mb, const CUtensorMap &mb3,
-                        TcArgs t, int m_tiles_ub, int groups, int n_cols, cudaStream_t st) {
+                        TcArgs t, int m_tiles_ub, int groups, int n_cols, bool wide,
+                        cudaStream_t st) {
   // output columns per 256 accumulator columns
   const int per_n = (EPI == EPI_SWIGLU) ? kMmaN / 2 : kMmaN;
   const long long pair_m_ub = (long long)(m_tiles_ub + groups + 1) / 2;
@@ -686,7 +693,7 @@ cudaError_t launch_gemm(const CUtensorMap &ma, const CUtensorMap &mb, const CUte
     t.n_tiles = ceil_div(n_cols, per_n);
     return launch_pair<EPI, 1>(ma, mb, mb3, t, std::max<long long>(pair_m_ub * t.n_tiles, 1), st);
   }
-  if (t.K >= kWideMinK) {
+  if (wide) {
     t.n_tiles = ceil_div(n_cols, 2 * per_n);
     return launch_pair<EPI, 2>(ma, mb, mb3, t, std::max<long long>(pair_m_ub * t.n_tiles, 1), st);
   }
@@ -701,7 +708,8 @@ cudaError_t launch_ffn_tc(const GroupedFfnArgs &a, cudaStream_t st) {
   const bool swiglu = a.act == MOE_ACT_SWIGLU;
   // single-CTA tiles load 256 B rows at once (SwiGLU: two 128-row halves); pair
   // tiles load 128 B rows per CTA and N half
-  const uint32_t b_box = (uses_pairs(a.d) || swiglu) ? kMmaN / 2 : kMmaN;
+  const bool wide_up = use_wide(a.d, a.a_rows, a.G), wide_down = use_wide(a.F, a.a_rows, a.G);
+  const uint32_t b_box = (uses_pairs(wide_up) || swiglu) ? kMmaN / 2 : kMmaN;
   CUtensorMap ma, mb, mb3;
   // up projection: [rows, d] x [G*F, d]^T -> h [rows, F]
   if (!make_map(&ma, a.a, (uint64_t)a.a_rows, (uint64_t)a.d, kTileM)) return cudaErrorInvalidValue;
@@ -724,11 +732,12 @@ cudaError_t launch_ffn_tc(const GroupedFfnArgs &a, cudaStream_t st) {
   t.bias = a.b1;
   t.act = a.act;
   t.err = a.err;
-  cudaError_t e = swiglu ? launch_gemm<EPI_SWIGLU>(ma, mb, mb3, t, a.m_tiles_ub, a.G, a.F, st)
-                         : launch_gemm<EPI_ACT>(ma, mb, mb3, t, a.m_tiles_ub, a.G, a.F, st);
+  cudaError_t e =
+      swiglu ? launch_gemm<EPI_SWIGLU>(ma, mb, mb3, t, a.m_tiles_ub, a.G, a.F, wide_up, st)
+             : launch_gemm<EPI_ACT>(ma, mb, mb3, t, a.m_tiles_ub, a.G, a.F, wide_up, st);
   if (e != cudaSuccess) return e;
   // down projection: h [rows, F] x [G*d, F]^T -> out [rows, d]
-  const uint32_t b_box2 = uses_pairs(a.F) ? kMmaN / 2 : kMmaN;
+  const uint32_t b_box2 = uses_pairs(wide_down) ? kMmaN / 2 : kMmaN;
   if (!make_map(&ma, a.h, (uint64_t)a.a_rows, (uint64_t)a.F, kTileM)) return cudaErrorInvalidValue;
   if (!make_map(&mb, a.w2, (uint64_t)a.G * a.d, (uint64_t)a.F, b_box2)) return cudaErrorInvalidValue;
   t.N = a.d;
@@ -738,7 +747,7 @@ cudaError_t launch_ffn_tc(const GroupedFfnArgs &a, cudaStream_t st) {
   t.out_f32 = a.out_f32;
   t.bias = a.b2;
   t.act = -1;
-  return launch_gemm<EPI_DOWN>(ma, mb, mb, t, a.m_tiles_ub, a.G, a.d, st);
+  return launch_gemm<EPI_DOWN>(ma, mb, mb, t, a.m_tiles_ub, a.G, a.d, wide_down, st);
 }
 
 }  // namespace moe

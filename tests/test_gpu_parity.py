@@ -181,11 +181,14 @@ FFN_CASES = [
     ("swiglu_bf16_medium", synth.ACT_SWIGLU, synth.DT_BF16, 256, 384, 5, [0, 1, 129, 60, 30]),
     ("gelu_bf16_medium_bias", synth.ACT_GELU, synth.DT_BF16, 128, 320, 4, [200, 0, 17, 33]),
     ("relu_bf16_medium_ntail", synth.ACT_RELU, synth.DT_BF16, 192, 192, 2, [100, 90]),
-    # reductions of 2048 and more: the 256 x 512 CTA-pair tile (ragged N, a pair
-    # tile whose second CTA holds one row)
-    ("swiglu_bf16_wide_up", synth.ACT_SWIGLU, synth.DT_BF16, 2112, 320, 3, [300, 0, 200]),
-    ("gelu_bf16_wide_down_bias", synth.ACT_GELU, synth.DT_BF16, 192, 2112, 3, [260, 5, 0]),
-    ("relu_bf16_wide_both", synth.ACT_RELU, synth.DT_BF16, 2048, 2048, 2, [129, 257]),
+    # reductions of 2048 and more over experts averaging 256+ rows: the 256 x 512
+    # CTA-pair tile (ragged N, pair tiles whose second CTA holds no row or one row)
+    ("swiglu_bf16_wide_up", synth.ACT_SWIGLU, synth.DT_BF16, 2112, 320, 3, [300, 0, 529]),
+    ("gelu_bf16_wide_down_bias", synth.ACT_GELU, synth.DT_BF16, 192, 2112, 3, [260, 5, 600]),
+    ("relu_bf16_wide_both", synth.ACT_RELU, synth.DT_BF16, 2048, 2048, 2, [129, 400]),
+    # the same reduction lengths over experts with few rows: 128-row single-CTA tiles
+    ("swiglu_bf16_long_k_few_rows", synth.ACT_SWIGLU, synth.DT_BF16, 2112, 320, 3,
+     [100, 0, 200]),
     # 80 wide tiles over the 74 CTA pairs of a B200: the last round runs as half tiles
     ("relu_bf16_wide_tail", synth.ACT_RELU, synth.DT_BF16, 2048, 2048, 4,
      [1300, 1300, 1000, 1000]),
