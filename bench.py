@@ -356,31 +356,63 @@ def run_ours(args, wl, rank, world, local_rank):
     roof["algorithmic"] = {"flops": flops, "bytes": alg_bytes, "rows": R,
                            "touched_experts": touched}
 
-    # ---- end to end through the public API with host buffers
+    # ---- end to end through the public API with host buffers. Every step copies
+    # its input from pinned host memory, runs moe_forward and copies its output
+    # (and the aux statistics) back to pinned host memory. Two buffer slots and
+    # three streams (copy in, compute, copy out) let step i+1's input copy and step
+    # i-1's output copy run under step i's compute; events order each slot's reuse.
     xh = inp["x"].pin_memory()
-    yh = torch.empty(x.shape, dtype=x.dtype).pin_memory()
+    slots = []
     for _ in range(2):
-        x.copy_(xh, non_blocking=True)
-        layer.forward(x, y, aux)
-        yh.copy_(y, non_blocking=True)
+        slots.append({"x": torch.empty_like(x), "y": torch.empty_like(y),
+                      "aux": None if aux is None else torch.empty_like(aux),
+                      "yh": torch.empty(x.shape, dtype=x.dtype).pin_memory(),
+                      "auxh": None if aux is None else torch.empty(aux.shape).pin_memory(),
+                      "in": torch.cuda.Event(), "comp": torch.cuda.Event(),
+                      "out": torch.cuda.Event()})
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+
+    def e2e_steps(n):
+        for i in range(n):
+            sl = slots[i % 2]
+            with torch.cuda.stream(s_in):
+                s_in.wait_event(sl["comp"])  # the slot's previous forward has read x
+                sl["x"].copy_(xh, non_blocking=True)
+                sl["in"].record(s_in)
+            stream.wait_event(sl["in"])
+            stream.wait_event(sl["out"])     # the slot's previous output has left
+            layer.forward(sl["x"], sl["y"], sl["aux"])
+            sl["comp"].record(stream)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(sl["comp"])
+                sl["yh"].copy_(sl["y"], non_blocking=True)
+                if sl["aux"] is not None:
+                    sl["auxh"].copy_(sl["aux"], non_blocking=True)
+                sl["out"].record(s_out)
+
+    e2e_steps(4)
     torch.cuda.synchronize()
     barrier(world)
     g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    g0.record(stream)
-    for _ in range(args.steps):
-        x.copy_(xh, non_blocking=True)
-        layer.forward(x, y, aux)
-        yh.copy_(y, non_blocking=True)
-        if aux is not None:
-            aux.cpu()
-    g1.record(stream)
+    g0.record(s_in)
+    s_in.wait_event(g0)
+    stream.wait_event(g0)
+    s_out.wait_event(g0)
+    e2e_steps(args.steps)
+    for sl in slots:  # the end: both slots' last outputs are on the host
+        s_out.wait_event(sl["out"])
+    g1.record(s_out)
     torch.cuda.synchronize()
     barrier(world)
     e2e_ms = max_over_ranks(g0.elapsed_time(g1), world, dev)
     e2e = {"value": tokens_per_second(wl.T, world, args.steps, e2e_ms), "unit": "tokens/s",
            "h2d_bytes_per_step": int(xh.numel() * xh.element_size()),
-           "d2h_bytes_per_step": int(yh.numel() * yh.element_size()) +
-           (int(aux.numel() * 4) if aux is not None else 0)}
+           "d2h_bytes_per_step": int(slots[0]["yh"].numel() * slots[0]["yh"].element_size()) +
+           (int(aux.numel() * 4) if aux is not None else 0),
+           "pipelining": "2 slots, copy-in / compute / copy-out streams"}
+    code, info = layer.last_device_error()
+    if code != 0:
+        raise RuntimeError(f"device error {code} ({info}) in the end-to-end loop")
 
     if rank != 0:
         return
