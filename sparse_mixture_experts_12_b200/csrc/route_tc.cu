@@ -10,11 +10,11 @@
 // top-k renormalised (youngju.dev ja "TopKGating"), softmax then top-1 raw
 // (SwitchRouter).
 //
-// One CTA per 128 tokens, 192 threads:
+// One CTA per 128 tokens, 320 threads:
 //   warp 0      TMA producer: 128 x 64 slices of x and EPAD x 64 slices of W_r
 //               (rows >= E read as zeros), 128-byte swizzle, 4..9-stage ring.
 //   warp 1      TMEM owner and MMA issuer (M = 128, N = EPAD, K = 16 per MMA).
-//   warps 2..5  epilogue, one token per thread (TMEM lane = token row).
+//   warps 2..9  epilogue, two threads per token.
 // Same results as the SIMT router up to the fp32 summation order of the dot
 // products: same bias order, NaN -> -inf before selection, ties to the lower
 // expert index, same gate formulas, same fixed-order per-tile sums.
@@ -31,7 +31,8 @@ using namespace tc;
 constexpr int kRtMaxStages = 10;
 constexpr int kRtRingBudget = 192 * 1024;  // shared memory for the operand ring
 constexpr int kRtM = 128;  // tokens per CTA
-constexpr int kRtThreads = 192;
+constexpr int kRtEpiThreads = 256;  // two threads per token
+constexpr int kRtThreads = 64 + kRtEpiThreads;
 constexpr int kRtABytes = kRtM * kBlockK * 2;
 constexpr int kRtMaxSubs = 4;  // permute tiles per CTA: 128 / router_bm(E)
 
@@ -47,6 +48,12 @@ struct RtCtl {
   float lb[kMaxExperts];  // per-expert logit bias (0 when absent)
   float lse[kRtM];
   int cnt[kRtMaxSubs][kMaxExperts];
+  // the two threads of a token meet here: max, top-k candidates (double-buffered
+  // by round parity), exp sums
+  float hmax[2][kRtM];
+  float cand_v[2][2][kRtM];
+  int cand_i[2][2][kRtM];
+  float hsum[2][kRtM];
 };
 
 template <int EPAD> struct RtCfg {
@@ -74,67 +81,83 @@ __device__ __forceinline__ bool rt_better(float v, int i, float bv, int bi) {
   return v > bv || (v == bv && i < bi);
 }
 
-// One token per thread (TMEM lane = token row). Pass 1 reads the logits from
-// TMEM in 32-column chunks, adds the biases, writes them out, keeps the running
-// max and parks z (NaN -> -inf) in the thread's row of the shared-memory tile.
-// Then k argmax rounds over that row give the top-k, and a last pass sums
-// exp(z - max) and leaves the probabilities in the row for the per-tile sums.
+__device__ __forceinline__ void rt_epi_sync() {
+  asm volatile("bar.sync 1, %0;" ::"n"(kRtEpiThreads) : "memory");
+}
+
+// Two threads per token. Pass 1: the two warps that may read a TMEM lane quarter
+// take alternate 32-column chunks of their 32 tokens: logits (+ biases in the
+// CUDA-core router's order) are written out and z (NaN -> -inf) parked in the
+// token's row of the shared-memory tile. Then thread (token r, half h) owns row r,
+// columns [h*E0, min(E, (h+1)*E0)): the max, k argmax rounds (each the best entry
+// ranked below the previous pick: value, then lower index) and sum exp(z - max) are
+// taken over each half and merged through shared memory in a fixed order.
 template <int EPAD>
 __device__ __forceinline__ void epilogue_rows(const RouterArgs &a, RtCtl *ctl, float *prob,
                                               uint32_t tmem, int t0, int NT, int BM, int warp,
                                               int lane) {
   constexpr int LDL = RtCfg<EPAD>::kLdl;
   const int E = a.E, T = a.T, k = a.k;
-  const int ew = warp & 3;           // TMEM lanes [32 ew, 32 ew + 32) (warp % 4)
-  const int r = ew * 32 + lane;      // token row within the tile
-  const int et = (warp - 2) * 32 + lane;  // 0..127 over the epilogue threads
+  const int et = (warp - 2) * 32 + lane;  // 0..255 over the epilogue threads
+  // one thread waits; the named barrier is reached by all epilogue threads
+  if (et == 0) ctl->epi_ok = rt_wait(&ctl->tfull, 0, ctl, a.err, 13) ? 1 : 0;
+  rt_epi_sync();
+  if (!ctl->epi_ok) return;
+  tc_fence_after();
+
+  {  // ---- pass 1: TMEM -> logits out, z into the row
+    const int ew = warp & 3;                // TMEM lanes [32 ew, 32 ew + 32) (warp % 4)
+    const int c_first = (warp - 2) >> 2;    // this warp's chunks: c_first, c_first + 2, ...
+    const int r = ew * 32 + lane;
+    const int t = t0 + r;
+    const bool valid = t < T;
+    float *row = prob + r * LDL;
+    const uint32_t tb = tmem + ((uint32_t)(ew * 32) << 16);
+    const bool vec_out = valid && a.logits_out != nullptr && (E & 3) == 0;
+#pragma unroll 1
+    for (int c = c_first; c < EPAD / 32; c += 2) {
+      uint32_t v[32];
+      tmem_ld32(tb + c * 32, v);
+      tmem_ld_wait();
+      float lo[32];
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        const int e = c * 32 + j;
+        float val = __uint_as_float(v[j]);
+        if (a.b_router) val += ctl->br[e];
+        if (a.logit_bias) val += ctl->lb[e];
+        lo[j] = val;
+        if (e < E) row[e] = (val != val) ? -INFINITY : val;  // a NaN logit never wins a slot
+      }
+      const int n_out = min(32, E - c * 32);
+      if (vec_out && n_out == 32) {
+        float4 *dst = reinterpret_cast<float4 *>(a.logits_out + (size_t)t * E + c * 32);
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+          dst[q] = make_float4(lo[4 * q], lo[4 * q + 1], lo[4 * q + 2], lo[4 * q + 3]);
+      } else if (valid && a.logits_out != nullptr) {
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+          if (j < n_out) a.logits_out[(size_t)t * E + c * 32 + j] = lo[j];
+      }
+    }
+  }
+  rt_epi_sync();
+
+  // ---- the rest: thread (token r, half h); a warp holds 32 consecutive tokens
+  const int r = et & (kRtM - 1), h = et / kRtM;
   const int t = t0 + r;
   const bool valid = t < T;
   float *row = prob + r * LDL;
-  // one thread waits; the named barrier below is reached by all 128 threads
-  if (et == 0) ctl->epi_ok = rt_wait(&ctl->tfull, 0, ctl, a.err, 13) ? 1 : 0;
-  asm volatile("bar.sync 1, 128;" ::: "memory");
-  if (!ctl->epi_ok) return;
-  tc_fence_after();
-  const uint32_t tb = tmem + ((uint32_t)(ew * 32) << 16);
+  const int E0 = (E + 1) >> 1;
+  const int e_lo = h * E0, e_hi = min(E, e_lo + E0);
 
   float mx = -INFINITY;
-  const bool vec_out = valid && a.logits_out != nullptr && (E & 3) == 0;
-#pragma unroll 1
-  for (int c = 0; c < EPAD / 32; ++c) {
-    uint32_t v[32];
-    tmem_ld32(tb + c * 32, v);
-    tmem_ld_wait();
-    float lo[32];
-#pragma unroll
-    for (int j = 0; j < 32; ++j) {
-      const int e = c * 32 + j;
-      float val = __uint_as_float(v[j]);
-      if (a.b_router) val += ctl->br[e];
-      if (a.logit_bias) val += ctl->lb[e];
-      lo[j] = val;
-      const float z = (val != val) ? -INFINITY : val;  // a NaN logit never wins a slot
-      if (e < E) {
-        mx = fmaxf(mx, z);
-        row[e] = z;
-      }
-    }
-    const int n_out = min(32, E - c * 32);
-    if (vec_out && n_out == 32) {
-      float4 *dst = reinterpret_cast<float4 *>(a.logits_out + (size_t)t * E + c * 32);
-#pragma unroll
-      for (int q = 0; q < 8; ++q)
-        dst[q] = make_float4(lo[4 * q], lo[4 * q + 1], lo[4 * q + 2], lo[4 * q + 3]);
-    } else if (valid && a.logits_out != nullptr) {
-#pragma unroll
-      for (int j = 0; j < 32; ++j)
-        if (j < n_out) a.logits_out[(size_t)t * E + c * 32 + j] = lo[j];
-    }
-  }
+  for (int e = e_lo; e < e_hi; ++e) mx = fmaxf(mx, row[e]);
+  ctl->hmax[h][r] = mx;
+  rt_epi_sync();
+  mx = fmaxf(ctl->hmax[0][r], ctl->hmax[1][r]);
 
-  // top-k as k argmax rounds over the row, each taking the best entry ranked below
-  // the previous pick (value descending, ties to the lower index): no marks, no
-  // divergence; four interleaved partial argmaxes per round for ILP
   float tv[kMaxTopK];
   int ti[kMaxTopK];
   float pv = INFINITY;
@@ -146,9 +169,9 @@ __device__ __forceinline__ void epilogue_rows(const RouterArgs &a, RtCtl *ctl, f
     if (s < k) {
       float bv[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
       int bi[4] = {0x7fffffff, 0x7fffffff, 0x7fffffff, 0x7fffffff};
-      int e = 0;
+      int e = e_lo;
 #pragma unroll 2
-      for (; e + 4 <= E; e += 4) {
+      for (; e + 4 <= e_hi; e += 4) {
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           const float z = row[e + q];
@@ -156,7 +179,7 @@ __device__ __forceinline__ void epilogue_rows(const RouterArgs &a, RtCtl *ctl, f
           if (below && rt_better(z, e + q, bv[q], bi[q])) { bv[q] = z; bi[q] = e + q; }
         }
       }
-      for (; e < E; ++e) {
+      for (; e < e_hi; ++e) {
         const float z = row[e];
         const bool below = z < pv || (z == pv && e > pi);
         if (below && rt_better(z, e, bv[0], bi[0])) { bv[0] = z; bi[0] = e; }
@@ -164,57 +187,68 @@ __device__ __forceinline__ void epilogue_rows(const RouterArgs &a, RtCtl *ctl, f
 #pragma unroll
       for (int q = 1; q < 4; ++q)
         if (rt_better(bv[q], bi[q], bv[0], bi[0])) { bv[0] = bv[q]; bi[0] = bi[q]; }
-      tv[s] = pv = bv[0];
-      ti[s] = pi = bi[0];
+      ctl->cand_v[s & 1][h][r] = bv[0];
+      ctl->cand_i[s & 1][h][r] = bi[0];
+      rt_epi_sync();
+      float b0 = ctl->cand_v[s & 1][0][r], b1 = ctl->cand_v[s & 1][1][r];
+      int i0 = ctl->cand_i[s & 1][0][r], i1 = ctl->cand_i[s & 1][1][r];
+      if (rt_better(b1, i1, b0, i0)) { b0 = b1; i0 = i1; }
+      tv[s] = pv = b0;
+      ti[s] = pi = i0;
     }
   }
 
   float ssum = 0.f;
 #pragma unroll 4
-  for (int e = 0; e < E; ++e) {
+  for (int e = e_lo; e < e_hi; ++e) {
     const float ex = expf(row[e] - mx);
     ssum += ex;
     row[e] = ex;
   }
+  ctl->hsum[h][r] = ssum;
+  rt_epi_sync();
+  ssum = ctl->hsum[0][r] + ctl->hsum[1][r];
   const float inv_s = 1.f / ssum;
-  ctl->lse[r] = mx + logf(ssum);
   if (a.tile_p != nullptr)
-    for (int e = 0; e < E; ++e) row[e] *= inv_s;
+    for (int e = e_lo; e < e_hi; ++e) row[e] *= inv_s;
 
-  float g[kMaxTopK];
-  float gs = 0.f;
-  if (a.gate_mode == MOE_GATE_TOPK_SOFTMAX) {
+  if (h == 0) {
+    ctl->lse[r] = mx + logf(ssum);
+    float g[kMaxTopK];
+    float gs = 0.f;
+    if (a.gate_mode == MOE_GATE_TOPK_SOFTMAX) {
 #pragma unroll
-    for (int s = 0; s < kMaxTopK; ++s)
-      if (s < k) { g[s] = expf(tv[s] - tv[0]); gs += g[s]; }
-    const float inv = 1.f / gs;
+      for (int s = 0; s < kMaxTopK; ++s)
+        if (s < k) { g[s] = expf(tv[s] - tv[0]); gs += g[s]; }
+      const float inv = 1.f / gs;
 #pragma unroll
-    for (int s = 0; s < kMaxTopK; ++s) if (s < k) g[s] *= inv;
-  } else {
+      for (int s = 0; s < kMaxTopK; ++s) if (s < k) g[s] *= inv;
+    } else {
 #pragma unroll
-    for (int s = 0; s < kMaxTopK; ++s)
-      if (s < k) { g[s] = expf(tv[s] - mx) * inv_s; gs += g[s]; }
-    if (a.gate_mode == MOE_GATE_SOFTMAX_TOPK_RENORM) {
+      for (int s = 0; s < kMaxTopK; ++s)
+        if (s < k) { g[s] = expf(tv[s] - mx) * inv_s; gs += g[s]; }
+      if (a.gate_mode == MOE_GATE_SOFTMAX_TOPK_RENORM) {
 #pragma unroll
-      for (int s = 0; s < kMaxTopK; ++s) if (s < k) g[s] = g[s] / gs;
+        for (int s = 0; s < kMaxTopK; ++s) if (s < k) g[s] = g[s] / gs;
+      }
     }
-  }
-  if (valid) {
+    if (valid) {
 #pragma unroll
-    for (int s = 0; s < kMaxTopK; ++s) {
-      if (s < k) {
-        a.topk_idx[(size_t)t * k + s] = ti[s];
-        a.topk_gate[(size_t)t * k + s] = g[s];
-        if (ti[s] < E) atomicAdd(&ctl->cnt[r / BM][ti[s]], 1);
+      for (int s = 0; s < kMaxTopK; ++s) {
+        if (s < k) {
+          a.topk_idx[(size_t)t * k + s] = ti[s];
+          a.topk_gate[(size_t)t * k + s] = g[s];
+          if (ti[s] < E) atomicAdd(&ctl->cnt[r / BM][ti[s]], 1);
+        }
       }
     }
   }
-  asm volatile("bar.sync 1, 128;" ::: "memory");
+  rt_epi_sync();
 
   // per permute tile (BM tokens): histogram, probability sums, sum of lse^2,
   // each in token order
   const int subs = kRtM / BM;
-  for (int i = et; i < subs * E; i += 128) {
+  for (int i = et; i < subs * E; i += kRtEpiThreads) {
     const int sub = i / E, e = i - sub * E;
     const int tile = blockIdx.x * subs + sub;
     if (tile >= NT) continue;
