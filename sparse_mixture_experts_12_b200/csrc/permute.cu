@@ -209,8 +209,13 @@ __global__ void __launch_bounds__(kScatterThreads) k_scatter(ScatterArgs a) {
   char *xp = static_cast<char *>(a.x_perm);
   for (int m = warp; m < rows; m += kScatterThreads / 32) {
     int dst[kMaxTopK];
+    bool any = false;
 #pragma unroll
-    for (int s = 0; s < kMaxTopK; ++s) dst[s] = (s < k) ? prow[m * k + s] : -1;
+    for (int s = 0; s < kMaxTopK; ++s) {
+      dst[s] = (s < k) ? prow[m * k + s] : -1;
+      any |= dst[s] >= 0;
+    }
+    if (!any) continue;  // every slot dropped: the row is not read at all
     const uint4 *src = reinterpret_cast<const uint4 *>(xb + (size_t)(t0 + m) * row_bytes);
     for (int v0 = lane; v0 < nvec; v0 += 32 * 4) {
       uint4 u[4];
@@ -234,17 +239,20 @@ __global__ void __launch_bounds__(kScatterThreads) k_scatter(ScatterArgs a) {
 }
 
 // ------------------------------------------------------------------- combine
-template <typename T>
+// A warp per token. Each lane takes NB 16-byte vectors of the row per batch and
+// requests every kept slot's vectors (and the shared-expert row) before using
+// any, so a warp keeps NB x k loads in flight; KMAX bounds k (register budget).
+template <typename T, int KMAX, int NB>
 __global__ void __launch_bounds__(256) k_combine(CombineArgs a) {
   constexpr int VE = Elem<T>::kPerVec;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t = blockIdx.x * 8 + warp;
   if (t >= a.T) return;
   const int k = a.k;
-  int row[kMaxTopK];
-  float g[kMaxTopK];
+  int row[KMAX];
+  float g[KMAX];
 #pragma unroll
-  for (int s = 0; s < kMaxTopK; ++s) {
+  for (int s = 0; s < KMAX; ++s) {
     row[s] = -1;
     g[s] = 0.f;
     if (s < k) {
@@ -260,34 +268,53 @@ __global__ void __launch_bounds__(256) k_combine(CombineArgs a) {
   const T *yp = static_cast<const T *>(a.y_perm);
   T *y = static_cast<T *>(a.y);
   const int nvec = a.d / VE;
-  for (int v = lane; v < nvec; v += 32) {
-    // every slot's row is requested before any is used (a dropped slot reads nothing
-    // and contributes zero)
-    uint4 u[kMaxTopK];
+  for (int v0 = lane; v0 < nvec; v0 += 32 * NB) {
+    // a dropped slot reads nothing and contributes zero
+    uint4 u[KMAX][NB];
 #pragma unroll
-    for (int s = 0; s < kMaxTopK; ++s)
-      u[s] = (row[s] >= 0) ? __ldg(reinterpret_cast<const uint4 *>(yp + (size_t)row[s] * a.d) + v)
-                           : make_uint4(0u, 0u, 0u, 0u);
-    float acc[VE];
+    for (int s = 0; s < KMAX; ++s)
 #pragma unroll
-    for (int i = 0; i < VE; ++i) acc[i] = 0.f;
-#pragma unroll
-    for (int s = 0; s < kMaxTopK; ++s) {
-      if (s >= k) break;
-      float f[VE];
-      unpack16(u[s], f);
-#pragma unroll
-      for (int i = 0; i < VE; ++i) acc[i] = fmaf(g[s], f[i], acc[i]);
-    }
+      for (int b = 0; b < NB; ++b) {
+        const int v = v0 + 32 * b;
+        u[s][b] = (row[s] >= 0 && v < nvec)
+                      ? __ldg(reinterpret_cast<const uint4 *>(yp + (size_t)row[s] * a.d) + v)
+                      : make_uint4(0u, 0u, 0u, 0u);
+      }
+    float4 sh[NB][VE / 4];
     if (a.shared_y) {
-      const float4 *sp = reinterpret_cast<const float4 *>(a.shared_y + (size_t)t * a.d + v * VE);
 #pragma unroll
-      for (int i = 0; i < VE; i += 4) {
-        const float4 q = __ldg(sp + i / 4);
-        acc[i] += q.x; acc[i + 1] += q.y; acc[i + 2] += q.z; acc[i + 3] += q.w;
+      for (int b = 0; b < NB; ++b) {
+        const int v = v0 + 32 * b;
+        const float4 *sp = reinterpret_cast<const float4 *>(a.shared_y + (size_t)t * a.d + v * VE);
+#pragma unroll
+        for (int i = 0; i < VE / 4; ++i)
+          sh[b][i] = (v < nvec) ? __ldg(sp + i) : make_float4(0.f, 0.f, 0.f, 0.f);
       }
     }
-    reinterpret_cast<uint4 *>(y + (size_t)t * a.d)[v] = pack16(acc);
+#pragma unroll
+    for (int b = 0; b < NB; ++b) {
+      const int v = v0 + 32 * b;
+      if (v >= nvec) break;
+      float acc[VE];
+#pragma unroll
+      for (int i = 0; i < VE; ++i) acc[i] = 0.f;
+#pragma unroll
+      for (int s = 0; s < KMAX; ++s) {
+        if (s >= k) break;
+        float f[VE];
+        unpack16(u[s][b], f);
+#pragma unroll
+        for (int i = 0; i < VE; ++i) acc[i] = fmaf(g[s], f[i], acc[i]);
+      }
+      if (a.shared_y) {
+#pragma unroll
+        for (int i = 0; i < VE; i += 4) {
+          const float4 q = sh[b][i / 4];
+          acc[i] += q.x; acc[i + 1] += q.y; acc[i + 2] += q.z; acc[i + 3] += q.w;
+        }
+      }
+      reinterpret_cast<uint4 *>(y + (size_t)t * a.d)[v] = pack16(acc);
+    }
   }
 }
 
@@ -344,10 +371,14 @@ cudaError_t launch_scatter(const ScatterArgs &a, cudaStream_t st) {
 cudaError_t launch_combine(const CombineArgs &a, int dtype, cudaStream_t st) {
   if (a.T == 0) return cudaSuccess;
   const int grid = ceil_div(a.T, 8);
-  if (dtype == MOE_DTYPE_F32)
-    k_combine<float><<<grid, 256, 0, st>>>(a);
-  else
-    k_combine<__nv_bfloat16><<<grid, 256, 0, st>>>(a);
+  const bool f32 = dtype == MOE_DTYPE_F32;
+  if (a.k <= 2) {
+    if (f32) k_combine<float, 2, 4><<<grid, 256, 0, st>>>(a);
+    else k_combine<__nv_bfloat16, 2, 4><<<grid, 256, 0, st>>>(a);
+  } else {
+    if (f32) k_combine<float, kMaxTopK, 1><<<grid, 256, 0, st>>>(a);
+    else k_combine<__nv_bfloat16, kMaxTopK, 1><<<grid, 256, 0, st>>>(a);
+  }
   return cudaGetLastError();
 }
 
