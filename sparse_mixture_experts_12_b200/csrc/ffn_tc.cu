@@ -64,7 +64,43 @@ struct TcArgs {
   int act;
   int32_t *err;
   int tile_mode;  // TILES_ALL, or the pair / tail halves of a split launch
+  int tma_store;  // pair kernel, bf16 output: full 32-row groups leave through TMA stores
 };
+
+// The output path of one epilogue warp for one tile. With a map, a chunk whose 32
+// rows are all the expert's is staged in the warp's 2 KB shared-memory buffer (64-
+// byte swizzle) and written by one TMA store; other chunks use masked direct stores.
+struct EpiStore {
+  const CUtensorMap *map;  // 32 x 32 bf16 output boxes, or nullptr
+  uint8_t *stage;          // this warp's staging buffer
+  bool rows_full;          // all 32 rows of the warp belong to the expert
+  int row0;                // output row of lane 0
+};
+constexpr int kStageOutBytes = kStoreBox * kStoreBox * 2;  // 2 KB per epilogue warp
+
+// one 32-row x 32-column bf16 chunk (pk = this lane's row) to global memory
+__device__ __forceinline__ void emit_chunk(const EpiStore &st, const uint4 (&pk)[4],
+                                           __nv_bfloat16 *dst_row, int col0) {
+  if (st.map != nullptr && st.rows_full) {
+    const int lane = threadIdx.x & 31;
+    if (lane == 0) bulk_wait_read_all();  // the previous store has read the buffer
+    __syncwarp();
+    uint4 *row = reinterpret_cast<uint4 *>(st.stage + lane * 64);
+    const int sw = (lane >> 1) & 3;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) row[q ^ sw] = pk[q];
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+      tma_store_2d(st.map, st.stage, col0, st.row0);
+      bulk_commit();
+    }
+  } else {
+    uint4 *dst = reinterpret_cast<uint4 *>(dst_row + col0);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) dst[q] = pk[q];
+  }
+}
 
 // Row tiles of an expert with c rows: mt = ceil(c / 128). A split launch gives the
 // CTA-pair kernel the floor(mt / 2) full pair tiles and, when mt is odd (the last
@@ -102,7 +138,7 @@ __device__ __forceinline__ bool wait_bounded(uint64_t *bar, uint32_t parity, Sme
 template <int EPI>
 __device__ __forceinline__ void epilogue_tile(const TcArgs &a, uint32_t tbase, int g, int acc_off,
                                               int out_base, int c0, int c1, bool valid,
-                                              size_t orow) {
+                                              size_t orow, const EpiStore &st) {
   if (EPI == EPI_SWIGLU) {
     __nv_bfloat16 *out = static_cast<__nv_bfloat16 *>(a.out);
 #pragma unroll 1
@@ -112,8 +148,8 @@ __device__ __forceinline__ void epilogue_tile(const TcArgs &a, uint32_t tbase, i
       tmem_ld32(tbase + acc_off + kMmaN / 2 + c * 32, uv);
       tmem_ld_wait();
       const int col0 = out_base + c * 32;
-      if (valid && col0 < a.N) {
-        uint4 *dst = reinterpret_cast<uint4 *>(out + orow * a.N + col0);
+      if (valid && col0 < a.N) {  // rows_full implies valid on every lane
+        uint4 pk[4];
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           float h[8];
@@ -123,8 +159,9 @@ __device__ __forceinline__ void epilogue_tile(const TcArgs &a, uint32_t tbase, i
             const float up = __uint_as_float(uv[q * 8 + j]);
             h[j] = __fdividef(gt, 1.f + __expf(-gt)) * up;
           }
-          dst[q] = pack16(h);
+          pk[q] = pack16(h);
         }
+        emit_chunk(st, pk, out + orow * a.N, col0);
       }
     }
   } else {
@@ -162,15 +199,15 @@ __device__ __forceinline__ void epilogue_tile(const TcArgs &a, uint32_t tbase, i
           for (int q = 0; q < 8; ++q)
             dst[q] = make_float4(f[4 * q], f[4 * q + 1], f[4 * q + 2], f[4 * q + 3]);
         } else {
-          uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(a.out) +
-                                                 orow * a.N + col0);
+          uint4 pk[4];
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
             float h[8];
 #pragma unroll
             for (int j = 0; j < 8; ++j) h[j] = f[q * 8 + j];
-            dst[q] = pack16(h);
+            pk[q] = pack16(h);
           }
+          emit_chunk(st, pk, static_cast<__nv_bfloat16 *>(a.out) + orow * a.N, col0);
         }
       }
     }
@@ -325,10 +362,12 @@ k_ffn_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtens
       const size_t orow = (size_t)offs[g] + grow;
       const uint32_t tbase = tmem + ((uint32_t)(ew * 32) << 16) + (uint32_t)(acc * kMmaN);
       // the two warps sharing a TMEM lane quarter take half the columns each
+      const EpiStore st{nullptr, nullptr, false, 0};
       if (EPI == EPI_SWIGLU)
-        epilogue_tile<EPI>(a, tbase, g, 0, n * (kMmaN / 2), 2 * half, 2 * half + 2, valid, orow);
+        epilogue_tile<EPI>(a, tbase, g, 0, n * (kMmaN / 2), 2 * half, 2 * half + 2, valid, orow,
+                           st);
       else
-        epilogue_tile<EPI>(a, tbase, g, 0, n * kMmaN, 4 * half, 4 * half + 4, valid, orow);
+        epilogue_tile<EPI>(a, tbase, g, 0, n * kMmaN, 4 * half, 4 * half + 4, valid, orow, st);
       tc_fence_before();
       mbar_arrive(&ctl->tempty[acc]);
       if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
@@ -380,7 +419,9 @@ struct SmemCtl2 {
 };
 
 template <int NH>
-constexpr size_t pair_smem_bytes() { return PairCfg<NH>::kRing + sizeof(SmemCtl2) + 1024; }
+constexpr size_t pair_smem_bytes() {
+  return PairCfg<NH>::kRing + (size_t)kEpiWarps * kStageOutBytes + sizeof(SmemCtl2) + 1024;
+}
 
 // Work items of the persistent pair kernel. With NH = 2, when the last round of
 // tiles would leave at least half of the CTA pairs idle (r = total % pairs tiles,
@@ -417,14 +458,16 @@ __device__ __forceinline__ bool wait_pair(uint64_t *bar, uint32_t parity, SmemCt
 template <int EPI, int NH>
 __global__ void __launch_bounds__(kThreads, 1)
 k_ffn_tc2(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-          const __grid_constant__ CUtensorMap tmB3, TcArgs a) {
+          const __grid_constant__ CUtensorMap tmB3, const __grid_constant__ CUtensorMap tmO,
+          TcArgs a) {
   using PC = PairCfg<NH>;
   constexpr int kS = PC::kStages;
   constexpr int kSB = PC::kStageBytes;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  SmemCtl2 *ctl = reinterpret_cast<SmemCtl2 *>(smem + PC::kRing);
+  // ring | 8 x 2 KB output staging (TMA stores) | control block
+  SmemCtl2 *ctl = reinterpret_cast<SmemCtl2 *>(smem + PC::kRing + kEpiWarps * kStageOutBytes);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const uint32_t rank = cluster_ctarank();
   const bool leader = rank == 0;
@@ -576,6 +619,7 @@ k_ffn_tc2(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
     const int ew = warp & 3;
     const int half = (warp - 4) >> 2;
     const uint32_t tempty0 = mapa_rank(smem_u32(&ctl->tempty[0]), 0);
+    uint8_t *stage_out = smem + PC::kRing + (warp - 4) * kStageOutBytes;
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int it = c0; it < work.items; it += cstep) {
@@ -589,23 +633,29 @@ k_ffn_tc2(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
       const bool valid = grow < offs[g + 1] - offs[g];
       const size_t orow = (size_t)offs[g] + grow;
       const uint32_t tbase = tmem + ((uint32_t)(ew * 32) << 16) + (uint32_t)(acc * kMmaN);
+      const bool rows_full = __all_sync(0xffffffffu, valid);
+      const EpiStore st{a.tma_store ? &tmO : nullptr, stage_out, rows_full,
+                        (int)(orow - (size_t)lane)};
       if (NH == 1) {  // the two warps sharing a lane quarter take half the columns each
         if (EPI == EPI_SWIGLU)
-          epilogue_tile<EPI>(a, tbase, g, 0, n * (kMmaN / 2), 2 * half, 2 * half + 2, valid, orow);
+          epilogue_tile<EPI>(a, tbase, g, 0, n * (kMmaN / 2), 2 * half, 2 * half + 2, valid, orow,
+                             st);
         else
-          epilogue_tile<EPI>(a, tbase, g, 0, n * kMmaN, 4 * half, 4 * half + 4, valid, orow);
+          epilogue_tile<EPI>(a, tbase, g, 0, n * kMmaN, 4 * half, 4 * half + 4, valid, orow, st);
       } else if (sel < 0 || sel == half) {  // ... or one N half (256 columns) each
         if (EPI == EPI_SWIGLU)
           epilogue_tile<EPI>(a, tbase, g, half * kMmaN, n * kMmaN + half * (kMmaN / 2), 0, 4,
-                             valid, orow);
+                             valid, orow, st);
         else
           epilogue_tile<EPI>(a, tbase, g, half * kMmaN, (2 * n + half) * kMmaN, 0, 8, valid,
-                             orow);
+                             orow, st);
       }
       tc_fence_before();
       mbar_arrive_cluster(tempty0 + (uint32_t)(acc * sizeof(uint64_t)));
       if (++acc == PC::kAccBufs) { acc = 0; acc_phase ^= 1u; }
     }
+    if (a.tma_store && lane == 0) bulk_wait_all();  // this warp's output stores are done
+    __syncwarp();
   }
   if (*(volatile int *)&ctl->abort_flag) settle_ns(100000);  // copies in flight land
   tc_fence_before();
@@ -671,7 +721,8 @@ cudaError_t launch_single(const CUtensorMap &ma, const CUtensorMap &mb, const CU
 
 template <int EPI, int NH>
 cudaError_t launch_pair(const CUtensorMap &ma, const CUtensorMap &mb, const CUtensorMap &mb3,
-                        const TcArgs &t, long long tiles_ub, cudaStream_t st) {
+                        const CUtensorMap &mo, const TcArgs &t, long long tiles_ub,
+                        cudaStream_t st) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
@@ -705,7 +756,7 @@ cudaError_t launch_pair(const CUtensorMap &ma, const CUtensorMap &mb, const CUte
   }
   const long long pairs = std::min<long long>(tiles_ub, info.max_pairs[slot]);
   cfg.gridDim = dim3((unsigned)(2 * pairs));
-  e = cudaLaunchKernelEx(&cfg, k_ffn_tc2<EPI, NH>, ma, mb, mb3, t);
+  e = cudaLaunchKernelEx(&cfg, k_ffn_tc2<EPI, NH>, ma, mb, mb3, mo, t);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
@@ -741,24 +792,27 @@ inline bool uses_pairs(bool wide) { return kUsePairs || wide; }
 // it is used below 1024 rows per expert on average.
 inline bool split_tails(long long rows, int groups) { return rows < 4LL * kPairM * groups; }
 
+// mo: the output map for the pair kernel's TMA stores (used when t.tma_store).
 template <int EPI>
 cudaError_t launch_gemm(const CUtensorMap &ma, const CUtensorMap &mb, const CUtensorMap &mb3,
-                        const CUtensorMap &mb1, const CUtensorMap &mb31, TcArgs t, int m_tiles_ub,
-                        int groups, int n_cols, bool wide, bool split, cudaStream_t st) {
+                        const CUtensorMap &mb1, const CUtensorMap &mb31, const CUtensorMap &mo,
+                        TcArgs t, int m_tiles_ub, int groups, int n_cols, bool wide, bool split,
+                        cudaStream_t st) {
   // output columns per 256 accumulator columns
   const int per_n = (EPI == EPI_SWIGLU) ? kMmaN / 2 : kMmaN;
   const long long pair_m_ub = (long long)(m_tiles_ub + groups + 1) / 2;
   if (kUsePairs) {
     t.n_tiles = ceil_div(n_cols, per_n);
     t.tile_mode = TILES_ALL;
-    return launch_pair<EPI, 1>(ma, mb, mb3, t, std::max<long long>(pair_m_ub * t.n_tiles, 1), st);
+    return launch_pair<EPI, 1>(ma, mb, mb3, mo, t,
+                               std::max<long long>(pair_m_ub * t.n_tiles, 1), st);
   }
   if (wide) {
     // full pair tiles on the wide kernel; with split, the odd last 128-row tiles
     // on the single-CTA kernel, which fills the SMs the pair grid's last round leaves
     t.n_tiles = ceil_div(n_cols, 2 * per_n);
     t.tile_mode = split ? TILES_PAIRS_NO_TAIL : TILES_ALL;
-    cudaError_t e = launch_pair<EPI, 2>(ma, mb, mb3, t,
+    cudaError_t e = launch_pair<EPI, 2>(ma, mb, mb3, mo, t,
                                         std::max<long long>(pair_m_ub * t.n_tiles, 1), st);
     if (e != cudaSuccess || !split) return e;
     t.n_tiles = ceil_div(n_cols, per_n);
@@ -813,11 +867,15 @@ cudaError_t launch_ffn_tc(const GroupedFfnArgs &a, cudaStream_t st) {
   t.bias = a.b1;
   t.act = a.act;
   t.err = a.err;
+  // pair tiles write bf16 outputs through TMA stores of 32 x 32 boxes
+  CUtensorMap mo;
+  if (!make_store_map(&mo, a.h, (uint64_t)a.a_rows, (uint64_t)a.F)) return cudaErrorInvalidValue;
+  t.tma_store = 1;
   cudaError_t e =
-      swiglu ? launch_gemm<EPI_SWIGLU>(ma, mb, mb3, mbs, mb3s, t, a.m_tiles_ub, a.G, a.F, wide_up,
-                                       split, st)
-             : launch_gemm<EPI_ACT>(ma, mb, mb3, mbs, mb3s, t, a.m_tiles_ub, a.G, a.F, wide_up,
-                                    split, st);
+      swiglu ? launch_gemm<EPI_SWIGLU>(ma, mb, mb3, mbs, mb3s, mo, t, a.m_tiles_ub, a.G, a.F,
+                                       wide_up, split, st)
+             : launch_gemm<EPI_ACT>(ma, mb, mb3, mbs, mb3s, mo, t, a.m_tiles_ub, a.G, a.F,
+                                    wide_up, split, st);
   if (e != cudaSuccess) return e;
   // down projection: h [rows, F] x [G*d, F]^T -> out [rows, d]
   if (!make_map(&ma, a.h, (uint64_t)a.a_rows, (uint64_t)a.F, kTileM)) return cudaErrorInvalidValue;
@@ -836,8 +894,11 @@ cudaError_t launch_ffn_tc(const GroupedFfnArgs &a, cudaStream_t st) {
   t.out_f32 = a.out_f32;
   t.bias = a.b2;
   t.act = -1;
-  return launch_gemm<EPI_DOWN>(ma, mb, mb, mbs, mbs, t, a.m_tiles_ub, a.G, a.d, wide_down, split,
-                               st);
+  t.tma_store = a.out_f32 ? 0 : 1;
+  if (!a.out_f32 && !make_store_map(&mo, a.out, (uint64_t)a.a_rows, (uint64_t)a.d))
+    return cudaErrorInvalidValue;
+  return launch_gemm<EPI_DOWN>(ma, mb, mb, mbs, mbs, mo, t, a.m_tiles_ub, a.G, a.d, wide_down,
+                               split, st);
 }
 
 }  // namespace moe
