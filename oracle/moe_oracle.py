@@ -19,10 +19,11 @@ Pages cited (by title and the listing or section that defines each step):
 * P3 — youngju.dev, "Mixture of Experts（MoE）架构深度解析：从 Switch Transformer 到
   Mixtral 的演进与高效扩展策略": ``GatingNetwork``, ``MoELayer`` (GELU),
   ``SwitchRouter``, ``load_balancing_loss``, ``MixtralMoELayer``, ``SwiGLUExpert``,
-  ``DeepSeekMoELayer``.
+  ``DeepSeekMoELayer``, ``ExpertChoiceRouter``.
 * P4 — youngju.dev, "Sparse Mixture of Experts（MoE）アーキテクチャ深層分析：設計原理
   からDeepSeek-V3・Qwen3まで": the gating equation, ``SwiGLUExpert``, ``TopKGating``,
-  ``compute_load_balancing_loss``, ``MoELayerWithAuxLoss``, ``router_z_loss``.
+  ``ExpertChoiceGating``, ``compute_load_balancing_loss``, ``MoELayerWithAuxLoss``,
+  ``router_z_loss``.
 * P5 — study-site lecture 03, "Mixture of Experts": "Token Routing" (gates 0.7/0.3,
   unselected experts are not computed), "SiLU · SwiGLU · MoE" table.
 
@@ -39,6 +40,10 @@ test):
 * f_i counts pre-drop assignments over T*k; P_i is the mean full softmax of the
   router logits (router bias and logit bias included).
 * GELU is the exact erf form; dropout and routing noise are off (inference).
+* Expert-Choice routing: each expert takes int(cf * T / E) tokens, chosen on the
+  fp32 logits (equal logits: lower token index first); a token's output is the
+  score-weighted sum over the experts that took it (P4's dispatch mask used as
+  the gate), 0 if none did.
 * No intermediate rounding: everything after the fp32 logits is fp64.
 
 Parity status: every function below is pinned by the CPU test suite; none is
@@ -362,3 +367,86 @@ def balance_sq_loss(idx, E: int) -> float:
         counts[int(e)] += 1
     share = counts / counts.sum()
     return float(((share - 1.0 / E) ** 2).sum())
+
+
+# ------------------------------------------------------------ Expert-Choice routing
+def expert_choice_capacity(capacity_factor: float, T: int, E: int) -> int:
+    """Tokens each expert takes: int(cf * N / E) with N = all tokens of the call
+    (P3 ``ExpertChoiceRouter``, P4 ``ExpertChoiceGating``: ``expert_capacity``)."""
+    return int(math.floor(float(capacity_factor) * T / E))
+
+
+def expert_choice_scores(logits32) -> np.ndarray:
+    """Scores [E, T]: for every expert, the softmax of its logits over the tokens
+    (P3: ``F.softmax(logits, dim=0)``; P4: ``F.softmax(gate_logits.T, dim=-1)``), fp64."""
+    z = _f64(logits32).T
+    m = z.max(axis=1, keepdims=True)
+    e = np.exp(z - m)
+    return e / e.sum(axis=1, keepdims=True)
+
+
+def expert_choice_select(logits32, C: int) -> np.ndarray:
+    """Token indices [E, C] each expert takes: its C highest-scoring tokens, in
+    descending score (``torch.topk(scores, C, dim=-1)``).
+
+    The per-expert softmax over tokens is monotone in the logit, so the choice is
+    made on the fp32 logits; equal logits go to the lower token index first.
+    """
+    z = np.asarray(logits32, dtype=np.float32)
+    T, E = z.shape
+    out = np.zeros((E, C), dtype=np.int32)
+    for e in range(E):
+        order = np.argsort(-z[:, e].astype(np.float64), kind="stable")
+        out[e] = order[:C]
+    return out
+
+
+def expert_choice_forward(x, params: dict, *, capacity_factor: float, act: str,
+                          logits=None, tokens: Optional[Sequence[int]] = None):
+    """Expert-Choice layer output y[t] = sum over experts e that took t of
+    score[e, t] * E_e(x_t): the dispatch mask of P4 ``ExpertChoiceGating``
+    (``dispatch_mask.scatter_(1, top_k_indices, top_k_scores)``) applied as the
+    gate of each expert's output. A token no expert took gets 0.
+
+    Returns (y [len(tokens) or T, d] fp64, dict(logits, C, idx [E, C], scores [E, C])).
+    """
+    x = _f64(x)
+    if logits is None:
+        logits = router_logits(x, params["w_router"], params.get("b_router"),
+                               params.get("logit_bias"))
+    logits = np.asarray(logits, dtype=np.float32)
+    T, E = logits.shape
+    C = expert_choice_capacity(capacity_factor, T, E)
+    idx = expert_choice_select(logits, C)
+    S = expert_choice_scores(logits)
+    scores = np.take_along_axis(S, idx.astype(np.int64), axis=1)
+    sel = np.arange(T) if tokens is None else np.asarray(tokens, dtype=np.int64)
+    pos = np.full(T, -1, dtype=np.int64)
+    pos[sel] = np.arange(len(sel))
+    y = np.zeros((len(sel), x.shape[1]), dtype=np.float64)
+    for e in range(E):
+        toks = idx[e].astype(np.int64)
+        keep = pos[toks] >= 0
+        if not keep.any():
+            continue
+        w3 = params["w3"][e] if params.get("w3") is not None else None
+        b1 = params["b1"][e] if params.get("b1") is not None else None
+        b2 = params["b2"][e] if params.get("b2") is not None else None
+        out = expert_ffn(x[toks[keep]], act, params["w1"][e], params["w2"][e], w3, b1, b2)
+        y[pos[toks[keep]]] += scores[e, keep][:, None] * out
+    return y, dict(logits=logits, C=C, idx=idx, scores=scores)
+
+
+def expert_choice_margin(logits32, C: int) -> np.ndarray:
+    """Per expert, the gap between its C-th and (C+1)-th largest fp32 logits (inf
+    when C >= T): a choice whose gap is tiny may flip under a different rounding
+    of the logits."""
+    z = np.asarray(logits32, dtype=np.float64)
+    T, E = z.shape
+    out = np.full(E, np.inf)
+    if C >= T or C <= 0:
+        return out
+    for e in range(E):
+        v = np.sort(z[:, e])[::-1]
+        out[e] = v[C - 1] - v[C]
+    return out

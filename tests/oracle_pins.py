@@ -355,7 +355,80 @@ def check_combine(O):
     assert np.allclose(out[2], sh[2], rtol=0, atol=1e-15)
 
 
+# ------------------------------------------------------------ Expert-Choice routing
+def check_expert_choice_capacity(O):
+    """int(cf * N / E) (P3 ``ExpertChoiceRouter``, P4 ``ExpertChoiceGating``), by hand."""
+    for cf, T, E, want in ((1.0, 16384, 128, 128), (1.0, 10, 3, 3), (2.0, 4096, 8, 1024),
+                           (1.25, 7, 2, 4), (0.5, 9, 4, 1), (3.0, 5, 3, 5)):
+        assert O.expert_choice_capacity(cf, T, E) == want, (cf, T, E)
+
+
+def check_expert_choice_bruteforce(O):
+    """Each expert's C tokens, by enumeration over all ordered C-subsets of the
+    tokens (value descending, equal values to the lower token first)."""
+    rng = np.random.default_rng(5)
+    for T, E in ((5, 2), (6, 3), (7, 1)):
+        for C in range(1, T + 1):
+            z = rng.normal(size=(T, E)).astype(np.float32)
+            zt = (np.round(rng.normal(size=(T, E)) * 2) / 2).astype(np.float32)
+            for zz in (z, zt):
+                got = O.expert_choice_select(zz, C)
+                assert got.shape == (E, C)
+                for e in range(E):
+                    assert list(got[e]) == _brute_topk(zz[:, e], C), (T, E, C, zz[:, e])
+
+
+def check_expert_choice_scores(O):
+    """Per expert, a softmax over the tokens: each expert's scores sum to 1 over
+    the tokens, and score ratios are exp of logit differences along a column."""
+    rng = np.random.default_rng(6)
+    z = (rng.normal(size=(9, 4)) * 3).astype(np.float32)
+    S = O.expert_choice_scores(z)
+    assert S.shape == (4, 9)
+    assert np.allclose(S.sum(axis=1), 1.0, rtol=0, atol=1e-14)
+    for e in range(4):
+        for t in range(1, 9):
+            assert abs(S[e, t] / S[e, 0] - math.exp(float(z[t, e]) - float(z[0, e]))) <= \
+                1e-12 * math.exp(float(z[t, e]) - float(z[0, e]))
+    # a column that is constant gives the uniform distribution over the tokens
+    S1 = O.expert_choice_scores(np.zeros((5, 2), dtype=np.float32))
+    assert np.allclose(S1, 0.2, rtol=0, atol=1e-15)
+
+
+def check_expert_choice_dense(O):
+    """The pages' form: dispatch mask [E, N] = scores scattered at each expert's
+    top-C tokens (torch.topk on torch.softmax over the token dim, P4
+    ``ExpertChoiceGating``), every expert computed on every token, masked and
+    summed, equals the oracle's sparse loop; with C = N it is the dense soft mix."""
+    for wl, cf in ((synth.SMALL["tiny"].replace(T=24), 1.0),
+                   (synth.SMALL["mixtral_small"].replace(T=20, d_model=16, d_ff=24, n_experts=4),
+                    1.5),
+                   (synth.SMALL["switch_small"].replace(T=12, d_model=8, d_ff=16, n_experts=3),
+                    3.0)):
+        inp, p = _small_inputs(wl, seed=13)
+        act = ACT[wl.act]
+        y, r = O.expert_choice_forward(p["x"], p, capacity_factor=cf, act=act)
+        T, E = r["logits"].shape
+        assert np.min(O.expert_choice_margin(r["logits"], r["C"])) > 1e-6, wl.name
+        zt = torch.as_tensor(np.asarray(r["logits"], dtype=np.float64))
+        scores = torch.softmax(zt.T, dim=-1)
+        top_s, top_i = torch.topk(scores, r["C"], dim=-1)
+        dispatch = torch.zeros(E, T, dtype=torch.float64)
+        dispatch.scatter_(1, top_i, top_s)
+        assert np.array_equal(np.asarray(r["idx"]), top_i.numpy()), wl.name
+        dense = np.zeros_like(y)
+        for e in range(E):
+            dense += dispatch[e].numpy()[:, None] * _dense_expert(p, e, act, p["x"])
+        assert np.abs(y - dense).max() <= 1e-12 * max(1.0, np.abs(dense).max()), wl.name
+        if r["C"] == T:
+            assert (dispatch > 0).all(), "C = N: every expert takes every token"
+        else:
+            assert (dispatch.sum(dim=0) == 0).any() or r["C"] * E >= T
+
+
 ALL_CHECKS = [check_combine, check_topk_bruteforce, check_gate_sums_and_ranges, check_worked_gates,
               check_softmax_closed_forms, check_router_logits_exact, check_capacity_golden,
               check_counts_and_drop_order, check_layout, check_forward_vs_pages_torch,
-              check_sparse_equals_dense_masked, check_special_cases, check_aux_closed_forms]
+              check_sparse_equals_dense_masked, check_special_cases, check_aux_closed_forms,
+              check_expert_choice_capacity, check_expert_choice_bruteforce,
+              check_expert_choice_scores, check_expert_choice_dense]

@@ -98,7 +98,41 @@ def _combine_ignores_gates(y_rows, inv, gates, shared=None):
     return _orig["combine"](y_rows, inv, np.ones_like(np.asarray(gates, dtype=float)), shared)
 
 
+def _ec_softmax_over_experts(logits32):
+    z = np.asarray(logits32, dtype=np.float64)
+    e = np.exp(z - z.max(axis=1, keepdims=True))
+    return (e / e.sum(axis=1, keepdims=True)).T
+
+
+def _ec_ties_to_higher_token(logits32, C):
+    z = np.asarray(logits32, dtype=np.float32)
+    T, E = z.shape
+    out = np.zeros((E, C), dtype=np.int32)
+    for e in range(E):
+        order = np.argsort(-z[::-1, e].astype(np.float64), kind="stable")
+        out[e] = (T - 1 - order)[:C]
+    return out
+
+
+def _ec_capacity_rounds_up(cf, T, E):
+    return int(np.ceil(float(cf) * T / E))
+
+
+def _ec_forward_ignores_scores(x, params, *, capacity_factor, act, logits=None, tokens=None):
+    orig = _orig["expert_choice_scores"]
+    O.expert_choice_scores = lambda z: np.ones_like(orig(z))
+    try:
+        return _orig["expert_choice_forward"](x, params, capacity_factor=capacity_factor,
+                                              act=act, logits=logits, tokens=tokens)
+    finally:
+        O.expert_choice_scores = orig
+
+
 MUTANTS = {
+    "ec_softmax_over_experts": ("expert_choice_scores", _ec_softmax_over_experts),
+    "ec_ties_to_higher_token": ("expert_choice_select", _ec_ties_to_higher_token),
+    "ec_capacity_rounds_up": ("expert_choice_capacity", _ec_capacity_rounds_up),
+    "ec_output_ignores_scores": ("expert_choice_forward", _ec_forward_ignores_scores),
     "combine_ignores_gates": ("combine", _combine_ignores_gates),
     "topk_ties_to_higher_index": ("select_topk", _topk_ties_high),
     "gates_not_renormalised": ("gate_values", _gates_no_renorm),
