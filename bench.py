@@ -17,6 +17,7 @@ import argparse
 import datetime
 import hashlib
 import json
+import math
 import os
 import statistics
 import sys
@@ -185,6 +186,22 @@ def oracle_sample_rate(wl, inp, n_tokens: int):
     acts = {0: "relu", 1: "gelu", 2: "swiglu"}
     modes = {0: "topk_softmax", 1: "softmax_topk_renorm", 2: "softmax_topk_raw"}
     P = _oracle_params(inp)
+    if wl.routing == synth.ROUTING_EXPERT_CHOICE:
+        t0 = time.perf_counter()
+        logits = O.router_logits(P["x"], P["w_router"], P.get("b_router"), P.get("logit_bias"))
+        O.expert_choice_select(logits, O.expert_choice_capacity(wl.capacity_factor, wl.T,
+                                                                wl.n_experts))
+        t_route = time.perf_counter() - t0
+        toks = synth.token_sample(wl.T, n_tokens).numpy()
+        t0 = time.perf_counter()
+        O.expert_choice_forward(P["x"], P, capacity_factor=wl.capacity_factor,
+                                act=acts[wl.act], logits=logits, tokens=toks)
+        t_ffn = time.perf_counter() - t0  # includes the (cheap) re-selection
+        per_token = t_route / wl.T + t_ffn / len(toks)
+        desc = (f"oracle (numpy fp64), expert choice: routing of all {wl.T} tokens "
+                f"({t_route:.2f} s) + expert FFNs of {len(toks)} strided tokens ({t_ffn:.2f} s)"
+                f"; tokens/s = 1 / (t_route/T + t_ffn/n)")
+        return 1.0 / per_token, desc, t_route + t_ffn
     kw = dict(top_k=wl.top_k, act=acts[wl.act], gate_mode=modes[wl.gate_mode],
               capacity_factor=wl.capacity_factor, n_shared=wl.n_shared)
     t0 = time.perf_counter()
@@ -234,6 +251,8 @@ def _config(wl, world):
     return {"workload": wl.name, "T": wl.T, "d_model": wl.d_model, "n_experts": wl.n_experts,
             "top_k": wl.top_k, "d_ff": wl.d_ff, "n_shared": wl.n_shared,
             "d_ff_shared": wl.d_ff_shared, "capacity_factor": wl.capacity_factor,
+            "routing": "expert choice" if wl.routing == synth.ROUTING_EXPERT_CHOICE
+            else "token choice",
             "global_batch": wl.T * world, "seq_len": wl.T,
             "parallelism": f"dp{world} (independent token batches, no data-path collective)",
             "l2": "working set > L2 (weights >= 2.8 GB per step); no flush"}
@@ -260,6 +279,37 @@ def _traffic(workload_name):
         return None
 
 
+def kernels_per_step(step, dev) -> int:
+    """Kernel launches of one step, counted from a CUDA-graph capture of it (the
+    graph is built, its kernel nodes counted, and destroyed without running)."""
+    from cuda.bindings import runtime as cudart
+
+    s = torch.cuda.Stream(dev)
+    s.wait_stream(torch.cuda.current_stream())
+    torch.cuda.synchronize()
+    with torch.cuda.stream(s):
+        (e,) = cudart.cudaStreamBeginCapture(
+            s.cuda_stream, cudart.cudaStreamCaptureMode.cudaStreamCaptureModeThreadLocal)
+        if e != cudart.cudaError_t.cudaSuccess:
+            raise RuntimeError(f"stream capture: {e}")
+        try:
+            step()
+        finally:
+            e, graph = cudart.cudaStreamEndCapture(s.cuda_stream)
+    if e != cudart.cudaError_t.cudaSuccess:
+        raise RuntimeError(f"stream capture: {e}")
+    try:
+        e, _, n = cudart.cudaGraphGetNodes(graph, 0)
+        e, nodes, n = cudart.cudaGraphGetNodes(graph, n)
+        kernels = 0
+        for node in nodes[:n]:
+            e, kind = cudart.cudaGraphNodeGetType(node)
+            kernels += kind == cudart.cudaGraphNodeType.cudaGraphNodeTypeKernel
+        return int(kernels)
+    finally:
+        cudart.cudaGraphDestroy(graph)
+
+
 # ---------------------------------------------------------------------- our arm
 def run_ours(args, wl, rank, world, local_rank):
     from sparse_mixture_experts_12_b200 import binding as B
@@ -278,10 +328,11 @@ def run_ours(args, wl, rank, world, local_rank):
     layer = B.MoELayer(wl, inp, dev)
     x = inp["x"].to(dev)
     y = torch.empty_like(x)
-    want_aux = wl.capacity_factor > 0  # the Switch workload also emits f, P and the aux loss
+    ec = wl.routing == synth.ROUTING_EXPERT_CHOICE
+    # the Switch workload also emits f, P and the aux loss (token choice only)
+    want_aux = wl.capacity_factor > 0 and not ec
     aux = layer.new_aux() if want_aux else None
     stream = torch.cuda.current_stream()
-    per_step_launches = 6 + (2 if wl.n_shared > 0 else 0)
 
     clocks = ClockSampler(local_rank)
     clocks.start()
@@ -291,6 +342,10 @@ def run_ours(args, wl, rank, world, local_rank):
     code, info = layer.last_device_error()
     if code != 0:
         raise RuntimeError(f"device error {code} ({info}) during warm-up")
+    clocks.stop()
+    per_step_launches = kernels_per_step(lambda: layer.forward(x, y, aux), dev)
+    clocks = ClockSampler(local_rank)
+    clocks.start()
     barrier(world)
     torch.cuda.synchronize()
     clocks.begin_load()
@@ -309,16 +364,26 @@ def run_ours(args, wl, rank, world, local_rank):
     value = tokens_per_second(wl.T, world, args.steps, ms)
 
     # ---- expert FFN (grouped GEMMs) timed alone on the same stream, for the roofline
-    taps = layer.new_taps()
-    layer.forward(x, y, aux, taps=taps)
     E, k = wl.n_experts, wl.top_k
-    xp = torch.empty((wl.T * k, wl.d_model), dtype=wl.torch_dtype, device=dev)
-    cnt = torch.empty(E, dtype=torch.int32, device=dev)
-    off = torch.empty(E + 1, dtype=torch.int32, device=dev)
-    perm = torch.empty(wl.T * k, dtype=torch.int32, device=dev)
-    inv = torch.empty(wl.T * k, dtype=torch.int32, device=dev)
-    layer.permute(x, taps["topk_idx"], cnt, off, perm, inv, xp)
+    if ec:  # each expert's C picked rows, expert-contiguous
+        C = int(math.floor(wl.capacity_factor * wl.T / E))
+        lg = torch.empty((wl.T, E), dtype=torch.float32, device=dev)
+        eci = torch.empty((E, C), dtype=torch.int32, device=dev)
+        ecs = torch.empty((E, C), dtype=torch.float32, device=dev)
+        layer.route_expert_choice(x, lg, eci, ecs)
+        xp = x[eci.reshape(-1).long()].contiguous()
+        off = (torch.arange(E + 1, device=dev, dtype=torch.int32) * C).contiguous()
+    else:
+        taps = layer.new_taps()
+        layer.forward(x, y, aux, taps=taps)
+        xp = torch.empty((wl.T * k, wl.d_model), dtype=wl.torch_dtype, device=dev)
+        cnt = torch.empty(E, dtype=torch.int32, device=dev)
+        off = torch.empty(E + 1, dtype=torch.int32, device=dev)
+        perm = torch.empty(wl.T * k, dtype=torch.int32, device=dev)
+        inv = torch.empty(wl.T * k, dtype=torch.int32, device=dev)
+        layer.permute(x, taps["topk_idx"], cnt, off, perm, inv, xp)
     yp = torch.empty_like(xp)
+    counts = np.diff(off.cpu().numpy()) if ec else taps["counts"].cpu().numpy()
     for _ in range(3):
         layer.expert_ffn(xp, off, yp)
     torch.cuda.synchronize()
@@ -331,7 +396,6 @@ def run_ours(args, wl, rank, world, local_rank):
     torch.cuda.synchronize()
     ffn_ms = f0.elapsed_time(f1) / n_ffn
     R = int(off[-1].item())
-    counts = taps["counts"].cpu().numpy()
     kept = np.diff(off.cpu().numpy())
     touched = int((kept > 0).sum())
     F, d = wl.d_ff, wl.d_model
@@ -428,7 +492,8 @@ def run_ours(args, wl, rank, world, local_rank):
             "data": "synthetic (seeded N(0,1) activations, random-init weights)",
             "config": _config(wl, world), "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": per_step_launches * args.steps, "clocks": clk,
-            "routing": {"rows_kept": R, "dropped": int(wl.T * k - R),
+            "routing": {"kind": "expert choice" if ec else "token choice", "rows_kept": R,
+                        "dropped": 0 if ec else int(wl.T * k - R),
                         "max_expert_load": int(counts.max()), "min_expert_load": int(counts.min())}}
     print(json.dumps(line), flush=True)
 

@@ -89,6 +89,14 @@ enum {
 
 enum { MOE_DTYPE_F32 = 0, MOE_DTYPE_BF16 = 1 };
 
+/* Routing. Token choice: every token picks its top-k experts (all gate modes,
+ * capacity drops). Expert choice (youngju.dev (zh) "ExpertChoiceRouter", youngju.dev
+ * (ja) "ExpertChoiceGating"): every expert takes the C = floor(cf * T / E) tokens with
+ * the highest score, score = its softmax over the tokens of the call; a token's
+ * output is the score-weighted sum over the experts that took it (the dispatch mask
+ * as the gate), 0 if none did. top_k and gate_mode are not used. */
+enum { MOE_ROUTING_TOKEN_CHOICE = 0, MOE_ROUTING_EXPERT_CHOICE = 1 };
+
 /* Layer configuration (MoEConfig of the ja page, plus routing and storage fields).
  * Limits: 1 <= E <= 256; 1 <= k <= min(E, 8); T >= 0 (T = 0 is a no-op);
  * d_model, d_ff, d_ff_shared multiples of 64 for bf16 (tensor-core path) and of
@@ -107,6 +115,8 @@ typedef struct {
   float aux_alpha;         /* weight of the load-balancing loss (0.01 on the pages) */
   int32_t n_shared;        /* always-on SwiGLU experts, added unweighted (0 = none) */
   int32_t d_ff_shared;     /* F of each shared expert */
+  int32_t routing;         /* MOE_ROUTING_*; expert choice: capacity_factor > 0 gives C,
+                              1 <= C <= 8192, T <= 32768, n_shared = 0 */
 } moe_cfg_t;
 
 /* Device pointers to the parameters. Unused entries must be NULL. */
@@ -186,10 +196,11 @@ moe_status_t moe_permute_noalloc(const moe_cfg_t *cfg, const void *x, const int3
                                  void *x_perm, moe_stream_t stream);
 
 /* Expert FFNs on expert-contiguous rows ("SwiGLUExpert", MLP experts).
- * Rows [offsets[e], offsets[e+1]) of x_perm [T*k, d] go through expert e and the
- * result is written to the same rows of y_perm [T*k, d] (dtype). offsets is a
- * device array [E+1]; it must be non-decreasing from 0 to at most T*k (checked on
- * the device: MOE_DEVERR_OFFSETS, nothing computed). For the shared experts call
+ * Rows [offsets[e], offsets[e+1]) of x_perm [R, d] go through expert e and the
+ * result is written to the same rows of y_perm [R, d] (dtype), R = T*k (token
+ * choice) or E*C (expert choice). offsets is a device array [E+1]; it must be
+ * non-decreasing from 0 to at most R (checked on the device: MOE_DEVERR_OFFSETS,
+ * nothing computed). For the shared experts call
  * it with n_experts = 1, d_ff = n_shared*F_sh, w1/w3/w2 = ws_gate/ws_up/ws_down. */
 moe_status_t moe_expert_ffn(const moe_cfg_t *cfg, const moe_weights_t *w, const void *x_perm,
                             const int32_t *offsets, void *y_perm, void *ws, size_t ws_bytes,
@@ -214,10 +225,32 @@ moe_status_t moe_aux_stats(const moe_cfg_t *cfg, const float *logits, const int3
 
 /* The whole layer: route, permute, expert FFNs, shared experts, combine.
  * x [T, d] and y [T, d] in dtype. aux_out (nullable) receives the moe_aux_stats
- * vector [3 + 2E]. taps (nullable) receives intermediates. */
+ * vector [3 + 2E]. taps (nullable) receives intermediates.
+ * With cfg->routing == MOE_ROUTING_EXPERT_CHOICE: router, expert choice, gather of
+ * each expert's C rows, expert FFNs, score-weighted combine; aux_out must be NULL
+ * and of the taps only `logits` is filled. */
 moe_status_t moe_forward(const moe_cfg_t *cfg, const moe_weights_t *w, const void *x, void *y,
                          float *aux_out, const moe_taps_t *taps, void *ws, size_t ws_bytes,
                          moe_stream_t stream);
+
+/* Expert-Choice routing step (youngju.dev (zh) "ExpertChoiceRouter", youngju.dev (ja)
+ * "ExpertChoiceGating"): logits as in moe_route, then for every expert e its C =
+ * floor(cf * T / E) tokens of highest logit in descending order (equal logits: lower
+ * token first; the per-expert softmax over tokens is monotone in the logit, so this
+ * is the order of the scores), and their scores exp(z - m_e) / sum_t exp(z_t - m_e)
+ * with m_e the expert's largest logit. A NaN logit counts as -inf.
+ *   x         [T, d] dtype, or NULL: then `logits` [T, E] fp32 is the input
+ *   logits    [T, E] fp32 output (input when x == NULL)
+ *   ec_idx    [E, C] int32 output: token index of expert e's j-th pick
+ *   ec_score  [E, C] fp32 output: its score
+ * Requires cfg->routing == MOE_ROUTING_EXPERT_CHOICE (MOE_ERR_INVALID_ARG otherwise)
+ * and the limits of moe_cfg_t (MOE_ERR_UNSUPPORTED beyond them). This is the pages'
+ * router module (scores and indices per expert); moe_forward runs it as its first
+ * step. */
+moe_status_t moe_route_expert_choice(const moe_cfg_t *cfg, const moe_weights_t *w,
+                                     const void *x, float *logits, int32_t *ec_idx,
+                                     float *ec_score, void *ws, size_t ws_bytes,
+                                     moe_stream_t stream);
 
 /* Synchronise `stream`, read and clear the sticky device error word.
  * Returns MOE_ERR_DEVICE when *code != 0, MOE_ERR_CUDA when the sync failed. */

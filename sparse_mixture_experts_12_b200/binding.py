@@ -26,8 +26,8 @@ STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED",
 DEVERR_NAMES = {0: "none", 1: "expert index out of range", 2: "invalid offsets",
                 3: "row index out of range", 4: "pipeline wait timeout"}
 
-EXPORTED = ("moe_workspace_size", "moe_workspace_init", "moe_route", "moe_permute",
-            "moe_permute_noalloc",
+EXPORTED = ("moe_workspace_size", "moe_workspace_init", "moe_route", "moe_route_expert_choice",
+            "moe_permute", "moe_permute_noalloc",
             "moe_expert_ffn", "moe_combine", "moe_aux_stats", "moe_forward",
             "moe_last_device_error", "moe_status_string")
 
@@ -44,7 +44,8 @@ class MoeCfg(ctypes.Structure):
                 ("d_ff", ctypes.c_int32), ("act", ctypes.c_int32),
                 ("gate_mode", ctypes.c_int32), ("dtype", ctypes.c_int32),
                 ("capacity_factor", ctypes.c_float), ("aux_alpha", ctypes.c_float),
-                ("n_shared", ctypes.c_int32), ("d_ff_shared", ctypes.c_int32)]
+                ("n_shared", ctypes.c_int32), ("d_ff_shared", ctypes.c_int32),
+                ("routing", ctypes.c_int32)]
 
 
 class MoeWeights(ctypes.Structure):
@@ -113,7 +114,7 @@ def make_cfg(w: synth.Workload, **over) -> MoeCfg:
     c = MoeCfg(n_tokens=w.T, d_model=w.d_model, n_experts=w.n_experts, top_k=w.top_k,
                d_ff=w.d_ff, act=w.act, gate_mode=w.gate_mode, dtype=w.dtype,
                capacity_factor=w.capacity_factor, aux_alpha=w.aux_alpha,
-               n_shared=w.n_shared, d_ff_shared=w.d_ff_shared)
+               n_shared=w.n_shared, d_ff_shared=w.d_ff_shared, routing=w.routing)
     for k, v in over.items():
         setattr(c, k, v)
     return c
@@ -185,6 +186,15 @@ class MoELayer:
         _check(self.lib.moe_route(ctypes.byref(self.cfg), ctypes.byref(self.weights), _ptr(x),
                                   _ptr(logits), _ptr(topk_idx), _ptr(topk_gate), _ptr(self.ws),
                                   self.ws.numel(), _stream()), "moe_route")
+
+    def route_expert_choice(self, x: Optional[torch.Tensor], logits: torch.Tensor,
+                            ec_idx: torch.Tensor, ec_score: torch.Tensor):
+        """Expert-Choice routing: logits [T, E] (input when x is None), ec_idx [E, C],
+        ec_score [E, C]."""
+        _check(self.lib.moe_route_expert_choice(
+            ctypes.byref(self.cfg), ctypes.byref(self.weights), _ptr(x), _ptr(logits),
+            _ptr(ec_idx), _ptr(ec_score), _ptr(self.ws), self.ws.numel(), _stream()),
+            "moe_route_expert_choice")
 
     def permute(self, x, topk_idx, counts, offsets, perm, inv, x_perm):
         _check(self.lib.moe_permute(ctypes.byref(self.cfg), _ptr(x), _ptr(topk_idx), _ptr(counts),

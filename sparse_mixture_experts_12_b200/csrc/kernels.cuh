@@ -79,6 +79,26 @@ struct GroupedFfnArgs {
   int32_t *err;
 };
 
+// Expert-Choice routing (see expert_choice.cu)
+constexpr int kEcMaxTokens = 32768;  // one CTA holds an expert's whole column of logits
+constexpr int kEcMaxPicks = 8192;    // C: the sort buffer of the picks
+struct EcArgs {
+  const float *logits;  // [T, E]
+  float *zt;            // [E, T] scratch: transposed logits, NaN -> -inf
+  int32_t *ec_idx;      // [E, C]
+  float *ec_score;      // [E, C]
+  int32_t *slot;        // [T, E] or nullptr: pick slot j of token t in expert e, -1 if none
+                        // (the caller sets it to -1 first)
+  int32_t *offsets;     // [E+1] or nullptr: e * C
+  int T, E, C;
+  int32_t *err;         // device error word or nullptr
+};
+cudaError_t launch_ec_route(const EcArgs &a, cudaStream_t st);
+cudaError_t launch_ec_gather(const void *x, int T, const int32_t *ec_idx, int rows,
+                             int row_bytes, void *x_perm, cudaStream_t st);
+cudaError_t launch_ec_combine(const void *y_perm, const int32_t *slot, const float *score,
+                              int T, int E, int C, int d, int dtype, void *y, cudaStream_t st);
+
 cudaError_t launch_router(const RouterArgs &a, int dtype, cudaStream_t st);
 // bf16 router on the tensor cores (x given, 16 <= E <= 256)
 cudaError_t launch_router_tc(const RouterArgs &a, cudaStream_t st);

@@ -15,7 +15,7 @@ namespace {
 enum Buf {
   B_ERR, B_TILE_COUNTS, B_TILE_BASE, B_TILE_P, B_TILE_Z, B_COUNTS, B_OFFSETS, B_MPREFIX, B_SH_TBL,
   B_LOGITS, B_IDX, B_GATE, B_PERM, B_INV, B_XPERM, B_H, B_YPERM, B_SH_H, B_SH_Y, B_YPART,
-  B_NBUF
+  B_EC_ZT, B_EC_IDX, B_EC_SCORE, B_EC_SLOT, B_NBUF
 };
 
 struct Layout {
@@ -25,12 +25,33 @@ struct Layout {
 
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
+bool expert_choice(const moe_cfg_t &c) { return c.routing == MOE_ROUTING_EXPERT_CHOICE; }
+long long ec_picks(const moe_cfg_t &c);
+
+// rows of the expert-contiguous buffers (x_perm, h, y_perm): T*k (token choice) or
+// E*C (expert choice)
+long long expert_rows(const moe_cfg_t &c) {
+  return expert_choice(c) ? (long long)c.n_experts * ec_picks(c)
+                          : (long long)c.n_tokens * c.top_k;
+}
+
+// tokens each expert takes under Expert-Choice routing: floor(cf * T / E)
+long long ec_picks(const moe_cfg_t &c) {
+  if (!(c.capacity_factor > 0.f)) return 0;
+  const double v = floor((double)c.capacity_factor * (double)c.n_tokens / (double)c.n_experts);
+  return v > 1e18 ? (long long)1e18 : (long long)v;
+}
+
 Layout layout_for(const moe_cfg_t &c) {
   const size_t T = (size_t)c.n_tokens, E = (size_t)c.n_experts, k = (size_t)c.top_k;
   const size_t d = (size_t)c.d_model, F = (size_t)c.d_ff;
   const size_t eb = c.dtype == MOE_DTYPE_F32 ? 4 : 2;
   const size_t NT = (size_t)ceil_div(c.n_tokens > 0 ? c.n_tokens : 1, router_bm(c.n_experts));
   const size_t Fs = (size_t)c.n_shared * (size_t)c.d_ff_shared;
+  const bool ec = expert_choice(c);
+  const size_t C = ec ? (size_t)ec_picks(c) : 0;
+  // rows of the expert-contiguous buffers: T*k (token choice) or E*C (expert choice)
+  const size_t R = ec ? E * C : T * k;
   size_t sz[B_NBUF];
   sz[B_ERR] = 2 * sizeof(int32_t);
   sz[B_TILE_COUNTS] = E * NT * 4;
@@ -46,15 +67,19 @@ Layout layout_for(const moe_cfg_t &c) {
   sz[B_GATE] = T * k * 4;
   sz[B_PERM] = T * k * 4;
   sz[B_INV] = T * k * 4;
-  sz[B_XPERM] = T * k * d * eb;
-  sz[B_H] = T * k * F * eb;
-  sz[B_YPERM] = T * k * d * eb;
+  sz[B_XPERM] = R * d * eb;
+  sz[B_H] = R * F * eb;
+  sz[B_YPERM] = R * d * eb;
   sz[B_SH_H] = Fs ? T * Fs * eb : 0;
   sz[B_SH_Y] = Fs ? T * d * 4 : 0;
   // split-K partials of the small-batch expert GEMM (bf16, few tokens)
   sz[B_YPART] = (c.dtype == MOE_DTYPE_BF16 && T <= (size_t)kDecodeMaxRows)
-                    ? ffn_decode_partial_bytes((int)(T * k > T ? T * k : T), (int)d)
+                    ? ffn_decode_partial_bytes((int)(R > T ? R : T), (int)d)
                     : 0;
+  sz[B_EC_ZT] = ec ? E * T * 4 : 0;
+  sz[B_EC_IDX] = ec ? E * C * 4 : 0;
+  sz[B_EC_SCORE] = ec ? E * C * 4 : 0;
+  sz[B_EC_SLOT] = ec ? T * E * 4 : 0;
   Layout L;
   size_t o = 0;
   for (int i = 0; i < B_NBUF; ++i) {
@@ -87,7 +112,18 @@ moe_status_t check_cfg(const moe_cfg_t *c) {
   if (c->dtype != MOE_DTYPE_F32 && c->dtype != MOE_DTYPE_BF16) return MOE_ERR_INVALID_ARG;
   if (!isfinite(c->capacity_factor) || !isfinite(c->aux_alpha)) return MOE_ERR_INVALID_ARG;
   if (c->n_shared < 0 || (c->n_shared > 0 && c->d_ff_shared <= 0)) return MOE_ERR_INVALID_ARG;
-  const long long rows = (long long)c->n_tokens * c->top_k;
+  if (c->routing != MOE_ROUTING_TOKEN_CHOICE && c->routing != MOE_ROUTING_EXPERT_CHOICE)
+    return MOE_ERR_INVALID_ARG;
+  if (expert_choice(*c)) {
+    if (!(c->capacity_factor > 0.f)) return MOE_ERR_INVALID_ARG;
+    const long long C = ec_picks(*c);
+    if (c->n_tokens > 0 && C < 1) return MOE_ERR_INVALID_ARG;  // every expert takes a token
+    if (C > c->n_tokens) return MOE_ERR_INVALID_ARG;           // cf > E: more picks than tokens
+    if (c->n_tokens > kEcMaxTokens || C > kEcMaxPicks || c->n_shared > 0)
+      return MOE_ERR_UNSUPPORTED;
+  }
+  const long long rows = expert_choice(*c) ? (long long)c->n_experts * ec_picks(*c)
+                                           : (long long)c->n_tokens * c->top_k;
   if (rows > INT_MAX / 2) return MOE_ERR_UNSUPPORTED;
   const long long fs = (long long)c->n_shared * c->d_ff_shared;
   if (fs > INT_MAX / 2 || c->d_model > INT_MAX / 4 || c->d_ff > INT_MAX / 4)
@@ -175,7 +211,7 @@ GroupedFfnArgs routed_ffn_args(const moe_cfg_t &c, const moe_weights_t &w, const
   a.max_group_rows = max_group_rows;
   a.part = part;
   a.a = x_perm;
-  a.a_rows = c.n_tokens * c.top_k;
+  a.a_rows = (int)expert_rows(c);
   a.offsets = offsets;
   a.mprefix = mprefix;
   a.G = c.n_experts;
@@ -193,6 +229,70 @@ GroupedFfnArgs routed_ffn_args(const moe_cfg_t &c, const moe_weights_t &w, const
   a.out_f32 = 0;
   a.err = err;
   return a;
+}
+
+// Expert-Choice routing: router logits (unless x is NULL: logits are the input),
+// then every expert's picks. slot/offsets (nullable) feed the forward's later steps.
+moe_status_t ec_route(const moe_cfg_t &c, const moe_weights_t *w, const void *x, float *logits,
+                      int32_t *ec_idx, float *ec_score, int32_t *slot, int32_t *offsets,
+                      void *ws, const Layout &L, cudaStream_t stream) {
+  if (x != nullptr) {
+    RouterArgs r{};
+    r.x = x;
+    r.w = w->w_router;
+    r.b_router = w->b_router;
+    r.logit_bias = w->logit_bias;
+    r.logits_out = logits;
+    r.topk_idx = at<int32_t>(ws, L, B_IDX);  // the router's own top-1, not used here
+    r.topk_gate = at<float>(ws, L, B_GATE);
+    r.T = c.n_tokens;
+    r.d = c.d_model;
+    r.E = c.n_experts;
+    r.k = 1;
+    r.gate_mode = MOE_GATE_TOPK_SOFTMAX;
+    r.err = at<int32_t>(ws, L, B_ERR);
+    MOE_CUDA(launch_router(r, c.dtype, stream));
+  }
+  if (slot != nullptr)
+    MOE_CUDA(cudaMemsetAsync(slot, 0xFF, (size_t)c.n_tokens * c.n_experts * sizeof(int32_t),
+                             stream));
+  EcArgs a{};
+  a.logits = logits;
+  a.zt = at<float>(ws, L, B_EC_ZT);
+  a.ec_idx = ec_idx;
+  a.ec_score = ec_score;
+  a.slot = slot;
+  a.offsets = offsets;
+  a.T = c.n_tokens;
+  a.E = c.n_experts;
+  a.C = (int)ec_picks(c);
+  a.err = at<int32_t>(ws, L, B_ERR);
+  MOE_CUDA(launch_ec_route(a, stream));
+  return MOE_OK;
+}
+
+// Expert-Choice forward: route, gather each expert's C rows, expert FFNs, combine.
+moe_status_t ec_forward(const moe_cfg_t &c, const moe_weights_t *w, const void *x, void *y,
+                        float *logits, void *ws, const Layout &L, cudaStream_t stream) {
+  const int T = c.n_tokens, E = c.n_experts, C = (int)ec_picks(c);
+  int32_t *err = at<int32_t>(ws, L, B_ERR);
+  int32_t *ec_idx = at<int32_t>(ws, L, B_EC_IDX);
+  float *ec_score = at<float>(ws, L, B_EC_SCORE);
+  int32_t *slot = at<int32_t>(ws, L, B_EC_SLOT);
+  int32_t *offsets = at<int32_t>(ws, L, B_OFFSETS);
+  int32_t *mprefix = at<int32_t>(ws, L, B_MPREFIX);
+  MOE_TRY(ec_route(c, w, x, logits, ec_idx, ec_score, slot, offsets, ws, L, stream));
+  const int eb = c.dtype == MOE_DTYPE_F32 ? 4 : 2;
+  void *x_perm = at<void>(ws, L, B_XPERM);
+  void *y_perm = at<void>(ws, L, B_YPERM);
+  MOE_CUDA(launch_ec_gather(x, T, ec_idx, E * C, c.d_model * eb, x_perm, stream));
+  MOE_CUDA(launch_tile_table(offsets, E, E * C, mprefix, err, stream));
+  float *part = layout_size(L, B_YPART) > 0 ? at<float>(ws, L, B_YPART) : nullptr;
+  GroupedFfnArgs a = routed_ffn_args(c, *w, x_perm, offsets, mprefix, at<void>(ws, L, B_H),
+                                     y_perm, err, C, part);  // E*C rows, C per expert
+  MOE_CUDA(run_ffn(c, a, stream));
+  MOE_CUDA(launch_ec_combine(y_perm, slot, ec_score, T, E, C, c.d_model, c.dtype, y, stream));
+  return MOE_OK;
 }
 
 }  // namespace
@@ -249,6 +349,24 @@ MOE_API moe_status_t moe_route(const moe_cfg_t *cfg, const moe_weights_t *w, con
   r.err = at<int32_t>(ws, L, B_ERR);
   MOE_CUDA(launch_router(r, c.dtype, stream));
   return MOE_OK;
+}
+
+MOE_API moe_status_t moe_route_expert_choice(const moe_cfg_t *cfg, const moe_weights_t *w,
+                                             const void *x, float *logits, int32_t *ec_idx,
+                                             float *ec_score, void *ws, size_t ws_bytes,
+                                             moe_stream_t stream) {
+  MOE_TRY(check_cfg(cfg));
+  MOE_TRY(check_ws(cfg, ws, ws_bytes));
+  if (!expert_choice(*cfg)) return MOE_ERR_INVALID_ARG;
+  if (cfg->n_tokens == 0) return MOE_OK;
+  if (x != nullptr) {
+    if (w == nullptr) return MOE_ERR_INVALID_ARG;
+    MOE_TRY(check_ptrs({{x, true}, {w->w_router, true}, {w->b_router, false},
+                        {w->logit_bias, false}}));
+  }
+  MOE_TRY(check_ptrs({{logits, true}, {ec_idx, true}, {ec_score, true}}));
+  const Layout L = layout_for(*cfg);
+  return ec_route(*cfg, w, x, logits, ec_idx, ec_score, nullptr, nullptr, ws, L, stream);
 }
 
 MOE_API moe_status_t moe_permute(const moe_cfg_t *cfg, const void *x, const int32_t *topk_idx,
@@ -312,9 +430,10 @@ MOE_API moe_status_t moe_expert_ffn(const moe_cfg_t *cfg, const moe_weights_t *w
   const Layout L = layout_for(c);
   int32_t *err = at<int32_t>(ws, L, B_ERR);
   int32_t *mprefix = at<int32_t>(ws, L, B_MPREFIX);
-  MOE_CUDA(launch_tile_table(offsets, c.n_experts, c.n_tokens * c.top_k, mprefix, err, stream));
+  const int rows = (int)expert_rows(c);
+  MOE_CUDA(launch_tile_table(offsets, c.n_experts, rows, mprefix, err, stream));
   GroupedFfnArgs a = routed_ffn_args(c, *w, x_perm, offsets, mprefix, at<void>(ws, L, B_H),
-                                     y_perm, err, c.n_tokens * c.top_k,
+                                     y_perm, err, rows,
                                      layout_size(L, B_YPART) > 0 ? at<float>(ws, L, B_YPART) : nullptr);
   MOE_CUDA(run_ffn(c, a, stream));
   return MOE_OK;
@@ -413,6 +532,10 @@ MOE_API moe_status_t moe_forward(const moe_cfg_t *cfg, const moe_weights_t *w, c
   const Layout L = layout_for(c);
   int32_t *err = at<int32_t>(ws, L, B_ERR);
   float *logits = tp.logits ? tp.logits : at<float>(ws, L, B_LOGITS);
+  if (expert_choice(c)) {
+    if (aux_out != nullptr) return MOE_ERR_INVALID_ARG;
+    return ec_forward(c, w, x, y, logits, ws, L, stream);
+  }
   int32_t *idx = tp.topk_idx ? tp.topk_idx : at<int32_t>(ws, L, B_IDX);
   float *gate = tp.topk_gate ? tp.topk_gate : at<float>(ws, L, B_GATE);
   int32_t *counts = tp.counts ? tp.counts : at<int32_t>(ws, L, B_COUNTS);

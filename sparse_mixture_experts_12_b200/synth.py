@@ -35,6 +35,7 @@ from typing import Optional
 import torch
 
 ACT_RELU, ACT_GELU, ACT_SWIGLU = 0, 1, 2
+ROUTING_TOKEN_CHOICE, ROUTING_EXPERT_CHOICE = 0, 1
 # gate modes: A = softmax over the top-k logits; B = top-k of the full softmax,
 # divided by their sum; C = top-k of the full softmax, raw (Switch).
 GATE_TOPK_SOFTMAX, GATE_SOFTMAX_TOPK_RENORM, GATE_SOFTMAX_TOPK_RAW = 0, 1, 2
@@ -63,6 +64,7 @@ class Workload:
     aux_alpha: float = 0.01
     router_std: float = 0.02
     bias_std: float = 0.0
+    routing: int = ROUTING_TOKEN_CHOICE  # expert choice: C = floor(cf * T / E) per expert
 
     def replace(self, **kw) -> "Workload":
         return dataclasses.replace(self, **kw)
@@ -93,6 +95,13 @@ SWITCH_CAPACITY = Workload("switch_top1_bf16_T16384_d1024_E128_gelu4096_cf1.25",
                            capacity_factor=1.25, expert_bias=True, logit_bias_std=1.5)
 
 
+# Expert-Choice routing on the Mixtral prefill layer: cf = 2 gives each of the 8
+# experts C = 1024 of the 4096 tokens (the same expert work as top-2 token choice)
+MIXTRAL_EC = MIXTRAL_PREFILL.replace(name="mixtral_ec_bf16_T4096_d4096_E8_cf2_swiglu14336",
+                                     capacity_factor=2.0, top_k=1,
+                                     routing=ROUTING_EXPERT_CHOICE)
+
+
 def mixtral_decode(T: int) -> Workload:
     return MIXTRAL_PREFILL.replace(name=f"mixtral_decode_bf16_T{T}_d4096_E8_k2_swiglu14336", T=T)
 
@@ -105,6 +114,7 @@ WORKLOADS = {
     "decode32": mixtral_decode(32),
     "decode8": mixtral_decode(8),
     "decode1": mixtral_decode(1),
+    "mixtral_ec": MIXTRAL_EC,
 }
 
 # ---- reduced shapes of the same families (several tiles plus a ragged tail) ------
@@ -131,6 +141,15 @@ SMALL = {
     "router_e256": SWITCH_CAPACITY.replace(name="router_e256", T=300, d_model=128, d_ff=64,
                                            n_experts=256, top_k=8, capacity_factor=0.0,
                                            bias_std=0.1),
+    # Expert-Choice routing: bf16 SwiGLU (C = 93 of 300 tokens for each of 8 experts),
+    # fp32 ReLU with biases, a bf16 GELU layer with 20 experts (C = 17)
+    "ec_small": MIXTRAL_EC.replace(name="ec_small", T=300, d_model=256, d_ff=384,
+                                   capacity_factor=2.5),
+    "ec_fp32": TINY_FP32.replace(name="ec_fp32", T=64, top_k=1, capacity_factor=1.0,
+                                 routing=ROUTING_EXPERT_CHOICE, bias_std=0.1),
+    "ec_gelu20": SWITCH_CAPACITY.replace(name="ec_gelu20", T=347, d_model=128, d_ff=192,
+                                         n_experts=20, capacity_factor=1.0, bias_std=0.1,
+                                         routing=ROUTING_EXPERT_CHOICE),
     "fp32_swiglu": DEEPSEEK_FINE.replace(name="fp32_swiglu", T=150, d_model=96, d_ff=160,
                                          n_experts=16, top_k=3, dtype=DT_F32,
                                          d_ff_shared=64),

@@ -141,3 +141,47 @@ def test_entry_points_reject_bad_pointers_before_launching(lib):
     code = ctypes.c_int32(0)
     assert lib.moe_last_device_error(None, ctypes.byref(code), None, None) == 1
     assert lib.moe_status_string(4) == b"workspace too small"
+
+
+@pytest.mark.parametrize("over,expect", [
+    ({}, B.MOE_OK),
+    ({"routing": 2}, 1),                           # no such routing
+    ({"capacity_factor": 0.0}, 1),                 # expert choice needs cf > 0
+    ({"capacity_factor": 0.001}, 1),               # C = 0: an expert would take nothing
+    ({"capacity_factor": 9.0}, 1),                 # C > T
+    ({"n_tokens": 40000, "capacity_factor": 0.1}, 2),   # T beyond one CTA's column
+    ({"capacity_factor": 8.0, "n_tokens": 16384}, 2),   # C = 16384 > 8192 picks
+    ({"n_shared": 2, "d_ff_shared": 8192}, 2),     # shared experts with expert choice
+])
+def test_expert_choice_config_validation(lib, over, expect):
+    cfg = B.make_cfg(synth.MIXTRAL_EC, **over)
+    st, n = _status(lib, cfg)
+    assert st == expect, (over, st)
+
+
+def test_expert_choice_workspace_holds_its_rows(lib):
+    """cf = 2 over 8 experts: 2T expert rows, twice top-1 token choice's."""
+    ec = _status(lib, B.make_cfg(synth.MIXTRAL_EC))[1]
+    tc = _status(lib, B.make_cfg(synth.MIXTRAL_EC, routing=0, capacity_factor=0.0))[1]
+    assert ec > tc
+
+
+def test_expert_choice_entry_points_reject_before_launching(lib):
+    wl = synth.SMALL["ec_small"]
+    cfg = B.make_cfg(wl)
+    ws_bytes = B.workspace_size(cfg)
+    ws = ctypes.c_void_p(0x100000)
+    good = ctypes.c_void_p(0x200000)
+    odd = ctypes.c_void_p(0x200008)
+    W = B.MoeWeights(w_router=good, w1=good, w3=good, w2=good)
+    route = lib.moe_route_expert_choice
+    assert route(ctypes.byref(cfg), ctypes.byref(W), None, None, good, good, ws, ws_bytes,
+                 None) == 1                          # logits input missing
+    assert route(ctypes.byref(cfg), ctypes.byref(W), None, good, odd, good, ws, ws_bytes,
+                 None) == 3                          # ec_idx misaligned
+    tc = B.make_cfg(wl, routing=0)
+    assert route(ctypes.byref(tc), ctypes.byref(W), None, good, good, good, ws,
+                 B.workspace_size(tc), None) == 1    # a token-choice configuration
+    # moe_forward: expert choice produces no load-balancing statistics
+    assert lib.moe_forward(ctypes.byref(cfg), ctypes.byref(W), good, good, good, None, ws,
+                           ws_bytes, None) == 1

@@ -402,7 +402,13 @@ def _routing_on_oracle_logits(wl, layer, inp, r):
     assert code == 0
 
 
-@pytest.mark.parametrize("name", sorted(synth.SMALL))
+TOKEN_CHOICE_SMALL = sorted(n for n, w in synth.SMALL.items()
+                            if w.routing == synth.ROUTING_TOKEN_CHOICE)
+EXPERT_CHOICE_SMALL = sorted(n for n, w in synth.SMALL.items()
+                             if w.routing == synth.ROUTING_EXPERT_CHOICE)
+
+
+@pytest.mark.parametrize("name", TOKEN_CHOICE_SMALL)
 def test_forward_small_matches_oracle(name):
     _forward_and_compare(synth.SMALL[name], seed=0)
 
@@ -436,3 +442,108 @@ def test_zero_tokens_is_a_noop():
     y = layer.forward(x)
     assert y.shape == (0, wl.d_model)
     assert layer.last_device_error() == (0, 0)
+
+
+# ============================================================ Expert-Choice routing
+EC_ROUTE_CASES = [
+    # E, T, cf (C = floor(cf * T / E))
+    (8, 300, 2.5), (20, 347, 1.0), (64, 1000, 1.0), (1, 64, 1.0), (3, 5000, 0.5),
+    (128, 4096, 1.0), (256, 2048, 3.0), (8, 32768, 2.0),
+]
+
+
+@pytest.mark.parametrize("E,T,cf", EC_ROUTE_CASES)
+def test_ec_route_given_logits_bitexact(E, T, cf):
+    """Each expert's picks (order included) are bit-exact and the scores match when
+    both sides see the same fp32 logits, ties included."""
+    wl = synth.SMALL["ec_small"].replace(T=T, n_experts=E, capacity_factor=cf)
+    C = O.expert_choice_capacity(cf, T, E)
+    z = synth.random_logits(T, E, seed=E * 7 + T, std=1.5, tie_fraction=0.3)
+    layer = B.MoELayer(wl, synth.generate(wl.replace(T=1), seed=0, with_weights=False), DEV)
+    logits = z.to(DEV)
+    idx = torch.empty((E, C), dtype=torch.int32, device=DEV)
+    score = torch.empty((E, C), dtype=torch.float32, device=DEV)
+    layer.route_expert_choice(None, logits, idx, score)
+    torch.cuda.synchronize()
+    zn = z.numpy()
+    ref_idx = O.expert_choice_select(zn, C)
+    assert np.array_equal(idx.cpu().numpy(), ref_idx)
+    ref_s = np.take_along_axis(O.expert_choice_scores(zn), ref_idx.astype(np.int64), axis=1)
+    assert np.allclose(score.cpu().numpy(), ref_s, rtol=2e-5, atol=1e-9)
+    _devcheck(layer.ws)
+
+
+def _ec_forward_and_compare(wl: synth.Workload, seed: int, n_sample=None):
+    inp = synth.generate(wl, seed=seed)
+    layer = B.MoELayer(wl, inp, DEV)
+    x = inp["x"].to(DEV)
+    taps = layer.new_taps()
+    y = layer.forward(x, taps=taps)
+    torch.cuda.synchronize()
+    code, info = layer.last_device_error()
+    assert code == 0, (code, info)
+    P = H.oracle_params(inp)
+    T, E = wl.T, wl.n_experts
+    tokens = None if n_sample is None else synth.token_sample(T, n_sample).numpy()
+    yref, r = O.expert_choice_forward(P["x"], P, capacity_factor=wl.capacity_factor,
+                                      act=H.ACT[wl.act], tokens=tokens)
+    extra = np.zeros(E)
+    if P["b_router"] is not None:
+        extra += np.abs(P["b_router"])
+    if P["logit_bias"] is not None:
+        extra += np.abs(P["logit_bias"])
+    zg = taps["logits"].cpu().numpy().astype(np.float64)
+    assert np.all(np.abs(zg - r["logits"]) <= H.logits_bound(P["x"], P["w_router"], extra))
+    # the forward's picks from its own logits: tokens within 1e-4 of an expert's
+    # C-th logit may be picked differently and are not compared
+    C = r["C"]
+    near = set()
+    zr = np.asarray(r["logits"], dtype=np.float64)
+    for e in range(E):
+        col = zr[:, e]
+        kth = np.sort(col)[::-1][C - 1]
+        near |= set(np.nonzero(np.abs(col - kth) < H.MARGIN)[0].tolist()) if C < T else set()
+    gidx = torch.empty((E, C), dtype=torch.int32, device=DEV)
+    gsc = torch.empty((E, C), dtype=torch.float32, device=DEV)
+    layer.route_expert_choice(None, taps["logits"], gidx, gsc)
+    torch.cuda.synchronize()
+    ref_own = O.expert_choice_select(taps["logits"].cpu().numpy(), C)
+    assert np.array_equal(gidx.cpu().numpy(), ref_own)  # bit-exact on the GPU's logits
+    sel = np.arange(T) if tokens is None else tokens
+    keep = np.array([t not in near for t in sel])
+    yg = y.cpu().to(torch.float64).numpy()[sel]
+    err = H.max_rel_err(yg[keep], yref[keep])
+    taken = np.zeros(T, dtype=bool)
+    taken[np.asarray(r["idx"]).ravel()] = True
+    H.report("forward_expert_choice", workload=wl.name, T=T, C=C, compared=int(keep.sum()),
+             near_tie_tokens=len(near), untaken_tokens=int((~taken).sum()),
+             worst_rel_err=float(err.max()) if len(err) else 0.0)
+    assert err.max() <= H.TOL[wl.dtype], (wl.name, float(err.max()))
+
+
+@pytest.mark.parametrize("name", EXPERT_CHOICE_SMALL)
+def test_ec_forward_small_matches_oracle(name):
+    _ec_forward_and_compare(synth.SMALL[name], seed=0)
+
+
+def test_ec_forward_full_size_sampled():
+    _ec_forward_and_compare(synth.WORKLOADS["mixtral_ec"], seed=0, n_sample=48)
+
+
+def test_ec_forward_is_deterministic():
+    wl = synth.SMALL["ec_gelu20"]
+    inp = synth.generate(wl, seed=4)
+    layer = B.MoELayer(wl, inp, DEV)
+    x = inp["x"].to(DEV)
+    y1 = layer.forward(x).clone()
+    y2 = layer.forward(x).clone()
+    torch.cuda.synchronize()
+    assert torch.equal(y1, y2)
+
+
+def test_ec_forward_rejects_aux():
+    wl = synth.SMALL["ec_small"]
+    layer = B.MoELayer(wl, synth.generate(wl, seed=1), DEV)
+    x = torch.zeros((wl.T, wl.d_model), dtype=wl.torch_dtype, device=DEV)
+    with pytest.raises(B.MoeError):
+        layer.forward(x, aux=layer.new_aux())
