@@ -281,20 +281,31 @@ __global__ void __launch_bounds__(256) k_ec_combine(const ET *__restrict__ y_per
     for (int b = 0; b < 2; ++b)
 #pragma unroll
       for (int i = 0; i < VE; ++i) acc[b][i] = 0.f;
-    for (int i = 0; i < n; ++i) {
-      const int row = l_row[warp][i];
-      const float g = l_g[warp][i];
-      const uint4 *src = reinterpret_cast<const uint4 *>(y_perm + (size_t)row * d);
-      uint4 u[2];
+    // two experts' rows requested together (four 16-byte loads in flight per lane),
+    // then added in expert order
+    for (int i = 0; i < n; i += 2) {
+      const bool two = i + 1 < n;
+      uint4 u[2][2];
 #pragma unroll
-      for (int b = 0; b < 2; ++b)
-        u[b] = (v0 + 32 * b < nvec) ? __ldg(src + v0 + 32 * b) : make_uint4(0u, 0u, 0u, 0u);
+      for (int h = 0; h < 2; ++h) {
+        const int row = l_row[warp][two || h == 0 ? i + h : i];
+        const uint4 *src = reinterpret_cast<const uint4 *>(y_perm + (size_t)row * d);
 #pragma unroll
-      for (int b = 0; b < 2; ++b) {
-        float f[VE];
-        unpack16(u[b], f);
+        for (int b = 0; b < 2; ++b)
+          u[h][b] = ((h == 0 || two) && v0 + 32 * b < nvec) ? __ldg(src + v0 + 32 * b)
+                                                             : make_uint4(0u, 0u, 0u, 0u);
+      }
 #pragma unroll
-        for (int q = 0; q < VE; ++q) acc[b][q] = fmaf(g, f[q], acc[b][q]);
+      for (int h = 0; h < 2; ++h) {
+        if (h == 1 && !two) break;
+        const float g = l_g[warp][i + h];
+#pragma unroll
+        for (int b = 0; b < 2; ++b) {
+          float f[VE];
+          unpack16(u[h][b], f);
+#pragma unroll
+          for (int q = 0; q < VE; ++q) acc[b][q] = fmaf(g, f[q], acc[b][q]);
+        }
       }
     }
 #pragma unroll

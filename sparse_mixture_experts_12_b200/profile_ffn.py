@@ -30,11 +30,20 @@ def main(argv=None) -> int:
     layer = B.MoELayer(wl, inp, dev)
     x = inp["x"].to(dev)
     T, E, k, d = wl.T, wl.n_experts, wl.top_k, wl.d_model
-    taps = layer.new_taps()
-    layer.route(x, taps["logits"], taps["topk_idx"], taps["topk_gate"])
-    xp = torch.empty((T * k, d), dtype=wl.torch_dtype, device=dev)
-    off = torch.empty(E + 1, dtype=torch.int32, device=dev)
-    layer.permute(x, taps["topk_idx"], taps["counts"], off, taps["perm"], taps["inv"], xp)
+    if wl.routing == synth.ROUTING_EXPERT_CHOICE:  # each expert's C picked rows
+        C = int(wl.capacity_factor * T // E)
+        logits = torch.empty((T, E), dtype=torch.float32, device=dev)
+        idx = torch.empty((E, C), dtype=torch.int32, device=dev)
+        score = torch.empty((E, C), dtype=torch.float32, device=dev)
+        layer.route_expert_choice(x, logits, idx, score)
+        xp = x[idx.reshape(-1).long()].contiguous()
+        off = (torch.arange(E + 1, dtype=torch.int32, device=dev) * C).contiguous()
+    else:
+        taps = layer.new_taps()
+        layer.route(x, taps["logits"], taps["topk_idx"], taps["topk_gate"])
+        xp = torch.empty((T * k, d), dtype=wl.torch_dtype, device=dev)
+        off = torch.empty(E + 1, dtype=torch.int32, device=dev)
+        layer.permute(x, taps["topk_idx"], taps["counts"], off, taps["perm"], taps["inv"], xp)
     yp = torch.empty_like(xp)
     torch.cuda.synchronize()
     for _ in range(args.reps):
