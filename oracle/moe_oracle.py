@@ -40,6 +40,8 @@ test):
 * f_i counts pre-drop assignments over T*k; P_i is the mean full softmax of the
   router logits (router bias and logit bias included).
 * GELU is the exact erf form; dropout and routing noise are off (inference).
+* Noisy top-k gating (training mode of P4 ``TopKGating``): the standard normal
+  draws eps [T, E] are an input, so both sides see the same draws.
 * Expert-Choice routing: each expert takes int(cf * T / E) tokens, chosen on the
   fp32 logits (equal logits: lower token index first); a token's output is the
   score-weighted sum over the experts that took it (P4's dispatch mask used as
@@ -450,3 +452,26 @@ def expert_choice_margin(logits32, C: int) -> np.ndarray:
         v = np.sort(z[:, e])[::-1]
         out[e] = v[C - 1] - v[C]
     return out
+
+
+# ----------------------------------------------------------------- noisy top-k gating
+def softplus(v):
+    """softplus(v) = log(1 + e^v), fp64 (``F.softplus`` of P4 ``TopKGating``, whose
+    default switches to the identity above 20)."""
+    v = _f64(v)
+    return np.where(v > 20.0, v, np.log1p(np.exp(np.minimum(v, 20.0))))
+
+
+def noisy_router_logits(x, w_router, w_noise, eps, b_router=None,
+                        logit_bias=None) -> np.ndarray:
+    """Training-mode logits of P4 ``TopKGating`` (Noisy Top-K Gating):
+    z + softplus(x W_noise^T) * eps, with z the plain router logits and eps [T, E]
+    the standard normal draws (passed in), exact in fp64, rounded once to fp32."""
+    x = _f64(x)
+    z = x @ _f64(w_router).T
+    if b_router is not None:
+        z = z + _f64(b_router)[None, :]
+    if logit_bias is not None:
+        z = z + _f64(logit_bias)[None, :]
+    zn = x @ _f64(w_noise).T
+    return (z + softplus(zn) * _f64(eps)).astype(np.float32)

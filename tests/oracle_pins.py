@@ -426,9 +426,34 @@ def check_expert_choice_dense(O):
             assert (dispatch.sum(dim=0) == 0).any() or r["C"] * E >= T
 
 
+# -------------------------------------------------------------- noisy top-k gating
+def check_noisy_logits(O):
+    """P4 ``TopKGating`` training logits: zero noise gives the plain router; a zero
+    noise projection adds ln(2) * eps; the noise term is linear in eps; softplus
+    against torch's, including its switch to the identity above 20."""
+    rng = np.random.default_rng(8)
+    T, d, E = 7, 6, 5
+    x = rng.integers(-3, 4, size=(T, d)).astype(np.float64)
+    wr = rng.integers(-2, 3, size=(E, d)).astype(np.float64) / 4
+    wn = rng.integers(-2, 3, size=(E, d)).astype(np.float64) / 8
+    eps = rng.normal(size=(T, E))
+    plain = O.router_logits(x, wr)
+    assert np.array_equal(O.noisy_router_logits(x, wr, wn, np.zeros((T, E))), plain)
+    z0 = O.noisy_router_logits(x, wr, np.zeros((E, d)), eps)
+    assert np.allclose(z0, (x @ wr.T + math.log(2.0) * eps).astype(np.float32), rtol=0,
+                       atol=1e-6)
+    z1 = O.noisy_router_logits(x, wr, wn, eps).astype(np.float64) - plain
+    z2 = O.noisy_router_logits(x, wr, wn, 2 * eps).astype(np.float64) - plain
+    assert np.allclose(z2, 2 * z1, rtol=1e-6, atol=1e-5)
+    v = np.array([-30.0, -3.0, -0.5, 0.0, 0.5, 3.0, 19.9, 20.0, 20.5, 40.0])
+    ref = F.softplus(torch.as_tensor(v)).numpy()
+    assert np.allclose(O.softplus(v), ref, rtol=1e-15, atol=1e-300)
+    assert O.softplus(np.array([0.0]))[0] == math.log(2.0)
+
+
 ALL_CHECKS = [check_combine, check_topk_bruteforce, check_gate_sums_and_ranges, check_worked_gates,
               check_softmax_closed_forms, check_router_logits_exact, check_capacity_golden,
               check_counts_and_drop_order, check_layout, check_forward_vs_pages_torch,
               check_sparse_equals_dense_masked, check_special_cases, check_aux_closed_forms,
               check_expert_choice_capacity, check_expert_choice_bruteforce,
-              check_expert_choice_scores, check_expert_choice_dense]
+              check_expert_choice_scores, check_expert_choice_dense, check_noisy_logits]

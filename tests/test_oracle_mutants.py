@@ -128,7 +128,18 @@ def _ec_forward_ignores_scores(x, params, *, capacity_factor, act, logits=None, 
         O.expert_choice_scores = orig
 
 
+def _softplus_is_exp(v):
+    return np.exp(np.asarray(v, dtype=np.float64))
+
+
+def _noise_sign_flipped(x, w_router, w_noise, eps, b_router=None, logit_bias=None):
+    return _orig["noisy_router_logits"](x, w_router, w_noise, -np.asarray(eps), b_router,
+                                        logit_bias)
+
+
 MUTANTS = {
+    "softplus_is_exp": ("softplus", _softplus_is_exp),
+    "noise_sign_flipped": ("noisy_router_logits", _noise_sign_flipped),
     "ec_softmax_over_experts": ("expert_choice_scores", _ec_softmax_over_experts),
     "ec_ties_to_higher_token": ("expert_choice_select", _ec_ties_to_higher_token),
     "ec_capacity_rounds_up": ("expert_choice_capacity", _ec_capacity_rounds_up),
