@@ -132,6 +132,8 @@ typedef struct {
   const void *ws_gate;      /* [n_shared*F_sh, d] dtype: shared experts' w_gate, concatenated */
   const void *ws_up;        /* [n_shared*F_sh, d] dtype */
   const void *ws_down;      /* [d, n_shared*F_sh] dtype */
+  const void *w_noise;      /* [E, d]  dtype: noise projection of noisy top-k gating
+                               (moe_route_noisy / moe_forward_noisy), else NULL */
 } moe_weights_t;
 
 /* Optional device buffers that moe_forward fills with its intermediates
@@ -232,6 +234,22 @@ moe_status_t moe_aux_stats(const moe_cfg_t *cfg, const float *logits, const int3
 moe_status_t moe_forward(const moe_cfg_t *cfg, const moe_weights_t *w, const void *x, void *y,
                          float *aux_out, const moe_taps_t *taps, void *ws, size_t ws_bytes,
                          moe_stream_t stream);
+
+/* Noisy top-k gating, the training mode of youngju.dev (ja) "TopKGating" (Noisy Top-K
+ * Gating): the logits are z + softplus(x W_noise^T) * eps, z as in moe_route, softplus
+ * the identity above 20 (as F.softplus), eps [T, E] fp32 standard normal draws made by
+ * the caller (device memory); then selection and gates exactly as moe_route on those
+ * logits (cfg->gate_mode; the page's mode is MOE_GATE_SOFTMAX_TOPK_RENORM). logits
+ * [T, E] fp32 receives the noisy logits. Token-choice configurations only. */
+moe_status_t moe_route_noisy(const moe_cfg_t *cfg, const moe_weights_t *w, const void *x,
+                             const float *eps, float *logits, int32_t *topk_idx,
+                             float *topk_gate, void *ws, size_t ws_bytes, moe_stream_t stream);
+
+/* moe_forward with noisy top-k gating (see moe_route_noisy): the whole layer, routed
+ * on the noisy logits; aux_out and the logits tap see the noisy logits. */
+moe_status_t moe_forward_noisy(const moe_cfg_t *cfg, const moe_weights_t *w, const void *x,
+                               const float *eps, void *y, float *aux_out, const moe_taps_t *taps,
+                               void *ws, size_t ws_bytes, moe_stream_t stream);
 
 /* Expert-Choice routing step (youngju.dev (zh) "ExpertChoiceRouter", youngju.dev (ja)
  * "ExpertChoiceGating"): logits as in moe_route, then for every expert e its C =

@@ -26,8 +26,8 @@ STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED",
 DEVERR_NAMES = {0: "none", 1: "expert index out of range", 2: "invalid offsets",
                 3: "row index out of range", 4: "pipeline wait timeout"}
 
-EXPORTED = ("moe_workspace_size", "moe_workspace_init", "moe_route", "moe_route_expert_choice",
-            "moe_permute", "moe_permute_noalloc",
+EXPORTED = ("moe_workspace_size", "moe_workspace_init", "moe_route", "moe_route_noisy",
+            "moe_route_expert_choice", "moe_permute", "moe_permute_noalloc", "moe_forward_noisy",
             "moe_expert_ffn", "moe_combine", "moe_aux_stats", "moe_forward",
             "moe_last_device_error", "moe_status_string")
 
@@ -51,7 +51,7 @@ class MoeCfg(ctypes.Structure):
 class MoeWeights(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in
                 ("w_router", "b_router", "logit_bias", "w1", "w3", "w2", "b1", "b2",
-                 "ws_gate", "ws_up", "ws_down")]
+                 "ws_gate", "ws_up", "ws_down", "w_noise")]
 
 
 class MoeTaps(ctypes.Structure):
@@ -167,6 +167,22 @@ class MoELayer:
                                     _ptr(self.ws), self.ws.numel(), _stream()), "moe_forward")
         return y
 
+    def forward_noisy(self, x: torch.Tensor, eps: torch.Tensor, y: Optional[torch.Tensor] = None,
+                      aux: Optional[torch.Tensor] = None,
+                      taps: Optional[dict] = None) -> torch.Tensor:
+        """The layer with noisy top-k gating; eps [T, E] fp32 standard normal draws."""
+        if y is None:
+            y = torch.empty_like(x)
+        tp = None
+        if taps is not None:
+            tp = MoeTaps(**{k: _ptr(taps.get(k)) for k, _ in MoeTaps._fields_})
+        _check(self.lib.moe_forward_noisy(ctypes.byref(self.cfg), ctypes.byref(self.weights),
+                                          _ptr(x), _ptr(eps), _ptr(y), _ptr(aux),
+                                          ctypes.byref(tp) if tp is not None else None,
+                                          _ptr(self.ws), self.ws.numel(), _stream()),
+               "moe_forward_noisy")
+        return y
+
     def new_taps(self) -> dict:
         T, E, k = self.w.T, self.w.n_experts, self.w.top_k
         dev = self.device
@@ -186,6 +202,13 @@ class MoELayer:
         _check(self.lib.moe_route(ctypes.byref(self.cfg), ctypes.byref(self.weights), _ptr(x),
                                   _ptr(logits), _ptr(topk_idx), _ptr(topk_gate), _ptr(self.ws),
                                   self.ws.numel(), _stream()), "moe_route")
+
+    def route_noisy(self, x: torch.Tensor, eps: torch.Tensor, logits: torch.Tensor,
+                    topk_idx: torch.Tensor, topk_gate: torch.Tensor):
+        _check(self.lib.moe_route_noisy(ctypes.byref(self.cfg), ctypes.byref(self.weights),
+                                        _ptr(x), _ptr(eps), _ptr(logits), _ptr(topk_idx),
+                                        _ptr(topk_gate), _ptr(self.ws), self.ws.numel(),
+                                        _stream()), "moe_route_noisy")
 
     def route_expert_choice(self, x: Optional[torch.Tensor], logits: torch.Tensor,
                             ec_idx: torch.Tensor, ec_score: torch.Tensor):

@@ -100,6 +100,9 @@ cudaError_t launch_ec_combine(const void *y_perm, const int32_t *slot, const flo
                               int T, int E, int C, int d, int dtype, void *y, cudaStream_t st);
 
 cudaError_t launch_router(const RouterArgs &a, int dtype, cudaStream_t st);
+// noisy top-k gating: z[i] += softplus(zn[i]) * eps[i] over n logits
+cudaError_t launch_noisy_logits(float *z, const float *zn, const float *eps, size_t n,
+                                cudaStream_t st);
 // bf16 router on the tensor cores (x given, 16 <= E <= 256)
 cudaError_t launch_router_tc(const RouterArgs &a, cudaStream_t st);
 cudaError_t launch_tile_counts(const int32_t *topk_idx, int T, int k, int E, int32_t *tile_counts,

@@ -15,7 +15,7 @@ namespace {
 enum Buf {
   B_ERR, B_TILE_COUNTS, B_TILE_BASE, B_TILE_P, B_TILE_Z, B_COUNTS, B_OFFSETS, B_MPREFIX, B_SH_TBL,
   B_LOGITS, B_IDX, B_GATE, B_PERM, B_INV, B_XPERM, B_H, B_YPERM, B_SH_H, B_SH_Y, B_YPART,
-  B_EC_ZT, B_EC_IDX, B_EC_SCORE, B_EC_SLOT, B_NBUF
+  B_EC_ZT, B_EC_IDX, B_EC_SCORE, B_EC_SLOT, B_NOISE, B_NBUF
 };
 
 struct Layout {
@@ -80,6 +80,7 @@ Layout layout_for(const moe_cfg_t &c) {
   sz[B_EC_IDX] = ec ? E * C * 4 : 0;
   sz[B_EC_SCORE] = ec ? E * C * 4 : 0;
   sz[B_EC_SLOT] = ec ? T * E * 4 : 0;
+  sz[B_NOISE] = T * E * 4;  // x W_noise^T of noisy top-k gating
   Layout L;
   size_t o = 0;
   for (int i = 0; i < B_NBUF; ++i) {
@@ -231,6 +232,36 @@ GroupedFfnArgs routed_ffn_args(const moe_cfg_t &c, const moe_weights_t &w, const
   return a;
 }
 
+// Noisy top-k gating logits: z (router, biases) + softplus(x W_noise^T) * eps, into
+// `logits`; the two router passes' own selections go to scratch.
+moe_status_t noisy_logits(const moe_cfg_t &c, const moe_weights_t *w, const void *x,
+                          const float *eps, float *logits, void *ws, const Layout &L,
+                          cudaStream_t stream) {
+  RouterArgs r{};
+  r.x = x;
+  r.w = w->w_router;
+  r.b_router = w->b_router;
+  r.logit_bias = w->logit_bias;
+  r.logits_out = logits;
+  r.topk_idx = at<int32_t>(ws, L, B_IDX);
+  r.topk_gate = at<float>(ws, L, B_GATE);
+  r.T = c.n_tokens;
+  r.d = c.d_model;
+  r.E = c.n_experts;
+  r.k = c.top_k;
+  r.gate_mode = c.gate_mode;
+  r.err = at<int32_t>(ws, L, B_ERR);
+  MOE_CUDA(launch_router(r, c.dtype, stream));
+  float *zn = at<float>(ws, L, B_NOISE);
+  r.w = w->w_noise;
+  r.b_router = nullptr;
+  r.logit_bias = nullptr;
+  r.logits_out = zn;
+  MOE_CUDA(launch_router(r, c.dtype, stream));
+  MOE_CUDA(launch_noisy_logits(logits, zn, eps, (size_t)c.n_tokens * c.n_experts, stream));
+  return MOE_OK;
+}
+
 // Expert-Choice routing: router logits (unless x is NULL: logits are the input),
 // then every expert's picks. slot/offsets (nullable) feed the forward's later steps.
 moe_status_t ec_route(const moe_cfg_t &c, const moe_weights_t *w, const void *x, float *logits,
@@ -338,6 +369,36 @@ MOE_API moe_status_t moe_route(const moe_cfg_t *cfg, const moe_weights_t *w, con
   r.logit_bias = w->logit_bias;
   r.logits_in = x ? nullptr : logits;
   r.logits_out = x ? logits : nullptr;
+  r.topk_idx = topk_idx;
+  r.topk_gate = topk_gate;
+  r.tile_counts = at<int32_t>(ws, L, B_TILE_COUNTS);
+  r.T = c.n_tokens;
+  r.d = c.d_model;
+  r.E = c.n_experts;
+  r.k = c.top_k;
+  r.gate_mode = c.gate_mode;
+  r.err = at<int32_t>(ws, L, B_ERR);
+  MOE_CUDA(launch_router(r, c.dtype, stream));
+  return MOE_OK;
+}
+
+MOE_API moe_status_t moe_route_noisy(const moe_cfg_t *cfg, const moe_weights_t *w,
+                                     const void *x, const float *eps, float *logits,
+                                     int32_t *topk_idx, float *topk_gate, void *ws,
+                                     size_t ws_bytes, moe_stream_t stream) {
+  MOE_TRY(check_cfg(cfg));
+  MOE_TRY(check_ws(cfg, ws, ws_bytes));
+  if (expert_choice(*cfg)) return MOE_ERR_INVALID_ARG;
+  if (cfg->n_tokens == 0) return MOE_OK;
+  if (w == nullptr) return MOE_ERR_INVALID_ARG;
+  MOE_TRY(check_ptrs({{x, true}, {eps, true}, {logits, true}, {topk_idx, true},
+                      {topk_gate, true}, {w->w_router, true}, {w->w_noise, true},
+                      {w->b_router, false}, {w->logit_bias, false}}));
+  const moe_cfg_t &c = *cfg;
+  const Layout L = layout_for(c);
+  MOE_TRY(noisy_logits(c, w, x, eps, logits, ws, L, stream));
+  RouterArgs r{};
+  r.logits_in = logits;
   r.topk_idx = topk_idx;
   r.topk_gate = topk_gate;
   r.tile_counts = at<int32_t>(ws, L, B_TILE_COUNTS);
@@ -510,9 +571,12 @@ MOE_API moe_status_t moe_aux_stats(const moe_cfg_t *cfg, const float *logits,
   return MOE_OK;
 }
 
-MOE_API moe_status_t moe_forward(const moe_cfg_t *cfg, const moe_weights_t *w, const void *x,
-                                 void *y, float *aux_out, const moe_taps_t *taps, void *ws,
-                                 size_t ws_bytes, moe_stream_t stream) {
+namespace moe {
+namespace {
+// the whole layer; eps != NULL: noisy top-k gating (token choice only)
+moe_status_t forward_impl(const moe_cfg_t *cfg, const moe_weights_t *w, const void *x,
+                          const float *eps, void *y, float *aux_out, const moe_taps_t *taps,
+                          void *ws, size_t ws_bytes, moe_stream_t stream) {
   MOE_TRY(check_cfg(cfg));
   MOE_TRY(check_ws(cfg, ws, ws_bytes));
   if (cfg->n_tokens == 0) return MOE_OK;  // nothing is read or written
@@ -533,9 +597,10 @@ MOE_API moe_status_t moe_forward(const moe_cfg_t *cfg, const moe_weights_t *w, c
   int32_t *err = at<int32_t>(ws, L, B_ERR);
   float *logits = tp.logits ? tp.logits : at<float>(ws, L, B_LOGITS);
   if (expert_choice(c)) {
-    if (aux_out != nullptr) return MOE_ERR_INVALID_ARG;
+    if (aux_out != nullptr || eps != nullptr) return MOE_ERR_INVALID_ARG;
     return ec_forward(c, w, x, y, logits, ws, L, stream);
   }
+  if (eps != nullptr) MOE_TRY(check_ptrs({{eps, true}, {w->w_noise, true}}));
   int32_t *idx = tp.topk_idx ? tp.topk_idx : at<int32_t>(ws, L, B_IDX);
   float *gate = tp.topk_gate ? tp.topk_gate : at<float>(ws, L, B_GATE);
   int32_t *counts = tp.counts ? tp.counts : at<int32_t>(ws, L, B_COUNTS);
@@ -546,13 +611,19 @@ MOE_API moe_status_t moe_forward(const moe_cfg_t *cfg, const moe_weights_t *w, c
   int32_t *sh_tbl = at<int32_t>(ws, L, B_SH_TBL);
   const bool want_aux = aux_out != nullptr;
 
-  // 1. router GEMM + softmax + top-k + gates + per-tile histogram
+  // 1. router GEMM + softmax + top-k + gates + per-tile histogram (noisy gating:
+  //    the noisy logits first, then the same steps on them as the input)
   RouterArgs r{};
-  r.x = x;
-  r.w = w->w_router;
-  r.b_router = w->b_router;
-  r.logit_bias = w->logit_bias;
-  r.logits_out = (tp.logits || want_aux) ? logits : nullptr;
+  if (eps != nullptr) {
+    MOE_TRY(noisy_logits(c, w, x, eps, logits, ws, L, stream));
+    r.logits_in = logits;
+  } else {
+    r.x = x;
+    r.w = w->w_router;
+    r.b_router = w->b_router;
+    r.logit_bias = w->logit_bias;
+    r.logits_out = (tp.logits || want_aux) ? logits : nullptr;
+  }
   r.topk_idx = idx;
   r.topk_gate = gate;
   r.tile_counts = at<int32_t>(ws, L, B_TILE_COUNTS);
@@ -645,6 +716,22 @@ MOE_API moe_status_t moe_forward(const moe_cfg_t *cfg, const moe_weights_t *w, c
   cb.err = err;
   MOE_CUDA(launch_combine(cb, c.dtype, stream));
   return MOE_OK;
+}
+}  // namespace
+}  // namespace moe
+
+MOE_API moe_status_t moe_forward(const moe_cfg_t *cfg, const moe_weights_t *w, const void *x,
+                                 void *y, float *aux_out, const moe_taps_t *taps, void *ws,
+                                 size_t ws_bytes, moe_stream_t stream) {
+  return forward_impl(cfg, w, x, nullptr, y, aux_out, taps, ws, ws_bytes, stream);
+}
+
+MOE_API moe_status_t moe_forward_noisy(const moe_cfg_t *cfg, const moe_weights_t *w,
+                                       const void *x, const float *eps, void *y,
+                                       float *aux_out, const moe_taps_t *taps, void *ws,
+                                       size_t ws_bytes, moe_stream_t stream) {
+  if (eps == nullptr) return MOE_ERR_INVALID_ARG;
+  return forward_impl(cfg, w, x, eps, y, aux_out, taps, ws, ws_bytes, stream);
 }
 
 MOE_API moe_status_t moe_last_device_error(void *ws, int32_t *code, int32_t *info,

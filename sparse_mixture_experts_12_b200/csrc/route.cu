@@ -589,6 +589,28 @@ cudaError_t launch_router(const RouterArgs &a, int dtype, cudaStream_t st) {
   return launch_router_e<256>(a, dtype, st);
 }
 
+// Noisy Top-K Gating (youngju.dev (ja) "TopKGating", training mode): the router
+// logits plus softplus(x W_noise^T) times the caller's standard normal draws.
+// softplus switches to the identity above 20, as F.softplus does.
+__global__ void __launch_bounds__(256) k_noisy_logits(float *__restrict__ z,
+                                                      const float *__restrict__ zn,
+                                                      const float *__restrict__ eps, size_t n) {
+  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+       i += (size_t)gridDim.x * blockDim.x) {
+    const float v = zn[i];
+    const float sp = v > 20.f ? v : log1pf(expf(v));
+    z[i] = z[i] + sp * eps[i];
+  }
+}
+
+cudaError_t launch_noisy_logits(float *z, const float *zn, const float *eps, size_t n,
+                                cudaStream_t st) {
+  if (n == 0) return cudaSuccess;
+  const size_t blocks = std::min<size_t>((n + 255) / 256, 148 * 16);
+  k_noisy_logits<<<(unsigned)blocks, 256, 0, st>>>(z, zn, eps, n);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_tile_counts(const int32_t *topk_idx, int T, int k, int E, int32_t *tile_counts,
                                int32_t *err, cudaStream_t st) {
   if (T == 0) return cudaSuccess;

@@ -17,6 +17,8 @@ seeded with ``seed``; every draw is fp32 ``normal_`` in this fixed order):
 7. per shared expert j: gate [F_sh, d], up [F_sh, d], down [d, F_sh] ~ N(0, 1/fan_in);
    the shared experts are stored concatenated along F_sh
    (``ws_gate``/``ws_up`` [n_sh*F_sh, d], ``ws_down`` [d, n_sh*F_sh]).
+8. ``w_noise`` [E, d] ~ N(0, 0.02^2) (noisy gating only); the noise draws eps
+   [T, E] ~ N(0, 1) come from ``noise_draws`` with a seed of their own.
 
 Weights and activations are then rounded once (round-to-nearest-even) to the
 workload's storage dtype (bf16 or fp32). Biases and ``logit_bias`` stay fp32.
@@ -65,6 +67,7 @@ class Workload:
     router_std: float = 0.02
     bias_std: float = 0.0
     routing: int = ROUTING_TOKEN_CHOICE  # expert choice: C = floor(cf * T / E) per expert
+    noisy: bool = False  # noisy top-k gating: draws w_noise (the draws of eps are separate)
 
     def replace(self, **kw) -> "Workload":
         return dataclasses.replace(self, **kw)
@@ -133,6 +136,13 @@ SMALL = {
     # SwiGLU experts with a capacity of 112 rows each
     "mixtral_cap": MIXTRAL_PREFILL.replace(name="mixtral_cap", T=900, d_model=256, d_ff=384,
                                            capacity_factor=0.5),
+    # noisy top-k gating (softmax, top-2, renormalised, as the ja page's TopKGating):
+    # bf16 with 16 experts (tensor-core router), fp32 with 8 (CUDA-core router)
+    "noisy_small": MIXTRAL_PREFILL.replace(name="noisy_small", T=500, d_model=256, d_ff=128,
+                                           n_experts=16, gate_mode=GATE_SOFTMAX_TOPK_RENORM,
+                                           noisy=True),
+    "noisy_fp32": TINY_FP32.replace(name="noisy_fp32", T=100, gate_mode=GATE_SOFTMAX_TOPK_RENORM,
+                                    noisy=True, bias_std=0.1),
     # bf16 routers with 20 and 256 experts (expert counts that pad to the MMA's N),
     # router and logit biases, ragged token tiles
     "router_e20": DEEPSEEK_FINE.replace(name="router_e20", T=700, d_model=256, d_ff=128,
@@ -209,7 +219,16 @@ def generate(w: Workload, seed: int = 0, with_weights: bool = True) -> dict:
         out["ws_gate"], out["ws_up"], out["ws_down"] = gate, up, down
     else:
         out["ws_gate"] = out["ws_up"] = out["ws_down"] = None
+    # 8. (noisy gating only) the noise projection, drawn last so that every other
+    #    draw is the same with and without it
+    out["w_noise"] = _normal(g, (E, d), w.router_std).to(dt) if w.noisy else None
     return out
+
+
+def noise_draws(T: int, E: int, seed: int) -> torch.Tensor:
+    """Standard normal draws eps [T, E] fp32 of noisy top-k gating, seeded."""
+    g = torch.Generator().manual_seed(seed)
+    return _normal(g, (T, E), 1.0)
 
 
 def random_logits(T: int, E: int, seed: int = 0, std: float = 1.0,

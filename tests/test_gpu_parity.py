@@ -325,14 +325,22 @@ def _forward_and_compare(wl: synth.Workload, seed: int, n_sample=None, check_ful
     x = inp["x"].to(DEV)
     taps = layer.new_taps()
     aux = layer.new_aux()
-    y = layer.forward(x, taps=taps, aux=aux)
+    eps = synth.noise_draws(wl.T, wl.n_experts, seed + 99) if wl.noisy else None
+    if eps is None:
+        y = layer.forward(x, taps=taps, aux=aux)
+    else:
+        y = layer.forward_noisy(x, eps.to(DEV), taps=taps, aux=aux)
     torch.cuda.synchronize()
     code, info = layer.last_device_error()
     assert code == 0, (code, info)
     P = H.oracle_params(inp)
     T, E, k = wl.T, wl.n_experts, wl.top_k
     tokens = None if n_sample is None else synth.token_sample(T, n_sample).numpy()
-    yref, r = O.moe_forward(P["x"], P, tokens=tokens, **H.oracle_kwargs(wl))
+    ref_logits = None
+    if eps is not None:
+        ref_logits = O.noisy_router_logits(P["x"], P["w_router"], P["w_noise"], eps.numpy(),
+                                           P["b_router"], P["logit_bias"])
+    yref, r = O.moe_forward(P["x"], P, tokens=tokens, logits=ref_logits, **H.oracle_kwargs(wl))
     # logits against the fp32 accumulation bound
     extra = np.zeros(E)
     if P["b_router"] is not None:
@@ -340,8 +348,25 @@ def _forward_and_compare(wl: synth.Workload, seed: int, n_sample=None, check_ful
     if P["logit_bias"] is not None:
         extra += np.abs(P["logit_bias"])
     bound = H.logits_bound(P["x"], P["w_router"], extra)
+    if eps is not None:  # + |eps| (bound of x W_noise^T + softplus rounding) + final roundings
+        e64 = eps.numpy().astype(np.float64)
+        zn = P["x"] @ P["w_noise"].T
+        sp = O.softplus(zn)
+        zpl = P["x"] @ P["w_router"].T
+        bound = bound + np.abs(e64) * (H.logits_bound(P["x"], P["w_noise"]) + 8 * H.U32 * sp) \
+            + 4 * H.U32 * (np.abs(zpl) + extra[None, :] + sp * np.abs(e64))
     zg = taps["logits"].cpu().numpy().astype(np.float64)
     assert np.all(np.abs(zg - r["logits"]) <= bound)
+    if eps is not None:  # the forward's selection, on its own noisy logits, is bit-exact
+        gi = torch.empty((T, k), dtype=torch.int32, device=DEV)
+        gg = torch.empty((T, k), dtype=torch.float32, device=DEV)
+        layer.route(None, taps["logits"], gi, gg)
+        torch.cuda.synchronize()
+        assert torch.equal(gi, taps["topk_idx"])
+        li = torch.empty((T, E), dtype=torch.float32, device=DEV)
+        layer.route_noisy(x, eps.to(DEV), li, gi, gg)
+        torch.cuda.synchronize()
+        assert torch.equal(li, taps["logits"]) and torch.equal(gi, taps["topk_idx"])
     # the forward's own routing: differences only on near-ties
     gidx = taps["topk_idx"].cpu().numpy()
     mism, affected, n_near = H.routing_compare(gidx, r["logits"], r["idx"], k, r["capacity"])
