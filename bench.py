@@ -205,8 +205,13 @@ def oracle_sample_rate(wl, inp, n_tokens: int):
     kw = dict(top_k=wl.top_k, act=acts[wl.act], gate_mode=modes[wl.gate_mode],
               capacity_factor=wl.capacity_factor, n_shared=wl.n_shared)
     t0 = time.perf_counter()
+    noisy = None
+    if wl.noisy:  # the same seeded draws as the GPU arm
+        eps = synth.noise_draws(wl.T, wl.n_experts, 99).numpy()
+        noisy = O.noisy_router_logits(P["x"], P["w_router"], P["w_noise"], eps,
+                                      P.get("b_router"), P.get("logit_bias"))
     r = O.route(P["x"], P, top_k=wl.top_k, gate_mode=kw["gate_mode"],
-                capacity_factor=wl.capacity_factor)
+                capacity_factor=wl.capacity_factor, logits=noisy)
     t_route = time.perf_counter() - t0
     toks = synth.token_sample(wl.T, n_tokens).numpy()
     t0 = time.perf_counter()
@@ -251,8 +256,8 @@ def _config(wl, world):
     return {"workload": wl.name, "T": wl.T, "d_model": wl.d_model, "n_experts": wl.n_experts,
             "top_k": wl.top_k, "d_ff": wl.d_ff, "n_shared": wl.n_shared,
             "d_ff_shared": wl.d_ff_shared, "capacity_factor": wl.capacity_factor,
-            "routing": "expert choice" if wl.routing == synth.ROUTING_EXPERT_CHOICE
-            else "token choice",
+            "routing": ("expert choice" if wl.routing == synth.ROUTING_EXPERT_CHOICE
+                        else "token choice") + (", noisy gating" if wl.noisy else ""),
             "global_batch": wl.T * world, "seq_len": wl.T,
             "parallelism": f"dp{world} (independent token batches, no data-path collective)",
             "l2": "working set > L2 (weights >= 2.8 GB per step); no flush"}
@@ -333,17 +338,25 @@ def run_ours(args, wl, rank, world, local_rank):
     want_aux = wl.capacity_factor > 0 and not ec
     aux = layer.new_aux() if want_aux else None
     stream = torch.cuda.current_stream()
+    # noisy gating: the step routes on logits + softplus(x W_noise^T) * eps; the draws
+    # eps are made once (seeded) and stay resident, like x
+    eps = synth.noise_draws(wl.T, wl.n_experts, 99 + rank).to(dev) if wl.noisy else None
+
+    def forward(xx, yy, aa, taps=None):
+        if eps is None:
+            return layer.forward(xx, yy, aa, taps=taps)
+        return layer.forward_noisy(xx, eps, yy, aa, taps=taps)
 
     clocks = ClockSampler(local_rank)
     clocks.start()
     for _ in range(args.warmup):
-        layer.forward(x, y, aux)
+        forward(x, y, aux)
     torch.cuda.synchronize()
     code, info = layer.last_device_error()
     if code != 0:
         raise RuntimeError(f"device error {code} ({info}) during warm-up")
     clocks.stop()
-    per_step_launches = kernels_per_step(lambda: layer.forward(x, y, aux), dev)
+    per_step_launches = kernels_per_step(lambda: forward(x, y, aux), dev)
     clocks = ClockSampler(local_rank)
     clocks.start()
     barrier(world)
@@ -352,7 +365,7 @@ def run_ours(args, wl, rank, world, local_rank):
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for _ in range(args.steps):
-        layer.forward(x, y, aux)
+        forward(x, y, aux)
     e1.record(stream)
     torch.cuda.synchronize()
     barrier(world)
@@ -375,7 +388,7 @@ def run_ours(args, wl, rank, world, local_rank):
         off = (torch.arange(E + 1, device=dev, dtype=torch.int32) * C).contiguous()
     else:
         taps = layer.new_taps()
-        layer.forward(x, y, aux, taps=taps)
+        forward(x, y, aux, taps=taps)
         xp = torch.empty((wl.T * k, wl.d_model), dtype=wl.torch_dtype, device=dev)
         cnt = torch.empty(E, dtype=torch.int32, device=dev)
         off = torch.empty(E + 1, dtype=torch.int32, device=dev)
@@ -445,7 +458,7 @@ def run_ours(args, wl, rank, world, local_rank):
                 sl["in"].record(s_in)
             stream.wait_event(sl["in"])
             stream.wait_event(sl["out"])     # the slot's previous output has left
-            layer.forward(sl["x"], sl["y"], sl["aux"])
+            forward(sl["x"], sl["y"], sl["aux"])
             sl["comp"].record(stream)
             with torch.cuda.stream(s_out):
                 s_out.wait_event(sl["comp"])

@@ -105,6 +105,13 @@ MIXTRAL_EC = MIXTRAL_PREFILL.replace(name="mixtral_ec_bf16_T4096_d4096_E8_cf2_sw
                                      routing=ROUTING_EXPERT_CHOICE)
 
 
+# Noisy top-k gating (training mode of the ja page's TopKGating: softmax, top-2,
+# renormalised) on the Mixtral prefill shapes
+MIXTRAL_NOISY = MIXTRAL_PREFILL.replace(
+    name="mixtral_noisy_bf16_T4096_d4096_E8_k2_swiglu14336", gate_mode=GATE_SOFTMAX_TOPK_RENORM,
+    noisy=True)
+
+
 def mixtral_decode(T: int) -> Workload:
     return MIXTRAL_PREFILL.replace(name=f"mixtral_decode_bf16_T{T}_d4096_E8_k2_swiglu14336", T=T)
 
@@ -118,6 +125,7 @@ WORKLOADS = {
     "decode8": mixtral_decode(8),
     "decode1": mixtral_decode(1),
     "mixtral_ec": MIXTRAL_EC,
+    "mixtral_noisy": MIXTRAL_NOISY,
 }
 
 # ---- reduced shapes of the same families (several tiles plus a ragged tail) ------
