@@ -475,3 +475,32 @@ def noisy_router_logits(x, w_router, w_noise, eps, b_router=None,
         z = z + _f64(logit_bias)[None, :]
     zn = x @ _f64(w_noise).T
     return (z + softplus(zn) * _f64(eps)).astype(np.float32)
+
+
+# ------------------------------------------------- token-sharded routing (several ranks)
+def shard_capacity(counts_all, rank: int, cap: Optional[int]):
+    """Capacity left to shard `rank` for each expert when the call's T tokens are
+    split into consecutive shards: cap minus the (pre-drop) assignments of the earlier
+    shards, at least 0 (None: unlimited). counts_all [W, E]. The drop order is then
+    the same as for the whole batch in one call (token-major over all tokens)."""
+    if cap is None:
+        return None
+    counts_all = np.asarray(counts_all, dtype=np.int64)
+    before = counts_all[:rank].sum(axis=0)
+    return np.maximum(0, cap - before)
+
+
+def dispatch_with_caps(idx, E: int, caps):
+    """``dispatch`` with a capacity per expert (token-major, then slot order)."""
+    idx = np.asarray(idx)
+    T, k = idx.shape
+    counts = np.zeros(E, dtype=np.int64)
+    rank = np.zeros((T, k), dtype=np.int64)
+    kept = np.zeros((T, k), dtype=bool)
+    for t in range(T):
+        for s in range(k):
+            e = int(idx[t, s])
+            rank[t, s] = counts[e]
+            kept[t, s] = caps is None or counts[e] < caps[e]
+            counts[e] += 1
+    return counts, rank, kept

@@ -451,9 +451,34 @@ def check_noisy_logits(O):
     assert O.softplus(np.array([0.0]))[0] == math.log(2.0)
 
 
+# ---------------------------------------------------------- token-sharded capacity
+def check_sharded_capacity(O):
+    """Splitting the tokens into consecutive shards, each dropping against the capacity
+    the earlier shards left, keeps exactly the (token, slot) pairs the single call
+    keeps (enumerated over shard splits of random routings with drops)."""
+    rng = np.random.default_rng(12)
+    for T, E, k, cf in ((30, 4, 2, 0.7), (25, 3, 1, 0.5), (40, 6, 3, 1.0)):
+        z = rng.normal(size=(T, E)).astype(np.float32)
+        idx = O.select_topk(z, k)
+        cap = O.capacity(cf, T, k, E)
+        _, _, kept = O.dispatch(idx, E, cap)
+        assert (~kept).any()
+        for cuts in ((T // 2,), (7, 19), (1, 2, T - 1)):
+            bounds = [0, *cuts, T]
+            shards = [idx[a:b] for a, b in zip(bounds, bounds[1:])]
+            counts_all = np.stack([np.bincount(sh.ravel(), minlength=E) for sh in shards])
+            got = []
+            for r, sh in enumerate(shards):
+                caps = O.shard_capacity(counts_all, r, cap)
+                got.append(O.dispatch_with_caps(sh, E, caps)[2])
+            assert np.array_equal(np.concatenate(got), kept), (T, E, k, cuts)
+    assert O.shard_capacity(np.ones((2, 3)), 1, None) is None
+
+
 ALL_CHECKS = [check_combine, check_topk_bruteforce, check_gate_sums_and_ranges, check_worked_gates,
               check_softmax_closed_forms, check_router_logits_exact, check_capacity_golden,
               check_counts_and_drop_order, check_layout, check_forward_vs_pages_torch,
               check_sparse_equals_dense_masked, check_special_cases, check_aux_closed_forms,
               check_expert_choice_capacity, check_expert_choice_bruteforce,
-              check_expert_choice_scores, check_expert_choice_dense, check_noisy_logits]
+              check_expert_choice_scores, check_expert_choice_dense, check_noisy_logits,
+              check_sharded_capacity]

@@ -137,7 +137,12 @@ def _noise_sign_flipped(x, w_router, w_noise, eps, b_router=None, logit_bias=Non
                                         logit_bias)
 
 
+def _shard_capacity_ignores_earlier(counts_all, rank, cap):
+    return _orig["shard_capacity"](counts_all, 0, cap)
+
+
 MUTANTS = {
+    "shard_capacity_ignores_earlier_shards": ("shard_capacity", _shard_capacity_ignores_earlier),
     "softplus_is_exp": ("softplus", _softplus_is_exp),
     "noise_sign_flipped": ("noisy_router_logits", _noise_sign_flipped),
     "ec_softmax_over_experts": ("expert_choice_scores", _ec_softmax_over_experts),
