@@ -270,6 +270,65 @@ moe_status_t moe_route_expert_choice(const moe_cfg_t *cfg, const moe_weights_t *
                                      float *ec_score, void *ws, size_t ws_bytes,
                                      moe_stream_t stream);
 
+/* ---------------------------------------------------------------------------
+ * Token-sharded batches. One batch of T_total tokens is split into n_shards
+ * consecutive slices (shard 0 first), one per rank, with the weights replicated.
+ * The pages define the layer on one batch; the entries below give each shard
+ * exactly its slice of that single call's results. Tokens are independent given
+ * the routing except in two places, and these entries carry both:
+ *  - the capacity drop of youngju.dev (zh) "SwitchRouter" takes every expert's
+ *    (token, slot) pairs in token-major order over the whole batch, with capacity
+ *    floor(cf * T_total * k / E); shard r may keep max(0, cap - before_e) pairs for
+ *    expert e, before_e = the pairs shards 0..r-1 routed to e before drops. So the
+ *    shards first exchange their pre-drop counts [E] (an all-gather, the caller's
+ *    collective) and pass them in as counts_all;
+ *  - the statistics of moe_aux_stats are means over the batch: each shard emits
+ *    fp64 sums, the caller adds them over the shards (a sum all-reduce), and
+ *    moe_aux_finalize turns the sums into the statistics.
+ * Sequence per rank: moe_route_shard -> all-gather counts, all-reduce aux_part ->
+ * moe_forward_shard (or moe_permute_shard + moe_expert_ffn + moe_combine) and
+ * moe_aux_finalize. Token-choice configurations only (MOE_ERR_INVALID_ARG with
+ * MOE_ROUTING_EXPERT_CHOICE). cfg->n_tokens is the shard's token count. */
+typedef struct {
+  long long n_tokens_total;   /* tokens of the whole batch, >= cfg->n_tokens */
+  int n_shards;               /* >= 1 */
+  int shard;                  /* this shard's place, 0 <= shard < n_shards */
+  const int32_t *counts_all;  /* device [n_shards, E] int32: every shard's pre-drop
+                                 counts (moe_route_shard's `counts`), shard-major */
+} moe_shard_t;
+
+/* moe_route on this shard's tokens, plus its pre-drop counts per expert
+ * (counts [E] int32, device) and, when aux_part != NULL, its fp64 sums for the
+ * statistics: aux_part [1 + 2E] = { sum_t logsumexp(z_t)^2, count[0..E),
+ * sum_t softmax(z_t)[0..E) } (device). x == NULL: logits is the input, as in
+ * moe_route. An empty shard writes zero counts and sums. */
+moe_status_t moe_route_shard(const moe_cfg_t *cfg, const moe_weights_t *w, const void *x,
+                             float *logits, int32_t *topk_idx, float *topk_gate,
+                             int32_t *counts, double *aux_part, void *ws, size_t ws_bytes,
+                             moe_stream_t stream);
+
+/* moe_permute for one shard: the same outputs, with the capacity of the whole batch
+ * shared out as described above (counts are this shard's, before drops; offsets,
+ * perm and inv index this shard's rows and tokens). */
+moe_status_t moe_permute_shard(const moe_cfg_t *cfg, const moe_shard_t *shard, const void *x,
+                               const int32_t *topk_idx, int32_t *counts, int32_t *offsets,
+                               int32_t *perm, int32_t *inv, void *x_perm, void *ws,
+                               size_t ws_bytes, moe_stream_t stream);
+
+/* moe_forward for one shard that moe_route_shard has routed: taps->topk_idx and
+ * taps->topk_gate are INPUTS (required); the other taps are outputs as in
+ * moe_forward (taps->logits is not written). Permute with the shared-out capacity,
+ * shared experts, expert FFNs and combine; y [n_tokens, d]. */
+moe_status_t moe_forward_shard(const moe_cfg_t *cfg, const moe_shard_t *shard,
+                               const moe_weights_t *w, const void *x, const moe_taps_t *taps,
+                               void *y, void *ws, size_t ws_bytes, moe_stream_t stream);
+
+/* The moe_aux_stats vector out [3 + 2E] fp32 (device) from aux_part [1 + 2E] fp64
+ * summed over all shards (device), for a batch of n_tokens_total >= 1 tokens.
+ * Needs no workspace. */
+moe_status_t moe_aux_finalize(const moe_cfg_t *cfg, long long n_tokens_total,
+                              const double *aux_part, float *out, moe_stream_t stream);
+
 /* Synchronise `stream`, read and clear the sticky device error word.
  * Returns MOE_ERR_DEVICE when *code != 0, MOE_ERR_CUDA when the sync failed. */
 moe_status_t moe_last_device_error(void *ws, int32_t *code, int32_t *info, moe_stream_t stream);

@@ -29,6 +29,7 @@ DEVERR_NAMES = {0: "none", 1: "expert index out of range", 2: "invalid offsets",
 EXPORTED = ("moe_workspace_size", "moe_workspace_init", "moe_route", "moe_route_noisy",
             "moe_route_expert_choice", "moe_permute", "moe_permute_noalloc", "moe_forward_noisy",
             "moe_expert_ffn", "moe_combine", "moe_aux_stats", "moe_forward",
+            "moe_route_shard", "moe_permute_shard", "moe_forward_shard", "moe_aux_finalize",
             "moe_last_device_error", "moe_status_string")
 
 
@@ -59,6 +60,11 @@ class MoeTaps(ctypes.Structure):
                 ("logits", "topk_idx", "topk_gate", "counts", "offsets", "perm", "inv")]
 
 
+class MoeShard(ctypes.Structure):
+    _fields_ = [("n_tokens_total", ctypes.c_longlong), ("n_shards", ctypes.c_int32),
+                ("shard", ctypes.c_int32), ("counts_all", ctypes.c_void_p)]
+
+
 def lib_path() -> str:
     return _LIB_PATH
 
@@ -84,6 +90,11 @@ def load() -> ctypes.CDLL:
         "moe_combine": [cfgp, P, P, P, P, P, P, S, P],
         "moe_aux_stats": [cfgp, P, P, P, P, S, P],
         "moe_forward": [cfgp, wp, P, P, P, ctypes.POINTER(MoeTaps), P, S, P],
+        "moe_route_shard": [cfgp, wp, P, P, P, P, P, P, P, S, P],
+        "moe_permute_shard": [cfgp, ctypes.POINTER(MoeShard), P, P, P, P, P, P, P, P, S, P],
+        "moe_forward_shard": [cfgp, ctypes.POINTER(MoeShard), wp, P, ctypes.POINTER(MoeTaps), P,
+                              P, S, P],
+        "moe_aux_finalize": [cfgp, ctypes.c_longlong, P, P, P],
         "moe_last_device_error": [P, ctypes.POINTER(ctypes.c_int32),
                                   ctypes.POINTER(ctypes.c_int32), P],
     }
@@ -240,6 +251,45 @@ class MoELayer:
         _check(self.lib.moe_aux_stats(ctypes.byref(self.cfg), _ptr(logits), _ptr(topk_idx),
                                       _ptr(out), _ptr(self.ws), self.ws.numel(), _stream()),
                "moe_aux_stats")
+
+    # ------------------------------------------------- one shard of a larger batch
+    def route_shard(self, x: Optional[torch.Tensor], logits: Optional[torch.Tensor],
+                    topk_idx: torch.Tensor, topk_gate: torch.Tensor, counts: torch.Tensor,
+                    aux_part: Optional[torch.Tensor] = None):
+        """moe_route on this shard + its pre-drop counts [E] int32 and, optionally, its
+        fp64 sums aux_part [1 + 2E] for the statistics."""
+        _check(self.lib.moe_route_shard(ctypes.byref(self.cfg), ctypes.byref(self.weights),
+                                        _ptr(x), _ptr(logits), _ptr(topk_idx), _ptr(topk_gate),
+                                        _ptr(counts), _ptr(aux_part), _ptr(self.ws),
+                                        self.ws.numel(), _stream()), "moe_route_shard")
+
+    def permute_shard(self, shard: MoeShard, x, topk_idx, counts, offsets, perm, inv, x_perm):
+        _check(self.lib.moe_permute_shard(ctypes.byref(self.cfg), ctypes.byref(shard), _ptr(x),
+                                          _ptr(topk_idx), _ptr(counts), _ptr(offsets),
+                                          _ptr(perm), _ptr(inv), _ptr(x_perm), _ptr(self.ws),
+                                          self.ws.numel(), _stream()), "moe_permute_shard")
+
+    def forward_shard(self, shard: MoeShard, x: torch.Tensor, taps: dict,
+                      y: Optional[torch.Tensor] = None) -> torch.Tensor:
+        """The layer on this shard, routed by route_shard: taps["topk_idx"] and
+        taps["topk_gate"] are inputs."""
+        if y is None:
+            y = torch.empty_like(x)
+        tp = MoeTaps(**{k: _ptr(taps.get(k)) for k, _ in MoeTaps._fields_})
+        _check(self.lib.moe_forward_shard(ctypes.byref(self.cfg), ctypes.byref(shard),
+                                          ctypes.byref(self.weights), _ptr(x), ctypes.byref(tp),
+                                          _ptr(y), _ptr(self.ws), self.ws.numel(), _stream()),
+               "moe_forward_shard")
+        return y
+
+    def aux_finalize(self, n_tokens_total: int, aux_part: torch.Tensor,
+                     out: Optional[torch.Tensor] = None) -> torch.Tensor:
+        if out is None:
+            out = self.new_aux()
+        _check(self.lib.moe_aux_finalize(ctypes.byref(self.cfg), int(n_tokens_total),
+                                         _ptr(aux_part), _ptr(out), _stream()),
+               "moe_aux_finalize")
+        return out
 
     def last_device_error(self):
         code, info = ctypes.c_int32(0), ctypes.c_int32(0)

@@ -5,7 +5,7 @@
 
 #include <climits>
 
-#include "kernels.cuh"
+#include "shard.cuh"
 
 #define MOE_API extern "C" __attribute__((visibility("default")))
 
@@ -15,7 +15,7 @@ namespace {
 enum Buf {
   B_ERR, B_TILE_COUNTS, B_TILE_BASE, B_TILE_P, B_TILE_Z, B_COUNTS, B_OFFSETS, B_MPREFIX, B_SH_TBL,
   B_LOGITS, B_IDX, B_GATE, B_PERM, B_INV, B_XPERM, B_H, B_YPERM, B_SH_H, B_SH_Y, B_YPART,
-  B_EC_ZT, B_EC_IDX, B_EC_SCORE, B_EC_SLOT, B_NOISE, B_NBUF
+  B_EC_ZT, B_EC_IDX, B_EC_SCORE, B_EC_SLOT, B_NOISE, B_CAP_E, B_NBUF
 };
 
 struct Layout {
@@ -81,6 +81,7 @@ Layout layout_for(const moe_cfg_t &c) {
   sz[B_EC_SCORE] = ec ? E * C * 4 : 0;
   sz[B_EC_SLOT] = ec ? T * E * 4 : 0;
   sz[B_NOISE] = T * E * 4;  // x W_noise^T of noisy top-k gating
+  sz[B_CAP_E] = E * 4;      // per-expert capacity left to one shard of a batch
   Layout L;
   size_t o = 0;
   for (int i = 0; i < B_NBUF; ++i) {
@@ -190,6 +191,24 @@ int capacity_of(const moe_cfg_t &c) {
   const double cap = floor((double)c.capacity_factor * (double)c.n_tokens * (double)c.top_k /
                            (double)c.n_experts);
   return cap > (double)INT_MAX ? INT_MAX : (int)cap;
+}
+
+// capacity of a batch of n_tokens tokens: floor(cf * n_tokens * k / E), -1 = unlimited
+int capacity_for_tokens(const moe_cfg_t &c, long long n_tokens) {
+  if (!(c.capacity_factor > 0.f)) return -1;
+  const double cap = floor((double)c.capacity_factor * (double)n_tokens * (double)c.top_k /
+                           (double)c.n_experts);
+  return cap > (double)INT_MAX ? INT_MAX : (int)cap;
+}
+
+// One shard of a token-sharded batch (see moe_shard_t).
+moe_status_t check_shard(const moe_cfg_t &c, const moe_shard_t *sh) {
+  if (sh == nullptr) return MOE_ERR_INVALID_ARG;
+  if (sh->n_shards < 1 || sh->shard < 0 || sh->shard >= sh->n_shards) return MOE_ERR_INVALID_ARG;
+  if (sh->n_tokens_total < c.n_tokens) return MOE_ERR_INVALID_ARG;
+  if (sh->counts_all == nullptr) return MOE_ERR_INVALID_ARG;
+  if (expert_choice(c)) return MOE_ERR_INVALID_ARG;  // picks are per expert over all tokens
+  return MOE_OK;
 }
 
 int m_tiles_ub(long long rows, int groups) {
@@ -574,14 +593,24 @@ MOE_API moe_status_t moe_aux_stats(const moe_cfg_t *cfg, const float *logits,
 namespace moe {
 namespace {
 // the whole layer; eps != NULL: noisy top-k gating (token choice only)
+// sh != NULL: one shard of a token-sharded batch, routed already (topk_idx and
+// topk_gate in taps, the capacity of the whole batch shared out per expert)
 moe_status_t forward_impl(const moe_cfg_t *cfg, const moe_weights_t *w, const void *x,
                           const float *eps, void *y, float *aux_out, const moe_taps_t *taps,
-                          void *ws, size_t ws_bytes, moe_stream_t stream) {
+                          void *ws, size_t ws_bytes, moe_stream_t stream,
+                          const moe_shard_t *sh = nullptr) {
   MOE_TRY(check_cfg(cfg));
   MOE_TRY(check_ws(cfg, ws, ws_bytes));
+  if (sh != nullptr) {
+    MOE_TRY(check_shard(*cfg, sh));
+    if (aux_out != nullptr || eps != nullptr) return MOE_ERR_INVALID_ARG;
+    if (cfg->n_tokens > 0 &&
+        (taps == nullptr || taps->topk_idx == nullptr || taps->topk_gate == nullptr))
+      return MOE_ERR_INVALID_ARG;
+  }
   if (cfg->n_tokens == 0) return MOE_OK;  // nothing is read or written
   if (w == nullptr) return MOE_ERR_INVALID_ARG;
-  MOE_TRY(check_ptrs({{x, true}, {y, true}, {aux_out, false}, {w->w_router, true},
+  MOE_TRY(check_ptrs({{x, true}, {y, true}, {aux_out, false}, {w->w_router, sh == nullptr},
                       {w->b_router, false}, {w->logit_bias, false}}));
   MOE_TRY(check_expert_weights(cfg, w));
   MOE_TRY(check_shared_weights(cfg, w));
@@ -635,7 +664,12 @@ moe_status_t forward_impl(const moe_cfg_t *cfg, const moe_weights_t *w, const vo
   r.k = c.top_k;
   r.gate_mode = c.gate_mode;
   r.err = err;
-  MOE_CUDA(launch_router(r, c.dtype, stream));
+  if (sh == nullptr) {
+    MOE_CUDA(launch_router(r, c.dtype, stream));
+  } else {  // routed by the caller: only the per-tile histogram
+    MOE_CUDA(launch_tile_counts(idx, c.n_tokens, c.top_k, c.n_experts, r.tile_counts, err,
+                                stream));
+  }
   // 2. scan: counts, capacity, offsets, GEMM tile table (+ aux statistics)
   ScanArgs s{};
   s.tile_counts = r.tile_counts;
@@ -653,7 +687,14 @@ moe_status_t forward_impl(const moe_cfg_t *cfg, const moe_weights_t *w, const vo
   s.k = c.top_k;
   s.alpha = c.aux_alpha;
   s.sh_tbl = c.n_shared > 0 ? sh_tbl : nullptr;
-  MOE_CUDA(launch_scan(s, stream));
+  ShardCaps sc{};
+  if (sh == nullptr) {
+    MOE_CUDA(launch_scan(s, stream));
+  } else {
+    s.cap = capacity_for_tokens(c, sh->n_tokens_total);
+    sc = ShardCaps{sh->counts_all, at<int32_t>(ws, L, B_CAP_E), sh->n_shards, sh->shard};
+    MOE_CUDA(launch_scan_shard(s, sc, stream));
+  }
   // 3. stable permutation with capacity drops + row gather
   ScatterArgs p{};
   p.x = x;
@@ -670,7 +711,8 @@ moe_status_t forward_impl(const moe_cfg_t *cfg, const moe_weights_t *w, const vo
   p.cap = s.cap;
   p.elem_bytes = c.dtype == MOE_DTYPE_F32 ? 4 : 2;
   p.err = err;
-  MOE_CUDA(launch_scatter(p, stream));
+  if (sh == nullptr) MOE_CUDA(launch_scatter(p, stream));
+  else MOE_CUDA(launch_scatter_shard(p, sc.cap_e, stream));
   // 4. always-on shared experts: one SwiGLU over all tokens, experts concatenated along F
   float *sh_y = nullptr;
   float *part = layout_size(L, B_YPART) > 0 ? at<float>(ws, L, B_YPART) : nullptr;
@@ -732,6 +774,142 @@ MOE_API moe_status_t moe_forward_noisy(const moe_cfg_t *cfg, const moe_weights_t
                                        size_t ws_bytes, moe_stream_t stream) {
   if (eps == nullptr) return MOE_ERR_INVALID_ARG;
   return forward_impl(cfg, w, x, eps, y, aux_out, taps, ws, ws_bytes, stream);
+}
+
+// ----------------------------------------------------- token-sharded batches
+MOE_API moe_status_t moe_route_shard(const moe_cfg_t *cfg, const moe_weights_t *w,
+                                     const void *x, float *logits, int32_t *topk_idx,
+                                     float *topk_gate, int32_t *counts, double *aux_part,
+                                     void *ws, size_t ws_bytes, moe_stream_t stream) {
+  MOE_TRY(check_cfg(cfg));
+  MOE_TRY(check_ws(cfg, ws, ws_bytes));
+  if (expert_choice(*cfg)) return MOE_ERR_INVALID_ARG;
+  MOE_TRY(check_ptrs({{counts, true}, {aux_part, false}}));
+  const moe_cfg_t &c = *cfg;
+  if (c.n_tokens == 0) {  // an empty shard: no assignments, zero sums
+    MOE_CUDA(cudaMemsetAsync(counts, 0, sizeof(int32_t) * c.n_experts, stream));
+    if (aux_part != nullptr)
+      MOE_CUDA(cudaMemsetAsync(aux_part, 0, sizeof(double) * (1 + 2 * c.n_experts), stream));
+    return MOE_OK;
+  }
+  if (w == nullptr) return MOE_ERR_INVALID_ARG;
+  if (x != nullptr) {
+    MOE_TRY(check_ptrs({{x, true}, {w->w_router, true}, {logits, false}}));
+  } else {
+    MOE_TRY(check_ptrs({{logits, true}}));
+  }
+  MOE_TRY(check_ptrs({{topk_idx, true}, {topk_gate, true}, {w->b_router, false},
+                      {w->logit_bias, false}}));
+  const Layout L = layout_for(c);
+  int32_t *err = at<int32_t>(ws, L, B_ERR);
+  RouterArgs r{};
+  r.x = x;
+  r.w = w->w_router;
+  r.b_router = w->b_router;
+  r.logit_bias = w->logit_bias;
+  r.logits_in = x ? nullptr : logits;
+  r.logits_out = x ? logits : nullptr;
+  r.topk_idx = topk_idx;
+  r.topk_gate = topk_gate;
+  r.tile_counts = at<int32_t>(ws, L, B_TILE_COUNTS);
+  r.tile_p = aux_part ? at<float>(ws, L, B_TILE_P) : nullptr;
+  r.tile_z = aux_part ? at<float>(ws, L, B_TILE_Z) : nullptr;
+  r.T = c.n_tokens;
+  r.d = c.d_model;
+  r.E = c.n_experts;
+  r.k = c.top_k;
+  r.gate_mode = c.gate_mode;
+  r.err = err;
+  MOE_CUDA(launch_router(r, c.dtype, stream));
+  // the shard's assignments per expert before any drop (offsets etc. to scratch)
+  const int NT = ceil_div(c.n_tokens, router_bm(c.n_experts));
+  ScanArgs s{};
+  s.tile_counts = r.tile_counts;
+  s.tile_base = at<int32_t>(ws, L, B_TILE_BASE);
+  s.counts = counts;
+  s.offsets = at<int32_t>(ws, L, B_OFFSETS);
+  s.mprefix = at<int32_t>(ws, L, B_MPREFIX);
+  s.E = c.n_experts;
+  s.NT = NT;
+  s.cap = -1;
+  s.T = c.n_tokens;
+  s.k = c.top_k;
+  MOE_CUDA(launch_scan(s, stream));
+  if (aux_part != nullptr)
+    MOE_CUDA(launch_aux_partials(r.tile_counts, r.tile_p, r.tile_z, c.n_experts, NT, aux_part,
+                                 stream));
+  return MOE_OK;
+}
+
+MOE_API moe_status_t moe_permute_shard(const moe_cfg_t *cfg, const moe_shard_t *shard,
+                                       const void *x, const int32_t *topk_idx, int32_t *counts,
+                                       int32_t *offsets, int32_t *perm, int32_t *inv,
+                                       void *x_perm, void *ws, size_t ws_bytes,
+                                       moe_stream_t stream) {
+  MOE_TRY(check_cfg(cfg));
+  MOE_TRY(check_ws(cfg, ws, ws_bytes));
+  MOE_TRY(check_shard(*cfg, shard));
+  MOE_TRY(check_ptrs({{x, true}, {topk_idx, true}, {counts, true}, {offsets, true}, {perm, true},
+                      {inv, true}, {x_perm, true}, {shard->counts_all, true}}));
+  const moe_cfg_t &c = *cfg;
+  if (c.n_tokens == 0) {
+    MOE_CUDA(cudaMemsetAsync(counts, 0, sizeof(int32_t) * c.n_experts, stream));
+    MOE_CUDA(cudaMemsetAsync(offsets, 0, sizeof(int32_t) * (c.n_experts + 1), stream));
+    return MOE_OK;
+  }
+  const Layout L = layout_for(c);
+  int32_t *err = at<int32_t>(ws, L, B_ERR);
+  int32_t *tile_counts = at<int32_t>(ws, L, B_TILE_COUNTS);
+  MOE_CUDA(launch_tile_counts(topk_idx, c.n_tokens, c.top_k, c.n_experts, tile_counts, err, stream));
+  ScanArgs s{};
+  s.tile_counts = tile_counts;
+  s.tile_base = at<int32_t>(ws, L, B_TILE_BASE);
+  s.counts = counts;
+  s.offsets = offsets;
+  s.mprefix = at<int32_t>(ws, L, B_MPREFIX);
+  s.E = c.n_experts;
+  s.NT = ceil_div(c.n_tokens, router_bm(c.n_experts));
+  s.cap = capacity_for_tokens(c, shard->n_tokens_total);
+  s.T = c.n_tokens;
+  s.k = c.top_k;
+  const ShardCaps sc{shard->counts_all, at<int32_t>(ws, L, B_CAP_E), shard->n_shards,
+                     shard->shard};
+  MOE_CUDA(launch_scan_shard(s, sc, stream));
+  ScatterArgs p{};
+  p.x = x;
+  p.topk_idx = topk_idx;
+  p.tile_base = s.tile_base;
+  p.offsets = offsets;
+  p.perm = perm;
+  p.inv = inv;
+  p.x_perm = x_perm;
+  p.T = c.n_tokens;
+  p.d = c.d_model;
+  p.E = c.n_experts;
+  p.k = c.top_k;
+  p.cap = s.cap;
+  p.elem_bytes = c.dtype == MOE_DTYPE_F32 ? 4 : 2;
+  p.err = err;
+  MOE_CUDA(launch_scatter_shard(p, sc.cap_e, stream));
+  return MOE_OK;
+}
+
+MOE_API moe_status_t moe_forward_shard(const moe_cfg_t *cfg, const moe_shard_t *shard,
+                                       const moe_weights_t *w, const void *x,
+                                       const moe_taps_t *taps, void *y, void *ws,
+                                       size_t ws_bytes, moe_stream_t stream) {
+  if (shard == nullptr) return MOE_ERR_INVALID_ARG;
+  return forward_impl(cfg, w, x, nullptr, y, nullptr, taps, ws, ws_bytes, stream, shard);
+}
+
+MOE_API moe_status_t moe_aux_finalize(const moe_cfg_t *cfg, long long n_tokens_total,
+                                      const double *aux_part, float *out, moe_stream_t stream) {
+  MOE_TRY(check_cfg(cfg));
+  if (n_tokens_total < 1) return MOE_ERR_INVALID_ARG;  // the statistics are means over tokens
+  MOE_TRY(check_ptrs({{aux_part, true}, {out, true}}));
+  MOE_CUDA(launch_aux_finalize(aux_part, cfg->n_experts, n_tokens_total, cfg->top_k,
+                               cfg->aux_alpha, out, stream));
+  return MOE_OK;
 }
 
 MOE_API moe_status_t moe_last_device_error(void *ws, int32_t *code, int32_t *info,

@@ -11,7 +11,7 @@
 //
 // Everything is atomic-free in global memory and deterministic: ranks come from
 // per-tile counts, an exclusive scan over (expert, tile), and in-tile warp matching.
-#include "kernels.cuh"
+#include "shard.cuh"
 
 namespace moe {
 
@@ -35,7 +35,10 @@ constexpr int kScanVPL = 8;  // tiles per lane per batch (loads issued together)
 // the token tiles (tile_counts is [E][NT], so a warp reads consecutive tiles).
 // Then one warp: counts, capacity, kept-row offsets and the 128-row tile prefix
 // over the experts. Optionally the load-balancing statistics (fixed-order sums).
-__global__ void __launch_bounds__(kScanThreads) k_scan(ScanArgs a) {
+// SHARD: the tokens are one shard of a larger batch; expert e keeps at most
+// max(0, cap - pairs routed to e by the earlier shards), written to sc.cap_e.
+template <bool SHARD>
+__global__ void __launch_bounds__(kScanThreads) k_scan(ScanArgs a, ShardCaps sc) {
   __shared__ int count_s[kMaxExperts];
   __shared__ float P_s[kMaxExperts];
   __shared__ float red[kScanThreads / 32];
@@ -83,7 +86,16 @@ __global__ void __launch_bounds__(kScanThreads) k_scan(ScanArgs a) {
       const int e = lane * 8 + j;
       const int c = e < E ? count_s[e] : 0;
       cnt[j] = c;
-      kept[j] = (a.cap < 0) ? c : min(c, a.cap);
+      int cap = a.cap;
+      if constexpr (SHARD) {
+        if (cap >= 0 && e < E) {
+          long long before = 0;
+          for (int r = 0; r < sc.rank; ++r) before += sc.counts_all[(size_t)r * E + e];
+          cap = (int)max(0LL, (long long)a.cap - before);
+          sc.cap_e[e] = cap;
+        }
+      }
+      kept[j] = (a.cap < 0) ? c : min(c, cap);
       mt[j] = ceil_div(kept[j], kRowTile);
       sk += kept[j];
       sm += mt[j];
@@ -150,7 +162,8 @@ __global__ void __launch_bounds__(kScanThreads) k_scan(ScanArgs a) {
 // ------------------------------------------------------------------- scatter
 constexpr int kScatterThreads = 256;
 
-__global__ void __launch_bounds__(kScatterThreads) k_scatter(ScatterArgs a) {
+template <bool SHARD>
+__global__ void __launch_bounds__(kScatterThreads) k_scatter(ScatterArgs a, const int32_t *cap_e) {
   extern __shared__ int32_t sh[];
   const int E = a.E, k = a.k, T = a.T;
   const int bm = router_bm(E);
@@ -193,7 +206,7 @@ __global__ void __launch_bounds__(kScatterThreads) k_scatter(ScatterArgs a) {
       report_error(a.err, MOE_DEVERR_EXPERT_INDEX, t0 * k + p);
     } else {
       const int rank = a.tile_base[(size_t)e * NT + tile] + hist[(p / 32) * E + e] + prow[p];
-      if (a.cap < 0 || rank < a.cap) {
+      if (a.cap < 0 || rank < (SHARD ? cap_e[e] : a.cap)) {
         row = a.offsets[e] + rank;
         a.perm[row] = t;
       }
@@ -354,18 +367,34 @@ __global__ void k_tile_table(const int32_t *offsets, int G, int max_rows, int32_
 }  // namespace
 
 cudaError_t launch_scan(const ScanArgs &a, cudaStream_t st) {
-  k_scan<<<1, kScanThreads, 0, st>>>(a);
+  k_scan<false><<<1, kScanThreads, 0, st>>>(a, ShardCaps{});
   return cudaGetLastError();
 }
 
-cudaError_t launch_scatter(const ScatterArgs &a, cudaStream_t st) {
+cudaError_t launch_scan_shard(const ScanArgs &a, const ShardCaps &sc, cudaStream_t st) {
+  k_scan<true><<<1, kScanThreads, 0, st>>>(a, sc);
+  return cudaGetLastError();
+}
+
+namespace {
+template <bool SHARD>
+cudaError_t scatter(const ScatterArgs &a, const int32_t *cap_e, cudaStream_t st) {
   if (a.T == 0) return cudaSuccess;
   const int bm = router_bm(a.E);
   const int NT = ceil_div(a.T, bm);
   const int NC = ceil_div(bm * a.k, 32);
   const size_t smem = (size_t)(NC * a.E + bm * a.k) * sizeof(int32_t);
-  k_scatter<<<NT, kScatterThreads, smem, st>>>(a);
+  k_scatter<SHARD><<<NT, kScatterThreads, smem, st>>>(a, cap_e);
   return cudaGetLastError();
+}
+}  // namespace
+
+cudaError_t launch_scatter(const ScatterArgs &a, cudaStream_t st) {
+  return scatter<false>(a, nullptr, st);
+}
+
+cudaError_t launch_scatter_shard(const ScatterArgs &a, const int32_t *cap_e, cudaStream_t st) {
+  return scatter<true>(a, cap_e, st);
 }
 
 cudaError_t launch_combine(const CombineArgs &a, int dtype, cudaStream_t st) {

@@ -55,8 +55,10 @@ def test_struct_layout_matches_header(tmp_path):
         + "".join(f"  F(moe_cfg_t, {n});\n" for n, _ in B.MoeCfg._fields_)
         + "".join(f"  F(moe_weights_t, {n});\n" for n, _ in B.MoeWeights._fields_)
         + "".join(f"  F(moe_taps_t, {n});\n" for n, _ in B.MoeTaps._fields_)
+        + "".join(f"  F(moe_shard_t, {n});\n" for n, _ in B.MoeShard._fields_)
         + '  printf("size moe_cfg_t %zu\\nsize moe_weights_t %zu\\nsize moe_taps_t %zu\\n",'
-          " sizeof(moe_cfg_t), sizeof(moe_weights_t), sizeof(moe_taps_t));\n  return 0;\n}\n")
+          " sizeof(moe_cfg_t), sizeof(moe_weights_t), sizeof(moe_taps_t));\n"
+        + '  printf("size moe_shard_t %zu\\n", sizeof(moe_shard_t));\n  return 0;\n}\n')
     exe = tmp_path / "layout"
     subprocess.run(["gcc", "-std=c99", f"-I{os.path.dirname(HEADER)}", str(prog), "-o", str(exe)],
                    check=True)
@@ -67,7 +69,7 @@ def test_struct_layout_matches_header(tmp_path):
             a, b, c = ln.split()
             got[(a, b)] = int(c)
     for st, cls in (("moe_cfg_t", B.MoeCfg), ("moe_weights_t", B.MoeWeights),
-                    ("moe_taps_t", B.MoeTaps)):
+                    ("moe_taps_t", B.MoeTaps), ("moe_shard_t", B.MoeShard)):
         for n, _ in cls._fields_:
             assert got[(st, n)] == getattr(cls, n).offset, (st, n)
         assert got[("size", st)] == ctypes.sizeof(cls)
