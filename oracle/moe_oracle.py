@@ -46,6 +46,9 @@ test):
   fp32 logits (equal logits: lower token index first); a token's output is the
   score-weighted sum over the experts that took it (P4's dispatch mask used as
   the gate), 0 if none did.
+* A batch split by tokens over several shards gives every token what the single
+  call over the whole batch gives: the capacity is that of the whole batch, and
+  each shard keeps per expert what the earlier shards' pre-drop pairs left.
 * No intermediate rounding: everything after the fp32 logits is fp64.
 
 Parity status: every function below is pinned by the CPU test suite; none is
