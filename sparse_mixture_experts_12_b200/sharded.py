@@ -70,6 +70,11 @@ class ShardedMoELayer:
 
     def __init__(self, workload: synth.Workload, params: dict, shard: int, n_shards: int,
                  device="cuda", group=None):
+        if not 0 <= shard < n_shards:
+            raise ValueError(f"shard {shard} is not one of {n_shards} shards")
+        if dist.is_initialized() and (dist.get_world_size(group) != n_shards
+                                      or dist.get_rank(group) != shard):
+            raise ValueError("shard / n_shards must be this rank's place in the process group")
         self.n_tokens_total = workload.T
         self.shard, self.n_shards, self.group = shard, n_shards, group
         a, b = shard_bounds(workload.T, n_shards)[shard]

@@ -95,6 +95,23 @@ class OracleSteps:
                     z=p[0] / T, bsq=float(((f - 1.0 / E) ** 2).sum()))
 
 
+def test_one_shard_needs_no_process_group():
+    """Without a process group the exchange is the identity: one shard is the batch."""
+    P = H.oracle_params(synth.generate(WL, seed=3))
+    steps = OracleSteps(WL, P, 0, 1)
+    y, aux = S.forward_sharded(steps, P["x"], WL.n_experts, want_aux=True)
+    yref, r = O.moe_forward(P["x"], P, **H.oracle_kwargs(WL))
+    assert np.array_equal(steps.kept, r["kept"])
+    assert np.allclose(y, yref, rtol=1e-12, atol=1e-12)
+    _, _, auxv = O.aux_stats(r["logits"], r["idx"], WL.n_experts, WL.top_k, WL.aux_alpha)
+    assert aux["aux"] == pytest.approx(auxv, rel=1e-12)
+
+
+def test_sharded_layer_checks_its_place():
+    with pytest.raises(ValueError):
+        S.ShardedMoELayer(WL, {}, shard=2, n_shards=2, device="cpu")
+
+
 def _free_port():
     with socket.socket() as s:
         s.bind(("127.0.0.1", 0))
