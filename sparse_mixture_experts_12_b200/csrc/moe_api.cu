@@ -379,7 +379,6 @@ MOE_API moe_status_t moe_route(const moe_cfg_t *cfg, const moe_weights_t *w, con
   MOE_TRY(check_ptrs({{topk_idx, true}, {topk_gate, true}, {w->b_router, false},
                       {w->logit_bias, false}}));
   const moe_cfg_t &c = *cfg;
-  if (c.n_tokens == 0) return MOE_OK;
   const Layout L = layout_for(c);
   RouterArgs r{};
   r.x = x;
@@ -506,7 +505,6 @@ MOE_API moe_status_t moe_expert_ffn(const moe_cfg_t *cfg, const moe_weights_t *w
   MOE_TRY(check_expert_weights(cfg, w));
   MOE_TRY(check_ptrs({{x_perm, true}, {offsets, true}, {y_perm, true}}));
   const moe_cfg_t &c = *cfg;
-  if (c.n_tokens == 0) return MOE_OK;
   const Layout L = layout_for(c);
   int32_t *err = at<int32_t>(ws, L, B_ERR);
   int32_t *mprefix = at<int32_t>(ws, L, B_MPREFIX);
@@ -528,7 +526,6 @@ MOE_API moe_status_t moe_combine(const moe_cfg_t *cfg, const void *y_perm, const
   MOE_TRY(check_ptrs({{y_perm, true}, {inv, true}, {topk_gate, true}, {shared_y, false},
                       {y, true}}));
   const moe_cfg_t &c = *cfg;
-  if (c.n_tokens == 0) return MOE_OK;
   const Layout L = layout_for(c);
   CombineArgs a{};
   a.y_perm = y_perm;
