@@ -188,9 +188,11 @@ moe_status_t moe_permute(const moe_cfg_t *cfg, const void *x, const int32_t *top
  * larger problems return MOE_ERR_WORKSPACE. d_model * element size must be a
  * multiple of 16 bytes.
  * All calls share the static array: calls that overlap on the GPU race, so the
- * caller must serialise them (one stream, or explicit ordering). The first call on
- * each device looks up the array's device address (cudaGetSymbolAddress); make
- * that first call before any stream capture. Out-of-range expert indices are not
+ * caller must serialise them (one stream, or explicit ordering). The array's
+ * address belongs to a CUDA context: the first call in each context (the device's
+ * primary context, a context the caller created, or a primary context re-created
+ * after a reset) looks it up with cudaGetSymbolAddress and caches it under the
+ * context's ID; make that first call before any stream capture. Out-of-range expert indices are not
  * reported (there is no workspace for the error word); such a pair is treated as
  * dropped (inv = -1). */
 moe_status_t moe_permute_noalloc(const moe_cfg_t *cfg, const void *x, const int32_t *topk_idx,
@@ -235,6 +237,43 @@ moe_status_t moe_forward(const moe_cfg_t *cfg, const moe_weights_t *w, const voi
                          float *aux_out, const moe_taps_t *taps, void *ws, size_t ws_bytes,
                          moe_stream_t stream);
 
+/* A cudaEvent_t. */
+typedef struct CUevent_st *moe_event_t;
+
+/* Stages of one layer call, in launch order. Token choice: ROUTE = router GEMM,
+ * softmax, top-k, gates and per-tile histogram (noisy gating: both projections and
+ * the noise); SCAN = counts, capacity, offsets and the GEMM tile table; PERMUTE =
+ * ranks, drops and the row gather; SHARED_FFN = the always-on experts; EXPERT_FFN =
+ * the routed experts' GEMMs; COMBINE = the gate-weighted sum. Expert choice: ROUTE =
+ * router and each expert's picks, SCAN = tile table, PERMUTE = row gather,
+ * SHARED_FFN = nothing. */
+enum {
+  MOE_STAGE_ROUTE = 0,
+  MOE_STAGE_SCAN = 1,
+  MOE_STAGE_PERMUTE = 2,
+  MOE_STAGE_SHARED_FFN = 3,
+  MOE_STAGE_EXPERT_FFN = 4,
+  MOE_STAGE_COMBINE = 5,
+  MOE_STAGE_COUNT = 6
+};
+
+/* Events that moe_forward_staged records on `stream`: ev[i] before stage i and
+ * ev[MOE_STAGE_COUNT] after the last one, so stage i's device time is the elapsed
+ * time from ev[i] to ev[i + 1]. NULL entries are not recorded. The caller creates the
+ * events (with timing enabled) and owns them. */
+typedef struct {
+  moe_event_t ev[MOE_STAGE_COUNT + 1];
+} moe_stage_events_t;
+
+/* moe_forward that also records `events` (nullable) at its stage boundaries and
+ * marks each stage with an NVTX range (named "moe_route", "moe_scan", ...). The
+ * kernels and results are those of moe_forward; a failed event record returns
+ * MOE_ERR_CUDA. */
+moe_status_t moe_forward_staged(const moe_cfg_t *cfg, const moe_weights_t *w, const void *x,
+                                void *y, float *aux_out, const moe_taps_t *taps,
+                                const moe_stage_events_t *events, void *ws, size_t ws_bytes,
+                                moe_stream_t stream);
+
 /* Noisy top-k gating, the training mode of youngju.dev (ja) "TopKGating" (Noisy Top-K
  * Gating): the logits are z + softplus(x W_noise^T) * eps, z as in moe_route, softplus
  * the identity above 20 (as F.softplus), eps [T, E] fp32 standard normal draws made by
@@ -250,6 +289,12 @@ moe_status_t moe_route_noisy(const moe_cfg_t *cfg, const moe_weights_t *w, const
 moe_status_t moe_forward_noisy(const moe_cfg_t *cfg, const moe_weights_t *w, const void *x,
                                const float *eps, void *y, float *aux_out, const moe_taps_t *taps,
                                void *ws, size_t ws_bytes, moe_stream_t stream);
+
+/* moe_forward_noisy with stage events (see moe_forward_staged). */
+moe_status_t moe_forward_noisy_staged(const moe_cfg_t *cfg, const moe_weights_t *w,
+                                      const void *x, const float *eps, void *y, float *aux_out,
+                                      const moe_taps_t *taps, const moe_stage_events_t *events,
+                                      void *ws, size_t ws_bytes, moe_stream_t stream);
 
 /* Expert-Choice routing step (youngju.dev (zh) "ExpertChoiceRouter", youngju.dev (ja)
  * "ExpertChoiceGating"): logits as in moe_route, then for every expert e its C =

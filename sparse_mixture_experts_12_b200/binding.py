@@ -30,7 +30,11 @@ EXPORTED = ("moe_workspace_size", "moe_workspace_init", "moe_route", "moe_route_
             "moe_route_expert_choice", "moe_permute", "moe_permute_noalloc", "moe_forward_noisy",
             "moe_expert_ffn", "moe_combine", "moe_aux_stats", "moe_forward",
             "moe_route_shard", "moe_permute_shard", "moe_forward_shard", "moe_aux_finalize",
+            "moe_forward_staged", "moe_forward_noisy_staged",
             "moe_last_device_error", "moe_status_string")
+
+# stages of one layer call (MOE_STAGE_*), in launch order
+STAGES = ("route", "scan", "permute", "shared_ffn", "expert_ffn", "combine")
 
 
 class MoeError(RuntimeError):
@@ -65,6 +69,10 @@ class MoeShard(ctypes.Structure):
                 ("shard", ctypes.c_int32), ("counts_all", ctypes.c_void_p)]
 
 
+class MoeStageEvents(ctypes.Structure):
+    _fields_ = [("ev", ctypes.c_void_p * (len(STAGES) + 1))]
+
+
 def lib_path() -> str:
     return _LIB_PATH
 
@@ -95,6 +103,10 @@ def load() -> ctypes.CDLL:
         "moe_forward_shard": [cfgp, ctypes.POINTER(MoeShard), wp, P, ctypes.POINTER(MoeTaps), P,
                               P, S, P],
         "moe_aux_finalize": [cfgp, ctypes.c_longlong, P, P, P],
+        "moe_forward_staged": [cfgp, wp, P, P, P, ctypes.POINTER(MoeTaps),
+                               ctypes.POINTER(MoeStageEvents), P, S, P],
+        "moe_forward_noisy_staged": [cfgp, wp, P, P, P, P, ctypes.POINTER(MoeTaps),
+                                     ctypes.POINTER(MoeStageEvents), P, S, P],
         "moe_last_device_error": [P, ctypes.POINTER(ctypes.c_int32),
                                   ctypes.POINTER(ctypes.c_int32), P],
     }
@@ -119,6 +131,22 @@ def _ptr(t: Optional[torch.Tensor]):
 
 def _stream():
     return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _taps(taps: Optional[dict]):
+    if taps is None:
+        return None
+    return MoeTaps(**{k: _ptr(taps.get(k)) for k, _ in MoeTaps._fields_})
+
+
+def stage_events(events) -> MoeStageEvents:
+    """MoeStageEvents from len(STAGES) + 1 torch.cuda.Event (None entries allowed)."""
+    if len(events) != len(STAGES) + 1:
+        raise ValueError(f"{len(STAGES) + 1} events expected, got {len(events)}")
+    ev = MoeStageEvents()
+    for i, e in enumerate(events):
+        ev.ev[i] = None if e is None else e.cuda_event
+    return ev
 
 
 def make_cfg(w: synth.Workload, **over) -> MoeCfg:
@@ -166,32 +194,45 @@ class MoELayer:
 
     # -------------------------------------------------------------- whole layer
     def forward(self, x: torch.Tensor, y: Optional[torch.Tensor] = None,
-                aux: Optional[torch.Tensor] = None, taps: Optional[dict] = None) -> torch.Tensor:
+                aux: Optional[torch.Tensor] = None, taps: Optional[dict] = None,
+                events: Optional[list] = None) -> torch.Tensor:
+        """The whole layer (moe_forward). ``events``: len(STAGES) + 1 torch.cuda.Event
+        objects recorded at the stage boundaries (moe_forward_staged)."""
         if y is None:
             y = torch.empty_like(x)
-        tp = None
-        if taps is not None:
-            tp = MoeTaps(**{k: _ptr(taps.get(k)) for k, _ in MoeTaps._fields_})
-        _check(self.lib.moe_forward(ctypes.byref(self.cfg), ctypes.byref(self.weights), _ptr(x),
-                                    _ptr(y), _ptr(aux),
-                                    ctypes.byref(tp) if tp is not None else None,
-                                    _ptr(self.ws), self.ws.numel(), _stream()), "moe_forward")
+        tp = _taps(taps)
+        tpr = ctypes.byref(tp) if tp is not None else None
+        if events is None:
+            _check(self.lib.moe_forward(ctypes.byref(self.cfg), ctypes.byref(self.weights),
+                                        _ptr(x), _ptr(y), _ptr(aux), tpr, _ptr(self.ws),
+                                        self.ws.numel(), _stream()), "moe_forward")
+        else:
+            ev = stage_events(events)
+            _check(self.lib.moe_forward_staged(ctypes.byref(self.cfg),
+                                               ctypes.byref(self.weights), _ptr(x), _ptr(y),
+                                               _ptr(aux), tpr, ctypes.byref(ev), _ptr(self.ws),
+                                               self.ws.numel(), _stream()), "moe_forward_staged")
         return y
 
     def forward_noisy(self, x: torch.Tensor, eps: torch.Tensor, y: Optional[torch.Tensor] = None,
-                      aux: Optional[torch.Tensor] = None,
-                      taps: Optional[dict] = None) -> torch.Tensor:
+                      aux: Optional[torch.Tensor] = None, taps: Optional[dict] = None,
+                      events: Optional[list] = None) -> torch.Tensor:
         """The layer with noisy top-k gating; eps [T, E] fp32 standard normal draws."""
         if y is None:
             y = torch.empty_like(x)
-        tp = None
-        if taps is not None:
-            tp = MoeTaps(**{k: _ptr(taps.get(k)) for k, _ in MoeTaps._fields_})
-        _check(self.lib.moe_forward_noisy(ctypes.byref(self.cfg), ctypes.byref(self.weights),
-                                          _ptr(x), _ptr(eps), _ptr(y), _ptr(aux),
-                                          ctypes.byref(tp) if tp is not None else None,
-                                          _ptr(self.ws), self.ws.numel(), _stream()),
-               "moe_forward_noisy")
+        tp = _taps(taps)
+        tpr = ctypes.byref(tp) if tp is not None else None
+        if events is None:
+            _check(self.lib.moe_forward_noisy(ctypes.byref(self.cfg), ctypes.byref(self.weights),
+                                              _ptr(x), _ptr(eps), _ptr(y), _ptr(aux), tpr,
+                                              _ptr(self.ws), self.ws.numel(), _stream()),
+                   "moe_forward_noisy")
+        else:
+            ev = stage_events(events)
+            _check(self.lib.moe_forward_noisy_staged(
+                ctypes.byref(self.cfg), ctypes.byref(self.weights), _ptr(x), _ptr(eps), _ptr(y),
+                _ptr(aux), tpr, ctypes.byref(ev), _ptr(self.ws), self.ws.numel(), _stream()),
+                "moe_forward_noisy_staged")
         return y
 
     def new_taps(self) -> dict:

@@ -5,6 +5,8 @@
 
 #include <climits>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "shard.cuh"
 
 #define MOE_API extern "C" __attribute__((visibility("default")))
@@ -186,6 +188,43 @@ moe_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE
   } while (0)
 #define MOE_CUDA(expr) MOE_TRY(cuda_status(expr))
 
+// Stage boundaries of one layer call: an event (when the caller gave one) and an
+// NVTX range per stage. Stages are entered in increasing order; skipped stages
+// still record their event, so every interval is defined.
+class Stages {
+ public:
+  Stages(const moe_stage_events_t *ev, cudaStream_t st) : ev_(ev), st_(st) {}
+  ~Stages() {
+    if (open_) nvtxRangePop();
+  }
+  moe_status_t enter(int stage) {
+    static const char *kNames[MOE_STAGE_COUNT] = {"moe_route", "moe_scan", "moe_permute",
+                                                  "moe_shared_ffn", "moe_expert_ffn",
+                                                  "moe_combine"};
+    for (; next_ <= stage; ++next_) MOE_TRY(record(next_));
+    if (open_) nvtxRangePop();
+    nvtxRangePushA(kNames[stage]);
+    open_ = true;
+    return MOE_OK;
+  }
+  moe_status_t finish() {
+    for (; next_ <= MOE_STAGE_COUNT; ++next_) MOE_TRY(record(next_));
+    if (open_) nvtxRangePop();
+    open_ = false;
+    return MOE_OK;
+  }
+
+ private:
+  moe_status_t record(int i) {
+    if (ev_ == nullptr || ev_->ev[i] == nullptr) return MOE_OK;
+    return cuda_status(cudaEventRecord(reinterpret_cast<cudaEvent_t>(ev_->ev[i]), st_));
+  }
+  const moe_stage_events_t *ev_;
+  cudaStream_t st_;
+  int next_ = 0;
+  bool open_ = false;
+};
+
 int capacity_of(const moe_cfg_t &c) {
   if (!(c.capacity_factor > 0.f)) return -1;
   const double cap = floor((double)c.capacity_factor * (double)c.n_tokens * (double)c.top_k /
@@ -323,7 +362,8 @@ moe_status_t ec_route(const moe_cfg_t &c, const moe_weights_t *w, const void *x,
 
 // Expert-Choice forward: route, gather each expert's C rows, expert FFNs, combine.
 moe_status_t ec_forward(const moe_cfg_t &c, const moe_weights_t *w, const void *x, void *y,
-                        float *logits, void *ws, const Layout &L, cudaStream_t stream) {
+                        float *logits, void *ws, const Layout &L, cudaStream_t stream,
+                        Stages &sg) {
   const int T = c.n_tokens, E = c.n_experts, C = (int)ec_picks(c);
   int32_t *err = at<int32_t>(ws, L, B_ERR);
   int32_t *ec_idx = at<int32_t>(ws, L, B_EC_IDX);
@@ -331,18 +371,23 @@ moe_status_t ec_forward(const moe_cfg_t &c, const moe_weights_t *w, const void *
   int32_t *slot = at<int32_t>(ws, L, B_EC_SLOT);
   int32_t *offsets = at<int32_t>(ws, L, B_OFFSETS);
   int32_t *mprefix = at<int32_t>(ws, L, B_MPREFIX);
+  MOE_TRY(sg.enter(MOE_STAGE_ROUTE));
   MOE_TRY(ec_route(c, w, x, logits, ec_idx, ec_score, slot, offsets, ws, L, stream));
   const int eb = c.dtype == MOE_DTYPE_F32 ? 4 : 2;
   void *x_perm = at<void>(ws, L, B_XPERM);
   void *y_perm = at<void>(ws, L, B_YPERM);
-  MOE_CUDA(launch_ec_gather(x, T, ec_idx, E * C, c.d_model * eb, x_perm, stream));
+  MOE_TRY(sg.enter(MOE_STAGE_SCAN));
   MOE_CUDA(launch_tile_table(offsets, E, E * C, mprefix, err, stream));
+  MOE_TRY(sg.enter(MOE_STAGE_PERMUTE));
+  MOE_CUDA(launch_ec_gather(x, T, ec_idx, E * C, c.d_model * eb, x_perm, stream));
   float *part = layout_size(L, B_YPART) > 0 ? at<float>(ws, L, B_YPART) : nullptr;
   GroupedFfnArgs a = routed_ffn_args(c, *w, x_perm, offsets, mprefix, at<void>(ws, L, B_H),
                                      y_perm, err, C, part);  // E*C rows, C per expert
+  MOE_TRY(sg.enter(MOE_STAGE_EXPERT_FFN));
   MOE_CUDA(run_ffn(c, a, stream));
+  MOE_TRY(sg.enter(MOE_STAGE_COMBINE));
   MOE_CUDA(launch_ec_combine(y_perm, slot, ec_score, T, E, C, c.d_model, c.dtype, y, stream));
-  return MOE_OK;
+  return sg.finish();
 }
 
 }  // namespace
@@ -595,7 +640,8 @@ namespace {
 moe_status_t forward_impl(const moe_cfg_t *cfg, const moe_weights_t *w, const void *x,
                           const float *eps, void *y, float *aux_out, const moe_taps_t *taps,
                           void *ws, size_t ws_bytes, moe_stream_t stream,
-                          const moe_shard_t *sh = nullptr) {
+                          const moe_shard_t *sh = nullptr,
+                          const moe_stage_events_t *events = nullptr) {
   MOE_TRY(check_cfg(cfg));
   MOE_TRY(check_ws(cfg, ws, ws_bytes));
   if (sh != nullptr) {
@@ -605,7 +651,8 @@ moe_status_t forward_impl(const moe_cfg_t *cfg, const moe_weights_t *w, const vo
         (taps == nullptr || taps->topk_idx == nullptr || taps->topk_gate == nullptr))
       return MOE_ERR_INVALID_ARG;
   }
-  if (cfg->n_tokens == 0) return MOE_OK;  // nothing is read or written
+  Stages sg(events, stream);
+  if (cfg->n_tokens == 0) return sg.finish();  // nothing is read or written
   if (w == nullptr) return MOE_ERR_INVALID_ARG;
   MOE_TRY(check_ptrs({{x, true}, {y, true}, {aux_out, false}, {w->w_router, sh == nullptr},
                       {w->b_router, false}, {w->logit_bias, false}}));
@@ -624,7 +671,7 @@ moe_status_t forward_impl(const moe_cfg_t *cfg, const moe_weights_t *w, const vo
   float *logits = tp.logits ? tp.logits : at<float>(ws, L, B_LOGITS);
   if (expert_choice(c)) {
     if (aux_out != nullptr || eps != nullptr) return MOE_ERR_INVALID_ARG;
-    return ec_forward(c, w, x, y, logits, ws, L, stream);
+    return ec_forward(c, w, x, y, logits, ws, L, stream, sg);
   }
   if (eps != nullptr) MOE_TRY(check_ptrs({{eps, true}, {w->w_noise, true}}));
   int32_t *idx = tp.topk_idx ? tp.topk_idx : at<int32_t>(ws, L, B_IDX);
@@ -639,6 +686,7 @@ moe_status_t forward_impl(const moe_cfg_t *cfg, const moe_weights_t *w, const vo
 
   // 1. router GEMM + softmax + top-k + gates + per-tile histogram (noisy gating:
   //    the noisy logits first, then the same steps on them as the input)
+  MOE_TRY(sg.enter(MOE_STAGE_ROUTE));
   RouterArgs r{};
   if (eps != nullptr) {
     MOE_TRY(noisy_logits(c, w, x, eps, logits, ws, L, stream));
@@ -668,6 +716,7 @@ moe_status_t forward_impl(const moe_cfg_t *cfg, const moe_weights_t *w, const vo
                                 stream));
   }
   // 2. scan: counts, capacity, offsets, GEMM tile table (+ aux statistics)
+  MOE_TRY(sg.enter(MOE_STAGE_SCAN));
   ScanArgs s{};
   s.tile_counts = r.tile_counts;
   s.tile_base = at<int32_t>(ws, L, B_TILE_BASE);
@@ -693,6 +742,7 @@ moe_status_t forward_impl(const moe_cfg_t *cfg, const moe_weights_t *w, const vo
     MOE_CUDA(launch_scan_shard(s, sc, stream));
   }
   // 3. stable permutation with capacity drops + row gather
+  MOE_TRY(sg.enter(MOE_STAGE_PERMUTE));
   ScatterArgs p{};
   p.x = x;
   p.topk_idx = idx;
@@ -713,6 +763,7 @@ moe_status_t forward_impl(const moe_cfg_t *cfg, const moe_weights_t *w, const vo
   // 4. always-on shared experts: one SwiGLU over all tokens, experts concatenated along F
   float *sh_y = nullptr;
   float *part = layout_size(L, B_YPART) > 0 ? at<float>(ws, L, B_YPART) : nullptr;
+  MOE_TRY(sg.enter(MOE_STAGE_SHARED_FFN));
   if (c.n_shared > 0) {
     GroupedFfnArgs a{};
     a.a = x;
@@ -740,8 +791,10 @@ moe_status_t forward_impl(const moe_cfg_t *cfg, const moe_weights_t *w, const vo
   //    any expert, so no group holds more than T rows)
   GroupedFfnArgs a = routed_ffn_args(c, *w, p.x_perm, offsets, mprefix, at<void>(ws, L, B_H),
                                      at<void>(ws, L, B_YPERM), err, c.n_tokens, part);
+  MOE_TRY(sg.enter(MOE_STAGE_EXPERT_FFN));
   MOE_CUDA(run_ffn(c, a, stream));
   // 6. gate-weighted combine (+ shared output)
+  MOE_TRY(sg.enter(MOE_STAGE_COMBINE));
   CombineArgs cb{};
   cb.y_perm = a.out;
   cb.inv = inv;
@@ -754,7 +807,7 @@ moe_status_t forward_impl(const moe_cfg_t *cfg, const moe_weights_t *w, const vo
   cb.R = c.n_tokens * c.top_k;
   cb.err = err;
   MOE_CUDA(launch_combine(cb, c.dtype, stream));
-  return MOE_OK;
+  return sg.finish();
 }
 }  // namespace
 }  // namespace moe
@@ -771,6 +824,24 @@ MOE_API moe_status_t moe_forward_noisy(const moe_cfg_t *cfg, const moe_weights_t
                                        size_t ws_bytes, moe_stream_t stream) {
   if (eps == nullptr) return MOE_ERR_INVALID_ARG;
   return forward_impl(cfg, w, x, eps, y, aux_out, taps, ws, ws_bytes, stream);
+}
+
+MOE_API moe_status_t moe_forward_staged(const moe_cfg_t *cfg, const moe_weights_t *w,
+                                        const void *x, void *y, float *aux_out,
+                                        const moe_taps_t *taps, const moe_stage_events_t *events,
+                                        void *ws, size_t ws_bytes, moe_stream_t stream) {
+  return forward_impl(cfg, w, x, nullptr, y, aux_out, taps, ws, ws_bytes, stream, nullptr,
+                      events);
+}
+
+MOE_API moe_status_t moe_forward_noisy_staged(const moe_cfg_t *cfg, const moe_weights_t *w,
+                                              const void *x, const float *eps, void *y,
+                                              float *aux_out, const moe_taps_t *taps,
+                                              const moe_stage_events_t *events, void *ws,
+                                              size_t ws_bytes, moe_stream_t stream) {
+  if (eps == nullptr) return MOE_ERR_INVALID_ARG;
+  return forward_impl(cfg, w, x, eps, y, aux_out, taps, ws, ws_bytes, stream, nullptr,
+                      events);
 }
 
 // ----------------------------------------------------- token-sharded batches

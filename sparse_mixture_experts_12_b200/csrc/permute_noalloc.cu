@@ -16,6 +16,8 @@
 // read is written earlier in the same call, so nothing needs clearing between
 // calls. Index errors are not recorded anywhere: a pair whose expert index is out
 // of range is treated as dropped (inv = -1).
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <math.h>
 
 #include <climits>
@@ -37,24 +39,81 @@ constexpr size_t kNoAllocInts = 2 * (size_t)kNoAllocMaxTileEntries + kMaxExperts
 
 static __device__ __align__(256) int32_t g_permute_scratch[kNoAllocInts];
 
-constexpr int kMaxDevices = 64;
-int32_t *g_scratch_addr[kMaxDevices];
+// The device address of g_permute_scratch belongs to a CUDA context: each context
+// that loads the library has its own copy of the array. So the address is cached per
+// context, keyed on the driver's context ID, which is unique for the life of the
+// process (a context created after a reset, or a non-primary context, gets a new
+// ID even where its handle repeats an old one). Where the ID cannot be read, the
+// address is looked up on every call (cudaGetSymbolAddress allocates nothing).
+struct ScratchEntry {
+  unsigned long long ctx_id;
+  int32_t *addr;
+};
+constexpr int kScratchCache = 64;
+ScratchEntry g_scratch_cache[kScratchCache];
+int g_scratch_used = 0;
+int g_scratch_next = 0;
 std::mutex g_scratch_mu;
 
-// Device address of g_permute_scratch on the current device, looked up once per
-// device (in host code the symbol itself is only a host-side stand-in).
-moe_status_t scratch_on_current_device(int32_t **out) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
-  if (dev < 0 || dev >= kMaxDevices) return MOE_ERR_UNSUPPORTED;
-  std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (g_scratch_addr[dev] == nullptr) {
+struct CtxQuery {
+  PFN_cuCtxGetCurrent_v4000 current = nullptr;
+  PFN_cuCtxGetId_v12000 get_id = nullptr;
+};
+
+const CtxQuery &ctx_query() {
+  static CtxQuery q;
+  static std::once_flag once;
+  std::call_once(once, [] {
     void *p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_permute_scratch) != cudaSuccess || p == nullptr)
-      return MOE_ERR_CUDA;
-    g_scratch_addr[dev] = static_cast<int32_t *>(p);
+    cudaDriverEntryPointQueryResult r;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &r) == cudaSuccess &&
+        r == cudaDriverEntryPointSuccess)
+      q.current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &r) == cudaSuccess &&
+        r == cudaDriverEntryPointSuccess)
+      q.get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(p);
+  });
+  return q;
+}
+
+// ID of the context current on this thread; false when there is none (the runtime
+// has not made the device's primary context current yet) or it cannot be read.
+bool current_context_id(unsigned long long *id) {
+  const CtxQuery &q = ctx_query();
+  if (q.current == nullptr || q.get_id == nullptr) return false;
+  CUcontext ctx = nullptr;
+  if (q.current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return false;
+  return q.get_id(ctx, id) == CUDA_SUCCESS;
+}
+
+// Device address of g_permute_scratch in the current context (in host code the
+// symbol itself is only a host-side stand-in).
+moe_status_t scratch_in_current_context(int32_t **out) {
+  unsigned long long id = 0;
+  bool have_id = current_context_id(&id);
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (have_id) {
+    for (int i = 0; i < g_scratch_used; ++i) {
+      if (g_scratch_cache[i].ctx_id == id) {
+        *out = g_scratch_cache[i].addr;
+        return MOE_OK;
+      }
+    }
   }
-  *out = g_scratch_addr[dev];
+  // also makes the current device's primary context current when none is
+  void *p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_permute_scratch) != cudaSuccess || p == nullptr)
+    return MOE_ERR_CUDA;
+  if (!have_id) have_id = current_context_id(&id);
+  if (have_id) {
+    ScratchEntry &slot = g_scratch_cache[g_scratch_next];
+    slot.ctx_id = id;
+    slot.addr = static_cast<int32_t *>(p);
+    g_scratch_next = (g_scratch_next + 1) % kScratchCache;
+    if (g_scratch_used < kScratchCache) ++g_scratch_used;
+  }
+  *out = static_cast<int32_t *>(p);
   return MOE_OK;
 }
 
@@ -87,7 +146,7 @@ MOE_API moe_status_t moe_permute_noalloc(const moe_cfg_t *cfg, const void *x,
   const int NT = ceil_div(c.n_tokens > 0 ? c.n_tokens : 1, router_bm(E));
   if ((long long)E * NT > kNoAllocMaxTileEntries) return MOE_ERR_WORKSPACE;  // beyond the static scratch
   int32_t *scratch = nullptr;
-  moe_status_t st = scratch_on_current_device(&scratch);
+  moe_status_t st = scratch_in_current_context(&scratch);
   if (st != MOE_OK) return st;
   cudaStream_t s = stream;
   if (c.n_tokens == 0) {

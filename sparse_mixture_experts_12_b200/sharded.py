@@ -40,6 +40,43 @@ def shard_bounds(n_tokens_total: int, n_shards: int):
     return out
 
 
+def check_placement(shard: int, n_shards: int, group=None):
+    """A shard's place must be its rank in the process group. Without a group only
+    the one-shard layout is valid: the other shards' counts would never arrive, and
+    the capacity left to this shard could not be computed."""
+    if not 0 <= shard < n_shards:
+        raise ValueError(f"shard {shard} is not one of {n_shards} shards")
+    if not dist.is_initialized():
+        if n_shards != 1:
+            raise ValueError(f"{n_shards} shards need a process group of {n_shards} ranks; "
+                             "none is initialised")
+        return
+    if dist.get_world_size(group) != n_shards or dist.get_rank(group) != shard:
+        raise ValueError("shard / n_shards must be this rank's place in the process group")
+
+
+def check_counts_all(counts_all: torch.Tensor, n_shards: int, n_experts: int, device):
+    """counts_all must be every shard's pre-drop counts, [n_shards, E] int32 on the
+    layer's device: the library reads n_shards * E of them through a raw pointer."""
+    if tuple(counts_all.shape) != (n_shards, n_experts):
+        raise ValueError(f"counts_all has shape {tuple(counts_all.shape)}, "
+                         f"expected ({n_shards}, {n_experts})")
+    if counts_all.dtype != torch.int32:
+        raise ValueError(f"counts_all must be int32, not {counts_all.dtype}")
+    if not _same_device(counts_all.device, device):
+        raise ValueError(f"counts_all is on {counts_all.device}, the layer on {device}")
+
+
+def _same_device(a, b) -> bool:
+    a, b = torch.device(a), torch.device(b)
+    if a.type != b.type:
+        return False
+    if a.type != "cuda":
+        return True
+    cur = torch.cuda.current_device()
+    return (cur if a.index is None else a.index) == (cur if b.index is None else b.index)
+
+
 def forward_sharded(steps, x, n_experts: int, group=None, want_aux: bool = False, y=None):
     """One rank's part of the layer over a token-sharded batch.
 
@@ -70,11 +107,7 @@ class ShardedMoELayer:
 
     def __init__(self, workload: synth.Workload, params: dict, shard: int, n_shards: int,
                  device="cuda", group=None):
-        if not 0 <= shard < n_shards:
-            raise ValueError(f"shard {shard} is not one of {n_shards} shards")
-        if dist.is_initialized() and (dist.get_world_size(group) != n_shards
-                                      or dist.get_rank(group) != shard):
-            raise ValueError("shard / n_shards must be this rank's place in the process group")
+        check_placement(shard, n_shards, group)
         self.n_tokens_total = workload.T
         self.shard, self.n_shards, self.group = shard, n_shards, group
         a, b = shard_bounds(workload.T, n_shards)[shard]
@@ -94,6 +127,7 @@ class ShardedMoELayer:
         return counts, part, routed
 
     def forward_shard(self, x, routed, counts_all, y=None):
+        check_counts_all(counts_all, self.n_shards, self.local.n_experts, self.layer.device)
         counts_all = counts_all.contiguous()
         desc = B.MoeShard(n_tokens_total=self.n_tokens_total, n_shards=self.n_shards,
                           shard=self.shard, counts_all=counts_all.data_ptr())

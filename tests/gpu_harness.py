@@ -104,3 +104,41 @@ def routing_compare(gpu_idx: np.ndarray, ref_logits: np.ndarray, ref_idx: np.nda
         hit = np.isin(ref_idx, list(experts)).any(axis=1) | np.isin(gpu_idx, list(experts)).any(axis=1)
         affected |= set(np.nonzero(later & hit)[0].tolist())
     return mism, affected, int((margin < MARGIN).sum())
+
+
+ROW_TILE = 128  # rows of one grouped-GEMM M tile
+
+
+def tile_rows(offsets) -> list:
+    """(expert, first row, last row) of every ROW_TILE-row tile of the expert-contiguous
+    rows: expert e owns rows [offsets[e], offsets[e+1])."""
+    out = []
+    offsets = np.asarray(offsets, dtype=np.int64)
+    for e in range(len(offsets) - 1):
+        a, b = int(offsets[e]), int(offsets[e + 1])
+        for r0 in range(a, b, ROW_TILE):
+            out.append((e, r0, min(r0 + ROW_TILE, b) - 1))
+    return out
+
+
+def tile_cover_tokens(row_token, offsets, T: int, n_strided: int = 48, extra=()):
+    """Tokens to compare at full size: the tokens of the first, the middle and the
+    last row of every expert tile (row_token maps a row to its token), plus a strided
+    sample and ``extra``. Returns (sorted unique tokens, tile list)."""
+    tiles = tile_rows(offsets)
+    toks = set(synth.token_sample(T, n_strided).tolist())
+    toks |= set(int(t) for t in extra)
+    for _, r0, r1 in tiles:
+        for r in (r0, (r0 + r1) // 2, r1):
+            toks.add(int(row_token[r]))
+    return np.array(sorted(toks), dtype=np.int64), tiles
+
+
+def tiles_covered(tiles, row_token, compared) -> int:
+    """Tiles with at least one row whose token is among ``compared``."""
+    cmp = set(int(t) for t in compared)
+    n = 0
+    for _, r0, r1 in tiles:
+        if any(int(row_token[r]) in cmp for r in range(r0, r1 + 1)):
+            n += 1
+    return n

@@ -58,7 +58,9 @@ def test_struct_layout_matches_header(tmp_path):
         + "".join(f"  F(moe_shard_t, {n});\n" for n, _ in B.MoeShard._fields_)
         + '  printf("size moe_cfg_t %zu\\nsize moe_weights_t %zu\\nsize moe_taps_t %zu\\n",'
           " sizeof(moe_cfg_t), sizeof(moe_weights_t), sizeof(moe_taps_t));\n"
-        + '  printf("size moe_shard_t %zu\\n", sizeof(moe_shard_t));\n  return 0;\n}\n')
+        + '  printf("size moe_shard_t %zu\\n", sizeof(moe_shard_t));\n'
+        + '  printf("size moe_stage_events_t %zu\\n", sizeof(moe_stage_events_t));\n'
+        + '  printf("stages count %d\\n", (int)MOE_STAGE_COUNT);\n  return 0;\n}\n')
     exe = tmp_path / "layout"
     subprocess.run(["gcc", "-std=c99", f"-I{os.path.dirname(HEADER)}", str(prog), "-o", str(exe)],
                    check=True)
@@ -73,6 +75,8 @@ def test_struct_layout_matches_header(tmp_path):
         for n, _ in cls._fields_:
             assert got[(st, n)] == getattr(cls, n).offset, (st, n)
         assert got[("size", st)] == ctypes.sizeof(cls)
+    assert got[("size", "moe_stage_events_t")] == ctypes.sizeof(B.MoeStageEvents)
+    assert got[("stages", "count")] == len(B.STAGES)
 
 
 def _status(lib, cfg):

@@ -335,12 +335,28 @@ def _forward_and_compare(wl: synth.Workload, seed: int, n_sample=None, check_ful
     assert code == 0, (code, info)
     P = H.oracle_params(inp)
     T, E, k = wl.T, wl.n_experts, wl.top_k
-    tokens = None if n_sample is None else synth.token_sample(T, n_sample).numpy()
     ref_logits = None
     if eps is not None:
         ref_logits = O.noisy_router_logits(P["x"], P["w_router"], P["w_noise"], eps.numpy(),
                                            P["b_router"], P["logit_bias"])
-    yref, r = O.moe_forward(P["x"], P, tokens=tokens, logits=ref_logits, **H.oracle_kwargs(wl))
+    kw = H.oracle_kwargs(wl)
+    tokens = tiles = None
+    if n_sample is not None:
+        # compared tokens from the oracle's routing: the first and the last row of
+        # every (expert, 128-row tile) of the grouped GEMMs, of every tile of the
+        # shared experts' GEMM (its rows are the tokens), some dropped tokens, and
+        # a strided sample
+        r0 = O.route(P["x"], P, top_k=k, gate_mode=kw["gate_mode"],
+                     capacity_factor=wl.capacity_factor, logits=ref_logits)
+        ref_logits = r0["logits"]
+        dropped = np.nonzero(~r0["kept"].all(axis=1))[0]
+        extra = list(dropped[np.unique(np.linspace(0, len(dropped) - 1, 8).astype(int))]) \
+            if len(dropped) else []
+        if wl.n_shared > 0:
+            for t0 in range(0, T, H.ROW_TILE):
+                extra += [t0, min(t0 + H.ROW_TILE, T) - 1]
+        tokens, tiles = H.tile_cover_tokens(r0["perm"], r0["offsets"], T, n_sample, extra)
+    yref, r = O.moe_forward(P["x"], P, tokens=tokens, logits=ref_logits, **kw)
     # logits against the fp32 accumulation bound
     extra = np.zeros(E)
     if P["b_router"] is not None:
@@ -389,7 +405,13 @@ def _forward_and_compare(wl: synth.Workload, seed: int, n_sample=None, check_ful
     assert np.abs(a[3:3 + E] - f).max() <= len(mism) / (T * k) + 1e-7
     assert np.allclose(a[3 + E:], Pm, rtol=1e-4, atol=1e-6)
     assert abs(a[0] - auxv) <= 1e-4 * auxv + wl.aux_alpha * E * len(mism) / (T * k)
-    H.report("forward", workload=wl.name, T=T, compared=int(keep.sum()),
+    cover = {}
+    if tiles is not None:
+        covered = H.tiles_covered(tiles, r["perm"], sel[keep])
+        cover = dict(tiles=len(tiles), tiles_covered=covered)
+        if len(mism) == 0:  # every expert tile of the GEMMs has a compared row
+            assert covered == len(tiles), (covered, len(tiles))
+    H.report("forward", workload=wl.name, T=T, compared=int(keep.sum()), **cover,
              worst_rel_err=float(err.max()) if len(err) else 0.0,
              p99_rel_err=float(np.quantile(err, 0.99)) if len(err) else 0.0,
              routing_mismatch=len(mism), near_tie_tokens=n_near, excluded=len(affected),
@@ -509,9 +531,17 @@ def _ec_forward_and_compare(wl: synth.Workload, seed: int, n_sample=None):
     assert code == 0, (code, info)
     P = H.oracle_params(inp)
     T, E = wl.T, wl.n_experts
-    tokens = None if n_sample is None else synth.token_sample(T, n_sample).numpy()
+    tokens = tiles = None
+    z0 = None
+    if n_sample is not None:
+        # the first and the last row of every 128-row tile of every expert's C picks
+        # (expert e owns rows [e*C, (e+1)*C), row e*C + j holding its j-th pick)
+        z0 = O.router_logits(P["x"], P["w_router"], P["b_router"], P["logit_bias"])
+        C0 = O.expert_choice_capacity(wl.capacity_factor, T, E)
+        picks = O.expert_choice_select(z0, C0)
+        tokens, tiles = H.tile_cover_tokens(picks.ravel(), np.arange(E + 1) * C0, T, n_sample)
     yref, r = O.expert_choice_forward(P["x"], P, capacity_factor=wl.capacity_factor,
-                                      act=H.ACT[wl.act], tokens=tokens)
+                                      act=H.ACT[wl.act], logits=z0, tokens=tokens)
     extra = np.zeros(E)
     if P["b_router"] is not None:
         extra += np.abs(P["b_router"])
@@ -540,7 +570,13 @@ def _ec_forward_and_compare(wl: synth.Workload, seed: int, n_sample=None):
     err = H.max_rel_err(yg[keep], yref[keep])
     taken = np.zeros(T, dtype=bool)
     taken[np.asarray(r["idx"]).ravel()] = True
+    cover = {}
+    if tiles is not None:
+        covered = H.tiles_covered(tiles, np.asarray(r["idx"]).ravel(), sel[keep])
+        cover = dict(tiles=len(tiles), tiles_covered=covered)
+        assert covered == len(tiles), (covered, len(tiles))
     H.report("forward_expert_choice", workload=wl.name, T=T, C=C, compared=int(keep.sum()),
+             **cover,
              near_tie_tokens=len(near), untaken_tokens=int((~taken).sum()),
              worst_rel_err=float(err.max()) if len(err) else 0.0)
     assert err.max() <= H.TOL[wl.dtype], (wl.name, float(err.max()))

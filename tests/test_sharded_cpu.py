@@ -112,6 +112,31 @@ def test_sharded_layer_checks_its_place():
         S.ShardedMoELayer(WL, {}, shard=2, n_shards=2, device="cpu")
 
 
+def test_several_shards_need_a_process_group():
+    """Without a process group, shard 1 of 2 would pass a one-row counts_all while
+    the library reads the counts of shard 0 from a second row: rejected up front."""
+    assert not dist.is_initialized()
+    with pytest.raises(ValueError, match="process group"):
+        S.ShardedMoELayer(WL, {}, shard=1, n_shards=2, device="cpu")
+    with pytest.raises(ValueError, match="process group"):
+        S.ShardedMoELayer(WL, {}, shard=0, n_shards=2, device="cpu")
+    S.check_placement(0, 1)  # one shard is the whole batch
+
+
+def test_counts_all_is_checked_before_the_descriptor_is_built():
+    E = WL.n_experts
+    ok = torch.zeros((2, E), dtype=torch.int32)
+    S.check_counts_all(ok, 2, E, "cpu")
+    with pytest.raises(ValueError, match="shape"):
+        S.check_counts_all(torch.zeros((1, E), dtype=torch.int32), 2, E, "cpu")
+    with pytest.raises(ValueError, match="shape"):
+        S.check_counts_all(torch.zeros((2, E + 1), dtype=torch.int32), 2, E, "cpu")
+    with pytest.raises(ValueError, match="int32"):
+        S.check_counts_all(torch.zeros((2, E), dtype=torch.int64), 2, E, "cpu")
+    with pytest.raises(ValueError, match="is on"):
+        S.check_counts_all(ok.to("meta"), 2, E, "cpu")
+
+
 def _free_port():
     with socket.socket() as s:
         s.bind(("127.0.0.1", 0))
@@ -158,6 +183,65 @@ def test_sharded_batch_matches_the_single_batch(world):
         assert aux["aux"] == pytest.approx(auxv, rel=1e-12)
         assert aux["z"] == pytest.approx(O.router_z_loss(r["logits"]), rel=1e-12)
         assert aux["bsq"] == pytest.approx(O.balance_sq_loss(r["idx"], WL.n_experts), rel=1e-9)
+
+
+def _bench_worker(rank, world, port, q):
+    """bench.py's sharded timing path on gloo ranks, the oracle doing the steps."""
+    import time
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world))
+    sys.path.insert(0, ROOT)
+    import bench
+    dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=60))
+    try:
+        P = H.oracle_params(synth.generate(WL, seed=3))
+        a, b = S.shard_bounds(WL.T, world)[rank]
+        steps = OracleSteps(WL, P, rank, world)
+
+        def clock():
+            t = {}
+
+            def start():
+                bench.barrier(world)
+                t[0] = time.perf_counter()
+
+            def stop():
+                bench.barrier(world)
+                return 1000.0 * (time.perf_counter() - t[0])
+
+            return start, stop
+
+        ms, (y, aux) = bench.sharded_steps_timing(steps, P["x"][a:b], WL.n_experts, 2, 3,
+                                                  None, clock)
+        worst = bench.max_over_ranks(ms, world)
+        q.put((rank, y, steps.kept, aux, ms, worst))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_bench_sharded_path_on_two_ranks():
+    """The timed loop bench.py runs for one batch split over N GPUs: every rank takes
+    the same collectives per step, the ranks' outputs put together are the single
+    batch's, and the reported time is the slowest rank's."""
+    world, port = 2, _free_port()
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_bench_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    got = sorted((q.get(timeout=300) for _ in range(world)), key=lambda g: g[0])
+    for p in procs:
+        p.join(timeout=120)
+        assert p.exitcode == 0
+    P = H.oracle_params(synth.generate(WL, seed=3))
+    yref, r = O.moe_forward(P["x"], P, **H.oracle_kwargs(WL))
+    assert np.array_equal(np.concatenate([g[2] for g in got]), r["kept"])
+    assert np.allclose(np.concatenate([g[1] for g in got]), yref, rtol=1e-12, atol=1e-12)
+    _, _, auxv = O.aux_stats(r["logits"], r["idx"], WL.n_experts, WL.top_k, WL.aux_alpha)
+    worst = max(g[4] for g in got)
+    for g in got:
+        assert g[3]["aux"] == pytest.approx(auxv, rel=1e-12)
+        assert g[5] == worst > 0
 
 
 # ----------------------------------------------------- C entry points, host checks
