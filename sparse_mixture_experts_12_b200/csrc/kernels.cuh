@@ -103,7 +103,8 @@ cudaError_t launch_router(const RouterArgs &a, int dtype, cudaStream_t st);
 // noisy top-k gating: z[i] += softplus(zn[i]) * eps[i] over n logits
 cudaError_t launch_noisy_logits(float *z, const float *zn, const float *eps, size_t n,
                                 cudaStream_t st);
-// bf16 router on the tensor cores (x given, 16 <= E <= 256)
+// bf16 router on the tensor cores (x given, d a multiple of 64, T > 0)
+bool router_tc_supported(const RouterArgs &a);
 cudaError_t launch_router_tc(const RouterArgs &a, cudaStream_t st);
 cudaError_t launch_tile_counts(const int32_t *topk_idx, int T, int k, int E, int32_t *tile_counts,
                                int32_t *err, cudaStream_t st);

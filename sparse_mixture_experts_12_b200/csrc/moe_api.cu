@@ -696,7 +696,7 @@ moe_status_t forward_impl(const moe_cfg_t *cfg, const moe_weights_t *w, const vo
     r.w = w->w_router;
     r.b_router = w->b_router;
     r.logit_bias = w->logit_bias;
-    r.logits_out = (tp.logits || want_aux) ? logits : nullptr;
+    r.logits_out = tp.logits;  // the statistics come from the router's own partial sums
   }
   r.topk_idx = idx;
   r.topk_gate = gate;

@@ -16,7 +16,6 @@ namespace {
 constexpr int kRouterThreads = 256;
 constexpr int kBK = 32;  // K elements per slice per iteration
 constexpr int kRouterStages = 3;  // cp.async ring depth
-constexpr int kRouterTcMinTokens = 256;
 
 template <int EPAD> struct RouterShape;
 template <> struct RouterShape<8>   { static constexpr int BM = 32, TM = 1, TN = 8, KS = 8; };
@@ -572,15 +571,14 @@ __global__ void __launch_bounds__(256) k_tile_counts(const int32_t *__restrict__
 cudaError_t launch_router(const RouterArgs &a, int dtype, cudaStream_t st) {
   if (a.T == 0) return cudaSuccess;
   const int E = a.E;
-  // small expert counts with W_r fitting in shared memory: the GEMV-shaped router
+  // bf16: the tensor-core router (x W_r^T is a contraction; on the CUDA cores it is
+  // bound by the FMA rate rather than by reading x)
+  if (dtype == MOE_DTYPE_BF16 && router_tc_supported(a)) return launch_router_tc(a, st);
+  // fp32, small expert counts with W_r fitting in shared memory: the GEMV-shaped router
   if (E <= 8 && a.x != nullptr &&
       8LL * a.d * (dtype == MOE_DTYPE_F32 ? 4 : 2) <= 96LL * 1024)
     return dtype == MOE_DTYPE_F32 ? launch_router_gemv<float>(a, st)
                                   : launch_router_gemv<__nv_bfloat16>(a, st);
-  // bf16 with many experts and enough tokens: the tensor-core router (the
-  // CUDA-core GEMM below is FMA-bound there)
-  if (dtype == MOE_DTYPE_BF16 && a.x != nullptr && E >= 16 && a.T >= kRouterTcMinTokens)
-    return launch_router_tc(a, st);
   if (E <= 8) return launch_router_e<8>(a, dtype, st);
   if (E <= 16) return launch_router_e<16>(a, dtype, st);
   if (E <= 32) return launch_router_e<32>(a, dtype, st);

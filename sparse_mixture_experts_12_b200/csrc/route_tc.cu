@@ -1,8 +1,8 @@
-// Router on the 5th-generation tensor cores for bf16 layers with 16..256
-// experts: logits = x W_r^T (+ router bias, + per-expert logit bias) by
-// tcgen05.mma with an fp32 TMEM accumulator, fused with the softmax, the top-k
-// selection, the gate values and the per-tile statistics that the permute step
-// (capacity ranks) and the auxiliary losses consume.
+// Router on the 5th-generation tensor cores for every bf16 layer: logits =
+// x W_r^T (+ router bias, + per-expert logit bias) by tcgen05.mma with an fp32
+// TMEM accumulator, fused with the softmax, the top-k selection, the gate values
+// and the per-tile statistics that the permute step (capacity ranks) and the
+// auxiliary losses consume.
 //
 // Gating network: youngju.dev (zh) "GatingNetwork" / "SwitchRouter" and the
 // devtips.kr "MoELayer" gate (a Linear over d_model, with or without bias);
@@ -10,14 +10,22 @@
 // top-k renormalised (youngju.dev ja "TopKGating"), softmax then top-1 raw
 // (SwitchRouter).
 //
-// One CTA per 128 tokens, 320 threads:
+// The router streams x (T x d) once and is bound by HBM. One cluster of S CTAs
+// (S = 1, 2 or 4) covers 128 tokens; CTA r of the cluster reduces its own share
+// of the d columns (a split of K), so that small batches still spread over the
+// SMs. Per CTA, 320 threads:
 //   warp 0      TMA producer: 128 x 64 slices of x and EPAD x 64 slices of W_r
-//               (rows >= E read as zeros), 128-byte swizzle, 4..9-stage ring.
+//               (rows >= E read as zeros), 128-byte swizzle, a ring of stages.
 //   warp 1      TMEM owner and MMA issuer (M = 128, N = EPAD, K = 16 per MMA).
-//   warps 2..9  epilogue, two threads per token.
-// Same results as the SIMT router up to the fp32 summation order of the dot
-// products: same bias order, NaN -> -inf before selection, ties to the lower
-// expert index, same gate formulas, same fixed-order per-tile sums.
+//   warps 2..9  epilogue.
+// The epilogue parks each CTA's fp32 partial logits in its shared memory; after a
+// cluster barrier, CTA r takes tokens [r * 128/S, (r+1) * 128/S) and sums the S
+// partials of each in rank order (distributed shared memory), so the result does
+// not depend on timing. G = 2S threads share a token (consecutive lanes), each
+// holding EPAD/G logits in registers: the max, the k argmax rounds (value, then
+// lower expert index), the exp sum and the probability column sums are register
+// work plus fixed shuffle trees. The permute tiles (router_bm(E) tokens) lie
+// inside one CTA's token share, so their histograms and sums need no exchange.
 #include <mutex>
 
 #include "tc_ptx.cuh"
@@ -28,13 +36,14 @@ namespace {
 
 using namespace tc;
 
-constexpr int kRtMaxStages = 10;
-constexpr int kRtRingBudget = 192 * 1024;  // shared memory for the operand ring
-constexpr int kRtM = 128;  // tokens per CTA
-constexpr int kRtEpiThreads = 256;  // two threads per token
+constexpr int kRtM = 128;           // tokens per cluster (the MMA's M)
+constexpr int kRtEpiWarps = 8;
+constexpr int kRtEpiThreads = 32 * kRtEpiWarps;
 constexpr int kRtThreads = 64 + kRtEpiThreads;
 constexpr int kRtABytes = kRtM * kBlockK * 2;
-constexpr int kRtMaxSubs = 4;  // permute tiles per CTA: 128 / router_bm(E)
+constexpr int kRtMaxStages = 8;
+constexpr int kRtRingBudget = 144 * 1024;  // shared memory for the operand ring
+constexpr int kRtMaxSubs = 4;              // permute tiles in one CTA's token share
 
 struct RtCtl {
   uint64_t full[kRtMaxStages];
@@ -46,29 +55,28 @@ struct RtCtl {
   int epi_ok;
   float br[kMaxExperts];  // router bias (0 when absent)
   float lb[kMaxExperts];  // per-expert logit bias (0 when absent)
-  float lse[kRtM];
   int cnt[kRtMaxSubs][kMaxExperts];
-  // the two threads of a token meet here: max, top-k candidates (double-buffered
-  // by round parity), exp sums
-  float hmax[2][kRtM];
-  float cand_v[2][2][kRtM];
-  int cand_i[2][2][kRtM];
-  float hsum[2][kRtM];
+  float psum[kRtEpiWarps][kMaxExperts];  // per-warp column sums of the probabilities
+  float lse[kRtM];
 };
 
-template <int EPAD> struct RtCfg {
-  static_assert(EPAD == 32 || EPAD == 64 || EPAD == 128 || EPAD == 256, "EPAD");
+template <int EPAD, int S> struct RtCfg {
+  static_assert(EPAD == 16 || EPAD == 32 || EPAD == 64 || EPAD == 128 || EPAD == 256, "EPAD");
+  static_assert(S == 1 || S == 2 || S == 4, "S");
   static constexpr int kBBytes = EPAD * kBlockK * 2;
   static constexpr int kStageBytes = kRtABytes + kBBytes;  // a multiple of 1024
-  // as many stages as the budget holds: one CTA per SM streams x, so the bytes in
-  // flight per SM set the achievable bandwidth
   static constexpr int kStages = kRtRingBudget / kStageBytes < kRtMaxStages
                                      ? kRtRingBudget / kStageBytes : kRtMaxStages;
   static constexpr int kRing = kStages * kStageBytes;
-  static constexpr int kLdl = EPAD + 1;  // probability tile row stride (floats)
-  static constexpr int kProbBytes = kRtM * kLdl * 4;
-  static constexpr int kBody = kRing > kProbBytes ? kRing : kProbBytes;
+  static constexpr int kLdp = EPAD + 1;             // partial tile row stride (floats)
+  static constexpr int kPartBytes = kRtM * kLdp * 4;
+  static constexpr int kBody = kRing > kPartBytes ? kRing : kPartBytes;
   static constexpr size_t kSmem = (size_t)kBody + sizeof(RtCtl) + 1024;
+  static constexpr int kTok = kRtM / S;             // tokens of one CTA's epilogue
+  static constexpr int kG = kRtEpiThreads / kTok;   // threads per token (2S)
+  static constexpr int kEpl = EPAD / kG;            // logits per thread
+  static constexpr uint32_t kTmemCols = EPAD < 32 ? 32 : EPAD;
+  static_assert(kEpl >= 1 && kEpl <= 64, "logits per thread");
 };
 
 __device__ __forceinline__ bool rt_wait(uint64_t *bar, uint32_t parity, RtCtl *ctl, int32_t *err,
@@ -85,79 +93,122 @@ __device__ __forceinline__ void rt_epi_sync() {
   asm volatile("bar.sync 1, %0;" ::"n"(kRtEpiThreads) : "memory");
 }
 
-// Two threads per token. Pass 1: the two warps that may read a TMEM lane quarter
-// take alternate 32-column chunks of their 32 tokens: logits (+ biases in the
-// CUDA-core router's order) are written out and z (NaN -> -inf) parked in the
-// token's row of the shared-memory tile. Then thread (token r, half h) owns row r,
-// columns [h*E0, min(E, (h+1)*E0)): the max, k argmax rounds (each the best entry
-// ranked below the previous pick: value, then lower index) and sum exp(z - max) are
-// taken over each half and merged through shared memory in a fixed order.
-template <int EPAD>
-__device__ __forceinline__ void epilogue_rows(const RouterArgs &a, RtCtl *ctl, float *prob,
-                                              uint32_t tmem, int t0, int NT, int BM, int warp,
-                                              int lane) {
-  constexpr int LDL = RtCfg<EPAD>::kLdl;
-  const int E = a.E, T = a.T, k = a.k;
-  const int et = (warp - 2) * 32 + lane;  // 0..255 over the epilogue threads
-  // one thread waits; the named barrier is reached by all epilogue threads
-  if (et == 0) ctl->epi_ok = rt_wait(&ctl->tfull, 0, ctl, a.err, 13) ? 1 : 0;
-  rt_epi_sync();
-  if (!ctl->epi_ok) return;
-  tc_fence_after();
+// every thread of the cluster (S > 1) or of the CTA (S = 1)
+template <int S>
+__device__ __forceinline__ void rt_sync_all() {
+  if constexpr (S == 1) {
+    __syncthreads();
+  } else {
+    __syncwarp();
+    cluster_sync_all();
+  }
+}
 
-  {  // ---- pass 1: TMEM -> logits out, z into the row
-    const int ew = warp & 3;                // TMEM lanes [32 ew, 32 ew + 32) (warp % 4)
-    const int c_first = (warp - 2) >> 2;    // this warp's chunks: c_first, c_first + 2, ...
-    const int r = ew * 32 + lane;
-    const int t = t0 + r;
-    const bool valid = t < T;
-    float *row = prob + r * LDL;
-    const uint32_t tb = tmem + ((uint32_t)(ew * 32) << 16);
-    const bool vec_out = valid && a.logits_out != nullptr && (E & 3) == 0;
+// TMEM -> this CTA's partial tile [128][EPAD] (row stride kLdp). Warp w reads TMEM
+// lanes [32 (w % 4), +32) (its lane quarter); the two warps of a quarter take
+// alternate 32-column chunks.
+template <int EPAD, int S>
+__device__ __forceinline__ void stage_partial(float *part, uint32_t tmem, int warp, int lane) {
+  using C = RtCfg<EPAD, S>;
+  const int q = warp & 3;
+  const int h = (warp - 2) >> 2;
+  const int r = q * 32 + lane;
+  float *row = part + r * C::kLdp;
+  const uint32_t tb = tmem + ((uint32_t)(q * 32) << 16);
+  if constexpr (EPAD == 16) {
+    if (h == 0) {
+      uint32_t v[16];
+      tmem_ld16(tb, v);
+      tmem_ld_wait();
+#pragma unroll
+      for (int j = 0; j < 16; ++j) row[j] = __uint_as_float(v[j]);
+    }
+  } else {
 #pragma unroll 1
-    for (int c = c_first; c < EPAD / 32; c += 2) {
+    for (int c = h; c < EPAD / 32; c += 2) {
       uint32_t v[32];
       tmem_ld32(tb + c * 32, v);
       tmem_ld_wait();
-      float lo[32];
 #pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        const int e = c * 32 + j;
-        float val = __uint_as_float(v[j]);
-        if (a.b_router) val += ctl->br[e];
-        if (a.logit_bias) val += ctl->lb[e];
-        lo[j] = val;
-        if (e < E) row[e] = (val != val) ? -INFINITY : val;  // a NaN logit never wins a slot
-      }
-      const int n_out = min(32, E - c * 32);
-      if (vec_out && n_out == 32) {
-        float4 *dst = reinterpret_cast<float4 *>(a.logits_out + (size_t)t * E + c * 32);
-#pragma unroll
-        for (int q = 0; q < 8; ++q)
-          dst[q] = make_float4(lo[4 * q], lo[4 * q + 1], lo[4 * q + 2], lo[4 * q + 3]);
-      } else if (valid && a.logits_out != nullptr) {
-#pragma unroll
-        for (int j = 0; j < 32; ++j)
-          if (j < n_out) a.logits_out[(size_t)t * E + c * 32 + j] = lo[j];
-      }
+      for (int j = 0; j < 32; ++j) row[c * 32 + j] = __uint_as_float(v[j]);
     }
   }
-  rt_epi_sync();
+}
 
-  // ---- the rest: thread (token r, half h); a warp holds 32 consecutive tokens
-  const int r = et & (kRtM - 1), h = et / kRtM;
-  const int t = t0 + r;
+// Group reductions over the G consecutive lanes that share a token (fixed trees).
+template <int G>
+__device__ __forceinline__ float group_max(float v) {
+#pragma unroll
+  for (int o = G / 2; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o, G));
+  return v;
+}
+template <int G>
+__device__ __forceinline__ float group_sum(float v) {
+#pragma unroll
+  for (int o = G / 2; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o, G);
+  return v;
+}
+template <int G>
+__device__ __forceinline__ void group_argmax(float &v, int &i) {
+#pragma unroll
+  for (int o = G / 2; o > 0; o >>= 1) {
+    const float ov = __shfl_xor_sync(0xffffffffu, v, o, G);
+    const int oi = __shfl_xor_sync(0xffffffffu, i, o, G);
+    if (rt_better(ov, oi, v, i)) { v = ov; i = oi; }
+  }
+}
+
+// The epilogue of CTA `rank`: tokens [rank * kTok, +kTok) of the cluster's 128.
+template <int EPAD, int S>
+__device__ __forceinline__ void epilogue_tokens(const RouterArgs &a, RtCtl *ctl, float *part,
+                                                int tile, int rank, int NT, int BM, int et) {
+  using C = RtCfg<EPAD, S>;
+  constexpr int G = C::kG, EPL = C::kEpl, TOK = C::kTok;
+  const int E = a.E, T = a.T, k = a.k;
+  const int m = et / G, g = et % G;        // token of this CTA's share, lane in its group
+  const int row = rank * TOK + m;          // row of the cluster's 128-token tile
+  const int t = tile * kRtM + row;
   const bool valid = t < T;
-  float *row = prob + r * LDL;
-  const int E0 = (E + 1) >> 1;
-  const int e_lo = h * E0, e_hi = min(E, e_lo + E0);
+  const int lane = et & 31, ew = et >> 5;
+
+  // ---- logits: the S partials in rank order (+ biases in the CUDA-core router's order)
+  float z[EPL];
+  {
+    float acc[EPL];
+#pragma unroll
+    for (int j = 0; j < EPL; ++j) acc[j] = 0.f;
+    const uint32_t base = smem_u32(part + row * C::kLdp);
+#pragma unroll
+    for (int r = 0; r < S; ++r) {
+      if constexpr (S == 1) {
+#pragma unroll
+        for (int j = 0; j < EPL; ++j) acc[j] = part[row * C::kLdp + j * G + g];
+      } else {
+        const uint32_t rb = mapa_rank(base, (uint32_t)r);
+        float v[EPL];
+#pragma unroll
+        for (int j = 0; j < EPL; ++j) v[j] = ld_cluster_f32(rb + 4u * (uint32_t)(j * G + g));
+#pragma unroll
+        for (int j = 0; j < EPL; ++j) acc[j] = (r == 0) ? v[j] : acc[j] + v[j];
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < EPL; ++j) {
+      const int e = j * G + g;
+      float v = acc[j];
+      if (a.b_router) v += ctl->br[e];
+      if (a.logit_bias) v += ctl->lb[e];
+      if (a.logits_out != nullptr && valid && e < E) a.logits_out[(size_t)t * E + e] = v;
+      z[j] = (e >= E || v != v) ? -INFINITY : v;  // padding and NaN never win a slot
+    }
+  }
 
   float mx = -INFINITY;
-  for (int e = e_lo; e < e_hi; ++e) mx = fmaxf(mx, row[e]);
-  ctl->hmax[h][r] = mx;
-  rt_epi_sync();
-  mx = fmaxf(ctl->hmax[0][r], ctl->hmax[1][r]);
+#pragma unroll
+  for (int j = 0; j < EPL; ++j) mx = fmaxf(mx, z[j]);
+  mx = group_max<G>(mx);
 
+  // ---- top-k: k rounds, each the best entry ranked below the previous pick
   float tv[kMaxTopK];
   int ti[kMaxTopK];
   float pv = INFINITY;
@@ -167,69 +218,49 @@ __device__ __forceinline__ void epilogue_rows(const RouterArgs &a, RtCtl *ctl, f
     tv[s] = -INFINITY;
     ti[s] = 0x7fffffff;
     if (s < k) {
-      float bv[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-      int bi[4] = {0x7fffffff, 0x7fffffff, 0x7fffffff, 0x7fffffff};
-      int e = e_lo;
-#pragma unroll 2
-      for (; e + 4 <= e_hi; e += 4) {
+      float bv = -INFINITY;
+      int bi = 0x7fffffff;
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const float z = row[e + q];
-          const bool below = z < pv || (z == pv && e + q > pi);
-          if (below && rt_better(z, e + q, bv[q], bi[q])) { bv[q] = z; bi[q] = e + q; }
-        }
+      for (int j = 0; j < EPL; ++j) {
+        const int e = j * G + g;
+        const bool below = z[j] < pv || (z[j] == pv && e > pi);
+        if (below && rt_better(z[j], e, bv, bi)) { bv = z[j]; bi = e; }
       }
-      for (; e < e_hi; ++e) {
-        const float z = row[e];
-        const bool below = z < pv || (z == pv && e > pi);
-        if (below && rt_better(z, e, bv[0], bi[0])) { bv[0] = z; bi[0] = e; }
-      }
-#pragma unroll
-      for (int q = 1; q < 4; ++q)
-        if (rt_better(bv[q], bi[q], bv[0], bi[0])) { bv[0] = bv[q]; bi[0] = bi[q]; }
-      ctl->cand_v[s & 1][h][r] = bv[0];
-      ctl->cand_i[s & 1][h][r] = bi[0];
-      rt_epi_sync();
-      float b0 = ctl->cand_v[s & 1][0][r], b1 = ctl->cand_v[s & 1][1][r];
-      int i0 = ctl->cand_i[s & 1][0][r], i1 = ctl->cand_i[s & 1][1][r];
-      if (rt_better(b1, i1, b0, i0)) { b0 = b1; i0 = i1; }
-      tv[s] = pv = b0;
-      ti[s] = pi = i0;
+      group_argmax<G>(bv, bi);
+      tv[s] = pv = bv;
+      ti[s] = pi = bi;
     }
   }
 
+  // ---- softmax denominators
+  float ex[EPL];
   float ssum = 0.f;
-#pragma unroll 4
-  for (int e = e_lo; e < e_hi; ++e) {
-    const float ex = expf(row[e] - mx);
-    ssum += ex;
-    row[e] = ex;
+#pragma unroll
+  for (int j = 0; j < EPL; ++j) {
+    ex[j] = expf(z[j] - mx);
+    ssum += ex[j];
   }
-  ctl->hsum[h][r] = ssum;
-  rt_epi_sync();
-  ssum = ctl->hsum[0][r] + ctl->hsum[1][r];
+  ssum = group_sum<G>(ssum);
   const float inv_s = 1.f / ssum;
-  if (a.tile_p != nullptr)
-    for (int e = e_lo; e < e_hi; ++e) row[e] *= inv_s;
 
-  if (h == 0) {
-    ctl->lse[r] = mx + logf(ssum);
-    float g[kMaxTopK];
+  if (g == 0) {
+    ctl->lse[m] = valid ? mx + logf(ssum) : 0.f;
+    float gv[kMaxTopK];
     float gs = 0.f;
     if (a.gate_mode == MOE_GATE_TOPK_SOFTMAX) {
 #pragma unroll
       for (int s = 0; s < kMaxTopK; ++s)
-        if (s < k) { g[s] = expf(tv[s] - tv[0]); gs += g[s]; }
+        if (s < k) { gv[s] = expf(tv[s] - tv[0]); gs += gv[s]; }
       const float inv = 1.f / gs;
 #pragma unroll
-      for (int s = 0; s < kMaxTopK; ++s) if (s < k) g[s] *= inv;
+      for (int s = 0; s < kMaxTopK; ++s) if (s < k) gv[s] *= inv;
     } else {
 #pragma unroll
       for (int s = 0; s < kMaxTopK; ++s)
-        if (s < k) { g[s] = expf(tv[s] - mx) * inv_s; gs += g[s]; }
+        if (s < k) { gv[s] = expf(tv[s] - mx) * inv_s; gs += gv[s]; }
       if (a.gate_mode == MOE_GATE_SOFTMAX_TOPK_RENORM) {
 #pragma unroll
-        for (int s = 0; s < kMaxTopK; ++s) if (s < k) g[s] = g[s] / gs;
+        for (int s = 0; s < kMaxTopK; ++s) if (s < k) gv[s] = gv[s] / gs;
       }
     }
     if (valid) {
@@ -237,57 +268,76 @@ __device__ __forceinline__ void epilogue_rows(const RouterArgs &a, RtCtl *ctl, f
       for (int s = 0; s < kMaxTopK; ++s) {
         if (s < k) {
           a.topk_idx[(size_t)t * k + s] = ti[s];
-          a.topk_gate[(size_t)t * k + s] = g[s];
-          if (ti[s] < E) atomicAdd(&ctl->cnt[r / BM][ti[s]], 1);
+          a.topk_gate[(size_t)t * k + s] = gv[s];
+          // integer counts: the result does not depend on the order of the adds
+          if (ti[s] < E) atomicAdd(&ctl->cnt[m / BM][ti[s]], 1);
         }
       }
     }
   }
+
+  // ---- probability column sums of this warp's tokens (lanes with the same g)
+  if (a.tile_p != nullptr) {
+    float p[EPL];
+#pragma unroll
+    for (int j = 0; j < EPL; ++j) p[j] = valid ? ex[j] * inv_s : 0.f;
+#pragma unroll
+    for (int o = G; o < 32; o <<= 1)
+#pragma unroll
+      for (int j = 0; j < EPL; ++j) p[j] += __shfl_xor_sync(0xffffffffu, p[j], o);
+    if (lane < G) {
+#pragma unroll
+      for (int j = 0; j < EPL; ++j) ctl->psum[ew][j * G + g] = p[j];
+    }
+  }
   rt_epi_sync();
 
-  // per permute tile (BM tokens): histogram, probability sums, sum of lse^2,
-  // each in token order
-  const int subs = kRtM / BM;
+  // ---- per permute tile (BM tokens, whole tiles inside this CTA's share)
+  const int subs = TOK / BM;
+  const int wpt = BM * G / 32;  // warps per permute tile
+  const int tile0 = (tile * kRtM + rank * TOK) / BM;
   for (int i = et; i < subs * E; i += kRtEpiThreads) {
     const int sub = i / E, e = i - sub * E;
-    const int tile = blockIdx.x * subs + sub;
-    if (tile >= NT) continue;
-    if (a.tile_counts) a.tile_counts[(size_t)e * NT + tile] = ctl->cnt[sub][e];
+    const int pt = tile0 + sub;
+    if (pt >= NT) continue;
+    if (a.tile_counts) a.tile_counts[(size_t)e * NT + pt] = ctl->cnt[sub][e];
     if (a.tile_p != nullptr) {
-      const int rows = min(BM, T - tile * BM);
       float s = 0.f;
-      for (int m = 0; m < rows; ++m) s += prob[(sub * BM + m) * LDL + e];
-      a.tile_p[(size_t)e * NT + tile] = s;
+      for (int w = 0; w < wpt; ++w) s += ctl->psum[sub * wpt + w][e];
+      a.tile_p[(size_t)e * NT + pt] = s;
     }
   }
   if (a.tile_z && et < subs) {
-    const int tile = blockIdx.x * subs + et;
-    if (tile < NT) {
-      const int rows = min(BM, T - tile * BM);
+    const int pt = tile0 + et;
+    if (pt < NT) {
+      const int rows = min(BM, T - pt * BM);
       float s = 0.f;
-      for (int m = 0; m < rows; ++m) {
-        const float l = ctl->lse[et * BM + m];
+      for (int mm = 0; mm < rows; ++mm) {
+        const float l = ctl->lse[et * BM + mm];
         s += l * l;
       }
-      a.tile_z[tile] = s;
+      a.tile_z[pt] = s;
     }
   }
 }
 
-template <int EPAD>
+template <int EPAD, int S>
 __global__ void __launch_bounds__(kRtThreads, 1)
 k_router_tc(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
             RouterArgs a, int NT, int BM) {
-  using C = RtCfg<EPAD>;
+  using C = RtCfg<EPAD, S>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   RtCtl *ctl = reinterpret_cast<RtCtl *>(smem + C::kBody);
-  float *prob = reinterpret_cast<float *>(smem);  // [128][EPAD+1], reuses the ring
+  float *part = reinterpret_cast<float *>(smem);  // [128][EPAD+1], reuses the ring
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int E = a.E;
-  const int t0 = blockIdx.x * kRtM;
+  const int rank = S == 1 ? 0 : (int)cluster_ctarank();
+  const int tile = blockIdx.x / S;
+  const int t0 = tile * kRtM;
   const int nkb = ceil_div(a.d, kBlockK);
+  const int kb0 = rank * nkb / S, kb1 = (rank + 1) * nkb / S;  // this CTA's K share
 
   for (int e = tid; e < kMaxExperts; e += kRtThreads) {
     ctl->br[e] = (a.b_router && e < E) ? a.b_router[e] : 0.f;
@@ -302,10 +352,11 @@ k_router_tc(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
     mbar_init(&ctl->tfull, 1);
     mbar_init(&ctl->drain, 1);
     ctl->abort_flag = 0;
+    ctl->epi_ok = 0;
     fence_mbar_init();
   }
   if (warp == 1) {
-    tmem_alloc(&ctl->tmem_base, EPAD);
+    tmem_alloc(&ctl->tmem_base, C::kTmemCols);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -320,7 +371,7 @@ k_router_tc(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
     int stage = 0;
     uint32_t phase = 0, issued = 0, last_phase = 0;
     bool ok = true;
-    for (int kb = 0; kb < nkb; ++kb) {
+    for (int kb = kb0; kb < kb1; ++kb) {
       if (!rt_wait(&ctl->empty[stage], phase ^ 1u, ctl, a.err, 11)) { ok = false; break; }
       uint8_t *sa = smem + (size_t)stage * C::kStageBytes;
       mbar_expect_tx(&ctl->full[stage], C::kStageBytes);
@@ -330,7 +381,7 @@ k_router_tc(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
       last_phase = (last_phase & ~(1u << stage)) | (phase << stage);
       if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
     }
-    if (!ok) {  // let the copies already in flight land before the CTA exits
+    if (!ok) {  // let the copies already in flight land before the ring is reused
       for (int s = 0; s < C::kStages; ++s)
         if (issued & (1u << s)) rt_wait(&ctl->full[s], (last_phase >> s) & 1u, ctl, nullptr, 0, false);
     }
@@ -340,7 +391,7 @@ k_router_tc(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
     int stage = 0;
     uint32_t phase = 0;
     bool ok = true, any = false;
-    for (int kb = 0; kb < nkb; ++kb) {
+    for (int kb = kb0; kb < kb1; ++kb) {
       if (!rt_wait(&ctl->full[stage], phase, ctl, a.err, 12)) { ok = false; break; }
       tc_fence_after();
       const uint32_t sa = smem_u32(smem + (size_t)stage * C::kStageBytes);
@@ -348,7 +399,7 @@ k_router_tc(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
       const uint64_t db = sw128_desc(sa + kRtABytes);
 #pragma unroll
       for (int kk = 0; kk < kBlockK / 16; ++kk)
-        umma_bf16(tmem, da + 2 * kk, db + 2 * kk, idesc, (kb | kk) != 0);
+        umma_bf16(tmem, da + 2 * kk, db + 2 * kk, idesc, (kb != kb0 || kk != 0) ? 1u : 0u);
       any = true;
       umma_commit(&ctl->empty[stage]);
       if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
@@ -360,21 +411,32 @@ k_router_tc(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
       rt_wait(&ctl->drain, 0, ctl, nullptr, 0, false);
     }
   } else if (warp >= 2) {
-    epilogue_rows<EPAD>(a, ctl, prob, tmem, t0, NT, BM, warp, lane);
+    // ------------------------------------------ epilogue, 1: TMEM -> partial tile
+    const int et = tid - 64;
+    // one thread waits; the named barrier is reached by all epilogue threads
+    if (et == 0) ctl->epi_ok = rt_wait(&ctl->tfull, 0, ctl, a.err, 13) ? 1 : 0;
+    rt_epi_sync();
+    if (ctl->epi_ok) {
+      tc_fence_after();
+      stage_partial<EPAD, S>(part, tmem, warp, lane);
+    }
   }
+  // the partial tiles of the whole cluster are complete
   tc_fence_before();
-  __syncthreads();
-  if (warp == 1) {
-    tc_fence_after();
-    tmem_dealloc(tmem, EPAD);
-  }
+  rt_sync_all<S>();
+  tc_fence_after();
+  if (warp >= 2 && ctl->epi_ok)
+    epilogue_tokens<EPAD, S>(a, ctl, part, tile, rank, NT, BM, tid - 64);
+  // no CTA leaves (its shared memory) while another may still read its partials
+  rt_sync_all<S>();
+  if (warp == 1) tmem_dealloc(tmem, C::kTmemCols);
 }
 
 std::mutex g_rt_mu;
 
-template <int EPAD>
+template <int EPAD, int S>
 cudaError_t launch_rt(const RouterArgs &a, cudaStream_t st) {
-  using C = RtCfg<EPAD>;
+  using C = RtCfg<EPAD, S>;
   static bool attr_set[64] = {};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -382,7 +444,7 @@ cudaError_t launch_rt(const RouterArgs &a, cudaStream_t st) {
   {
     std::lock_guard<std::mutex> lock(g_rt_mu);
     if (!attr_set[dev & 63]) {
-      e = cudaFuncSetAttribute(k_router_tc<EPAD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+      e = cudaFuncSetAttribute(k_router_tc<EPAD, S>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                (int)C::kSmem);
       if (e != cudaSuccess) return e;
       attr_set[dev & 63] = true;
@@ -393,19 +455,58 @@ cudaError_t launch_rt(const RouterArgs &a, cudaStream_t st) {
   if (!make_map(&mw, a.w, (uint64_t)a.E, (uint64_t)a.d, EPAD)) return cudaErrorInvalidValue;
   const int BM = router_bm(a.E);
   const int NT = ceil_div(a.T, BM);
-  k_router_tc<EPAD><<<ceil_div(a.T, kRtM), kRtThreads, C::kSmem, st>>>(mx, mw, a, NT, BM);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3((unsigned)(ceil_div(a.T, kRtM) * S));
+  cfg.blockDim = dim3(kRtThreads);
+  cfg.dynamicSmemBytes = C::kSmem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = S;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, k_router_tc<EPAD, S>, mx, mw, a, NT, BM);
+}
+
+// K splits: at most four, each CTA's token share (128 / S) a whole number of permute
+// tiles, at least two 64-column blocks of K per split, and only while the grid
+// stays under one CTA per SM.
+int router_splits(int T, int d, int E, int epad) {
+  const int BM = router_bm(E);
+  const int tiles = ceil_div(T, kRtM);
+  const int nkb = d / kBlockK;
+  const int sms = sm_count();
+  int S = 1;
+  while (S < 4 && kRtM / (2 * S) >= BM && 2 * S <= nkb && tiles * 2 * S <= sms) S *= 2;
+  if (epad == 256 && S == 1 && nkb >= 2) S = 2;  // at most 64 logits per epilogue thread
+  return S;
+}
+
+template <int EPAD>
+cudaError_t launch_rt_e(const RouterArgs &a, cudaStream_t st) {
+  const int S = router_splits(a.T, a.d, a.E, EPAD);
+  if (S == 4) return launch_rt<EPAD, 4>(a, st);
+  if (S == 2) return launch_rt<EPAD, 2>(a, st);
+  if constexpr (EPAD == 256) return cudaErrorInvalidValue;  // needs a split (d >= 128)
+  else return launch_rt<EPAD, 1>(a, st);
 }
 
 }  // namespace
 
+bool router_tc_supported(const RouterArgs &a) {
+  return a.x != nullptr && a.E >= 1 && a.E <= kMaxExperts && a.d % kBlockK == 0 && a.T > 0 &&
+         !(a.E > 128 && a.d < 2 * kBlockK);
+}
+
 cudaError_t launch_router_tc(const RouterArgs &a, cudaStream_t st) {
-  if (a.x == nullptr || a.E < 1 || a.E > kMaxExperts || a.d % kBlockK != 0)
-    return cudaErrorInvalidValue;
-  if (a.E <= 32) return launch_rt<32>(a, st);
-  if (a.E <= 64) return launch_rt<64>(a, st);
-  if (a.E <= 128) return launch_rt<128>(a, st);
-  return launch_rt<256>(a, st);
+  if (!router_tc_supported(a)) return cudaErrorInvalidValue;
+  if (a.E <= 16) return launch_rt_e<16>(a, st);
+  if (a.E <= 32) return launch_rt_e<32>(a, st);
+  if (a.E <= 64) return launch_rt_e<64>(a, st);
+  if (a.E <= 128) return launch_rt_e<128>(a, st);
+  return launch_rt_e<256>(a, st);
 }
 
 }  // namespace moe

@@ -40,12 +40,16 @@ def shard_bounds(n_tokens_total: int, n_shards: int):
     return out
 
 
-def check_placement(shard: int, n_shards: int, group=None):
+def check_placement(shard: int, n_shards: int, group=None, caller_exchanges: bool = False):
     """A shard's place must be its rank in the process group. Without a group only
     the one-shard layout is valid: the other shards' counts would never arrive, and
-    the capacity left to this shard could not be computed."""
+    the capacity left to this shard could not be computed. A caller that gathers
+    the counts itself (caller_exchanges) may place shards freely: it then passes
+    every shard's counts to forward_shard, whose check guards the library's read."""
     if not 0 <= shard < n_shards:
         raise ValueError(f"shard {shard} is not one of {n_shards} shards")
+    if caller_exchanges:
+        return
     if not dist.is_initialized():
         if n_shards != 1:
             raise ValueError(f"{n_shards} shards need a process group of {n_shards} ranks; "
@@ -106,8 +110,12 @@ class ShardedMoELayer:
     this rank runs ``shard_bounds(T, n_shards)[shard]`` of it."""
 
     def __init__(self, workload: synth.Workload, params: dict, shard: int, n_shards: int,
-                 device="cuda", group=None):
-        check_placement(shard, n_shards, group)
+                 device="cuda", group=None, caller_exchanges: bool = False):
+        """caller_exchanges: the caller gathers every shard's counts itself and calls
+        route_shard / forward_shard / aux_finalize directly (forward, which runs the
+        collectives over the process group, is then unavailable)."""
+        check_placement(shard, n_shards, group, caller_exchanges)
+        self.caller_exchanges = caller_exchanges
         self.n_tokens_total = workload.T
         self.shard, self.n_shards, self.group = shard, n_shards, group
         a, b = shard_bounds(workload.T, n_shards)[shard]
@@ -138,4 +146,7 @@ class ShardedMoELayer:
 
     def forward(self, x: torch.Tensor, y: Optional[torch.Tensor] = None, want_aux: bool = False):
         """x: this rank's tokens [T_shard, d] on the device. Returns (y, aux or None)."""
+        if self.caller_exchanges:
+            raise RuntimeError("a layer built with caller_exchanges=True has no process "
+                               "group to exchange over; call its three steps directly")
         return forward_sharded(self, x, self.local.n_experts, self.group, want_aux, y)

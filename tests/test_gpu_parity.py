@@ -81,6 +81,49 @@ def test_route_given_logits_bitexact(E, k, mode):
     _devcheck(ws)
 
 
+# shapes of the tensor-core router: expert counts padded to N = 16 .. 256, K split
+# over 1, 2 or 4 CTAs of a cluster, token tiles with ragged tails, one-token batches
+ROUTE_TC_CASES = [
+    # E, k, T, d, gate mode, biases
+    (1, 1, 77, 128, 0, False), (8, 2, 1, 4096, 0, False), (8, 2, 129, 256, 1, True),
+    (8, 2, 4096, 4096, 0, False), (16, 4, 300, 192, 2, True), (33, 3, 1000, 512, 0, True),
+    (64, 6, 257, 2048, 1, False), (64, 6, 8192, 2048, 1, False), (128, 1, 5000, 1024, 2, True),
+    (200, 8, 130, 256, 1, True), (256, 8, 64, 128, 0, False), (20, 5, 33, 64, 2, True),
+]
+
+
+@pytest.mark.parametrize("E,k,T,d,mode,bias", ROUTE_TC_CASES,
+                         ids=[f"E{c[0]}_k{c[1]}_T{c[2]}_d{c[3]}" for c in ROUTE_TC_CASES])
+def test_route_tc_matches_oracle(E, k, T, d, mode, bias):
+    """moe_route with x (bf16): logits within the fp32 accumulation bound; the
+    selection and the gates exactly those the oracle takes from the same logits."""
+    wl = synth.SMALL["mixtral_small"].replace(T=T, n_experts=E, top_k=k, gate_mode=mode,
+                                              d_model=d, router_bias=bias, bias_std=0.1,
+                                              logit_bias_std=0.5 if bias else 0.0)
+    inp = synth.generate(wl, seed=E + T + d, with_weights=False)
+    layer = B.MoELayer(wl, inp, DEV)
+    x = inp["x"].to(DEV)
+    logits = torch.empty((T, E), dtype=torch.float32, device=DEV)
+    idx = torch.empty((T, k), dtype=torch.int32, device=DEV)
+    gate = torch.empty((T, k), dtype=torch.float32, device=DEV)
+    layer.route(x, logits, idx, gate)
+    torch.cuda.synchronize()
+    P = H.oracle_params(inp)
+    extra = np.zeros(E)
+    for key in ("b_router", "logit_bias"):
+        if P[key] is not None:
+            extra += np.abs(P[key])
+    z64 = O.router_logits(P["x"], P["w_router"], P["b_router"], P["logit_bias"])
+    zg = logits.cpu().numpy()
+    assert np.all(np.abs(zg.astype(np.float64) - z64) <=
+                  H.logits_bound(P["x"], P["w_router"], extra))
+    ref_idx = O.select_topk(zg, k)
+    assert np.array_equal(idx.cpu().numpy(), ref_idx)
+    assert np.allclose(gate.cpu().numpy(), O.gate_values(zg, ref_idx, H.MODE[mode]),
+                       rtol=4e-6, atol=1e-7)
+    _devcheck(layer.ws)
+
+
 # ============================================================= permute (bit-exact)
 PERMUTE_CASES = [
     # E, k, T, cf, dtype

@@ -50,7 +50,9 @@ def test_sharded_batch_matches_oracle(name, wl, world):
     P = H.oracle_params(inp)
     T, E, k = wl.T, wl.n_experts, wl.top_k
     x = inp["x"].to(DEV)
-    shards = [S.ShardedMoELayer(wl, inp, s, world, DEV) for s in range(world)]
+    # every shard in this one process: the test gathers the counts itself
+    shards = [S.ShardedMoELayer(wl, inp, s, world, DEV, caller_exchanges=True)
+              for s in range(world)]
     # phase 1: every shard routes its tokens, counts them and sums its statistics
     logits, taps, counts, parts = [], [], [], []
     for sh in shards:

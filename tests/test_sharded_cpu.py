@@ -121,6 +121,9 @@ def test_several_shards_need_a_process_group():
     with pytest.raises(ValueError, match="process group"):
         S.ShardedMoELayer(WL, {}, shard=0, n_shards=2, device="cpu")
     S.check_placement(0, 1)  # one shard is the whole batch
+    S.check_placement(1, 2, caller_exchanges=True)  # the caller gathers the counts itself
+    with pytest.raises(ValueError):
+        S.check_placement(2, 2, caller_exchanges=True)
 
 
 def test_counts_all_is_checked_before_the_descriptor_is_built():
