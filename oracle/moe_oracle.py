@@ -41,7 +41,10 @@ test):
   router logits (router bias and logit bias included).
 * GELU is the exact erf form; dropout and routing noise are off (inference).
 * Noisy top-k gating (training mode of P4 ``TopKGating``): the standard normal
-  draws eps [T, E] are an input, so both sides see the same draws.
+  draws eps [T, E] are either an input, so both sides see the same draws, or the
+  counter-based draws of ``noise_draws`` (Philox4x32-10 and Box-Muller) for a seed
+  and an offset, which both sides compute from the generator's published
+  definition.
 * Expert-Choice routing: each expert takes int(cf * T / E) tokens, chosen on the
   fp32 logits (equal logits: lower token index first); a token's output is the
   score-weighted sum over the experts that took it (P4's dispatch mask used as
@@ -478,6 +481,82 @@ def noisy_router_logits(x, w_router, w_noise, eps, b_router=None,
         z = z + _f64(logit_bias)[None, :]
     zn = x @ _f64(w_noise).T
     return (z + softplus(zn) * _f64(eps)).astype(np.float32)
+
+
+# ------------------------------------------- counter-based noise draws (Philox + Box-Muller)
+# The noisy gate of P4 ``TopKGating`` draws ``torch.randn_like`` inside the layer. With
+# a seed and an offset instead of a caller's tensor, the draws must be a pure function
+# of (seed, offset, token, expert) so that the CUDA path and this oracle produce the
+# same numbers: a counter-based generator. Philox4x32-10 is restated here from J. K.
+# Salmon, M. A. Moraes, R. O. Dror and D. E. Shaw, "Parallel Random Numbers: As Easy
+# as 1, 2, 3" (SC'11), and the normal deviates from its uniforms by the transform of
+# G. E. P. Box and M. E. Muller, "A Note on the Generation of Random Normal Deviates"
+# (Ann. Math. Statist. 29, 1958).
+PHILOX_M0, PHILOX_M1 = 0xD2511F53, 0xCD9E8D57   # round multipliers
+PHILOX_W0, PHILOX_W1 = 0x9E3779B9, 0xBB67AE85   # Weyl increments of the key
+_MASK32 = np.uint64(0xFFFFFFFF)
+
+
+def philox4x32(counter, key, rounds: int = 10) -> np.ndarray:
+    """Philox4x32-R: counter [..., 4] and key [..., 2] (uint32) -> [..., 4] uint32.
+
+    One round maps (c0, c1, c2, c3) with key (k0, k1) to
+    (hi(M1*c2) ^ c1 ^ k0, lo(M1*c2), hi(M0*c0) ^ c3 ^ k1, lo(M0*c0)), where hi/lo are
+    the upper and lower 32 bits of the 64-bit product; the key is advanced by
+    (W0, W1) mod 2^32 before every round but the first."""
+    counter = np.asarray(counter, dtype=np.uint64)
+    key = np.asarray(key, dtype=np.uint64)
+    c0, c1, c2, c3 = (counter[..., i] for i in range(4))
+    k0, k1 = key[..., 0], key[..., 1]
+    for r in range(rounds):
+        if r > 0:
+            k0 = (k0 + np.uint64(PHILOX_W0)) & _MASK32
+            k1 = (k1 + np.uint64(PHILOX_W1)) & _MASK32
+        p0 = c0 * np.uint64(PHILOX_M0)   # < 2^64: exact in uint64
+        p1 = c2 * np.uint64(PHILOX_M1)
+        c0, c1, c2, c3 = ((p1 >> np.uint64(32)) ^ c1 ^ k0, p1 & _MASK32,
+                          (p0 >> np.uint64(32)) ^ c3 ^ k1, p0 & _MASK32)
+    return np.stack([c0, c1, c2, c3], axis=-1).astype(np.uint32)
+
+
+def uniform_open(r) -> np.ndarray:
+    """A uint32 word to a uniform in (0, 1): u = (2 * (r >> 9) + 1) * 2^-24, an odd
+    multiple of 2^-24 (exact in fp32 and fp64; never 0 or 1)."""
+    r = np.asarray(r, dtype=np.uint64)
+    return ((r >> np.uint64(9)).astype(np.float64) * 2.0 + 1.0) * 2.0 ** -24
+
+
+def box_muller(u_a, u_b):
+    """Two independent standard normals from two uniforms in (0, 1):
+    rho = sqrt(-2 ln u_a), (rho cos(2 pi u_b), rho sin(2 pi u_b)), in fp64."""
+    rho = np.sqrt(-2.0 * np.log(u_a))
+    ang = 2.0 * math.pi * np.asarray(u_b, dtype=np.float64)
+    return rho * np.cos(ang), rho * np.sin(ang)
+
+
+def noise_draws(T: int, E: int, seed: int, offset: int):
+    """The noise eps [T, E] of the seeded noisy gate, fp64, and the raw Philox words
+    [T, ceil(E/4), 4].
+
+    Token t and expert group q = e // 4 use counter (t, q, offset mod 2^32,
+    offset >> 32) and key (seed mod 2^32, seed >> 32); with the four words (r0, r1,
+    r2, r3) and u_i = uniform_open(r_i), Box-Muller of (u0, u1) gives experts 4q and
+    4q + 1 (cos, then sin) and of (u2, u3) experts 4q + 2 and 4q + 3."""
+    Q = (E + 3) // 4
+    t = np.arange(T, dtype=np.uint64)[:, None]
+    q = np.arange(Q, dtype=np.uint64)[None, :]
+    ctr = np.zeros((T, Q, 4), dtype=np.uint64)
+    ctr[..., 0] = t
+    ctr[..., 1] = q
+    ctr[..., 2] = offset & 0xFFFFFFFF
+    ctr[..., 3] = (offset >> 32) & 0xFFFFFFFF
+    key = np.array([seed & 0xFFFFFFFF, (seed >> 32) & 0xFFFFFFFF], dtype=np.uint64)
+    raw = philox4x32(ctr, np.broadcast_to(key, (T, Q, 2)))
+    u = uniform_open(raw)
+    eps = np.empty((T, Q, 4), dtype=np.float64)
+    eps[..., 0], eps[..., 1] = box_muller(u[..., 0], u[..., 1])
+    eps[..., 2], eps[..., 3] = box_muller(u[..., 2], u[..., 3])
+    return eps.reshape(T, 4 * Q)[:, :E], raw
 
 
 # ------------------------------------------------- token-sharded routing (several ranks)

@@ -475,10 +475,54 @@ def check_sharded_capacity(O):
     assert O.shard_capacity(np.ones((2, 3)), 1, None) is None
 
 
+# ------------------------------------------------- counter-based noise (Philox, Box-Muller)
+def check_philox_kat(O):
+    """Philox4x32-10 reproduces the generator's published known-answer vectors."""
+    kat = _golden("philox_kat.json")
+    for case in kat["cases"]:
+        ctr = np.array([int(v, 16) for v in case["counter"]], dtype=np.uint64)
+        key = np.array([int(v, 16) for v in case["key"]], dtype=np.uint64)
+        out = O.philox4x32(ctr, key, rounds=kat["rounds"])
+        assert [int(v) for v in out] == [int(v, 16) for v in case["out"]], case
+
+
+def check_noise_draws(O):
+    """The seeded noise: uniforms strictly inside (0, 1) and exact in fp32; the draws
+    a function of (seed, offset) alone; standard normal (Kolmogorov-Smirnov, mean,
+    variance) with the two members of a Box-Muller pair uncorrelated, also in their
+    squares (which a shared uniform would correlate)."""
+    from scipy import stats
+
+    u = O.uniform_open(np.array([0, 1, 511, 512, 2 ** 31, 2 ** 32 - 1], dtype=np.uint64))
+    assert u.min() > 0 and u.max() < 1
+    assert np.array_equal(u.astype(np.float32).astype(np.float64), u)
+    assert u[0] == 2.0 ** -24 and u[-1] == 1.0 - 2.0 ** -24 and u[2] == u[0] and u[3] > u[2]
+    T, E = 4096, 64
+    eps, raw = O.noise_draws(T, E, seed=1234, offset=5)
+    assert eps.shape == (T, E) and raw.shape == (T, E // 4, 4)
+    again, _ = O.noise_draws(T, E, seed=1234, offset=5)
+    assert np.array_equal(eps, again)
+    assert not np.array_equal(O.noise_draws(8, E, seed=1234, offset=6)[0], eps[:8])
+    assert not np.array_equal(O.noise_draws(8, E, seed=1235, offset=5)[0], eps[:8])
+    # a ragged expert count takes the first E columns of the same draws
+    assert np.array_equal(O.noise_draws(16, 6, seed=1234, offset=5)[0], eps[:16, :6])
+    n = eps.size
+    v = eps.ravel()
+    assert abs(v.mean()) < 5.0 / math.sqrt(n)
+    assert abs(v.var() - 1.0) < 5.0 * math.sqrt(2.0 / n)
+    assert stats.kstest(v, "norm").pvalue > 1e-4
+    a, b = eps[:, 0::2].ravel(), eps[:, 1::2].ravel()  # the two members of each pair
+    assert abs(np.corrcoef(a, b)[0, 1]) < 5.0 / math.sqrt(a.size)
+    assert abs(np.corrcoef(a * a, b * b)[0, 1]) < 5.0 / math.sqrt(a.size)
+    # nothing repeats across tokens, expert groups or offsets
+    words = np.concatenate([raw.ravel(), O.noise_draws(64, E, 1234, 6)[1].ravel()])
+    assert len(np.unique(words)) > 0.999 * len(words)
+
+
 ALL_CHECKS = [check_combine, check_topk_bruteforce, check_gate_sums_and_ranges, check_worked_gates,
               check_softmax_closed_forms, check_router_logits_exact, check_capacity_golden,
               check_counts_and_drop_order, check_layout, check_forward_vs_pages_torch,
               check_sparse_equals_dense_masked, check_special_cases, check_aux_closed_forms,
               check_expert_choice_capacity, check_expert_choice_bruteforce,
               check_expert_choice_scores, check_expert_choice_dense, check_noisy_logits,
-              check_sharded_capacity]
+              check_sharded_capacity, check_philox_kat, check_noise_draws]

@@ -141,7 +141,42 @@ def _shard_capacity_ignores_earlier(counts_all, rank, cap):
     return _orig["shard_capacity"](counts_all, 0, cap)
 
 
+def _philox_nine_rounds(counter, key, rounds=10):
+    return _orig["philox4x32"](counter, key, rounds - 1)
+
+
+def _philox_key_not_advanced(counter, key, rounds=10):
+    c = [np.asarray(counter, dtype=np.uint64)[..., i] for i in range(4)]
+    k0, k1 = (np.asarray(key, dtype=np.uint64)[..., i] for i in range(2))
+    m = np.uint64(0xFFFFFFFF)
+    for _ in range(rounds):
+        p0 = c[0] * np.uint64(O.PHILOX_M0)
+        p1 = c[2] * np.uint64(O.PHILOX_M1)
+        c = [(p1 >> np.uint64(32)) ^ c[1] ^ k0, p1 & m, (p0 >> np.uint64(32)) ^ c[3] ^ k1,
+             p0 & m]
+    return np.stack(c, axis=-1).astype(np.uint32)
+
+
+def _box_muller_without_two(u_a, u_b):
+    rho = np.sqrt(-np.log(u_a))
+    ang = 2.0 * math.pi * np.asarray(u_b, dtype=np.float64)
+    return rho * np.cos(ang), rho * np.sin(ang)
+
+
+def _box_muller_one_uniform(u_a, u_b):
+    return _orig["box_muller"](u_a, u_a)
+
+
+def _uniform_includes_zero(r):
+    return (np.asarray(r, dtype=np.uint64) >> np.uint64(8)).astype(np.float64) * 2.0 ** -24
+
+
 MUTANTS = {
+    "philox_nine_rounds": ("philox4x32", _philox_nine_rounds),
+    "philox_key_not_advanced": ("philox4x32", _philox_key_not_advanced),
+    "box_muller_without_factor_two": ("box_muller", _box_muller_without_two),
+    "box_muller_one_uniform_for_both": ("box_muller", _box_muller_one_uniform),
+    "uniform_includes_zero": ("uniform_open", _uniform_includes_zero),
     "shard_capacity_ignores_earlier_shards": ("shard_capacity", _shard_capacity_ignores_earlier),
     "softplus_is_exp": ("softplus", _softplus_is_exp),
     "noise_sign_flipped": ("noisy_router_logits", _noise_sign_flipped),
