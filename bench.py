@@ -202,8 +202,8 @@ def oracle_sample_rate(wl, P, n_tokens: int):
                   capacity_factor=wl.capacity_factor, n_shared=wl.n_shared)
         t0 = time.perf_counter()
         noisy = None
-        if wl.noisy:  # the same seeded draws as the GPU arm
-            eps = synth.noise_draws(wl.T, wl.n_experts, 99).numpy()
+        if wl.noisy:  # the counter-based draws of the GPU arm's first step
+            eps = O.noise_draws(wl.T, wl.n_experts, 1234, 1)[0]
             noisy = O.noisy_router_logits(P["x"], P["w_router"], P["w_noise"], eps,
                                           P.get("b_router"), P.get("logit_bias"))
         r = O.route(P["x"], P, top_k=wl.top_k, gate_mode=kw["gate_mode"],
@@ -448,17 +448,20 @@ class Workbench:
         # the capacity workloads also emit f, P and the aux loss (token choice only)
         self.want_aux = wl.capacity_factor > 0 and not self.ec
         self.aux = self.layer.new_aux() if self.want_aux else None
-        # noisy gating: the step routes on logits + softplus(x W_noise^T) * eps; the
-        # draws eps are made once (seeded) and stay resident, like x
-        self.eps = synth.noise_draws(wl.T, wl.n_experts, 99 + rank).to(dev) if wl.noisy else None
+        # noisy gating: the step routes on logits + softplus(x W_noise^T) * eps, the
+        # draws eps made inside the library for (seed, offset), a new offset per step
+        self.noise_seed = 1234 + rank if wl.noisy else None
+        self.noise_offset = 0
 
     def forward(self, x=None, y=None, aux=None, taps=None, events=None):
         x = self.x if x is None else x
         y = self.y if y is None else y
         aux = self.aux if aux is None else aux
-        if self.eps is None:
+        if self.noise_seed is None:
             return self.layer.forward(x, y, aux, taps=taps, events=events)
-        return self.layer.forward_noisy(x, self.eps, y, aux, taps=taps, events=events)
+        self.noise_offset += 1
+        return self.layer.forward_noisy(x, None, y, aux, taps=taps, events=events,
+                                        seed=self.noise_seed, offset=self.noise_offset)
 
     def check(self, where):
         code, info = self.layer.last_device_error()

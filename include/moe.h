@@ -265,21 +265,33 @@ typedef struct {
   moe_event_t ev[MOE_STAGE_COUNT + 1];
 } moe_stage_events_t;
 
-/* moe_forward that also records `events` (nullable) at its stage boundaries and
- * marks each stage with an NVTX range (named "moe_route", "moe_scan", ...). The
- * kernels and results are those of moe_forward; a failed event record returns
+/* The noise of noisy top-k gating for moe_forward_staged: the caller's draws eps
+ * [T, E] fp32 (device), or, when eps is NULL, the counter-based draws for (seed,
+ * offset) (see moe_noise_draws). */
+typedef struct {
+  const float *eps;
+  uint64_t seed;
+  uint64_t offset;
+} moe_noise_t;
+
+/* moe_forward (noise == NULL) or moe_forward_noisy / moe_forward_noisy_seeded (noise
+ * given) that also records `events` (nullable) at its stage boundaries and marks
+ * each stage with an NVTX range (named "moe_route", "moe_scan", ...). The kernels and
+ * results are those of the plain entry points; a failed event record returns
  * MOE_ERR_CUDA. */
 moe_status_t moe_forward_staged(const moe_cfg_t *cfg, const moe_weights_t *w, const void *x,
-                                void *y, float *aux_out, const moe_taps_t *taps,
-                                const moe_stage_events_t *events, void *ws, size_t ws_bytes,
-                                moe_stream_t stream);
+                                const moe_noise_t *noise, void *y, float *aux_out,
+                                const moe_taps_t *taps, const moe_stage_events_t *events,
+                                void *ws, size_t ws_bytes, moe_stream_t stream);
 
 /* Noisy top-k gating, the training mode of youngju.dev (ja) "TopKGating" (Noisy Top-K
  * Gating): the logits are z + softplus(x W_noise^T) * eps, z as in moe_route, softplus
  * the identity above 20 (as F.softplus), eps [T, E] fp32 standard normal draws made by
  * the caller (device memory); then selection and gates exactly as moe_route on those
  * logits (cfg->gate_mode; the page's mode is MOE_GATE_SOFTMAX_TOPK_RENORM). logits
- * [T, E] fp32 receives the noisy logits. Token-choice configurations only. */
+ * [T, E] fp32 receives the noisy logits. Token-choice configurations only. bf16 layers
+ * with at most 128 experts compute both projections in one tensor-core pass over x;
+ * the others take two router passes and an elementwise step. */
 moe_status_t moe_route_noisy(const moe_cfg_t *cfg, const moe_weights_t *w, const void *x,
                              const float *eps, float *logits, int32_t *topk_idx,
                              float *topk_gate, void *ws, size_t ws_bytes, moe_stream_t stream);
@@ -290,11 +302,32 @@ moe_status_t moe_forward_noisy(const moe_cfg_t *cfg, const moe_weights_t *w, con
                                const float *eps, void *y, float *aux_out, const moe_taps_t *taps,
                                void *ws, size_t ws_bytes, moe_stream_t stream);
 
-/* moe_forward_noisy with stage events (see moe_forward_staged). */
-moe_status_t moe_forward_noisy_staged(const moe_cfg_t *cfg, const moe_weights_t *w,
-                                      const void *x, const float *eps, void *y, float *aux_out,
-                                      const moe_taps_t *taps, const moe_stage_events_t *events,
-                                      void *ws, size_t ws_bytes, moe_stream_t stream);
+/* The standard normal draws of the seeded noisy gate, for (seed, offset): eps [T, E]
+ * fp32 (device) and, when raw != NULL, the generator's words raw [T, ceil(E/4), 4]
+ * uint32 (device, 16-byte aligned). A pure function of (seed, offset, token, expert),
+ * so calls may be repeated or split freely. Generator: Philox4x32-10 (J. K. Salmon,
+ * M. A. Moraes, R. O. Dror, D. E. Shaw, "Parallel Random Numbers: As Easy as 1, 2,
+ * 3", SC'11) with counter (t, e / 4, offset mod 2^32, offset >> 32) and key (seed mod
+ * 2^32, seed >> 32); each output word r gives u = (2 (r >> 9) + 1) 2^-24 in (0, 1),
+ * and the Box-Muller transform (rho = sqrt(-2 ln u0), rho cos 2 pi u1, rho sin 2 pi
+ * u1) of words (0, 1) gives experts 4q, 4q + 1 and of words (2, 3) experts 4q + 2,
+ * 4q + 3 (computed in fp32 with the device's logf, sqrtf and sincospif). A training
+ * loop advances `offset` once per call: different offsets use disjoint counters. */
+moe_status_t moe_noise_draws(int32_t n_tokens, int32_t n_experts, uint64_t seed,
+                             uint64_t offset, float *eps, uint32_t *raw, moe_stream_t stream);
+
+/* moe_route_noisy with the noise drawn inside the library for (seed, offset), the
+ * draws of moe_noise_draws (kept in the workspace). */
+moe_status_t moe_route_noisy_seeded(const moe_cfg_t *cfg, const moe_weights_t *w,
+                                    const void *x, uint64_t seed, uint64_t offset,
+                                    float *logits, int32_t *topk_idx, float *topk_gate,
+                                    void *ws, size_t ws_bytes, moe_stream_t stream);
+
+/* moe_forward_noisy with the noise drawn inside the library for (seed, offset). */
+moe_status_t moe_forward_noisy_seeded(const moe_cfg_t *cfg, const moe_weights_t *w,
+                                      const void *x, uint64_t seed, uint64_t offset, void *y,
+                                      float *aux_out, const moe_taps_t *taps, void *ws,
+                                      size_t ws_bytes, moe_stream_t stream);
 
 /* Expert-Choice routing step (youngju.dev (zh) "ExpertChoiceRouter", youngju.dev (ja)
  * "ExpertChoiceGating"): logits as in moe_route, then for every expert e its C =

@@ -30,7 +30,8 @@ EXPORTED = ("moe_workspace_size", "moe_workspace_init", "moe_route", "moe_route_
             "moe_route_expert_choice", "moe_permute", "moe_permute_noalloc", "moe_forward_noisy",
             "moe_expert_ffn", "moe_combine", "moe_aux_stats", "moe_forward",
             "moe_route_shard", "moe_permute_shard", "moe_forward_shard", "moe_aux_finalize",
-            "moe_forward_staged", "moe_forward_noisy_staged",
+            "moe_forward_staged", "moe_noise_draws", "moe_route_noisy_seeded",
+            "moe_forward_noisy_seeded",
             "moe_last_device_error", "moe_status_string")
 
 # stages of one layer call (MOE_STAGE_*), in launch order
@@ -73,6 +74,10 @@ class MoeStageEvents(ctypes.Structure):
     _fields_ = [("ev", ctypes.c_void_p * (len(STAGES) + 1))]
 
 
+class MoeNoise(ctypes.Structure):
+    _fields_ = [("eps", ctypes.c_void_p), ("seed", ctypes.c_uint64), ("offset", ctypes.c_uint64)]
+
+
 def lib_path() -> str:
     return _LIB_PATH
 
@@ -103,10 +108,15 @@ def load() -> ctypes.CDLL:
         "moe_forward_shard": [cfgp, ctypes.POINTER(MoeShard), wp, P, ctypes.POINTER(MoeTaps), P,
                               P, S, P],
         "moe_aux_finalize": [cfgp, ctypes.c_longlong, P, P, P],
-        "moe_forward_staged": [cfgp, wp, P, P, P, ctypes.POINTER(MoeTaps),
-                               ctypes.POINTER(MoeStageEvents), P, S, P],
-        "moe_forward_noisy_staged": [cfgp, wp, P, P, P, P, ctypes.POINTER(MoeTaps),
-                                     ctypes.POINTER(MoeStageEvents), P, S, P],
+        "moe_forward_staged": [cfgp, wp, P, ctypes.POINTER(MoeNoise), P, P,
+                               ctypes.POINTER(MoeTaps), ctypes.POINTER(MoeStageEvents), P, S,
+                               P],
+        "moe_noise_draws": [ctypes.c_int32, ctypes.c_int32, ctypes.c_uint64, ctypes.c_uint64, P,
+                            P, P],
+        "moe_route_noisy_seeded": [cfgp, wp, P, ctypes.c_uint64, ctypes.c_uint64, P, P, P, P, S,
+                                   P],
+        "moe_forward_noisy_seeded": [cfgp, wp, P, ctypes.c_uint64, ctypes.c_uint64, P, P,
+                                     ctypes.POINTER(MoeTaps), P, S, P],
         "moe_last_device_error": [P, ctypes.POINTER(ctypes.c_int32),
                                   ctypes.POINTER(ctypes.c_int32), P],
     }
@@ -207,32 +217,42 @@ class MoELayer:
                                         _ptr(x), _ptr(y), _ptr(aux), tpr, _ptr(self.ws),
                                         self.ws.numel(), _stream()), "moe_forward")
         else:
-            ev = stage_events(events)
-            _check(self.lib.moe_forward_staged(ctypes.byref(self.cfg),
-                                               ctypes.byref(self.weights), _ptr(x), _ptr(y),
-                                               _ptr(aux), tpr, ctypes.byref(ev), _ptr(self.ws),
-                                               self.ws.numel(), _stream()), "moe_forward_staged")
+            self._staged(x, None, y, aux, tpr, events)
         return y
 
-    def forward_noisy(self, x: torch.Tensor, eps: torch.Tensor, y: Optional[torch.Tensor] = None,
-                      aux: Optional[torch.Tensor] = None, taps: Optional[dict] = None,
-                      events: Optional[list] = None) -> torch.Tensor:
-        """The layer with noisy top-k gating; eps [T, E] fp32 standard normal draws."""
+    def _staged(self, x, noise, y, aux, tpr, events):
+        ev = stage_events(events)
+        _check(self.lib.moe_forward_staged(ctypes.byref(self.cfg), ctypes.byref(self.weights),
+                                           _ptr(x), ctypes.byref(noise) if noise else None,
+                                           _ptr(y), _ptr(aux), tpr, ctypes.byref(ev),
+                                           _ptr(self.ws), self.ws.numel(), _stream()),
+               "moe_forward_staged")
+
+    def forward_noisy(self, x: torch.Tensor, eps: Optional[torch.Tensor] = None,
+                      y: Optional[torch.Tensor] = None, aux: Optional[torch.Tensor] = None,
+                      taps: Optional[dict] = None, events: Optional[list] = None,
+                      seed: Optional[int] = None, offset: int = 0) -> torch.Tensor:
+        """The layer with noisy top-k gating: eps [T, E] fp32 standard normal draws, or
+        (eps None) the library's counter-based draws for (seed, offset)."""
+        if (eps is None) == (seed is None):
+            raise ValueError("give either eps or seed")
         if y is None:
             y = torch.empty_like(x)
         tp = _taps(taps)
         tpr = ctypes.byref(tp) if tp is not None else None
-        if events is None:
+        if events is not None:
+            self._staged(x, MoeNoise(eps=_ptr(eps), seed=seed or 0, offset=offset), y, aux, tpr,
+                         events)
+        elif eps is not None:
             _check(self.lib.moe_forward_noisy(ctypes.byref(self.cfg), ctypes.byref(self.weights),
                                               _ptr(x), _ptr(eps), _ptr(y), _ptr(aux), tpr,
                                               _ptr(self.ws), self.ws.numel(), _stream()),
                    "moe_forward_noisy")
         else:
-            ev = stage_events(events)
-            _check(self.lib.moe_forward_noisy_staged(
-                ctypes.byref(self.cfg), ctypes.byref(self.weights), _ptr(x), _ptr(eps), _ptr(y),
-                _ptr(aux), tpr, ctypes.byref(ev), _ptr(self.ws), self.ws.numel(), _stream()),
-                "moe_forward_noisy_staged")
+            _check(self.lib.moe_forward_noisy_seeded(
+                ctypes.byref(self.cfg), ctypes.byref(self.weights), _ptr(x), seed, offset,
+                _ptr(y), _ptr(aux), tpr, _ptr(self.ws), self.ws.numel(), _stream()),
+                "moe_forward_noisy_seeded")
         return y
 
     def new_taps(self) -> dict:
@@ -261,6 +281,14 @@ class MoELayer:
                                         _ptr(x), _ptr(eps), _ptr(logits), _ptr(topk_idx),
                                         _ptr(topk_gate), _ptr(self.ws), self.ws.numel(),
                                         _stream()), "moe_route_noisy")
+
+    def route_noisy_seeded(self, x: torch.Tensor, seed: int, offset: int, logits: torch.Tensor,
+                           topk_idx: torch.Tensor, topk_gate: torch.Tensor):
+        _check(self.lib.moe_route_noisy_seeded(ctypes.byref(self.cfg), ctypes.byref(self.weights),
+                                               _ptr(x), seed, offset, _ptr(logits),
+                                               _ptr(topk_idx), _ptr(topk_gate), _ptr(self.ws),
+                                               self.ws.numel(), _stream()),
+               "moe_route_noisy_seeded")
 
     def route_expert_choice(self, x: Optional[torch.Tensor], logits: torch.Tensor,
                             ec_idx: torch.Tensor, ec_score: torch.Tensor):
@@ -339,6 +367,14 @@ class MoELayer:
         if st not in (MOE_OK, 6):
             raise MoeError(st, "moe_last_device_error")
         return code.value, info.value
+
+
+def noise_draws(n_tokens: int, n_experts: int, seed: int, offset: int, eps: torch.Tensor,
+                raw: Optional[torch.Tensor] = None):
+    """moe_noise_draws: eps [T, E] fp32 and optionally raw [T, ceil(E/4), 4] int32 words
+    (the uint32 bit patterns), both on the current device and stream."""
+    _check(load().moe_noise_draws(n_tokens, n_experts, seed, offset, _ptr(eps), _ptr(raw),
+                                  _stream()), "moe_noise_draws")
 
 
 def shared_as_experts(layer: MoELayer):

@@ -19,6 +19,10 @@ struct RouterArgs {
   float *tile_z;            // [NT] or nullptr: per-tile sums of logsumexp^2
   int T, d, E, k, gate_mode;
   int32_t *err;             // device error word (pipeline timeouts) or nullptr
+  // noisy top-k gating (tensor-core router only): when w_noise != nullptr the logits
+  // are z + softplus(x W_noise^T) * eps before the selection
+  const void *w_noise;      // [E, d] dtype
+  const float *eps;         // [T, E] standard normal draws
 };
 
 struct ScanArgs {
@@ -103,8 +107,12 @@ cudaError_t launch_router(const RouterArgs &a, int dtype, cudaStream_t st);
 // noisy top-k gating: z[i] += softplus(zn[i]) * eps[i] over n logits
 cudaError_t launch_noisy_logits(float *z, const float *zn, const float *eps, size_t n,
                                 cudaStream_t st);
-// bf16 router on the tensor cores (x given, d a multiple of 64, T > 0)
+// bf16 router on the tensor cores (x given, d a multiple of 64, T > 0; with
+// w_noise, at most 128 experts)
 bool router_tc_supported(const RouterArgs &a);
+// the seeded noise draws eps [T, E] (and the raw Philox words [T, ceil(E/4), 4])
+cudaError_t launch_noise_draws(int T, int E, uint64_t seed, uint64_t offset, float *eps,
+                               uint32_t *raw, cudaStream_t st);
 cudaError_t launch_router_tc(const RouterArgs &a, cudaStream_t st);
 cudaError_t launch_tile_counts(const int32_t *topk_idx, int T, int k, int E, int32_t *tile_counts,
                                int32_t *err, cudaStream_t st);

@@ -17,7 +17,7 @@ namespace {
 enum Buf {
   B_ERR, B_TILE_COUNTS, B_TILE_BASE, B_TILE_P, B_TILE_Z, B_COUNTS, B_OFFSETS, B_MPREFIX, B_SH_TBL,
   B_LOGITS, B_IDX, B_GATE, B_PERM, B_INV, B_XPERM, B_H, B_YPERM, B_SH_H, B_SH_Y, B_YPART,
-  B_EC_ZT, B_EC_IDX, B_EC_SCORE, B_EC_SLOT, B_NOISE, B_CAP_E, B_NBUF
+  B_EC_ZT, B_EC_IDX, B_EC_SCORE, B_EC_SLOT, B_NOISE, B_CAP_E, B_EPS, B_NBUF
 };
 
 struct Layout {
@@ -84,6 +84,7 @@ Layout layout_for(const moe_cfg_t &c) {
   sz[B_EC_SLOT] = ec ? T * E * 4 : 0;
   sz[B_NOISE] = T * E * 4;  // x W_noise^T of noisy top-k gating
   sz[B_CAP_E] = E * 4;      // per-expert capacity left to one shard of a batch
+  sz[B_EPS] = T * E * 4;    // the seeded noise draws of noisy top-k gating
   Layout L;
   size_t o = 0;
   for (int i = 0; i < B_NBUF; ++i) {
@@ -320,6 +321,49 @@ moe_status_t noisy_logits(const moe_cfg_t &c, const moe_weights_t *w, const void
   return MOE_OK;
 }
 
+// The noise of noisy top-k gating: the caller's draws, or the counter-based draws
+// for (seed, offset).
+struct NoiseSpec {
+  const float *eps;  // [T, E] or nullptr: draw from (seed, offset)
+  uint64_t seed, offset;
+};
+
+// Noisy routing: r carries the selection outputs (topk_idx, topk_gate, the per-tile
+// partials, logits_out = the noisy-logits tap or nullptr). For bf16 layers with at
+// most 128 experts one tensor-core pass computes both projections and the noisy
+// logits and selects on them; otherwise the noisy logits go to logits_buf by two
+// router passes and an elementwise kernel, and a second pass selects on them.
+moe_status_t route_noisy(const moe_cfg_t &c, const moe_weights_t *w, const void *x,
+                         const NoiseSpec &ns, RouterArgs r, float *logits_buf, void *ws,
+                         const Layout &L, cudaStream_t stream) {
+  const float *eps = ns.eps;
+  if (eps == nullptr) {
+    float *draws = at<float>(ws, L, B_EPS);
+    MOE_CUDA(launch_noise_draws(c.n_tokens, c.n_experts, ns.seed, ns.offset, draws, nullptr,
+                                stream));
+    eps = draws;
+  }
+  RouterArgs f = r;
+  f.x = x;
+  f.w = w->w_router;
+  f.b_router = w->b_router;
+  f.logit_bias = w->logit_bias;
+  f.logits_in = nullptr;
+  f.w_noise = w->w_noise;
+  f.eps = eps;
+  if (c.dtype == MOE_DTYPE_BF16 && router_tc_supported(f)) {
+    MOE_CUDA(launch_router(f, c.dtype, stream));
+    return MOE_OK;
+  }
+  MOE_TRY(noisy_logits(c, w, x, eps, logits_buf, ws, L, stream));
+  RouterArgs sel = r;
+  sel.x = nullptr;
+  sel.logits_in = logits_buf;
+  sel.logits_out = nullptr;
+  MOE_CUDA(launch_router(sel, c.dtype, stream));
+  return MOE_OK;
+}
+
 // Expert-Choice routing: router logits (unless x is NULL: logits are the input),
 // then every expert's picks. slot/offsets (nullable) feed the forward's later steps.
 moe_status_t ec_route(const moe_cfg_t &c, const moe_weights_t *w, const void *x, float *logits,
@@ -445,23 +489,23 @@ MOE_API moe_status_t moe_route(const moe_cfg_t *cfg, const moe_weights_t *w, con
   return MOE_OK;
 }
 
-MOE_API moe_status_t moe_route_noisy(const moe_cfg_t *cfg, const moe_weights_t *w,
-                                     const void *x, const float *eps, float *logits,
-                                     int32_t *topk_idx, float *topk_gate, void *ws,
-                                     size_t ws_bytes, moe_stream_t stream) {
+namespace moe {
+namespace {
+moe_status_t route_noisy_entry(const moe_cfg_t *cfg, const moe_weights_t *w, const void *x,
+                               const NoiseSpec &ns, float *logits, int32_t *topk_idx,
+                               float *topk_gate, void *ws, size_t ws_bytes, cudaStream_t stream) {
   MOE_TRY(check_cfg(cfg));
   MOE_TRY(check_ws(cfg, ws, ws_bytes));
   if (expert_choice(*cfg)) return MOE_ERR_INVALID_ARG;
   if (cfg->n_tokens == 0) return MOE_OK;
   if (w == nullptr) return MOE_ERR_INVALID_ARG;
-  MOE_TRY(check_ptrs({{x, true}, {eps, true}, {logits, true}, {topk_idx, true},
-                      {topk_gate, true}, {w->w_router, true}, {w->w_noise, true},
-                      {w->b_router, false}, {w->logit_bias, false}}));
+  MOE_TRY(check_ptrs({{x, true}, {logits, true}, {topk_idx, true}, {topk_gate, true},
+                      {w->w_router, true}, {w->w_noise, true}, {w->b_router, false},
+                      {w->logit_bias, false}}));
   const moe_cfg_t &c = *cfg;
   const Layout L = layout_for(c);
-  MOE_TRY(noisy_logits(c, w, x, eps, logits, ws, L, stream));
   RouterArgs r{};
-  r.logits_in = logits;
+  r.logits_out = logits;
   r.topk_idx = topk_idx;
   r.topk_gate = topk_gate;
   r.tile_counts = at<int32_t>(ws, L, B_TILE_COUNTS);
@@ -471,7 +515,35 @@ MOE_API moe_status_t moe_route_noisy(const moe_cfg_t *cfg, const moe_weights_t *
   r.k = c.top_k;
   r.gate_mode = c.gate_mode;
   r.err = at<int32_t>(ws, L, B_ERR);
-  MOE_CUDA(launch_router(r, c.dtype, stream));
+  return route_noisy(c, w, x, ns, r, logits, ws, L, stream);
+}
+}  // namespace
+}  // namespace moe
+
+MOE_API moe_status_t moe_route_noisy(const moe_cfg_t *cfg, const moe_weights_t *w,
+                                     const void *x, const float *eps, float *logits,
+                                     int32_t *topk_idx, float *topk_gate, void *ws,
+                                     size_t ws_bytes, moe_stream_t stream) {
+  if (eps == nullptr) return MOE_ERR_INVALID_ARG;
+  MOE_TRY(check_ptrs({{eps, true}}));
+  return route_noisy_entry(cfg, w, x, NoiseSpec{eps, 0, 0}, logits, topk_idx, topk_gate, ws,
+                           ws_bytes, stream);
+}
+
+MOE_API moe_status_t moe_route_noisy_seeded(const moe_cfg_t *cfg, const moe_weights_t *w,
+                                            const void *x, uint64_t seed, uint64_t offset,
+                                            float *logits, int32_t *topk_idx, float *topk_gate,
+                                            void *ws, size_t ws_bytes, moe_stream_t stream) {
+  return route_noisy_entry(cfg, w, x, NoiseSpec{nullptr, seed, offset}, logits, topk_idx,
+                           topk_gate, ws, ws_bytes, stream);
+}
+
+MOE_API moe_status_t moe_noise_draws(int32_t n_tokens, int32_t n_experts, uint64_t seed,
+                                     uint64_t offset, float *eps, uint32_t *raw,
+                                     moe_stream_t stream) {
+  if (n_tokens < 0 || n_experts < 1 || n_experts > kMaxExperts) return MOE_ERR_INVALID_ARG;
+  MOE_TRY(check_ptrs({{eps, true}, {raw, false}}));
+  MOE_CUDA(launch_noise_draws(n_tokens, n_experts, seed, offset, eps, raw, stream));
   return MOE_OK;
 }
 
@@ -634,11 +706,11 @@ MOE_API moe_status_t moe_aux_stats(const moe_cfg_t *cfg, const float *logits,
 
 namespace moe {
 namespace {
-// the whole layer; eps != NULL: noisy top-k gating (token choice only)
+// the whole layer; noise != NULL: noisy top-k gating (token choice only)
 // sh != NULL: one shard of a token-sharded batch, routed already (topk_idx and
 // topk_gate in taps, the capacity of the whole batch shared out per expert)
 moe_status_t forward_impl(const moe_cfg_t *cfg, const moe_weights_t *w, const void *x,
-                          const float *eps, void *y, float *aux_out, const moe_taps_t *taps,
+                          const NoiseSpec *noise, void *y, float *aux_out, const moe_taps_t *taps,
                           void *ws, size_t ws_bytes, moe_stream_t stream,
                           const moe_shard_t *sh = nullptr,
                           const moe_stage_events_t *events = nullptr) {
@@ -646,7 +718,7 @@ moe_status_t forward_impl(const moe_cfg_t *cfg, const moe_weights_t *w, const vo
   MOE_TRY(check_ws(cfg, ws, ws_bytes));
   if (sh != nullptr) {
     MOE_TRY(check_shard(*cfg, sh));
-    if (aux_out != nullptr || eps != nullptr) return MOE_ERR_INVALID_ARG;
+    if (aux_out != nullptr || noise != nullptr) return MOE_ERR_INVALID_ARG;
     if (cfg->n_tokens > 0 &&
         (taps == nullptr || taps->topk_idx == nullptr || taps->topk_gate == nullptr))
       return MOE_ERR_INVALID_ARG;
@@ -670,10 +742,10 @@ moe_status_t forward_impl(const moe_cfg_t *cfg, const moe_weights_t *w, const vo
   int32_t *err = at<int32_t>(ws, L, B_ERR);
   float *logits = tp.logits ? tp.logits : at<float>(ws, L, B_LOGITS);
   if (expert_choice(c)) {
-    if (aux_out != nullptr || eps != nullptr) return MOE_ERR_INVALID_ARG;
+    if (aux_out != nullptr || noise != nullptr) return MOE_ERR_INVALID_ARG;
     return ec_forward(c, w, x, y, logits, ws, L, stream, sg);
   }
-  if (eps != nullptr) MOE_TRY(check_ptrs({{eps, true}, {w->w_noise, true}}));
+  if (noise != nullptr) MOE_TRY(check_ptrs({{noise->eps, false}, {w->w_noise, true}}));
   int32_t *idx = tp.topk_idx ? tp.topk_idx : at<int32_t>(ws, L, B_IDX);
   float *gate = tp.topk_gate ? tp.topk_gate : at<float>(ws, L, B_GATE);
   int32_t *counts = tp.counts ? tp.counts : at<int32_t>(ws, L, B_COUNTS);
@@ -685,19 +757,16 @@ moe_status_t forward_impl(const moe_cfg_t *cfg, const moe_weights_t *w, const vo
   const bool want_aux = aux_out != nullptr;
 
   // 1. router GEMM + softmax + top-k + gates + per-tile histogram (noisy gating:
-  //    the noisy logits first, then the same steps on them as the input)
+  //    on z + softplus(x W_noise^T) * eps)
   MOE_TRY(sg.enter(MOE_STAGE_ROUTE));
   RouterArgs r{};
-  if (eps != nullptr) {
-    MOE_TRY(noisy_logits(c, w, x, eps, logits, ws, L, stream));
-    r.logits_in = logits;
-  } else {
+  if (noise == nullptr) {
     r.x = x;
     r.w = w->w_router;
     r.b_router = w->b_router;
     r.logit_bias = w->logit_bias;
-    r.logits_out = tp.logits;  // the statistics come from the router's own partial sums
   }
+  r.logits_out = tp.logits;  // the statistics come from the router's own partial sums
   r.topk_idx = idx;
   r.topk_gate = gate;
   r.tile_counts = at<int32_t>(ws, L, B_TILE_COUNTS);
@@ -709,7 +778,9 @@ moe_status_t forward_impl(const moe_cfg_t *cfg, const moe_weights_t *w, const vo
   r.k = c.top_k;
   r.gate_mode = c.gate_mode;
   r.err = err;
-  if (sh == nullptr) {
+  if (noise != nullptr) {
+    MOE_TRY(route_noisy(c, w, x, *noise, r, logits, ws, L, stream));
+  } else if (sh == nullptr) {
     MOE_CUDA(launch_router(r, c.dtype, stream));
   } else {  // routed by the caller: only the per-tile histogram
     MOE_CUDA(launch_tile_counts(idx, c.n_tokens, c.top_k, c.n_experts, r.tile_counts, err,
@@ -823,25 +894,28 @@ MOE_API moe_status_t moe_forward_noisy(const moe_cfg_t *cfg, const moe_weights_t
                                        float *aux_out, const moe_taps_t *taps, void *ws,
                                        size_t ws_bytes, moe_stream_t stream) {
   if (eps == nullptr) return MOE_ERR_INVALID_ARG;
-  return forward_impl(cfg, w, x, eps, y, aux_out, taps, ws, ws_bytes, stream);
+  const NoiseSpec ns{eps, 0, 0};
+  return forward_impl(cfg, w, x, &ns, y, aux_out, taps, ws, ws_bytes, stream);
+}
+
+MOE_API moe_status_t moe_forward_noisy_seeded(const moe_cfg_t *cfg, const moe_weights_t *w,
+                                              const void *x, uint64_t seed, uint64_t offset,
+                                              void *y, float *aux_out, const moe_taps_t *taps,
+                                              void *ws, size_t ws_bytes, moe_stream_t stream) {
+  const NoiseSpec ns{nullptr, seed, offset};
+  return forward_impl(cfg, w, x, &ns, y, aux_out, taps, ws, ws_bytes, stream);
 }
 
 MOE_API moe_status_t moe_forward_staged(const moe_cfg_t *cfg, const moe_weights_t *w,
-                                        const void *x, void *y, float *aux_out,
-                                        const moe_taps_t *taps, const moe_stage_events_t *events,
-                                        void *ws, size_t ws_bytes, moe_stream_t stream) {
-  return forward_impl(cfg, w, x, nullptr, y, aux_out, taps, ws, ws_bytes, stream, nullptr,
-                      events);
-}
-
-MOE_API moe_status_t moe_forward_noisy_staged(const moe_cfg_t *cfg, const moe_weights_t *w,
-                                              const void *x, const float *eps, void *y,
-                                              float *aux_out, const moe_taps_t *taps,
-                                              const moe_stage_events_t *events, void *ws,
-                                              size_t ws_bytes, moe_stream_t stream) {
-  if (eps == nullptr) return MOE_ERR_INVALID_ARG;
-  return forward_impl(cfg, w, x, eps, y, aux_out, taps, ws, ws_bytes, stream, nullptr,
-                      events);
+                                        const void *x, const moe_noise_t *noise, void *y,
+                                        float *aux_out, const moe_taps_t *taps,
+                                        const moe_stage_events_t *events, void *ws,
+                                        size_t ws_bytes, moe_stream_t stream) {
+  if (noise == nullptr)
+    return forward_impl(cfg, w, x, nullptr, y, aux_out, taps, ws, ws_bytes, stream, nullptr,
+                        events);
+  const NoiseSpec ns{noise->eps, noise->seed, noise->offset};
+  return forward_impl(cfg, w, x, &ns, y, aux_out, taps, ws, ws_bytes, stream, nullptr, events);
 }
 
 // ----------------------------------------------------- token-sharded batches

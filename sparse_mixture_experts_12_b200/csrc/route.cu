@@ -571,6 +571,9 @@ __global__ void __launch_bounds__(256) k_tile_counts(const int32_t *__restrict__
 cudaError_t launch_router(const RouterArgs &a, int dtype, cudaStream_t st) {
   if (a.T == 0) return cudaSuccess;
   const int E = a.E;
+  // the fused noisy gate exists on the tensor-core router only
+  if (a.w_noise != nullptr && !(dtype == MOE_DTYPE_BF16 && router_tc_supported(a)))
+    return cudaErrorInvalidValue;
   // bf16: the tensor-core router (x W_r^T is a contraction; on the CUDA cores it is
   // bound by the FMA rate rather than by reading x)
   if (dtype == MOE_DTYPE_BF16 && router_tc_supported(a)) return launch_router_tc(a, st);

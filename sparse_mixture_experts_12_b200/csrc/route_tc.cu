@@ -26,6 +26,11 @@
 // lower expert index), the exp sum and the probability column sums are register
 // work plus fixed shuffle trees. The permute tiles (router_bm(E) tokens) lie
 // inside one CTA's token share, so their histograms and sums need no exchange.
+//
+// Noisy top-k gating (youngju.dev (ja) "TopKGating", training mode): W_r and W_noise
+// are stacked on the MMA's N side (EX columns each), so one pass over x gives both
+// x W_r^T and x W_noise^T; the epilogue forms z + softplus(x W_noise^T) * eps, with
+// softplus the identity above 20 (as F.softplus), before the selection.
 #include <mutex>
 
 #include "tc_ptx.cuh"
@@ -60,9 +65,12 @@ struct RtCtl {
   float lse[kRtM];
 };
 
-template <int EPAD, int S> struct RtCfg {
+template <int EPAD, int S, bool NOISY> struct RtCfg {
   static_assert(EPAD == 16 || EPAD == 32 || EPAD == 64 || EPAD == 128 || EPAD == 256, "EPAD");
   static_assert(S == 1 || S == 2 || S == 4, "S");
+  // expert columns the selection runs over: all of N, or its first half when the
+  // noise projection fills the second
+  static constexpr int kEx = NOISY ? EPAD / 2 : EPAD;
   static constexpr int kBBytes = EPAD * kBlockK * 2;
   static constexpr int kStageBytes = kRtABytes + kBBytes;  // a multiple of 1024
   static constexpr int kStages = kRtRingBudget / kStageBytes < kRtMaxStages
@@ -74,7 +82,7 @@ template <int EPAD, int S> struct RtCfg {
   static constexpr size_t kSmem = (size_t)kBody + sizeof(RtCtl) + 1024;
   static constexpr int kTok = kRtM / S;             // tokens of one CTA's epilogue
   static constexpr int kG = kRtEpiThreads / kTok;   // threads per token (2S)
-  static constexpr int kEpl = EPAD / kG;            // logits per thread
+  static constexpr int kEpl = kEx / kG;             // logits per thread
   static constexpr uint32_t kTmemCols = EPAD < 32 ? 32 : EPAD;
   static_assert(kEpl >= 1 && kEpl <= 64, "logits per thread");
 };
@@ -107,9 +115,9 @@ __device__ __forceinline__ void rt_sync_all() {
 // TMEM -> this CTA's partial tile [128][EPAD] (row stride kLdp). Warp w reads TMEM
 // lanes [32 (w % 4), +32) (its lane quarter); the two warps of a quarter take
 // alternate 32-column chunks.
-template <int EPAD, int S>
+template <int EPAD, int S, bool NOISY>
 __device__ __forceinline__ void stage_partial(float *part, uint32_t tmem, int warp, int lane) {
-  using C = RtCfg<EPAD, S>;
+  using C = RtCfg<EPAD, S, NOISY>;
   const int q = warp & 3;
   const int h = (warp - 2) >> 2;
   const int r = q * 32 + lane;
@@ -159,10 +167,11 @@ __device__ __forceinline__ void group_argmax(float &v, int &i) {
 }
 
 // The epilogue of CTA `rank`: tokens [rank * kTok, +kTok) of the cluster's 128.
-template <int EPAD, int S>
+template <int EPAD, int S, bool NOISY>
 __device__ __forceinline__ void epilogue_tokens(const RouterArgs &a, RtCtl *ctl, float *part,
                                                 int tile, int rank, int NT, int BM, int et) {
-  using C = RtCfg<EPAD, S>;
+  using C = RtCfg<EPAD, S, NOISY>;
+  constexpr int EX = C::kEx;
   constexpr int G = C::kG, EPL = C::kEpl, TOK = C::kTok;
   const int E = a.E, T = a.T, k = a.k;
   const int m = et / G, g = et % G;        // token of this CTA's share, lane in its group
@@ -172,32 +181,42 @@ __device__ __forceinline__ void epilogue_tokens(const RouterArgs &a, RtCtl *ctl,
   const int lane = et & 31, ew = et >> 5;
 
   // ---- logits: the S partials in rank order (+ biases in the CUDA-core router's order)
+  constexpr int NC = NOISY ? 2 : 1;  // columns e (and EX + e, the noise projection)
   float z[EPL];
   {
-    float acc[EPL];
-#pragma unroll
-    for (int j = 0; j < EPL; ++j) acc[j] = 0.f;
+    float acc[NC][EPL];
     const uint32_t base = smem_u32(part + row * C::kLdp);
 #pragma unroll
     for (int r = 0; r < S; ++r) {
-      if constexpr (S == 1) {
 #pragma unroll
-        for (int j = 0; j < EPL; ++j) acc[j] = part[row * C::kLdp + j * G + g];
-      } else {
-        const uint32_t rb = mapa_rank(base, (uint32_t)r);
-        float v[EPL];
+      for (int h = 0; h < NC; ++h) {
+        if constexpr (S == 1) {
 #pragma unroll
-        for (int j = 0; j < EPL; ++j) v[j] = ld_cluster_f32(rb + 4u * (uint32_t)(j * G + g));
+          for (int j = 0; j < EPL; ++j) acc[h][j] = part[row * C::kLdp + h * EX + j * G + g];
+        } else {
+          const uint32_t rb = mapa_rank(base, (uint32_t)r);
+          float v[EPL];
 #pragma unroll
-        for (int j = 0; j < EPL; ++j) acc[j] = (r == 0) ? v[j] : acc[j] + v[j];
+          for (int j = 0; j < EPL; ++j)
+            v[j] = ld_cluster_f32(rb + 4u * (uint32_t)(h * EX + j * G + g));
+#pragma unroll
+          for (int j = 0; j < EPL; ++j) acc[h][j] = (r == 0) ? v[j] : acc[h][j] + v[j];
+        }
       }
     }
 #pragma unroll
     for (int j = 0; j < EPL; ++j) {
       const int e = j * G + g;
-      float v = acc[j];
+      float v = acc[0][j];
       if (a.b_router) v += ctl->br[e];
       if (a.logit_bias) v += ctl->lb[e];
+      if constexpr (NOISY) {
+        if (valid && e < E) {
+          const float zn = acc[NC - 1][j];
+          const float sp = zn > 20.f ? zn : log1pf(expf(zn));
+          v = v + sp * a.eps[(size_t)t * E + e];
+        }
+      }
       if (a.logits_out != nullptr && valid && e < E) a.logits_out[(size_t)t * E + e] = v;
       z[j] = (e >= E || v != v) ? -INFINITY : v;  // padding and NaN never win a slot
     }
@@ -291,6 +310,7 @@ __device__ __forceinline__ void epilogue_tokens(const RouterArgs &a, RtCtl *ctl,
     }
   }
   rt_epi_sync();
+  (void)EX;
 
   // ---- per permute tile (BM tokens, whole tiles inside this CTA's share)
   const int subs = TOK / BM;
@@ -321,11 +341,11 @@ __device__ __forceinline__ void epilogue_tokens(const RouterArgs &a, RtCtl *ctl,
   }
 }
 
-template <int EPAD, int S>
+template <int EPAD, int S, bool NOISY>
 __global__ void __launch_bounds__(kRtThreads, 1)
 k_router_tc(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
-            RouterArgs a, int NT, int BM) {
-  using C = RtCfg<EPAD, S>;
+            const __grid_constant__ CUtensorMap tmN, RouterArgs a, int NT, int BM) {
+  using C = RtCfg<EPAD, S, NOISY>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -368,6 +388,7 @@ k_router_tc(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
     // ------------------------------------------------------------ TMA producer
     prefetch_map(&tmX);
     prefetch_map(&tmW);
+    if (NOISY) prefetch_map(&tmN);
     int stage = 0;
     uint32_t phase = 0, issued = 0, last_phase = 0;
     bool ok = true;
@@ -377,6 +398,9 @@ k_router_tc(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
       mbar_expect_tx(&ctl->full[stage], C::kStageBytes);
       tma_load_2d(&tmX, &ctl->full[stage], sa, kb * kBlockK, t0);
       tma_load_2d(&tmW, &ctl->full[stage], sa + kRtABytes, kb * kBlockK, 0);
+      if (NOISY)  // the noise projection's rows follow W_r's (whole 1024-byte atoms)
+        tma_load_2d(&tmN, &ctl->full[stage], sa + kRtABytes + C::kEx * kBlockK * 2,
+                    kb * kBlockK, 0);
       issued |= 1u << stage;
       last_phase = (last_phase & ~(1u << stage)) | (phase << stage);
       if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
@@ -418,7 +442,7 @@ k_router_tc(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
     rt_epi_sync();
     if (ctl->epi_ok) {
       tc_fence_after();
-      stage_partial<EPAD, S>(part, tmem, warp, lane);
+      stage_partial<EPAD, S, NOISY>(part, tmem, warp, lane);
     }
   }
   // the partial tiles of the whole cluster are complete
@@ -426,7 +450,7 @@ k_router_tc(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
   rt_sync_all<S>();
   tc_fence_after();
   if (warp >= 2 && ctl->epi_ok)
-    epilogue_tokens<EPAD, S>(a, ctl, part, tile, rank, NT, BM, tid - 64);
+    epilogue_tokens<EPAD, S, NOISY>(a, ctl, part, tile, rank, NT, BM, tid - 64);
   // no CTA leaves (its shared memory) while another may still read its partials
   rt_sync_all<S>();
   if (warp == 1) tmem_dealloc(tmem, C::kTmemCols);
@@ -434,9 +458,9 @@ k_router_tc(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
 
 std::mutex g_rt_mu;
 
-template <int EPAD, int S>
+template <int EPAD, int S, bool NOISY>
 cudaError_t launch_rt(const RouterArgs &a, cudaStream_t st) {
-  using C = RtCfg<EPAD, S>;
+  using C = RtCfg<EPAD, S, NOISY>;
   static bool attr_set[64] = {};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -444,15 +468,21 @@ cudaError_t launch_rt(const RouterArgs &a, cudaStream_t st) {
   {
     std::lock_guard<std::mutex> lock(g_rt_mu);
     if (!attr_set[dev & 63]) {
-      e = cudaFuncSetAttribute(k_router_tc<EPAD, S>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               (int)C::kSmem);
+      e = cudaFuncSetAttribute(k_router_tc<EPAD, S, NOISY>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::kSmem);
       if (e != cudaSuccess) return e;
       attr_set[dev & 63] = true;
     }
   }
-  CUtensorMap mx, mw;
+  CUtensorMap mx, mw, mn;
   if (!make_map(&mx, a.x, (uint64_t)a.T, (uint64_t)a.d, kRtM)) return cudaErrorInvalidValue;
-  if (!make_map(&mw, a.w, (uint64_t)a.E, (uint64_t)a.d, EPAD)) return cudaErrorInvalidValue;
+  if (!make_map(&mw, a.w, (uint64_t)a.E, (uint64_t)a.d, C::kEx)) return cudaErrorInvalidValue;
+  if (NOISY) {
+    if (!make_map(&mn, a.w_noise, (uint64_t)a.E, (uint64_t)a.d, C::kEx))
+      return cudaErrorInvalidValue;
+  } else {
+    mn = mw;
+  }
   const int BM = router_bm(a.E);
   const int NT = ceil_div(a.T, BM);
   cudaLaunchConfig_t cfg{};
@@ -467,46 +497,56 @@ cudaError_t launch_rt(const RouterArgs &a, cudaStream_t st) {
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, k_router_tc<EPAD, S>, mx, mw, a, NT, BM);
+  return cudaLaunchKernelEx(&cfg, k_router_tc<EPAD, S, NOISY>, mx, mw, mn, a, NT, BM);
 }
 
 // K splits: at most four, each CTA's token share (128 / S) a whole number of permute
 // tiles, at least two 64-column blocks of K per split, and only while the grid
 // stays under one CTA per SM.
-int router_splits(int T, int d, int E, int epad) {
+int router_splits(int T, int d, int E, int ex) {
   const int BM = router_bm(E);
   const int tiles = ceil_div(T, kRtM);
   const int nkb = d / kBlockK;
   const int sms = sm_count();
   int S = 1;
   while (S < 4 && kRtM / (2 * S) >= BM && 2 * S <= nkb && tiles * 2 * S <= sms) S *= 2;
-  if (epad == 256 && S == 1 && nkb >= 2) S = 2;  // at most 64 logits per epilogue thread
+  if (ex == 256 && S == 1 && nkb >= 2) S = 2;  // at most 64 logits per epilogue thread
   return S;
 }
 
-template <int EPAD>
+template <int EPAD, bool NOISY>
 cudaError_t launch_rt_e(const RouterArgs &a, cudaStream_t st) {
-  const int S = router_splits(a.T, a.d, a.E, EPAD);
-  if (S == 4) return launch_rt<EPAD, 4>(a, st);
-  if (S == 2) return launch_rt<EPAD, 2>(a, st);
-  if constexpr (EPAD == 256) return cudaErrorInvalidValue;  // needs a split (d >= 128)
-  else return launch_rt<EPAD, 1>(a, st);
+  constexpr int kEx = NOISY ? EPAD / 2 : EPAD;  // the expert columns of the selection
+  const int S = router_splits(a.T, a.d, a.E, kEx);
+  if (S == 4) return launch_rt<EPAD, 4, NOISY>(a, st);
+  if (S == 2) return launch_rt<EPAD, 2, NOISY>(a, st);
+  if constexpr (EPAD == 256 && !NOISY) return cudaErrorInvalidValue;  // needs a split
+  else return launch_rt<EPAD, 1, NOISY>(a, st);
 }
 
 }  // namespace
 
 bool router_tc_supported(const RouterArgs &a) {
-  return a.x != nullptr && a.E >= 1 && a.E <= kMaxExperts && a.d % kBlockK == 0 && a.T > 0 &&
-         !(a.E > 128 && a.d < 2 * kBlockK);
+  if (a.x == nullptr || a.E < 1 || a.E > kMaxExperts || a.d % kBlockK != 0 || a.T <= 0)
+    return false;
+  if (a.w_noise != nullptr) return a.E <= 128 && a.eps != nullptr;
+  return !(a.E > 128 && a.d < 2 * kBlockK);
 }
 
 cudaError_t launch_router_tc(const RouterArgs &a, cudaStream_t st) {
   if (!router_tc_supported(a)) return cudaErrorInvalidValue;
-  if (a.E <= 16) return launch_rt_e<16>(a, st);
-  if (a.E <= 32) return launch_rt_e<32>(a, st);
-  if (a.E <= 64) return launch_rt_e<64>(a, st);
-  if (a.E <= 128) return launch_rt_e<128>(a, st);
-  return launch_rt_e<256>(a, st);
+  if (a.w_noise != nullptr) {  // N = 2 x (E rounded up to 8 .. 128)
+    if (a.E <= 8) return launch_rt_e<16, true>(a, st);
+    if (a.E <= 16) return launch_rt_e<32, true>(a, st);
+    if (a.E <= 32) return launch_rt_e<64, true>(a, st);
+    if (a.E <= 64) return launch_rt_e<128, true>(a, st);
+    return launch_rt_e<256, true>(a, st);
+  }
+  if (a.E <= 16) return launch_rt_e<16, false>(a, st);
+  if (a.E <= 32) return launch_rt_e<32, false>(a, st);
+  if (a.E <= 64) return launch_rt_e<64, false>(a, st);
+  if (a.E <= 128) return launch_rt_e<128, false>(a, st);
+  return launch_rt_e<256, false>(a, st);
 }
 
 }  // namespace moe

@@ -18,6 +18,9 @@ TOL = {synth.DT_F32: 1e-5, synth.DT_BF16: 2e-2}
 # Tokens whose sorted top-(k+1) logits are closer than this are near-ties.
 MARGIN = 1e-4
 U32 = 2.0 ** -24
+# the device's fp32 Box-Muller draws against the oracle's fp64 ones (logf, sincospif
+# within 1 ulp each, sqrtf and the products correctly rounded): 8 ulp, relative
+EPS_REL = 8 * 2.0 ** -23
 
 
 class F64View:

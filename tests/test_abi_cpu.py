@@ -56,10 +56,12 @@ def test_struct_layout_matches_header(tmp_path):
         + "".join(f"  F(moe_weights_t, {n});\n" for n, _ in B.MoeWeights._fields_)
         + "".join(f"  F(moe_taps_t, {n});\n" for n, _ in B.MoeTaps._fields_)
         + "".join(f"  F(moe_shard_t, {n});\n" for n, _ in B.MoeShard._fields_)
+        + "".join(f"  F(moe_noise_t, {n});\n" for n, _ in B.MoeNoise._fields_)
         + '  printf("size moe_cfg_t %zu\\nsize moe_weights_t %zu\\nsize moe_taps_t %zu\\n",'
           " sizeof(moe_cfg_t), sizeof(moe_weights_t), sizeof(moe_taps_t));\n"
         + '  printf("size moe_shard_t %zu\\n", sizeof(moe_shard_t));\n'
         + '  printf("size moe_stage_events_t %zu\\n", sizeof(moe_stage_events_t));\n'
+        + '  printf("size moe_noise_t %zu\\n", sizeof(moe_noise_t));\n'
         + '  printf("stages count %d\\n", (int)MOE_STAGE_COUNT);\n  return 0;\n}\n')
     exe = tmp_path / "layout"
     subprocess.run(["gcc", "-std=c99", f"-I{os.path.dirname(HEADER)}", str(prog), "-o", str(exe)],
@@ -76,6 +78,9 @@ def test_struct_layout_matches_header(tmp_path):
             assert got[(st, n)] == getattr(cls, n).offset, (st, n)
         assert got[("size", st)] == ctypes.sizeof(cls)
     assert got[("size", "moe_stage_events_t")] == ctypes.sizeof(B.MoeStageEvents)
+    for n, _ in B.MoeNoise._fields_:
+        assert got[("moe_noise_t", n)] == getattr(B.MoeNoise, n).offset, n
+    assert got[("size", "moe_noise_t")] == ctypes.sizeof(B.MoeNoise)
     assert got[("stages", "count")] == len(B.STAGES)
 
 

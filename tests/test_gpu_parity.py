@@ -362,25 +362,39 @@ def test_aux_stats_matches_oracle(E, k):
 
 
 # ====================================================================== whole layer
-def _forward_and_compare(wl: synth.Workload, seed: int, n_sample=None, check_full_routing=True):
+NOISE_OFFSET = 7
+
+
+def _forward_and_compare(wl: synth.Workload, seed: int, n_sample=None, check_full_routing=True,
+                         noise_seed=None):
+    """noise_seed (noisy workloads): the library draws the noise for (noise_seed,
+    NOISE_OFFSET) and the oracle the same counter-based draws; otherwise the noise is
+    a seeded input both sides read."""
     inp = synth.generate(wl, seed=seed)
     layer = B.MoELayer(wl, inp, DEV)
     x = inp["x"].to(DEV)
     taps = layer.new_taps()
     aux = layer.new_aux()
-    eps = synth.noise_draws(wl.T, wl.n_experts, seed + 99) if wl.noisy else None
-    if eps is None:
+    eps = e64 = None
+    if wl.noisy and noise_seed is None:
+        eps = synth.noise_draws(wl.T, wl.n_experts, seed + 99)
+        e64 = eps.numpy().astype(np.float64)
+    elif wl.noisy:
+        e64 = O.noise_draws(wl.T, wl.n_experts, noise_seed, NOISE_OFFSET)[0]
+    if not wl.noisy:
         y = layer.forward(x, taps=taps, aux=aux)
-    else:
+    elif eps is not None:
         y = layer.forward_noisy(x, eps.to(DEV), taps=taps, aux=aux)
+    else:
+        y = layer.forward_noisy(x, seed=noise_seed, offset=NOISE_OFFSET, taps=taps, aux=aux)
     torch.cuda.synchronize()
     code, info = layer.last_device_error()
     assert code == 0, (code, info)
     P = H.oracle_params(inp)
     T, E, k = wl.T, wl.n_experts, wl.top_k
     ref_logits = None
-    if eps is not None:
-        ref_logits = O.noisy_router_logits(P["x"], P["w_router"], P["w_noise"], eps.numpy(),
+    if wl.noisy:
+        ref_logits = O.noisy_router_logits(P["x"], P["w_router"], P["w_noise"], e64,
                                            P["b_router"], P["logit_bias"])
     kw = H.oracle_kwargs(wl)
     tokens = tiles = None
@@ -407,23 +421,27 @@ def _forward_and_compare(wl: synth.Workload, seed: int, n_sample=None, check_ful
     if P["logit_bias"] is not None:
         extra += np.abs(P["logit_bias"])
     bound = H.logits_bound(P["x"], P["w_router"], extra)
-    if eps is not None:  # + |eps| (bound of x W_noise^T + softplus rounding) + final roundings
-        e64 = eps.numpy().astype(np.float64)
+    if wl.noisy:  # + |eps| (bound of x W_noise^T + softplus rounding) + final roundings
         zn = P["x"] @ P["w_noise"].T
         sp = O.softplus(zn)
         zpl = P["x"] @ P["w_router"].T
         bound = bound + np.abs(e64) * (H.logits_bound(P["x"], P["w_noise"]) + 8 * H.U32 * sp) \
             + 4 * H.U32 * (np.abs(zpl) + extra[None, :] + sp * np.abs(e64))
+        if eps is None:  # the device's fp32 draws differ from the fp64 ones by <= 8 ulp
+            bound = bound + sp * H.EPS_REL * np.abs(e64)
     zg = taps["logits"].cpu().numpy().astype(np.float64)
     assert np.all(np.abs(zg - r["logits"]) <= bound)
-    if eps is not None:  # the forward's selection, on its own noisy logits, is bit-exact
+    if wl.noisy:  # the forward's selection, on its own noisy logits, is bit-exact
         gi = torch.empty((T, k), dtype=torch.int32, device=DEV)
         gg = torch.empty((T, k), dtype=torch.float32, device=DEV)
         layer.route(None, taps["logits"], gi, gg)
         torch.cuda.synchronize()
         assert torch.equal(gi, taps["topk_idx"])
         li = torch.empty((T, E), dtype=torch.float32, device=DEV)
-        layer.route_noisy(x, eps.to(DEV), li, gi, gg)
+        if eps is not None:
+            layer.route_noisy(x, eps.to(DEV), li, gi, gg)
+        else:
+            layer.route_noisy_seeded(x, noise_seed, NOISE_OFFSET, li, gi, gg)
         torch.cuda.synchronize()
         assert torch.equal(li, taps["logits"]) and torch.equal(gi, taps["topk_idx"])
     # the forward's own routing: differences only on near-ties
@@ -503,15 +521,50 @@ def test_forward_small_matches_oracle(name):
     _forward_and_compare(synth.SMALL[name], seed=0)
 
 
-FULL = ["tiny", "mixtral_prefill", "deepseek", "switch", "decode32", "decode8", "decode1"]
+FULL = ["tiny", "mixtral_prefill", "deepseek", "switch", "decode32", "decode8", "decode1",
+        "mixtral_noisy"]
 
 
 @pytest.mark.parametrize("name", FULL)
 def test_forward_full_size_sampled(name):
     wl = synth.WORKLOADS[name]
     n = None if wl.T <= 64 else 48
-    _forward_and_compare(wl, seed=0, n_sample=n)
+    # the noisy layer at full size draws its noise inside the library, as in the benchmark
+    _forward_and_compare(wl, seed=0, n_sample=n, noise_seed=2024 if wl.noisy else None)
     torch.cuda.empty_cache()
+
+
+NOISY_SMALL = sorted(n for n, w in synth.SMALL.items() if w.noisy)
+
+
+@pytest.mark.parametrize("name", NOISY_SMALL)
+def test_forward_noisy_seeded_matches_oracle(name):
+    """The noise drawn inside the library for (seed, offset), the oracle drawing the
+    same counter-based noise: the whole layer as with the noise as an input."""
+    _forward_and_compare(synth.SMALL[name], seed=0, noise_seed=(1 << 40) + 17)
+
+
+NOISE_CASES = [(1, 1, 0, 0), (333, 6, 42, 3), (4096, 64, (1 << 40) + 3, (1 << 33) + 5),
+               (5000, 128, 7, 123456789), (17, 250, 2 ** 64 - 1, 2 ** 64 - 1)]
+
+
+@pytest.mark.parametrize("T,E,seed,offset", NOISE_CASES)
+def test_noise_draws_match_oracle(T, E, seed, offset):
+    """moe_noise_draws: the Philox words bit-exact, the normal draws within 8 ulp
+    (relative) of the oracle's fp64 Box-Muller on the same uniforms."""
+    Q = (E + 3) // 4
+    eps = torch.full((T, E), float("nan"), dtype=torch.float32, device=DEV)
+    raw = torch.zeros((T, Q, 4), dtype=torch.int32, device=DEV)
+    B.noise_draws(T, E, seed, offset, eps, raw)
+    torch.cuda.synchronize()
+    ref, ref_raw = O.noise_draws(T, E, seed, offset)
+    got_raw = raw.cpu().numpy().view(np.uint32)
+    assert np.array_equal(got_raw, ref_raw)
+    got = eps.cpu().numpy().astype(np.float64)
+    err = np.abs(got - ref)
+    assert np.all(err <= H.EPS_REL * np.abs(ref) + 1e-30), float((err / np.abs(ref)).max())
+    H.report("noise_draws", T=T, E=E, max_rel_err=float((err / np.abs(ref)).max()),
+             max_ulp=float((err / (np.abs(ref) * 2.0 ** -23)).max()))
 
 
 def test_forward_is_deterministic():
