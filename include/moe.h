@@ -407,6 +407,20 @@ moe_status_t moe_forward_shard(const moe_cfg_t *cfg, const moe_shard_t *shard,
 moe_status_t moe_aux_finalize(const moe_cfg_t *cfg, long long n_tokens_total,
                               const double *aux_part, float *out, moe_stream_t stream);
 
+/* ---------------------------------------------------------------------------
+ * Test hooks for failure detection (no counterpart on the pages). Every pipeline
+ * wait inside the tensor-core kernels is bounded; a wait that runs out records
+ * MOE_DEVERR_WAIT_TIMEOUT (info = the wait's site), lets the copies and MMAs the CTA
+ * already issued finish, frees its tensor memory and returns, so the context stays
+ * usable. These two calls make that happen on purpose, without a fault:
+ * moe_test_set_wait_limit sets the bound (ns; 0 restores 2 s) of the single-CTA
+ * expert GEMM's pipeline waits in launches that follow; moe_test_withhold_load makes
+ * the next n_calls launches of that GEMM's up projection withhold each CTA's first
+ * operand load, so its MMA issuer waits for data that never comes. Both are
+ * process-wide host settings read at launch. */
+moe_status_t moe_test_set_wait_limit(uint64_t ns);
+moe_status_t moe_test_withhold_load(int32_t n_calls);
+
 /* Synchronise `stream`, read and clear the sticky device error word.
  * Returns MOE_ERR_DEVICE when *code != 0, MOE_ERR_CUDA when the sync failed. */
 moe_status_t moe_last_device_error(void *ws, int32_t *code, int32_t *info, moe_stream_t stream);

@@ -31,7 +31,7 @@ EXPORTED = ("moe_workspace_size", "moe_workspace_init", "moe_route", "moe_route_
             "moe_expert_ffn", "moe_combine", "moe_aux_stats", "moe_forward",
             "moe_route_shard", "moe_permute_shard", "moe_forward_shard", "moe_aux_finalize",
             "moe_forward_staged", "moe_noise_draws", "moe_route_noisy_seeded",
-            "moe_forward_noisy_seeded",
+            "moe_forward_noisy_seeded", "moe_test_set_wait_limit", "moe_test_withhold_load",
             "moe_last_device_error", "moe_status_string")
 
 # stages of one layer call (MOE_STAGE_*), in launch order
@@ -117,6 +117,8 @@ def load() -> ctypes.CDLL:
                                    P],
         "moe_forward_noisy_seeded": [cfgp, wp, P, ctypes.c_uint64, ctypes.c_uint64, P, P,
                                      ctypes.POINTER(MoeTaps), P, S, P],
+        "moe_test_set_wait_limit": [ctypes.c_uint64],
+        "moe_test_withhold_load": [ctypes.c_int32],
         "moe_last_device_error": [P, ctypes.POINTER(ctypes.c_int32),
                                   ctypes.POINTER(ctypes.c_int32), P],
     }

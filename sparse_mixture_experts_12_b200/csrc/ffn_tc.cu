@@ -65,6 +65,9 @@ struct TcArgs {
   int32_t *err;
   int tile_mode;  // TILES_ALL, or the pair / tail halves of a split launch
   int tma_store;  // pair kernel, bf16 output: full 32-row groups leave through TMA stores
+  uint64_t wait_limit_ns;  // single-CTA kernel: bound on its pipeline waits
+  int withhold_load;       // single-CTA kernel, test hook: the first operand load of each
+                           // CTA is never issued, so the waits on it run out
 };
 
 // The output path of one epilogue warp for one tile. With a map, a chunk whose 32
@@ -123,8 +126,9 @@ constexpr size_t kSmemBytes = (size_t)kStages * kStageBytes + sizeof(SmemCtl) + 
 
 
 __device__ __forceinline__ bool wait_bounded(uint64_t *bar, uint32_t parity, SmemCtl *ctl,
-                                             int32_t *err, int site, bool honour_abort = true) {
-  return wait_mbar(bar, parity, &ctl->abort_flag, 0u, err, site, honour_abort, kWaitLimitNs);
+                                             int32_t *err, int site, bool honour_abort = true,
+                                             uint64_t limit_ns = kWaitLimitNs) {
+  return wait_mbar(bar, parity, &ctl->abort_flag, 0u, err, site, honour_abort, limit_ns);
 }
 
 // ------------------------------------------------------------ shared epilogue
@@ -282,7 +286,7 @@ k_ffn_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtens
     if (EPI == EPI_SWIGLU) prefetch_map(&tmB3);
     int stage = 0;
     uint32_t phase = 0;
-    uint32_t issued = 0, last_phase = 0;  // per-stage bit sets, for the abort drain
+    uint32_t issued = 0, last_phase = 0;  // per-stage bit sets, for the end-of-role drain
     bool ok = true;
     for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
       int g, n, m;
@@ -291,27 +295,36 @@ k_ffn_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtens
       const int arow = offs[g] + m * kTileM;
       const int brow = g * a.b_rows + n * kBStep;
       for (int kb = 0; kb < nkb; ++kb) {
-        if (!wait_bounded(&ctl->empty[stage], phase ^ 1u, ctl, a.err, 1)) { ok = false; break; }
-        uint8_t *sa = smem + (size_t)stage * kStageBytes;
-        uint8_t *sb = sa + kABytes;
-        mbar_expect_tx(&ctl->full[stage], kStageBytes);
-        tma_load_2d(&tmA, &ctl->full[stage], sa, kb * kBlockK, arow);
-        if (EPI == EPI_SWIGLU) {
-          tma_load_2d(&tmB, &ctl->full[stage], sb, kb * kBlockK, brow);
-          tma_load_2d(&tmB3, &ctl->full[stage], sb + kBBytes / 2, kb * kBlockK, brow);
-        } else {
-          tma_load_2d(&tmB, &ctl->full[stage], sb, kb * kBlockK, brow);
+        if (!wait_bounded(&ctl->empty[stage], phase ^ 1u, ctl, a.err, 1, true,
+                          a.wait_limit_ns)) {
+          ok = false;
+          break;
         }
-        issued |= 1u << stage;
-        last_phase = (last_phase & ~(1u << stage)) | (phase << stage);
+        // test hook: the CTA's first stage is never loaded, so the MMA issuer's wait
+        // on it (and then the producer's wait for that stage to drain) runs out
+        const bool withhold = a.withhold_load && tile == (int)blockIdx.x && kb == 0;
+        if (!withhold) {
+          uint8_t *sa = smem + (size_t)stage * kStageBytes;
+          uint8_t *sb = sa + kABytes;
+          mbar_expect_tx(&ctl->full[stage], kStageBytes);
+          tma_load_2d(&tmA, &ctl->full[stage], sa, kb * kBlockK, arow);
+          if (EPI == EPI_SWIGLU) {
+            tma_load_2d(&tmB, &ctl->full[stage], sb, kb * kBlockK, brow);
+            tma_load_2d(&tmB3, &ctl->full[stage], sb + kBBytes / 2, kb * kBlockK, brow);
+          } else {
+            tma_load_2d(&tmB, &ctl->full[stage], sb, kb * kBlockK, brow);
+          }
+          issued |= 1u << stage;
+          last_phase = (last_phase & ~(1u << stage)) | (phase << stage);
+        }
         if (++stage == kStages) { stage = 0; phase ^= 1u; }
       }
     }
-    if (!ok) {  // let the copies already in flight land before the CTA exits
-      for (int s = 0; s < kStages; ++s)
-        if (issued & (1u << s))
-          wait_bounded(&ctl->full[s], (last_phase >> s) & 1u, ctl, nullptr, 0, false);
-    }
+    // every copy this CTA issued has landed before it can exit, whichever role gave
+    // up (a no-op wait on a normal run: the MMAs consumed them all)
+    for (int s = 0; s < kStages; ++s)
+      if (issued & (1u << s))
+        wait_bounded(&ctl->full[s], (last_phase >> s) & 1u, ctl, nullptr, 0, false);
   } else if (warp == 1 && lane == 0) {
     // --------------------------------------------------------------- MMA issuer
     constexpr uint32_t idesc = make_idesc(kTileM, kMmaN);
@@ -319,11 +332,18 @@ k_ffn_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtens
     uint32_t phase = 0, acc_phase = 0;
     bool ok = true, any = false;
     for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
-      if (!wait_bounded(&ctl->tempty[acc], acc_phase ^ 1u, ctl, a.err, 2)) { ok = false; break; }
+      if (!wait_bounded(&ctl->tempty[acc], acc_phase ^ 1u, ctl, a.err, 2, true,
+                        a.wait_limit_ns)) {
+        ok = false;
+        break;
+      }
       tc_fence_after();
       const uint32_t d_tmem = tmem + (uint32_t)(acc * kMmaN);
       for (int kb = 0; kb < nkb; ++kb) {
-        if (!wait_bounded(&ctl->full[stage], phase, ctl, a.err, 3)) { ok = false; break; }
+        if (!wait_bounded(&ctl->full[stage], phase, ctl, a.err, 3, true, a.wait_limit_ns)) {
+          ok = false;
+          break;
+        }
         tc_fence_after();
         const uint32_t sa = smem_u32(smem + (size_t)stage * kStageBytes);
         const uint64_t da = sw128_desc(sa);
@@ -353,7 +373,7 @@ k_ffn_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtens
       int g, n, m;
       decode_tile(tile, mpre, G, a.n_tiles, g, n, m);
       if (a.tile_mode == TILES_TAIL_ONLY) m = ceil_div(offs[g + 1] - offs[g], kTileM) - 1;
-      bool ok = wait_bounded(&ctl->tfull[acc], acc_phase, ctl, a.err, 4);
+      bool ok = wait_bounded(&ctl->tfull[acc], acc_phase, ctl, a.err, 4, true, a.wait_limit_ns);
       __syncwarp();
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
@@ -867,6 +887,8 @@ cudaError_t launch_ffn_tc(const GroupedFfnArgs &a, cudaStream_t st) {
   t.bias = a.b1;
   t.act = a.act;
   t.err = a.err;
+  t.wait_limit_ns = a.wait_limit_ns ? a.wait_limit_ns : kWaitLimitNs;
+  t.withhold_load = a.withhold_load;  // the up projection only
   // pair tiles write bf16 outputs through TMA stores of 32 x 32 boxes
   CUtensorMap mo;
   if (!make_store_map(&mo, a.h, (uint64_t)a.a_rows, (uint64_t)a.F)) return cudaErrorInvalidValue;
@@ -894,6 +916,7 @@ cudaError_t launch_ffn_tc(const GroupedFfnArgs &a, cudaStream_t st) {
   t.out_f32 = a.out_f32;
   t.bias = a.b2;
   t.act = -1;
+  t.withhold_load = 0;
   t.tma_store = a.out_f32 ? 0 : 1;
   if (!a.out_f32 && !make_store_map(&mo, a.out, (uint64_t)a.a_rows, (uint64_t)a.d))
     return cudaErrorInvalidValue;

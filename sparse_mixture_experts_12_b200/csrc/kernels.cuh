@@ -81,6 +81,9 @@ struct GroupedFfnArgs {
   int max_group_rows;     // host bound on the rows of any one group
   float *part;            // fp32 split-K partials of the small-batch path, or nullptr
   int32_t *err;
+  uint64_t wait_limit_ns; // bound on the pipeline waits of the single-CTA GEMM (0: default)
+  int withhold_load;      // test hook: the single-CTA up-projection GEMM withholds one
+                          // operand load per CTA (its bounded waits run out)
 };
 
 // Expert-Choice routing (see expert_choice.cu)

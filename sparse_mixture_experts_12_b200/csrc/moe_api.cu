@@ -3,6 +3,7 @@
 #include <math.h>
 #include <string.h>
 
+#include <atomic>
 #include <climits>
 
 #include <nvtx3/nvToolsExt.h>
@@ -257,8 +258,21 @@ int m_tiles_ub(long long rows, int groups) {
   return (int)ub;
 }
 
-cudaError_t run_ffn(const moe_cfg_t &c, const GroupedFfnArgs &a, cudaStream_t st) {
+// Process-wide test settings of the single-CTA tensor-core GEMM (see
+// moe_test_set_wait_limit and moe_test_withhold_load).
+std::atomic<uint64_t> g_wait_limit_ns{0};
+std::atomic<int> g_withhold_loads{0};
+
+cudaError_t run_ffn(const moe_cfg_t &c, GroupedFfnArgs a, cudaStream_t st) {
   if (c.dtype == MOE_DTYPE_F32) return launch_ffn_simt(a, st);
+  a.wait_limit_ns = g_wait_limit_ns.load();
+  // the test hook is taken by the next call that reaches the single-CTA kernel path
+  if (a.max_group_rows > kDecodeMaxRows && g_withhold_loads.load() > 0) {
+    int n = g_withhold_loads.load();
+    while (n > 0 && !g_withhold_loads.compare_exchange_weak(n, n - 1)) {
+    }
+    a.withhold_load = n > 0 ? 1 : 0;
+  }
   // few rows in any group: stream the weights with the tokens on the MMA's N side
   if (a.max_group_rows <= kDecodeMaxRows) return launch_ffn_tc_decode(a, st);
   return launch_ffn_tc(a, st);
@@ -1065,6 +1079,17 @@ MOE_API moe_status_t moe_last_device_error(void *ws, int32_t *code, int32_t *inf
   *code = h[0];
   if (info) *info = h[1];
   return h[0] != 0 ? MOE_ERR_DEVICE : MOE_OK;
+}
+
+MOE_API moe_status_t moe_test_set_wait_limit(uint64_t ns) {
+  g_wait_limit_ns.store(ns);
+  return MOE_OK;
+}
+
+MOE_API moe_status_t moe_test_withhold_load(int32_t n_calls) {
+  if (n_calls < 0) return MOE_ERR_INVALID_ARG;
+  g_withhold_loads.store(n_calls);
+  return MOE_OK;
 }
 
 MOE_API const char *moe_status_string(moe_status_t s) {

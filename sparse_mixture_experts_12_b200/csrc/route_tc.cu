@@ -405,10 +405,11 @@ k_router_tc(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
       last_phase = (last_phase & ~(1u << stage)) | (phase << stage);
       if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
     }
-    if (!ok) {  // let the copies already in flight land before the ring is reused
-      for (int s = 0; s < C::kStages; ++s)
-        if (issued & (1u << s)) rt_wait(&ctl->full[s], (last_phase >> s) & 1u, ctl, nullptr, 0, false);
-    }
+    // every copy issued has landed before the ring is reused, whichever role gave up
+    // (a no-op wait on a normal run: the MMAs consumed them all)
+    for (int s = 0; s < C::kStages; ++s)
+      if (issued & (1u << s)) rt_wait(&ctl->full[s], (last_phase >> s) & 1u, ctl, nullptr, 0, false);
+    (void)ok;
   } else if (warp == 1 && lane == 0) {
     // --------------------------------------------------------------- MMA issuer
     constexpr uint32_t idesc = make_idesc(kRtM, EPAD);
