@@ -400,6 +400,12 @@ class StepTimer:
         self.steps = steps
         self.ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(STAGES) + 1)]
                    for _ in range(steps)]
+        # torch creates an event at its first record: do that here, so that the
+        # library records (and torch later reads) real event handles
+        for evs in self.ev:
+            for e in evs:
+                e.record()
+        torch.cuda.synchronize()
         self.e0 = torch.cuda.Event(enable_timing=True)
         self.e1 = torch.cuda.Event(enable_timing=True)
 

@@ -157,6 +157,8 @@ def stage_events(events) -> MoeStageEvents:
         raise ValueError(f"{len(STAGES) + 1} events expected, got {len(events)}")
     ev = MoeStageEvents()
     for i, e in enumerate(events):
+        if e is not None and not e.cuda_event:
+            raise ValueError("a torch.cuda.Event has no CUDA event until its first record()")
         ev.ev[i] = None if e is None else e.cuda_event
     return ev
 
