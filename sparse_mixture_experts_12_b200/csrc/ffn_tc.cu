@@ -7,14 +7,15 @@
 // an expert are multiplied by its weights ("Token Routing": unselected experts
 // are not computed at all).
 //
-// Design (persistent, warp-specialised, 384 threads per CTA):
+// Design (persistent, warp-specialised):
 //   warp 0      TMA producer: A rows of the expert-contiguous activations and the
 //               expert's weight rows, 64-element K slices with 128-byte swizzle,
 //               into a shared-memory ring.
 //   warp 1      MMA issuer: tcgen05.mma (kind::f16, fp32 accumulate in TMEM).
 //   warp 2      TMEM allocator.
-//   warps 4..11 epilogue (two warps per TMEM lane quarter, half the columns
-//               each): tcgen05.ld, fused silu(g)*u / bias+ReLU / bias+GELU,
+//   warps 4..   epilogue (the warps of a TMEM lane quarter split the columns:
+//               two per quarter in the CTA-pair kernel, four in the single-CTA
+//               kernel): tcgen05.ld, fused silu(g)*u / bias+ReLU / bias+GELU,
 //               bf16 (or fp32) stores masked to the expert's rows.
 // Tile shapes, chosen per projection by its reduction length K:
 //   K >= 2048  a CTA pair (cluster of 2, tcgen05.mma.cta_group::2): 256 rows x 512
@@ -49,6 +50,12 @@ constexpr int kStageBytes = kABytes + kBBytes;
 constexpr int kTmemCols = 2 * kMmaN;
 constexpr int kThreads = 384;  // warps 0-3: producer, MMA, TMEM, spare; 4-11: epilogue
 constexpr int kEpiWarps = 8;
+// single-CTA kernel: sixteen epilogue warps (four per TMEM lane quarter, a quarter
+// of the columns each). Its tiles are short (K < 2048), so the fused activation of
+// one tile must keep up with the next tile's main loop; the erf-GELU epilogue of
+// eight warps did not (latency-bound, about a third of an instruction per cycle).
+constexpr int kEpiWarps1 = 16;
+constexpr int kThreads1 = 128 + 32 * kEpiWarps1;
 
 enum { EPI_SWIGLU = 0, EPI_ACT = 1, EPI_DOWN = 2 };
 
@@ -220,7 +227,7 @@ __device__ __forceinline__ void epilogue_tile(const TcArgs &a, uint32_t tbase, i
 
 // =========================================================== single-CTA kernel
 template <int EPI>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads1, 1)
 k_ffn_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
          const __grid_constant__ CUtensorMap tmB3, TcArgs a) {
   extern __shared__ uint8_t smem_raw[];
@@ -231,7 +238,7 @@ k_ffn_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtens
   const int G = a.G;
   int *mpre = ctl->tbl;
   int *offs = ctl->tbl + (G + 1);
-  for (int i = tid; i <= G; i += kThreads) {
+  for (int i = tid; i <= G; i += kThreads1) {
     if (a.tile_mode != TILES_TAIL_ONLY) mpre[i] = a.mprefix[i];
     offs[i] = a.offsets[i];
   }
@@ -261,7 +268,7 @@ k_ffn_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtens
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&ctl->tfull[s], 1);
-      mbar_init(&ctl->tempty[s], kEpiWarps * 32);
+      mbar_init(&ctl->tempty[s], kEpiWarps1 * 32);
     }
     mbar_init(&ctl->drain, 1);
     ctl->abort_flag = 0;
@@ -366,7 +373,7 @@ k_ffn_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtens
   } else if (warp >= 4) {
     // ----------------------------------------------------------------- epilogue
     const int ew = warp & 3;          // TMEM lanes [32*ew, 32*ew + 32) (warp % 4)
-    const int half = (warp - 4) >> 2;  // which half of the tile's columns
+    const int quarter = (warp - 4) >> 2;  // which quarter of the tile's columns
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
@@ -381,13 +388,14 @@ k_ffn_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtens
       const bool valid = grow < offs[g + 1] - offs[g];
       const size_t orow = (size_t)offs[g] + grow;
       const uint32_t tbase = tmem + ((uint32_t)(ew * 32) << 16) + (uint32_t)(acc * kMmaN);
-      // the two warps sharing a TMEM lane quarter take half the columns each
+      // the four warps sharing a TMEM lane quarter take a quarter of the columns each
       const EpiStore st{nullptr, nullptr, false, 0};
       if (EPI == EPI_SWIGLU)
-        epilogue_tile<EPI>(a, tbase, g, 0, n * (kMmaN / 2), 2 * half, 2 * half + 2, valid, orow,
+        epilogue_tile<EPI>(a, tbase, g, 0, n * (kMmaN / 2), quarter, quarter + 1, valid, orow,
                            st);
       else
-        epilogue_tile<EPI>(a, tbase, g, 0, n * kMmaN, 4 * half, 4 * half + 4, valid, orow, st);
+        epilogue_tile<EPI>(a, tbase, g, 0, n * kMmaN, 2 * quarter, 2 * quarter + 2, valid, orow,
+                           st);
       tc_fence_before();
       mbar_arrive(&ctl->tempty[acc]);
       if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
@@ -721,7 +729,7 @@ cudaError_t launch_single(const CUtensorMap &ma, const CUtensorMap &mb, const CU
   }
   const int grid = (int)std::max<long long>(1, std::min<long long>(tiles_ub, sm_count()));
   if (!overlap) {
-    k_ffn_tc<EPI><<<grid, kThreads, kSmemBytes, st>>>(ma, mb, mb3, t);
+    k_ffn_tc<EPI><<<grid, kThreads1, kSmemBytes, st>>>(ma, mb, mb3, t);
     return cudaGetLastError();
   }
   cudaLaunchConfig_t cfg = {};
@@ -729,7 +737,7 @@ cudaError_t launch_single(const CUtensorMap &ma, const CUtensorMap &mb, const CU
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3(kThreads);
+  cfg.blockDim = dim3(kThreads1);
   cfg.dynamicSmemBytes = kSmemBytes;
   cfg.stream = st;
   cfg.attrs = attr;

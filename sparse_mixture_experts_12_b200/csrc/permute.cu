@@ -45,6 +45,48 @@ __global__ void __launch_bounds__(kScanThreads) k_scan(ScanArgs a, ShardCaps sc)
   const int E = a.E, NT = a.NT;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   constexpr int nw = kScanThreads / 32;
+  if (NT <= 32 * kScanVPL) {
+    // one batch of tiles per expert: the next expert's counts and probability sums
+    // are requested before this expert's are scanned, so a warp's experts overlap
+    // their load latencies instead of paying one each
+    const bool want_p = a.aux_out != nullptr;
+    int v[kScanVPL], vn[kScanVPL];
+    float pv[kScanVPL], pn[kScanVPL];
+    auto fetch = [&](int e, int (&cv)[kScanVPL], float (&cp)[kScanVPL]) {
+#pragma unroll
+      for (int j = 0; j < kScanVPL; ++j) {
+        const int t = j * 32 + lane;
+        const bool in = e < E && t < NT;
+        cv[j] = in ? a.tile_counts[(size_t)e * NT + t] : 0;
+        cp[j] = (want_p && in) ? a.tile_p[(size_t)e * NT + t] : 0.f;
+      }
+    };
+    fetch(warp, v, pv);
+    for (int e = warp; e < E; e += nw) {
+      fetch(e + nw, vn, pn);
+      int32_t *tb = a.tile_base + (size_t)e * NT;
+      int run = 0;
+      float p = 0.f;
+#pragma unroll
+      for (int j = 0; j < kScanVPL; ++j) {
+        const int incl = warp_incl_scan(v[j]);
+        const int t = j * 32 + lane;
+        if (t < NT) tb[t] = run + incl - v[j];
+        run += __shfl_sync(0xffffffffu, incl, 31);
+        p += pv[j];
+      }
+      if (lane == 0) count_s[e] = run;
+      if (want_p) {
+        p = warp_sum(p);
+        if (lane == 0) P_s[e] = p / (float)a.T;
+      }
+#pragma unroll
+      for (int j = 0; j < kScanVPL; ++j) {
+        v[j] = vn[j];
+        pv[j] = pn[j];
+      }
+    }
+  } else {
   for (int e = warp; e < E; e += nw) {
     const int32_t *tc = a.tile_counts + (size_t)e * NT;
     int32_t *tb = a.tile_base + (size_t)e * NT;
@@ -75,6 +117,7 @@ __global__ void __launch_bounds__(kScanThreads) k_scan(ScanArgs a, ShardCaps sc)
       p = warp_sum(p);
       if (lane == 0) P_s[e] = p / (float)a.T;
     }
+  }
   }
   __syncthreads();
   if (warp == 0) {

@@ -61,8 +61,10 @@ struct RtCtl {
   float br[kMaxExperts];  // router bias (0 when absent)
   float lb[kMaxExperts];  // per-expert logit bias (0 when absent)
   int cnt[kRtMaxSubs][kMaxExperts];
-  float psum[kRtEpiWarps][kMaxExperts];  // per-warp column sums of the probabilities
-  float lse[kRtM];
+  float lse[kRtM];      // per token of the CTA's share: logsumexp of the logits
+  float inv_s[kRtM];    // 1 / sum exp(z - max)
+  float sel_v[kRtM][kMaxTopK];  // the top-k picks, value and expert
+  int sel_i[kRtM][kMaxTopK];
 };
 
 template <int EPAD, int S, bool NOISY> struct RtCfg {
@@ -78,13 +80,17 @@ template <int EPAD, int S, bool NOISY> struct RtCfg {
   static constexpr int kRing = kStages * kStageBytes;
   static constexpr int kLdp = EPAD + 1;             // partial tile row stride (floats)
   static constexpr int kPartBytes = kRtM * kLdp * 4;
-  static constexpr int kBody = kRing > kPartBytes ? kRing : kPartBytes;
+  // the share's logits (zb): in place of the partial tile when S = 1, after it when
+  // the cluster's other CTAs still read the partials
+  static constexpr int kZBytes = S == 1 ? 0 : (kRtM / S) * kLdp * 4;
+  static constexpr int kBody =
+      kRing > kPartBytes + kZBytes ? kRing : kPartBytes + kZBytes;
   static constexpr size_t kSmem = (size_t)kBody + sizeof(RtCtl) + 1024;
   static constexpr int kTok = kRtM / S;             // tokens of one CTA's epilogue
   static constexpr int kG = kRtEpiThreads / kTok;   // threads per token (2S)
-  static constexpr int kEpl = kEx / kG;             // logits per thread
   static constexpr uint32_t kTmemCols = EPAD < 32 ? 32 : EPAD;
-  static_assert(kEpl >= 1 && kEpl <= 64, "logits per thread");
+  static_assert(kEx >= kG, "every thread of a token's group owns an expert column");
+  static_assert(kSmem <= 227 * 1024, "shared memory");
 };
 
 __device__ __forceinline__ bool rt_wait(uint64_t *bar, uint32_t parity, RtCtl *ctl, int32_t *err,
@@ -166,164 +172,166 @@ __device__ __forceinline__ void group_argmax(float &v, int &i) {
   }
 }
 
-// The epilogue of CTA `rank`: tokens [rank * kTok, +kTok) of the cluster's 128.
+// The epilogue of CTA `rank`: tokens [rank * kTok, +kTok) of the cluster's 128. The
+// logits live in shared memory and every pass is a compact loop: the router's
+// epilogue runs once per call, after the expert GEMMs have flushed its code from
+// L2, so code size (instruction fetch) costs more here than a few shared loads.
+//  1. (token, expert) pairs over all threads, consecutive threads on consecutive
+//     experts: the S partials summed in rank order, the biases, the noise term, the
+//     logits written out (coalesced) and z (NaN and padding -> -inf) kept in zb.
+//  2. G threads per token (consecutive lanes): the max, k argmax rounds (each the
+//     best entry ranked below the previous pick), sum exp(z - max) with exp(z - max)
+//     kept in zb; fixed shuffle trees across the G threads; one thread per token
+//     forms the gates and writes the token's outputs.
+//  3. per permute tile: counts, and (statistics) the probability sums, each column
+//     summed over the tile's tokens in token order, and the sum of lse^2.
 template <int EPAD, int S, bool NOISY>
 __device__ __forceinline__ void epilogue_tokens(const RouterArgs &a, RtCtl *ctl, float *part,
-                                                int tile, int rank, int NT, int BM, int et) {
+                                                float *zb, int tile, int rank, int NT, int BM,
+                                                int et) {
   using C = RtCfg<EPAD, S, NOISY>;
-  constexpr int EX = C::kEx;
-  constexpr int G = C::kG, EPL = C::kEpl, TOK = C::kTok;
+  constexpr int EX = C::kEx, G = C::kG, TOK = C::kTok, LD = C::kLdp;
   const int E = a.E, T = a.T, k = a.k;
-  const int m = et / G, g = et % G;        // token of this CTA's share, lane in its group
-  const int row = rank * TOK + m;          // row of the cluster's 128-token tile
-  const int t = tile * kRtM + row;
-  const bool valid = t < T;
-  const int lane = et & 31, ew = et >> 5;
+  const int t_base = tile * kRtM + rank * TOK;  // token of this CTA's first row
 
-  // ---- logits: the S partials in rank order (+ biases in the CUDA-core router's order)
-  constexpr int NC = NOISY ? 2 : 1;  // columns e (and EX + e, the noise projection)
-  float z[EPL];
+  // ---- 1. logits
   {
-    float acc[NC][EPL];
-    const uint32_t base = smem_u32(part + row * C::kLdp);
+    const uint32_t part_s = smem_u32(part);
+#pragma unroll 2
+    for (int i = et; i < TOK * EX; i += kRtEpiThreads) {
+      const int m = i / EX, e = i - m * EX;
+      const int row = rank * TOK + m;
+      const int t = t_base + m;
+      float acc, accn = 0.f;
+      if constexpr (S == 1) {
+        acc = part[row * LD + e];
+        if constexpr (NOISY) accn = part[row * LD + EX + e];
+      } else {
+        const uint32_t off = 4u * (uint32_t)(row * LD + e);
+        float v[S], vn[S];
 #pragma unroll
-    for (int r = 0; r < S; ++r) {
+        for (int r = 0; r < S; ++r) {
+          const uint32_t rb = mapa_rank(part_s, (uint32_t)r) + off;
+          v[r] = ld_cluster_f32(rb);
+          if constexpr (NOISY) vn[r] = ld_cluster_f32(rb + 4u * EX);
+        }
+        acc = v[0];
 #pragma unroll
-      for (int h = 0; h < NC; ++h) {
-        if constexpr (S == 1) {
+        for (int r = 1; r < S; ++r) acc += v[r];
+        if constexpr (NOISY) {
+          accn = vn[0];
 #pragma unroll
-          for (int j = 0; j < EPL; ++j) acc[h][j] = part[row * C::kLdp + h * EX + j * G + g];
-        } else {
-          const uint32_t rb = mapa_rank(base, (uint32_t)r);
-          float v[EPL];
-#pragma unroll
-          for (int j = 0; j < EPL; ++j)
-            v[j] = ld_cluster_f32(rb + 4u * (uint32_t)(h * EX + j * G + g));
-#pragma unroll
-          for (int j = 0; j < EPL; ++j) acc[h][j] = (r == 0) ? v[j] : acc[h][j] + v[j];
+          for (int r = 1; r < S; ++r) accn += vn[r];
         }
       }
-    }
-#pragma unroll
-    for (int j = 0; j < EPL; ++j) {
-      const int e = j * G + g;
-      float v = acc[0][j];
+      const bool live = t < T && e < E;
+      float v = acc;
       if (a.b_router) v += ctl->br[e];
       if (a.logit_bias) v += ctl->lb[e];
       if constexpr (NOISY) {
-        if (valid && e < E) {
-          const float zn = acc[NC - 1][j];
-          const float sp = zn > 20.f ? zn : log1pf(expf(zn));
+        if (live) {
+          const float sp = accn > 20.f ? accn : log1pf(expf(accn));
           v = v + sp * a.eps[(size_t)t * E + e];
         }
       }
-      if (a.logits_out != nullptr && valid && e < E) a.logits_out[(size_t)t * E + e] = v;
-      z[j] = (e >= E || v != v) ? -INFINITY : v;  // padding and NaN never win a slot
+      if (a.logits_out != nullptr && live) a.logits_out[(size_t)t * E + e] = v;
+      zb[m * LD + e] = (e >= E || v != v) ? -INFINITY : v;  // padding, NaN never win a slot
     }
   }
+  rt_epi_sync();
 
-  float mx = -INFINITY;
-#pragma unroll
-  for (int j = 0; j < EPL; ++j) mx = fmaxf(mx, z[j]);
-  mx = group_max<G>(mx);
-
-  // ---- top-k: k rounds, each the best entry ranked below the previous pick
-  float tv[kMaxTopK];
-  int ti[kMaxTopK];
-  float pv = INFINITY;
-  int pi = -1;
-#pragma unroll
-  for (int s = 0; s < kMaxTopK; ++s) {
-    tv[s] = -INFINITY;
-    ti[s] = 0x7fffffff;
-    if (s < k) {
+  // ---- 2. per token: G consecutive lanes, expert columns e = g, g + G, ...
+  {
+    const int m = et / G, g = et % G;
+    const int t = t_base + m;
+    const bool valid = t < T;
+    float *zr = zb + m * LD;
+    float mx = -INFINITY;
+#pragma unroll 4
+    for (int e = g; e < EX; e += G) mx = fmaxf(mx, zr[e]);
+    mx = group_max<G>(mx);
+    float pv = INFINITY;
+    int pi = -1;
+#pragma unroll 1
+    for (int s = 0; s < k; ++s) {
       float bv = -INFINITY;
       int bi = 0x7fffffff;
-#pragma unroll
-      for (int j = 0; j < EPL; ++j) {
-        const int e = j * G + g;
-        const bool below = z[j] < pv || (z[j] == pv && e > pi);
-        if (below && rt_better(z[j], e, bv, bi)) { bv = z[j]; bi = e; }
+#pragma unroll 4
+      for (int e = g; e < EX; e += G) {
+        const float z = zr[e];
+        const bool below = z < pv || (z == pv && e > pi);
+        if (below && rt_better(z, e, bv, bi)) { bv = z; bi = e; }
       }
       group_argmax<G>(bv, bi);
-      tv[s] = pv = bv;
-      ti[s] = pi = bi;
-    }
-  }
-
-  // ---- softmax denominators
-  float ex[EPL];
-  float ssum = 0.f;
-#pragma unroll
-  for (int j = 0; j < EPL; ++j) {
-    ex[j] = expf(z[j] - mx);
-    ssum += ex[j];
-  }
-  ssum = group_sum<G>(ssum);
-  const float inv_s = 1.f / ssum;
-
-  if (g == 0) {
-    ctl->lse[m] = valid ? mx + logf(ssum) : 0.f;
-    float gv[kMaxTopK];
-    float gs = 0.f;
-    if (a.gate_mode == MOE_GATE_TOPK_SOFTMAX) {
-#pragma unroll
-      for (int s = 0; s < kMaxTopK; ++s)
-        if (s < k) { gv[s] = expf(tv[s] - tv[0]); gs += gv[s]; }
-      const float inv = 1.f / gs;
-#pragma unroll
-      for (int s = 0; s < kMaxTopK; ++s) if (s < k) gv[s] *= inv;
-    } else {
-#pragma unroll
-      for (int s = 0; s < kMaxTopK; ++s)
-        if (s < k) { gv[s] = expf(tv[s] - mx) * inv_s; gs += gv[s]; }
-      if (a.gate_mode == MOE_GATE_SOFTMAX_TOPK_RENORM) {
-#pragma unroll
-        for (int s = 0; s < kMaxTopK; ++s) if (s < k) gv[s] = gv[s] / gs;
+      pv = bv;
+      pi = bi;
+      if (g == 0) {
+        ctl->sel_v[m][s] = bv;
+        ctl->sel_i[m][s] = bi;
       }
     }
-    if (valid) {
+    float ssum = 0.f;
+#pragma unroll 4
+    for (int e = g; e < EX; e += G) {
+      const float ex = expf(zr[e] - mx);
+      ssum += ex;
+      zr[e] = ex;  // kept for the probability sums
+    }
+    ssum = group_sum<G>(ssum);
+    const float inv_s = 1.f / ssum;
+    __syncwarp();  // the group's sel_v / sel_i are written
+    if (g == 0) {
+      ctl->lse[m] = valid ? mx + logf(ssum) : 0.f;
+      ctl->inv_s[m] = valid ? inv_s : 0.f;
+      const float *tv = ctl->sel_v[m];
+      const int *ti = ctl->sel_i[m];
+      float gv[kMaxTopK];
+      float gs = 0.f;
+      if (a.gate_mode == MOE_GATE_TOPK_SOFTMAX) {
 #pragma unroll
-      for (int s = 0; s < kMaxTopK; ++s) {
-        if (s < k) {
-          a.topk_idx[(size_t)t * k + s] = ti[s];
-          a.topk_gate[(size_t)t * k + s] = gv[s];
-          // integer counts: the result does not depend on the order of the adds
-          if (ti[s] < E) atomicAdd(&ctl->cnt[m / BM][ti[s]], 1);
+        for (int s = 0; s < kMaxTopK; ++s)
+          if (s < k) { gv[s] = expf(tv[s] - tv[0]); gs += gv[s]; }
+        const float inv = 1.f / gs;
+#pragma unroll
+        for (int s = 0; s < kMaxTopK; ++s) if (s < k) gv[s] *= inv;
+      } else {
+#pragma unroll
+        for (int s = 0; s < kMaxTopK; ++s)
+          if (s < k) { gv[s] = expf(tv[s] - mx) * inv_s; gs += gv[s]; }
+        if (a.gate_mode == MOE_GATE_SOFTMAX_TOPK_RENORM) {
+#pragma unroll
+          for (int s = 0; s < kMaxTopK; ++s) if (s < k) gv[s] = gv[s] / gs;
+        }
+      }
+      if (valid) {
+#pragma unroll
+        for (int s = 0; s < kMaxTopK; ++s) {
+          if (s < k) {
+            a.topk_idx[(size_t)t * k + s] = ti[s];
+            a.topk_gate[(size_t)t * k + s] = gv[s];
+            // integer counts: the result does not depend on the order of the adds
+            if (ti[s] < E) atomicAdd(&ctl->cnt[m / BM][ti[s]], 1);
+          }
         }
       }
     }
   }
-
-  // ---- probability column sums of this warp's tokens (lanes with the same g)
-  if (a.tile_p != nullptr) {
-    float p[EPL];
-#pragma unroll
-    for (int j = 0; j < EPL; ++j) p[j] = valid ? ex[j] * inv_s : 0.f;
-#pragma unroll
-    for (int o = G; o < 32; o <<= 1)
-#pragma unroll
-      for (int j = 0; j < EPL; ++j) p[j] += __shfl_xor_sync(0xffffffffu, p[j], o);
-    if (lane < G) {
-#pragma unroll
-      for (int j = 0; j < EPL; ++j) ctl->psum[ew][j * G + g] = p[j];
-    }
-  }
   rt_epi_sync();
-  (void)EX;
 
-  // ---- per permute tile (BM tokens, whole tiles inside this CTA's share)
+  // ---- 3. per permute tile (BM tokens, whole tiles inside this CTA's share)
   const int subs = TOK / BM;
-  const int wpt = BM * G / 32;  // warps per permute tile
-  const int tile0 = (tile * kRtM + rank * TOK) / BM;
+  const int tile0 = t_base / BM;
   for (int i = et; i < subs * E; i += kRtEpiThreads) {
     const int sub = i / E, e = i - sub * E;
     const int pt = tile0 + sub;
     if (pt >= NT) continue;
     if (a.tile_counts) a.tile_counts[(size_t)e * NT + pt] = ctl->cnt[sub][e];
     if (a.tile_p != nullptr) {
+      const int rows = min(BM, T - pt * BM);
+      const float *col = zb + sub * BM * LD + e;
+      const float *is = ctl->inv_s + sub * BM;
       float s = 0.f;
-      for (int w = 0; w < wpt; ++w) s += ctl->psum[sub * wpt + w][e];
+      for (int mm = 0; mm < rows; ++mm) s += col[mm * LD] * is[mm];
       a.tile_p[(size_t)e * NT + pt] = s;
     }
   }
@@ -451,7 +459,8 @@ k_router_tc(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
   rt_sync_all<S>();
   tc_fence_after();
   if (warp >= 2 && ctl->epi_ok)
-    epilogue_tokens<EPAD, S, NOISY>(a, ctl, part, tile, rank, NT, BM, tid - 64);
+    epilogue_tokens<EPAD, S, NOISY>(a, ctl, part, S == 1 ? part : part + kRtM * C::kLdp, tile,
+                                    rank, NT, BM, tid - 64);
   // no CTA leaves (its shared memory) while another may still read its partials
   rt_sync_all<S>();
   if (warp == 1) tmem_dealloc(tmem, C::kTmemCols);
@@ -511,7 +520,7 @@ int router_splits(int T, int d, int E, int ex) {
   const int sms = sm_count();
   int S = 1;
   while (S < 4 && kRtM / (2 * S) >= BM && 2 * S <= nkb && tiles * 2 * S <= sms) S *= 2;
-  if (ex == 256 && S == 1 && nkb >= 2) S = 2;  // at most 64 logits per epilogue thread
+  (void)ex;
   return S;
 }
 
@@ -521,8 +530,7 @@ cudaError_t launch_rt_e(const RouterArgs &a, cudaStream_t st) {
   const int S = router_splits(a.T, a.d, a.E, kEx);
   if (S == 4) return launch_rt<EPAD, 4, NOISY>(a, st);
   if (S == 2) return launch_rt<EPAD, 2, NOISY>(a, st);
-  if constexpr (EPAD == 256 && !NOISY) return cudaErrorInvalidValue;  // needs a split
-  else return launch_rt<EPAD, 1, NOISY>(a, st);
+  return launch_rt<EPAD, 1, NOISY>(a, st);
 }
 
 }  // namespace
@@ -531,7 +539,7 @@ bool router_tc_supported(const RouterArgs &a) {
   if (a.x == nullptr || a.E < 1 || a.E > kMaxExperts || a.d % kBlockK != 0 || a.T <= 0)
     return false;
   if (a.w_noise != nullptr) return a.E <= 128 && a.eps != nullptr;
-  return !(a.E > 128 && a.d < 2 * kBlockK);
+  return true;
 }
 
 cudaError_t launch_router_tc(const RouterArgs &a, cudaStream_t st) {

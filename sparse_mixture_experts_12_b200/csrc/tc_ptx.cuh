@@ -175,10 +175,16 @@ __device__ __forceinline__ void decode_tile(int tile, const int *mpre, int G, in
 }
 
 // erf by Abramowitz & Stegun, Handbook of Mathematical Functions, formula 7.1.26
-// (|error| <= 1.5e-7), well below the bf16 rounding of the stored activation.
+// (|error| <= 1.5e-7 in exact arithmetic; with the approximate reciprocal below, a
+// few 1e-7), far below the bf16 rounding of the stored activation.
+__device__ __forceinline__ float rcp_approx(float x) {
+  float r;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+  return r;
+}
 __device__ __forceinline__ float erf_as7126(float x) {
   const float ax = fabsf(x);
-  const float t = __frcp_rn(fmaf(0.3275911f, ax, 1.f));
+  const float t = rcp_approx(fmaf(0.3275911f, ax, 1.f));
   const float p =
       fmaf(fmaf(fmaf(fmaf(1.061405429f, t, -1.453152027f), t, 1.421413741f), t, -0.284496736f), t,
            0.254829592f) * t;
