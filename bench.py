@@ -8,11 +8,11 @@ inputs already resident in HBM. Prints ONE JSON line on rank 0.
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
                   [--workloads LIST|all|none] [--impl ours|reference]
 
-The timed steps record CUDA events at the layer's stage boundaries
-(``moe_forward_staged``), so every stage's device time, the expert FFN's among
-them, comes from the measured steps themselves. After the headline workload the
-other workloads of the layer run the same way, each reported under
-``workloads``.
+The timed steps are plain layer calls (the throughput); the same number of steps
+follows with CUDA events at the layer's stage boundaries (``moe_forward_staged``),
+which gives every stage's device time, the expert FFN's among them, from steps of
+the same run. After the headline workload the other workloads of the layer run
+the same way, each reported under ``workloads``.
 
 Multi-GPU (torchrun, one rank per GPU): every rank runs the same layer on its
 own batch of T tokens (weak scaling, no data-path collective); the elapsed time
@@ -501,8 +501,11 @@ class Workbench:
 
 def time_workload(wb: Workbench, steps: int, warmup: int, peaks, peaks_src, local_rank,
                   world=1, flush_buf=None):
-    """Warm-up, then K timed steps with stage events; returns the workload's report
-    (and the loop time, max over ranks)."""
+    """Warm-up, then K timed steps of the plain layer call (the throughput: kernels
+    that overlap their neighbours' launch through programmatic dependent launch stay
+    overlapped), then K steps with events at every stage boundary (the breakdown:
+    an event between two kernels keeps them apart). Returns the workload's report,
+    the plain loop time (max over ranks) and the kernels per step."""
     wl, dev = wb.wl, wb.dev
     stream = torch.cuda.current_stream()
     for _ in range(warmup):
@@ -519,24 +522,32 @@ def time_workload(wb: Workbench, steps: int, warmup: int, peaks, peaks_src, loca
     barrier(world)
     torch.cuda.synchronize()
     clocks.begin_load()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if flush is None:
+        e0.record(stream)
+        for _ in range(steps):
+            wb.forward()
+        e1.record(stream)
     timer.run(lambda ev: wb.forward(events=ev), stream, flush)
     torch.cuda.synchronize()
     barrier(world)
     clk = clocks.stop()
     wb.check("in the timed region")
-    loop_ms = max_over_ranks(timer.loop_ms(), world, dev)
     stage_ms = timer.stage_ms()
     if flush is None:
+        loop_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
         ms_step = loop_ms / steps
         timing = "back-to-back steps, working set > L2"
     else:
-        ms_step = timer.step_ms()
+        ms_step = max_over_ranks(timer.step_ms(), world, dev)
+        loop_ms = ms_step * steps
         timing = "per step (first to last stage event), L2 flushed between steps"
     rs = wb.routing()
     work = stage_work(wl, rs, wb.want_aux)
     ffn_ms = stage_ms[STAGES.index("expert_ffn")] + stage_ms[STAGES.index("shared_ffn")]
     rep = {"workload": wl.name, "T": wl.T, "ms_per_step": ms_step,
            "tokens_per_s": wl.T * world / (ms_step * 1e-3), "timing": timing,
+           "staged_ms_per_step": timer.step_ms(),
            "stages": stage_report(work, stage_ms, peaks),
            "roofline": ffn_roofline(wl, work, ffn_ms, peaks, peaks_src),
            "kernels_per_step": launches, "routing": rs, "clocks": clk}

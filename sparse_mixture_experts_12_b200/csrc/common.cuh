@@ -61,6 +61,20 @@ __device__ __forceinline__ void report_error(int32_t *err, int32_t code, int32_t
   if (atomicCAS(err, 0, code) == 0) atomicExch(err + 1, info);
 }
 
+// ------------------------------------------------- programmatic dependent launch
+// A kernel launched with programmatic stream serialisation may begin while the
+// kernel before it in the stream is still running. pdl_wait() blocks until that
+// kernel has completed and its writes are visible: it comes before the first
+// access to anything an earlier kernel writes, or reads while this one writes it.
+// pdl_trigger() lets the next kernel in the stream begin its launch; a kernel
+// calls it only after its own pdl_wait(), so every kernel that passes its wait
+// knows that all earlier kernels have completed. Both are no-ops in a kernel
+// launched without the attribute.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- warp helpers
 __device__ __forceinline__ float warp_max(float v) {
 #pragma unroll
@@ -89,5 +103,22 @@ __host__ __device__ constexpr int router_bm(int E) {
 }
 
 __host__ __device__ constexpr int ceil_div(int a, int b) { return (a + b - 1) / b; }
+
+// Launch `kernel` with programmatic stream serialisation (see pdl_wait).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t st, Args... args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
 
 }  // namespace moe

@@ -72,6 +72,8 @@ struct TcArgs {
   int32_t *err;
   int tile_mode;  // TILES_ALL, or the pair / tail halves of a split launch
   int tma_store;  // pair kernel, bf16 output: full 32-row groups leave through TMA stores
+  int pdl_mode;            // PDL_NONE, PDL_WAIT (wait before the first dependent access)
+                           // or PDL_TAIL (the tail-tile launch: wait only before exit)
   uint64_t wait_limit_ns;  // single-CTA kernel: bound on its pipeline waits
   int withhold_load;       // single-CTA kernel, test hook: the first operand load of each
                            // CTA is never issued, so the waits on it run out
@@ -117,6 +119,12 @@ __device__ __forceinline__ void emit_chunk(const EpiStore &st, const uint4 (&pk)
 // 128-row tile holds at most 128 rows), hands that tile to the single-CTA kernel
 // instead of a 256-row pair tile that would be at least half empty.
 enum { TILES_ALL = 0, TILES_PAIRS_NO_TAIL = 1, TILES_TAIL_ONLY = 2 };
+
+// Programmatic dependent launch of a GEMM (see pdl_wait). PDL_TAIL: the tail-tile
+// launch reads nothing the pair grid before it writes, so it starts at once; it
+// waits for that grid only before it exits, so that its completion tells the
+// kernels after it that the pair grid has completed too.
+enum { PDL_NONE = 0, PDL_WAIT = 1, PDL_TAIL = 2 };
 
 struct SmemCtl {
   uint64_t full[kStages];
@@ -238,6 +246,26 @@ k_ffn_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtens
   const int G = a.G;
   int *mpre = ctl->tbl;
   int *offs = ctl->tbl + (G + 1);
+  if (tid == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&ctl->full[s], 1);
+      mbar_init(&ctl->empty[s], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&ctl->tfull[s], 1);
+      mbar_init(&ctl->tempty[s], kEpiWarps1 * 32);
+    }
+    mbar_init(&ctl->drain, 1);
+    ctl->abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 2) {
+    tmem_alloc(&ctl->tmem_base, kTmemCols);
+    tmem_relinquish();
+  }
+  // the set-up above overlaps the previous kernel; the tile tables, the operands
+  // and the outputs are touched only after it has completed
+  if (a.pdl_mode == PDL_WAIT) pdl_wait();
   for (int i = tid; i <= G; i += kThreads1) {
     if (a.tile_mode != TILES_TAIL_ONLY) mpre[i] = a.mprefix[i];
     offs[i] = a.offsets[i];
@@ -261,26 +289,10 @@ k_ffn_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtens
     }
     if (lane == 31) mpre[G] = incl;
   }
-  if (tid == 0) {
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(&ctl->full[s], 1);
-      mbar_init(&ctl->empty[s], 1);
-    }
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(&ctl->tfull[s], 1);
-      mbar_init(&ctl->tempty[s], kEpiWarps1 * 32);
-    }
-    mbar_init(&ctl->drain, 1);
-    ctl->abort_flag = 0;
-    fence_mbar_init();
-  }
-  if (warp == 2) {
-    tmem_alloc(&ctl->tmem_base, kTmemCols);
-    tmem_relinquish();
-  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  if (a.pdl_mode == PDL_WAIT) pdl_trigger();
   const uint32_t tmem = ctl->tmem_base;
   const int total = mpre[G] * a.n_tiles;
   const int nkb = ceil_div(a.K, kBlockK);
@@ -407,6 +419,7 @@ k_ffn_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtens
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
+  if (a.pdl_mode == PDL_TAIL) pdl_wait();
 }
 
 // ============================================================= CTA-pair kernel
@@ -502,7 +515,6 @@ k_ffn_tc2(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
   const int G = a.G;
   int *ppre = ctl->tbl;
   int *offs = ctl->tbl + (G + 1);
-  for (int i = tid; i <= G; i += kThreads) offs[i] = a.offsets[i];
   if (tid == 0) {
     for (int s = 0; s < kS; ++s) {
       mbar_init(&ctl->full[s], 1);
@@ -516,6 +528,14 @@ k_ffn_tc2(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
     ctl->abort_flag = 0;
     fence_mbar_init();
   }
+  if (warp == 2) {
+    tmem_alloc_pair(&ctl->tmem_base, kTmemCols);
+    tmem_relinquish_pair();
+  }
+  // the set-up above overlaps the previous kernel; the tile tables, the operands
+  // and the outputs are touched only after it has completed
+  if (a.pdl_mode == PDL_WAIT) pdl_wait();
+  for (int i = tid; i <= G; i += kThreads) offs[i] = a.offsets[i];
   if (warp == 1) {
     // pair tiles per group = ceil(ceil(rows / 128) / 2) from the 128-row tile prefix
     // (all zero when the offsets failed validation); warp scan over the groups
@@ -536,10 +556,6 @@ k_ffn_tc2(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
       run += (a.mprefix[j + 1] - a.mprefix[j] + round_up) >> 1;
     }
     if (lane == 31) ppre[G] = incl;
-  }
-  if (warp == 2) {
-    tmem_alloc_pair(&ctl->tmem_base, kTmemCols);
-    tmem_relinquish_pair();
   }
   tc_fence_before();
   __syncthreads();
@@ -713,7 +729,7 @@ std::mutex g_attr_mu;
 // Only for a grid that neither reads nor writes anything the preceding grid writes.
 template <int EPI>
 cudaError_t launch_single(const CUtensorMap &ma, const CUtensorMap &mb, const CUtensorMap &mb3,
-                          const TcArgs &t, long long tiles_ub, bool overlap, cudaStream_t st) {
+                          TcArgs t, long long tiles_ub, bool overlap, cudaStream_t st) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
@@ -728,7 +744,9 @@ cudaError_t launch_single(const CUtensorMap &ma, const CUtensorMap &mb, const CU
     }
   }
   const int grid = (int)std::max<long long>(1, std::min<long long>(tiles_ub, sm_count()));
-  if (!overlap) {
+  if (overlap) {
+    t.pdl_mode = PDL_TAIL;
+  } else if (t.pdl_mode == PDL_NONE) {
     k_ffn_tc<EPI><<<grid, kThreads1, kSmemBytes, st>>>(ma, mb, mb3, t);
     return cudaGetLastError();
   }
@@ -784,6 +802,13 @@ cudaError_t launch_pair(const CUtensorMap &ma, const CUtensorMap &mb, const CUte
   }
   const long long pairs = std::min<long long>(tiles_ub, info.max_pairs[slot]);
   cfg.gridDim = dim3((unsigned)(2 * pairs));
+  cudaLaunchAttribute attr2[2] = {attr[0], attr[0]};
+  if (t.pdl_mode == PDL_WAIT) {  // the cluster shape and programmatic serialisation
+    attr2[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr2[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr2;
+    cfg.numAttrs = 2;
+  }
   e = cudaLaunchKernelEx(&cfg, k_ffn_tc2<EPI, NH>, ma, mb, mb3, mo, t);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
@@ -897,6 +922,10 @@ cudaError_t launch_ffn_tc(const GroupedFfnArgs &a, cudaStream_t st) {
   t.err = a.err;
   t.wait_limit_ns = a.wait_limit_ns ? a.wait_limit_ns : kWaitLimitNs;
   t.withhold_load = a.withhold_load;  // the up projection only
+  // both projections start while the kernel before them finishes (a tail-tile
+  // launch of the up projection waits for its pair grid before it exits, so the
+  // down projection's wait covers both)
+  t.pdl_mode = PDL_WAIT;
   // pair tiles write bf16 outputs through TMA stores of 32 x 32 boxes
   CUtensorMap mo;
   if (!make_store_map(&mo, a.h, (uint64_t)a.a_rows, (uint64_t)a.F)) return cudaErrorInvalidValue;

@@ -42,6 +42,8 @@ __global__ void __launch_bounds__(kScanThreads) k_scan(ScanArgs a, ShardCaps sc)
   __shared__ int count_s[kMaxExperts];
   __shared__ float P_s[kMaxExperts];
   __shared__ float red[kScanThreads / 32];
+  pdl_wait();
+  pdl_trigger();
   const int E = a.E, NT = a.NT;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   constexpr int nw = kScanThreads / 32;
@@ -219,6 +221,8 @@ __global__ void __launch_bounds__(kScatterThreads) k_scatter(ScatterArgs a, cons
   int32_t *prow = hist + NC * E;    // [bm*k]: in-chunk rank, then the destination row
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int32_t *idx = a.topk_idx + (size_t)t0 * k;
+  pdl_wait();
+  pdl_trigger();
 
   for (int i = tid; i < NC * E; i += kScatterThreads) hist[i] = 0;
   __syncthreads();
@@ -303,6 +307,8 @@ __global__ void __launch_bounds__(256) k_combine(CombineArgs a) {
   constexpr int VE = Elem<T>::kPerVec;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t = blockIdx.x * 8 + warp;
+  pdl_wait();
+  pdl_trigger();
   if (t >= a.T) return;
   const int k = a.k;
   int row[KMAX];
@@ -410,8 +416,7 @@ __global__ void k_tile_table(const int32_t *offsets, int G, int max_rows, int32_
 }  // namespace
 
 cudaError_t launch_scan(const ScanArgs &a, cudaStream_t st) {
-  k_scan<false><<<1, kScanThreads, 0, st>>>(a, ShardCaps{});
-  return cudaGetLastError();
+  return launch_pdl(k_scan<false>, dim3(1), dim3(kScanThreads), 0, st, a, ShardCaps{});
 }
 
 cudaError_t launch_scan_shard(const ScanArgs &a, const ShardCaps &sc, cudaStream_t st) {
@@ -427,8 +432,7 @@ cudaError_t scatter(const ScatterArgs &a, const int32_t *cap_e, cudaStream_t st)
   const int NT = ceil_div(a.T, bm);
   const int NC = ceil_div(bm * a.k, 32);
   const size_t smem = (size_t)(NC * a.E + bm * a.k) * sizeof(int32_t);
-  k_scatter<SHARD><<<NT, kScatterThreads, smem, st>>>(a, cap_e);
-  return cudaGetLastError();
+  return launch_pdl(k_scatter<SHARD>, dim3(NT), dim3(kScatterThreads), smem, st, a, cap_e);
 }
 }  // namespace
 
@@ -444,14 +448,13 @@ cudaError_t launch_combine(const CombineArgs &a, int dtype, cudaStream_t st) {
   if (a.T == 0) return cudaSuccess;
   const int grid = ceil_div(a.T, 8);
   const bool f32 = dtype == MOE_DTYPE_F32;
+  const dim3 g(grid), b(256);
   if (a.k <= 2) {
-    if (f32) k_combine<float, 2, 4><<<grid, 256, 0, st>>>(a);
-    else k_combine<__nv_bfloat16, 2, 4><<<grid, 256, 0, st>>>(a);
-  } else {
-    if (f32) k_combine<float, kMaxTopK, 1><<<grid, 256, 0, st>>>(a);
-    else k_combine<__nv_bfloat16, kMaxTopK, 1><<<grid, 256, 0, st>>>(a);
+    if (f32) return launch_pdl(k_combine<float, 2, 4>, g, b, 0, st, a);
+    return launch_pdl(k_combine<__nv_bfloat16, 2, 4>, g, b, 0, st, a);
   }
-  return cudaGetLastError();
+  if (f32) return launch_pdl(k_combine<float, kMaxTopK, 1>, g, b, 0, st, a);
+  return launch_pdl(k_combine<__nv_bfloat16, kMaxTopK, 1>, g, b, 0, st, a);
 }
 
 cudaError_t launch_tile_table(const int32_t *offsets, int G, int max_rows, int32_t *mprefix,

@@ -391,6 +391,10 @@ k_router_tc(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUt
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = ctl->tmem_base;
+  // the set-up above overlaps the previous kernel; x, the weights and every output
+  // are touched only after it has completed
+  pdl_wait();
+  pdl_trigger();
 
   if (warp == 0 && lane == 0) {
     // ------------------------------------------------------------ TMA producer
@@ -500,13 +504,15 @@ cudaError_t launch_rt(const RouterArgs &a, cudaStream_t st) {
   cfg.blockDim = dim3(kRtThreads);
   cfg.dynamicSmemBytes = C::kSmem;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = S;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   return cudaLaunchKernelEx(&cfg, k_router_tc<EPAD, S, NOISY>, mx, mw, mn, a, NT, BM);
 }
 
