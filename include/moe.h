@@ -23,7 +23,10 @@
  * - Ownership: the caller allocates and owns every buffer (device memory unless
  *   stated). The library never allocates, frees or keeps pointers after a call.
  * - Asynchrony: every call only enqueues kernels on `stream` and returns; none
- *   synchronises except moe_last_device_error().
+ *   synchronises except moe_last_device_error(). The layer's kernels are launched
+ *   with programmatic stream serialisation: each may begin its set-up while the
+ *   kernel before it in the stream finishes, and waits for that kernel before it
+ *   touches memory.
  * - Layout: row-major. Weights use the nn.Linear [out_features, in_features]
  *   layout, stacked over experts. Activations, weights, x_perm, y_perm and y are
  *   stored in cfg->dtype (fp32 or bf16); biases, logits, gates are fp32; index
@@ -277,8 +280,10 @@ typedef struct {
 /* moe_forward (noise == NULL) or moe_forward_noisy / moe_forward_noisy_seeded (noise
  * given) that also records `events` (nullable) at its stage boundaries and marks
  * each stage with an NVTX range (named "moe_route", "moe_scan", ...). The kernels and
- * results are those of the plain entry points; a failed event record returns
- * MOE_ERR_CUDA. */
+ * results are those of the plain entry points. The plain entry points launch each
+ * kernel so that it may begin while the one before it finishes (programmatic
+ * dependent launch); with events, the kernels run one after another, so that each
+ * stage's time is its kernels' own. A failed event record returns MOE_ERR_CUDA. */
 moe_status_t moe_forward_staged(const moe_cfg_t *cfg, const moe_weights_t *w, const void *x,
                                 const moe_noise_t *noise, void *y, float *aux_out,
                                 const moe_taps_t *taps, const moe_stage_events_t *events,

@@ -104,7 +104,13 @@ __host__ __device__ constexpr int router_bm(int E) {
 
 __host__ __device__ constexpr int ceil_div(int a, int b) { return (a + b - 1) / b; }
 
-// Launch `kernel` with programmatic stream serialisation (see pdl_wait).
+// Whether this host thread's launches use programmatic dependent launch. A layer call
+// that records stage events turns it off for its launches: an event between two
+// kernels keeps them apart anyway, and the timed stages should be the kernels' own.
+extern thread_local bool t_allow_pdl;
+
+// Launch `kernel` with programmatic stream serialisation (see pdl_wait) when
+// t_allow_pdl, else as a plain launch.
 template <typename... KArgs, typename... Args>
 cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
                        cudaStream_t st, Args... args) {
@@ -117,7 +123,7 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = t_allow_pdl ? 1 : 0;
   return cudaLaunchKernelEx(&cfg, kernel, args...);
 }
 

@@ -925,7 +925,7 @@ cudaError_t launch_ffn_tc(const GroupedFfnArgs &a, cudaStream_t st) {
   // both projections start while the kernel before them finishes (a tail-tile
   // launch of the up projection waits for its pair grid before it exits, so the
   // down projection's wait covers both)
-  t.pdl_mode = PDL_WAIT;
+  t.pdl_mode = t_allow_pdl ? PDL_WAIT : PDL_NONE;
   // pair tiles write bf16 outputs through TMA stores of 32 x 32 boxes
   CUtensorMap mo;
   if (!make_store_map(&mo, a.h, (uint64_t)a.a_rows, (uint64_t)a.F)) return cudaErrorInvalidValue;

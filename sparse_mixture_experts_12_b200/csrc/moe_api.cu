@@ -13,7 +13,22 @@
 #define MOE_API extern "C" __attribute__((visibility("default")))
 
 namespace moe {
+
+thread_local bool t_allow_pdl = true;
+
 namespace {
+
+// Turns programmatic dependent launch off for the launches of one layer call.
+class PdlOff {
+ public:
+  explicit PdlOff(bool off) : prev_(t_allow_pdl) {
+    if (off) t_allow_pdl = false;
+  }
+  ~PdlOff() { t_allow_pdl = prev_; }
+
+ private:
+  bool prev_;
+};
 
 enum Buf {
   B_ERR, B_TILE_COUNTS, B_TILE_BASE, B_TILE_P, B_TILE_Z, B_COUNTS, B_OFFSETS, B_MPREFIX, B_SH_TBL,
@@ -738,6 +753,7 @@ moe_status_t forward_impl(const moe_cfg_t *cfg, const moe_weights_t *w, const vo
       return MOE_ERR_INVALID_ARG;
   }
   Stages sg(events, stream);
+  const PdlOff pdl_off(events != nullptr);  // the timed stages are the kernels' own
   if (cfg->n_tokens == 0) return sg.finish();  // nothing is read or written
   if (w == nullptr) return MOE_ERR_INVALID_ARG;
   MOE_TRY(check_ptrs({{x, true}, {y, true}, {aux_out, false}, {w->w_router, sh == nullptr},
