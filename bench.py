@@ -8,10 +8,10 @@ inputs already resident in HBM. Prints ONE JSON line on rank 0.
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
                   [--workloads LIST|all|none] [--impl ours|reference]
 
-The timed steps are plain layer calls (the throughput); the same number of steps
-follows with CUDA events at the layer's stage boundaries (``moe_forward_staged``),
-which gives every stage's device time, the expert FFN's among them, from steps of
-the same run. After the headline workload the other workloads of the layer run
+Every timed step records CUDA events at the start of its expert FFNs and of its
+combine (``moe_forward_staged``), so the expert GEMMs' time comes from the timed
+steps themselves; the same number of steps follows with an event at every stage
+boundary, for the per-stage breakdown. After the headline workload the other workloads of the layer run
 the same way, each reported under ``workloads``.
 
 Multi-GPU (torchrun, one rank per GPU): every rank runs the same layer on its
@@ -398,14 +398,7 @@ class StepTimer:
 
     def __init__(self, steps: int):
         self.steps = steps
-        self.ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(STAGES) + 1)]
-                   for _ in range(steps)]
-        # torch creates an event at its first record: do that here, so that the
-        # library records (and torch later reads) real event handles
-        for evs in self.ev:
-            for e in evs:
-                e.record()
-        torch.cuda.synchronize()
+        self.ev = [_made_events(len(STAGES) + 1) for _ in range(steps)]
         self.e0 = torch.cuda.Event(enable_timing=True)
         self.e1 = torch.cuda.Event(enable_timing=True)
 
@@ -499,13 +492,29 @@ class Workbench:
         return rs
 
 
+def _made_events(n: int):
+    """n timing events, each already created on the device (torch creates an event
+    at its first record, and the library records the raw handle)."""
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+    for e in evs:
+        e.record()
+    torch.cuda.synchronize()
+    return evs
+
+
+FFN_FIRST, FFN_END = STAGES.index("shared_ffn"), STAGES.index("combine")
+
+
 def time_workload(wb: Workbench, steps: int, warmup: int, peaks, peaks_src, local_rank,
                   world=1, flush_buf=None):
-    """Warm-up, then K timed steps of the plain layer call (the throughput: kernels
-    that overlap their neighbours' launch through programmatic dependent launch stay
-    overlapped), then K steps with events at every stage boundary (the breakdown:
-    an event between two kernels keeps them apart). Returns the workload's report,
-    the plain loop time (max over ranks) and the kernels per step."""
+    """Warm-up, then the timed region: K steps of the layer call, each recording two
+    events, at the start of its expert FFNs (shared experts first) and at the start of
+    its combine, so that the expert GEMMs' time comes from the timed steps. The layer
+    launches each kernel so that it may begin while the one before it finishes; the
+    kernel right after an event does not, so these two events cost the steps a little.
+    Then, for the breakdown, K more steps with an event at every stage boundary.
+    Returns the workload's report, the timed loop's time (max over ranks) and the
+    kernels per step."""
     wl, dev = wb.wl, wb.dev
     stream = torch.cuda.current_stream()
     for _ in range(warmup):
@@ -514,6 +523,7 @@ def time_workload(wb: Workbench, steps: int, warmup: int, peaks, peaks_src, loca
     wb.check("during warm-up")
     launches = kernels_per_step(lambda: wb.forward(), dev)
     timer = StepTimer(steps)
+    ffn_ev = [_made_events(2) for _ in range(steps)]
     flush = None
     if flush_buf is not None:
         flush = flush_buf.zero_
@@ -523,16 +533,22 @@ def time_workload(wb: Workbench, steps: int, warmup: int, peaks, peaks_src, loca
     torch.cuda.synchronize()
     clocks.begin_load()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    if flush is None:
-        e0.record(stream)
-        for _ in range(steps):
-            wb.forward()
-        e1.record(stream)
-    timer.run(lambda ev: wb.forward(events=ev), stream, flush)
+    e0.record(stream)
+    for i in range(steps):
+        if flush is not None:
+            flush()
+        ev = [None] * (len(STAGES) + 1)
+        ev[FFN_FIRST], ev[FFN_END] = ffn_ev[i]
+        wb.forward(events=ev)
+    e1.record(stream)
     torch.cuda.synchronize()
     barrier(world)
     clk = clocks.stop()
     wb.check("in the timed region")
+    ffn_ms = float(np.mean([a.elapsed_time(b) for a, b in ffn_ev]))
+    timer.run(lambda ev: wb.forward(events=ev), stream, flush)  # the breakdown
+    torch.cuda.synchronize()
+    wb.check("in the breakdown steps")
     stage_ms = timer.stage_ms()
     if flush is None:
         loop_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
@@ -544,11 +560,11 @@ def time_workload(wb: Workbench, steps: int, warmup: int, peaks, peaks_src, loca
         timing = "per step (first to last stage event), L2 flushed between steps"
     rs = wb.routing()
     work = stage_work(wl, rs, wb.want_aux)
-    ffn_ms = stage_ms[STAGES.index("expert_ffn")] + stage_ms[STAGES.index("shared_ffn")]
     rep = {"workload": wl.name, "T": wl.T, "ms_per_step": ms_step,
            "tokens_per_s": wl.T * world / (ms_step * 1e-3), "timing": timing,
-           "staged_ms_per_step": timer.step_ms(),
            "stages": stage_report(work, stage_ms, peaks),
+           "stages_note": "a second run of K steps with an event at every stage boundary; "
+                          "the kernel after each event starts after it",
            "roofline": ffn_roofline(wl, work, ffn_ms, peaks, peaks_src),
            "kernels_per_step": launches, "routing": rs, "clocks": clk}
     return rep, loop_ms, launches

@@ -280,10 +280,11 @@ typedef struct {
 /* moe_forward (noise == NULL) or moe_forward_noisy / moe_forward_noisy_seeded (noise
  * given) that also records `events` (nullable) at its stage boundaries and marks
  * each stage with an NVTX range (named "moe_route", "moe_scan", ...). The kernels and
- * results are those of the plain entry points. The plain entry points launch each
- * kernel so that it may begin while the one before it finishes (programmatic
- * dependent launch); with events, the kernels run one after another, so that each
- * stage's time is its kernels' own. A failed event record returns MOE_ERR_CUDA. */
+ * results are those of the plain entry points. The entry points launch each kernel
+ * so that it may begin while the one before it finishes (programmatic dependent
+ * launch); the kernel launched right after a recorded event starts after the event
+ * instead, so that each timed stage is its own kernels' time. A failed event record
+ * returns MOE_ERR_CUDA. */
 moe_status_t moe_forward_staged(const moe_cfg_t *cfg, const moe_weights_t *w, const void *x,
                                 const moe_noise_t *noise, void *y, float *aux_out,
                                 const moe_taps_t *taps, const moe_stage_events_t *events,

@@ -104,13 +104,21 @@ __host__ __device__ constexpr int router_bm(int E) {
 
 __host__ __device__ constexpr int ceil_div(int a, int b) { return (a + b - 1) / b; }
 
-// Whether this host thread's launches use programmatic dependent launch. A layer call
-// that records stage events turns it off for its launches: an event between two
-// kernels keeps them apart anyway, and the timed stages should be the kernels' own.
-extern thread_local bool t_allow_pdl;
+// Set when a layer call has just recorded a stage event on this host thread: the
+// next launch is a plain one (it starts after the event, so that the stage's time is
+// its kernels' own) and clears the flag; every other launch uses programmatic
+// dependent launch.
+extern thread_local bool t_pdl_blocked;
 
-// Launch `kernel` with programmatic stream serialisation (see pdl_wait) when
-// t_allow_pdl, else as a plain launch.
+// Whether the next launch may use programmatic dependent launch (consumes the flag).
+inline bool take_pdl() {
+  const bool ok = !t_pdl_blocked;
+  t_pdl_blocked = false;
+  return ok;
+}
+
+// Launch `kernel` with programmatic stream serialisation (see pdl_wait), or as a
+// plain launch right after a stage event.
 template <typename... KArgs, typename... Args>
 cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
                        cudaStream_t st, Args... args) {
@@ -123,7 +131,7 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = t_allow_pdl ? 1 : 0;
+  cfg.numAttrs = take_pdl() ? 1 : 0;
   return cudaLaunchKernelEx(&cfg, kernel, args...);
 }
 

@@ -925,7 +925,7 @@ cudaError_t launch_ffn_tc(const GroupedFfnArgs &a, cudaStream_t st) {
   // both projections start while the kernel before them finishes (a tail-tile
   // launch of the up projection waits for its pair grid before it exits, so the
   // down projection's wait covers both)
-  t.pdl_mode = t_allow_pdl ? PDL_WAIT : PDL_NONE;
+  t.pdl_mode = take_pdl() ? PDL_WAIT : PDL_NONE;
   // pair tiles write bf16 outputs through TMA stores of 32 x 32 boxes
   CUtensorMap mo;
   if (!make_store_map(&mo, a.h, (uint64_t)a.a_rows, (uint64_t)a.F)) return cudaErrorInvalidValue;
@@ -954,6 +954,7 @@ cudaError_t launch_ffn_tc(const GroupedFfnArgs &a, cudaStream_t st) {
   t.bias = a.b2;
   t.act = -1;
   t.withhold_load = 0;
+  t.pdl_mode = PDL_WAIT;  // follows the up projection's kernels directly
   t.tma_store = a.out_f32 ? 0 : 1;
   if (!a.out_f32 && !make_store_map(&mo, a.out, (uint64_t)a.a_rows, (uint64_t)a.d))
     return cudaErrorInvalidValue;

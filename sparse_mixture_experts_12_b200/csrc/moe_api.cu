@@ -14,21 +14,9 @@
 
 namespace moe {
 
-thread_local bool t_allow_pdl = true;
+thread_local bool t_pdl_blocked = false;
 
 namespace {
-
-// Turns programmatic dependent launch off for the launches of one layer call.
-class PdlOff {
- public:
-  explicit PdlOff(bool off) : prev_(t_allow_pdl) {
-    if (off) t_allow_pdl = false;
-  }
-  ~PdlOff() { t_allow_pdl = prev_; }
-
- private:
-  bool prev_;
-};
 
 enum Buf {
   B_ERR, B_TILE_COUNTS, B_TILE_BASE, B_TILE_P, B_TILE_Z, B_COUNTS, B_OFFSETS, B_MPREFIX, B_SH_TBL,
@@ -228,12 +216,14 @@ class Stages {
     for (; next_ <= MOE_STAGE_COUNT; ++next_) MOE_TRY(record(next_));
     if (open_) nvtxRangePop();
     open_ = false;
+    t_pdl_blocked = false;  // a flag left by the last event stays in this call
     return MOE_OK;
   }
 
  private:
   moe_status_t record(int i) {
     if (ev_ == nullptr || ev_->ev[i] == nullptr) return MOE_OK;
+    t_pdl_blocked = true;  // the kernel after the event starts after it
     return cuda_status(cudaEventRecord(reinterpret_cast<cudaEvent_t>(ev_->ev[i]), st_));
   }
   const moe_stage_events_t *ev_;
@@ -753,7 +743,6 @@ moe_status_t forward_impl(const moe_cfg_t *cfg, const moe_weights_t *w, const vo
       return MOE_ERR_INVALID_ARG;
   }
   Stages sg(events, stream);
-  const PdlOff pdl_off(events != nullptr);  // the timed stages are the kernels' own
   if (cfg->n_tokens == 0) return sg.finish();  // nothing is read or written
   if (w == nullptr) return MOE_ERR_INVALID_ARG;
   MOE_TRY(check_ptrs({{x, true}, {y, true}, {aux_out, false}, {w->w_router, sh == nullptr},

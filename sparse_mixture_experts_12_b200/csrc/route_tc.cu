@@ -512,7 +512,7 @@ cudaError_t launch_rt(const RouterArgs &a, cudaStream_t st) {
   attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = t_allow_pdl ? 2 : 1;
+  cfg.numAttrs = take_pdl() ? 2 : 1;
   return cudaLaunchKernelEx(&cfg, k_router_tc<EPAD, S, NOISY>, mx, mw, mn, a, NT, BM);
 }
 
