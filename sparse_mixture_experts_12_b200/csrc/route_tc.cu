@@ -194,48 +194,66 @@ __device__ __forceinline__ void epilogue_tokens(const RouterArgs &a, RtCtl *ctl,
   const int E = a.E, T = a.T, k = a.k;
   const int t_base = tile * kRtM + rank * TOK;  // token of this CTA's first row
 
-  // ---- 1. logits
+  // ---- 1. logits. kB pairs per thread at a time: all their loads (the S ranks'
+  // partials) are issued before any of them is used or any zb store is made, since
+  // a store between two loads of the same array keeps them apart.
   {
+    constexpr int kB = 4;
+    constexpr int kPairs = TOK * EX;
     const uint32_t part_s = smem_u32(part);
-#pragma unroll 2
-    for (int i = et; i < TOK * EX; i += kRtEpiThreads) {
-      const int m = i / EX, e = i - m * EX;
-      const int row = rank * TOK + m;
-      const int t = t_base + m;
-      float acc, accn = 0.f;
-      if constexpr (S == 1) {
-        acc = part[row * LD + e];
-        if constexpr (NOISY) accn = part[row * LD + EX + e];
-      } else {
-        const uint32_t off = 4u * (uint32_t)(row * LD + e);
-        float v[S], vn[S];
+#pragma unroll 1
+    for (int i0 = et; i0 < kPairs; i0 += kB * kRtEpiThreads) {
+      float acc[kB], accn[kB];
 #pragma unroll
-        for (int r = 0; r < S; ++r) {
-          const uint32_t rb = mapa_rank(part_s, (uint32_t)r) + off;
-          v[r] = ld_cluster_f32(rb);
-          if constexpr (NOISY) vn[r] = ld_cluster_f32(rb + 4u * EX);
+      for (int u = 0; u < kB; ++u) {
+        const int i = i0 + u * kRtEpiThreads;
+        acc[u] = 0.f;
+        accn[u] = 0.f;
+        if (i < kPairs) {
+          const int m = i / EX, e = i - m * EX;
+          const int row = rank * TOK + m;
+          if constexpr (S == 1) {
+            acc[u] = part[row * LD + e];
+            if constexpr (NOISY) accn[u] = part[row * LD + EX + e];
+          } else {
+            const uint32_t off = 4u * (uint32_t)(row * LD + e);
+            float v[S], vn[S];
+#pragma unroll
+            for (int r = 0; r < S; ++r) {
+              const uint32_t rb = mapa_rank(part_s, (uint32_t)r) + off;
+              v[r] = ld_cluster_f32(rb);
+              if constexpr (NOISY) vn[r] = ld_cluster_f32(rb + 4u * EX);
+            }
+            acc[u] = v[0];  // the ranks' partials in rank order
+#pragma unroll
+            for (int r = 1; r < S; ++r) acc[u] += v[r];
+            if constexpr (NOISY) {
+              accn[u] = vn[0];
+#pragma unroll
+              for (int r = 1; r < S; ++r) accn[u] += vn[r];
+            }
+          }
         }
-        acc = v[0];
+      }
 #pragma unroll
-        for (int r = 1; r < S; ++r) acc += v[r];
+      for (int u = 0; u < kB; ++u) {
+        const int i = i0 + u * kRtEpiThreads;
+        if (i >= kPairs) continue;
+        const int m = i / EX, e = i - m * EX;
+        const int t = t_base + m;
+        const bool live = t < T && e < E;
+        float v = acc[u];
+        if (a.b_router) v += ctl->br[e];
+        if (a.logit_bias) v += ctl->lb[e];
         if constexpr (NOISY) {
-          accn = vn[0];
-#pragma unroll
-          for (int r = 1; r < S; ++r) accn += vn[r];
+          if (live) {
+            const float sp = accn[u] > 20.f ? accn[u] : log1pf(expf(accn[u]));
+            v = v + sp * a.eps[(size_t)t * E + e];
+          }
         }
+        if (a.logits_out != nullptr && live) a.logits_out[(size_t)t * E + e] = v;
+        zb[m * LD + e] = (e >= E || v != v) ? -INFINITY : v;  // padding, NaN never win
       }
-      const bool live = t < T && e < E;
-      float v = acc;
-      if (a.b_router) v += ctl->br[e];
-      if (a.logit_bias) v += ctl->lb[e];
-      if constexpr (NOISY) {
-        if (live) {
-          const float sp = accn > 20.f ? accn : log1pf(expf(accn));
-          v = v + sp * a.eps[(size_t)t * E + e];
-        }
-      }
-      if (a.logits_out != nullptr && live) a.logits_out[(size_t)t * E + e] = v;
-      zb[m * LD + e] = (e >= E || v != v) ? -INFINITY : v;  // padding, NaN never win a slot
     }
   }
   rt_epi_sync();
@@ -271,11 +289,20 @@ __device__ __forceinline__ void epilogue_tokens(const RouterArgs &a, RtCtl *ctl,
       }
     }
     float ssum = 0.f;
-#pragma unroll 4
-    for (int e = g; e < EX; e += G) {
-      const float ex = expf(zr[e] - mx);
-      ssum += ex;
-      zr[e] = ex;  // kept for the probability sums
+    constexpr int kEpl = EX / G;  // expert columns of this thread
+    constexpr int kB = kEpl < 4 ? kEpl : 4;
+#pragma unroll 1
+    for (int j0 = 0; j0 < kEpl; j0 += kB) {  // kB loads before the kB stores
+      float ex[kB];
+#pragma unroll
+      for (int u = 0; u < kB; ++u) ex[u] = zr[g + (j0 + u) * G];
+#pragma unroll
+      for (int u = 0; u < kB; ++u) {
+        ex[u] = expf(ex[u] - mx);
+        ssum += ex[u];
+      }
+#pragma unroll
+      for (int u = 0; u < kB; ++u) zr[g + (j0 + u) * G] = ex[u];  // for the probability sums
     }
     ssum = group_sum<G>(ssum);
     const float inv_s = 1.f / ssum;
