@@ -8,9 +8,9 @@ inputs already resident in HBM. Prints ONE JSON line on rank 0.
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
                   [--workloads LIST|all|none] [--impl ours|reference]
 
-Every timed step records CUDA events at the start of its expert FFNs and of its
-combine (``moe_forward_staged``), so the expert GEMMs' time comes from the timed
-steps themselves; the same number of steps follows with an event at every stage
+Every fourth timed step records CUDA events at the start of its expert FFNs and of
+its combine (``moe_forward_staged``), so the expert GEMMs' time comes from the
+timed steps themselves; the same number of steps follows with an event at every stage
 boundary, for the per-stage breakdown. After the headline workload the other workloads of the layer run
 the same way, each reported under ``workloads``.
 
@@ -503,15 +503,17 @@ def _made_events(n: int):
 
 
 FFN_FIRST, FFN_END = STAGES.index("shared_ffn"), STAGES.index("combine")
+FFN_EVERY = 4  # every 4th timed step also times its expert GEMMs
 
 
 def time_workload(wb: Workbench, steps: int, warmup: int, peaks, peaks_src, local_rank,
                   world=1, flush_buf=None):
-    """Warm-up, then the timed region: K steps of the layer call, each recording two
-    events, at the start of its expert FFNs (shared experts first) and at the start of
-    its combine, so that the expert GEMMs' time comes from the timed steps. The layer
-    launches each kernel so that it may begin while the one before it finishes; the
-    kernel right after an event does not, so these two events cost the steps a little.
+    """Warm-up, then the timed region: K steps of the layer call; every FFN_EVERY-th
+    step records two events, at the start of its expert FFNs (shared experts first)
+    and at the start of its combine, so that the expert GEMMs' time comes from the
+    timed steps. The layer launches each kernel so that it may begin while the one
+    before it finishes; the kernel right after an event does not, so these events
+    cost those steps a little.
     Then, for the breakdown, K more steps with an event at every stage boundary.
     Returns the workload's report, the timed loop's time (max over ranks) and the
     kernels per step."""
@@ -523,7 +525,7 @@ def time_workload(wb: Workbench, steps: int, warmup: int, peaks, peaks_src, loca
     wb.check("during warm-up")
     launches = kernels_per_step(lambda: wb.forward(), dev)
     timer = StepTimer(steps)
-    ffn_ev = [_made_events(2) for _ in range(steps)]
+    ffn_ev = [_made_events(2) for _ in range(0, steps, FFN_EVERY)]
     flush = None
     if flush_buf is not None:
         flush = flush_buf.zero_
@@ -537,9 +539,12 @@ def time_workload(wb: Workbench, steps: int, warmup: int, peaks, peaks_src, loca
     for i in range(steps):
         if flush is not None:
             flush()
-        ev = [None] * (len(STAGES) + 1)
-        ev[FFN_FIRST], ev[FFN_END] = ffn_ev[i]
-        wb.forward(events=ev)
+        if i % FFN_EVERY == 0:
+            ev = [None] * (len(STAGES) + 1)
+            ev[FFN_FIRST], ev[FFN_END] = ffn_ev[i // FFN_EVERY]
+            wb.forward(events=ev)
+        else:
+            wb.forward()
     e1.record(stream)
     torch.cuda.synchronize()
     barrier(world)
