@@ -13,19 +13,19 @@
 // The router streams x (T x d) once and is bound by HBM. One cluster of S CTAs
 // (S = 1, 2 or 4) covers 128 tokens; CTA r of the cluster reduces its own share
 // of the d columns (a split of K), so that small batches still spread over the
-// SMs. Per CTA, 320 threads:
-//   warp 0      TMA producer: 128 x 64 slices of x and EPAD x 64 slices of W_r
-//               (rows >= E read as zeros), 128-byte swizzle, a ring of stages.
-//   warp 1      TMEM owner and MMA issuer (M = 128, N = EPAD, K = 16 per MMA).
-//   warps 2..9  epilogue.
+// SMs. Per CTA, 576 threads:
+//   warp 0       TMA producer: 128 x 64 slices of x and EPAD x 64 slices of W_r
+//                (rows >= E read as zeros), 128-byte swizzle, a ring of stages.
+//   warp 1       TMEM owner and MMA issuer (M = 128, N = EPAD, K = 16 per MMA).
+//   warps 2..17  epilogue.
 // The epilogue parks each CTA's fp32 partial logits in its shared memory; after a
 // cluster barrier, CTA r takes tokens [r * 128/S, (r+1) * 128/S) and sums the S
 // partials of each in rank order (distributed shared memory), so the result does
-// not depend on timing. G = 2S threads share a token (consecutive lanes), each
-// holding EPAD/G logits in registers: the max, the k argmax rounds (value, then
-// lower expert index), the exp sum and the probability column sums are register
-// work plus fixed shuffle trees. The permute tiles (router_bm(E) tokens) lie
-// inside one CTA's token share, so their histograms and sums need no exchange.
+// not depend on timing. G threads share a token (consecutive lanes, expert columns
+// e = g, g + G, ...): the max and the k argmax rounds (value, then lower expert
+// index) and the exp sum run over shared memory with fixed shuffle trees across
+// the G lanes. The permute tiles (router_bm(E) tokens) lie inside one CTA's token
+// share, so their histograms and sums need no exchange.
 //
 // Noisy top-k gating (youngju.dev (ja) "TopKGating", training mode): W_r and W_noise
 // are stacked on the MMA's N side (EX columns each), so one pass over x gives both
@@ -42,7 +42,7 @@ namespace {
 using namespace tc;
 
 constexpr int kRtM = 128;           // tokens per cluster (the MMA's M)
-constexpr int kRtEpiWarps = 8;
+constexpr int kRtEpiWarps = 16;
 constexpr int kRtEpiThreads = 32 * kRtEpiWarps;
 constexpr int kRtThreads = 64 + kRtEpiThreads;
 constexpr int kRtABytes = kRtM * kBlockK * 2;
@@ -78,7 +78,13 @@ template <int EPAD, int S, bool NOISY> struct RtCfg {
   static constexpr int kStages = kRtRingBudget / kStageBytes < kRtMaxStages
                                      ? kRtRingBudget / kStageBytes : kRtMaxStages;
   static constexpr int kRing = kStages * kStageBytes;
-  static constexpr int kLdp = EPAD + 1;             // partial tile row stride (floats)
+  static constexpr int kTok = kRtM / S;             // tokens of one CTA's epilogue
+  static constexpr int kGmax = kRtEpiThreads / kTok;
+  static constexpr int kG = kGmax < kEx ? kGmax : kEx;  // threads per token
+  // Row stride (floats) of the logit tiles: at least EPAD and congruent to G modulo
+  // 32, so that the 32 / G tokens x G lanes of a warp, reading column g + j G of
+  // their token, hit 32 different banks. A multiple of 4 (G >= 4): 16-byte rows.
+  static constexpr int kLdp = EPAD + ((kG - EPAD) % 32 + 32) % 32;
   static constexpr int kPartBytes = kRtM * kLdp * 4;
   // the share's logits (zb): in place of the partial tile when S = 1, after it when
   // the cluster's other CTAs still read the partials
@@ -86,10 +92,9 @@ template <int EPAD, int S, bool NOISY> struct RtCfg {
   static constexpr int kBody =
       kRing > kPartBytes + kZBytes ? kRing : kPartBytes + kZBytes;
   static constexpr size_t kSmem = (size_t)kBody + sizeof(RtCtl) + 1024;
-  static constexpr int kTok = kRtM / S;             // tokens of one CTA's epilogue
-  static constexpr int kG = kRtEpiThreads / kTok;   // threads per token (2S)
   static constexpr uint32_t kTmemCols = EPAD < 32 ? 32 : EPAD;
-  static_assert(kEx >= kG, "every thread of a token's group owns an expert column");
+  static_assert(kG >= 4 && kG <= 32 && kEx % kG == 0, "token groups");
+  static_assert(kLdp % 4 == 0, "16-byte rows");
   static_assert(kSmem <= 227 * 1024, "shared memory");
 };
 
@@ -119,15 +124,15 @@ __device__ __forceinline__ void rt_sync_all() {
 }
 
 // TMEM -> this CTA's partial tile [128][EPAD] (row stride kLdp). Warp w reads TMEM
-// lanes [32 (w % 4), +32) (its lane quarter); the two warps of a quarter take
-// alternate 32-column chunks.
+// lanes [32 (w % 4), +32) (its lane quarter); the four warps of a quarter take
+// every fourth 32-column chunk. 16-byte stores.
 template <int EPAD, int S, bool NOISY>
 __device__ __forceinline__ void stage_partial(float *part, uint32_t tmem, int warp, int lane) {
   using C = RtCfg<EPAD, S, NOISY>;
   const int q = warp & 3;
   const int h = (warp - 2) >> 2;
   const int r = q * 32 + lane;
-  float *row = part + r * C::kLdp;
+  float4 *row = reinterpret_cast<float4 *>(part + r * C::kLdp);
   const uint32_t tb = tmem + ((uint32_t)(q * 32) << 16);
   if constexpr (EPAD == 16) {
     if (h == 0) {
@@ -135,16 +140,20 @@ __device__ __forceinline__ void stage_partial(float *part, uint32_t tmem, int wa
       tmem_ld16(tb, v);
       tmem_ld_wait();
 #pragma unroll
-      for (int j = 0; j < 16; ++j) row[j] = __uint_as_float(v[j]);
+      for (int j = 0; j < 4; ++j)
+        row[j] = make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
+                             __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]));
     }
   } else {
 #pragma unroll 1
-    for (int c = h; c < EPAD / 32; c += 2) {
+    for (int c = h; c < EPAD / 32; c += 4) {
       uint32_t v[32];
       tmem_ld32(tb + c * 32, v);
       tmem_ld_wait();
 #pragma unroll
-      for (int j = 0; j < 32; ++j) row[c * 32 + j] = __uint_as_float(v[j]);
+      for (int j = 0; j < 8; ++j)
+        row[c * 8 + j] = make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
+                                     __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]));
     }
   }
 }
@@ -176,13 +185,15 @@ __device__ __forceinline__ void group_argmax(float &v, int &i) {
 // logits live in shared memory and every pass is a compact loop: the router's
 // epilogue runs once per call, after the expert GEMMs have flushed its code from
 // L2, so code size (instruction fetch) costs more here than a few shared loads.
-//  1. (token, expert) pairs over all threads, consecutive threads on consecutive
-//     experts: the S partials summed in rank order, the biases, the noise term, the
-//     logits written out (coalesced) and z (NaN and padding -> -inf) kept in zb.
-//  2. G threads per token (consecutive lanes): the max, k argmax rounds (each the
-//     best entry ranked below the previous pick), sum exp(z - max) with exp(z - max)
-//     kept in zb; fixed shuffle trees across the G threads; one thread per token
-//     forms the gates and writes the token's outputs.
+// G threads per token (consecutive lanes), thread g on expert columns g, g + G, ...
+//  1. one pass over the thread's columns, kB at a time: the S partials summed in
+//     rank order, the biases, the noise term, the logits written out, z (NaN and
+//     padding -> -inf) kept in zb, and the best (value, then lower index) entry,
+//     which after a fixed shuffle tree across the G lanes is both the maximum and
+//     the first pick;
+//  2. the other k - 1 argmax rounds (each the best entry ranked below the previous
+//     pick), then sum exp(z - max) with exp(z - max) kept in zb; one thread per
+//     token forms the gates and writes the token's outputs;
 //  3. per permute tile: counts, and (statistics) the probability sums, each column
 //     summed over the tile's tokens in token order, and the sum of lse^2.
 template <int EPAD, int S, bool NOISY>
@@ -194,24 +205,29 @@ __device__ __forceinline__ void epilogue_tokens(const RouterArgs &a, RtCtl *ctl,
   const int E = a.E, T = a.T, k = a.k;
   const int t_base = tile * kRtM + rank * TOK;  // token of this CTA's first row
 
-  // ---- 1. logits. kB pairs per thread at a time: all their loads (the S ranks'
-  // partials) are issued before any of them is used or any zb store is made, since
-  // a store between two loads of the same array keeps them apart.
-  {
-    constexpr int kB = 4;
-    constexpr int kPairs = TOK * EX;
-    const uint32_t part_s = smem_u32(part);
+  if (et < TOK * G) {  // whole warps
+    const int m = et / G, g = et % G;
+    const int t = t_base + m;
+    const bool valid = t < T;
+    const int row = rank * TOK + m;  // the token's row in every rank's partial tile
+    float *zr = zb + m * LD;
+    constexpr int kEpl = EX / G;  // expert columns of this thread
+    constexpr int kB = kEpl < 4 ? kEpl : 4;
+
+    // ---- 1. logits, the maximum and the first pick. All kB columns' loads (the S
+    // ranks' partials) are issued before any is used or any zb store is made, since
+    // a store between two loads of the same array keeps them apart.
+    float bv = -INFINITY;
+    int bi = 0x7fffffff;
+    {
+      const uint32_t part_s = smem_u32(part);
 #pragma unroll 1
-    for (int i0 = et; i0 < kPairs; i0 += kB * kRtEpiThreads) {
-      float acc[kB], accn[kB];
+      for (int j0 = 0; j0 < kEpl; j0 += kB) {
+        float acc[kB], accn[kB];
 #pragma unroll
-      for (int u = 0; u < kB; ++u) {
-        const int i = i0 + u * kRtEpiThreads;
-        acc[u] = 0.f;
-        accn[u] = 0.f;
-        if (i < kPairs) {
-          const int m = i / EX, e = i - m * EX;
-          const int row = rank * TOK + m;
+        for (int u = 0; u < kB; ++u) {
+          const int e = g + (j0 + u) * G;
+          accn[u] = 0.f;
           if constexpr (S == 1) {
             acc[u] = part[row * LD + e];
             if constexpr (NOISY) accn[u] = part[row * LD + EX + e];
@@ -234,46 +250,40 @@ __device__ __forceinline__ void epilogue_tokens(const RouterArgs &a, RtCtl *ctl,
             }
           }
         }
-      }
 #pragma unroll
-      for (int u = 0; u < kB; ++u) {
-        const int i = i0 + u * kRtEpiThreads;
-        if (i >= kPairs) continue;
-        const int m = i / EX, e = i - m * EX;
-        const int t = t_base + m;
-        const bool live = t < T && e < E;
-        float v = acc[u];
-        if (a.b_router) v += ctl->br[e];
-        if (a.logit_bias) v += ctl->lb[e];
-        if constexpr (NOISY) {
-          if (live) {
-            const float sp = accn[u] > 20.f ? accn[u] : log1pf(expf(accn[u]));
-            v = v + sp * a.eps[(size_t)t * E + e];
+        for (int u = 0; u < kB; ++u) {
+          const int e = g + (j0 + u) * G;
+          const bool live = valid && e < E;
+          float v = acc[u];
+          if (a.b_router) v += ctl->br[e];
+          if (a.logit_bias) v += ctl->lb[e];
+          if constexpr (NOISY) {
+            if (live) {
+              const float sp = accn[u] > 20.f ? accn[u] : log1pf(expf(accn[u]));
+              v = v + sp * a.eps[(size_t)t * E + e];
+            }
           }
+          if (a.logits_out != nullptr && live) a.logits_out[(size_t)t * E + e] = v;
+          const float z = (e >= E || v != v) ? -INFINITY : v;  // padding, NaN never win
+          zr[e] = z;
+          if (rt_better(z, e, bv, bi)) { bv = z; bi = e; }
         }
-        if (a.logits_out != nullptr && live) a.logits_out[(size_t)t * E + e] = v;
-        zb[m * LD + e] = (e >= E || v != v) ? -INFINITY : v;  // padding, NaN never win
       }
     }
-  }
-  rt_epi_sync();
+    group_argmax<G>(bv, bi);
+    const float mx = bv;
+    if (g == 0) {
+      ctl->sel_v[m][0] = bv;
+      ctl->sel_i[m][0] = bi;
+    }
 
-  // ---- 2. per token: G consecutive lanes, expert columns e = g, g + G, ...
-  {
-    const int m = et / G, g = et % G;
-    const int t = t_base + m;
-    const bool valid = t < T;
-    float *zr = zb + m * LD;
-    float mx = -INFINITY;
-#pragma unroll 4
-    for (int e = g; e < EX; e += G) mx = fmaxf(mx, zr[e]);
-    mx = group_max<G>(mx);
-    float pv = INFINITY;
-    int pi = -1;
+    // ---- 2. the other picks, the exp sum, the gates
+    float pv = bv;
+    int pi = bi;
 #pragma unroll 1
-    for (int s = 0; s < k; ++s) {
-      float bv = -INFINITY;
-      int bi = 0x7fffffff;
+    for (int s = 1; s < k; ++s) {
+      bv = -INFINITY;
+      bi = 0x7fffffff;
 #pragma unroll 4
       for (int e = g; e < EX; e += G) {
         const float z = zr[e];
@@ -289,8 +299,6 @@ __device__ __forceinline__ void epilogue_tokens(const RouterArgs &a, RtCtl *ctl,
       }
     }
     float ssum = 0.f;
-    constexpr int kEpl = EX / G;  // expert columns of this thread
-    constexpr int kB = kEpl < 4 ? kEpl : 4;
 #pragma unroll 1
     for (int j0 = 0; j0 < kEpl; j0 += kB) {  // kB loads before the kB stores
       float ex[kB];
