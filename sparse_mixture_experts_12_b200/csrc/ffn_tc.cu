@@ -520,7 +520,7 @@ k_ffn_tc2(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
       mbar_init(&ctl->full[s], 1);
       mbar_init(&ctl->empty[s], 1);
     }
-    for (int s = 0; s < PC::kAccBufs; ++s) {
+    for (int s = 0; s < 2; ++s) {  // NH = 1: two accumulators; NH = 2: two N halves
       mbar_init(&ctl->tfull[s], 1);
       mbar_init(&ctl->tempty[s], 2 * kEpiWarps * 32);
     }
@@ -620,39 +620,124 @@ k_ffn_tc2(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
     int stage = 0, acc = 0;
     uint32_t phase = 0, acc_phase = 0;
     bool ok = true, any = false;
-    for (int it = c0; ok && it < work.items; it += cstep) {
-      int sel;
-      work.tile(it, sel);
-      const int h0 = sel < 0 ? 0 : sel, h1 = sel < 0 ? NH : sel + 1;
-      if (!wait_pair(&ctl->tempty[acc], acc_phase ^ 1u, ctl, peer_abort, a.err, 2)) {
-        ok = false;
-        break;
-      }
+    // the MMAs of one K step (one ring stage) for N half h
+    auto issue_half = [&](int st, int kb, int h) {
+      const uint32_t sa = smem_u32(smem + (size_t)st * kSB);
+      const uint64_t da = sw128_desc(sa), db = sw128_desc(sa + kAHalf + h * kBHalf);
+#pragma unroll
+      for (int kk = 0; kk < kBlockK / 16; ++kk)
+        umma_bf16_pair(tmem + (uint32_t)(h * kMmaN), da + 2 * kk, db + 2 * kk, idesc,
+                       (kb | kk) != 0);
+    };
+    // wait for the next stage to fill; returns its index and advances the ring
+    auto next_full = [&](int &st) -> bool {
+      if (!wait_pair(&ctl->full[stage], phase, ctl, peer_abort, a.err, 3)) return false;
       tc_fence_after();
-      const uint32_t d_tmem = tmem + (uint32_t)(acc * kMmaN);
-      for (int kb = 0; kb < nkb; ++kb) {
-        if (!wait_pair(&ctl->full[stage], phase, ctl, peer_abort, a.err, 3)) {
+      st = stage;
+      if (++stage == kS) { stage = 0; phase ^= 1u; }
+      return true;
+    };
+    if constexpr (NH == 2) {
+      // The accumulator's two N halves are handed over one at a time. At the end of
+      // a tile, half 0 of the last kS K steps is issued before half 1, so the
+      // epilogue drains half 0 while half 1 finishes; at the start of the next tile,
+      // half 0 of its first kS K steps runs as soon as half 0 is drained, while the
+      // epilogue drains half 1. Tiles of one N half (sel >= 0) run in plain order.
+      const bool split = nkb >= 2 * kS;
+      for (int it = c0; ok && it < work.items; it += cstep) {
+        int sel;
+        work.tile(it, sel);
+        if (!wait_pair(&ctl->tempty[0], acc_phase ^ 1u, ctl, peer_abort, a.err, 2)) {
+          ok = false;
+          break;
+        }
+        if (sel >= 0 || !split) {
+          if (!wait_pair(&ctl->tempty[1], acc_phase ^ 1u, ctl, peer_abort, a.err, 2)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          for (int kb = 0; kb < nkb; ++kb) {
+            int st;
+            if (!(ok = next_full(st))) break;
+            if (sel != 1) issue_half(st, kb, 0);
+            if (sel != 0) issue_half(st, kb, 1);
+            any = true;
+            umma_commit_pair_both(&ctl->empty[st]);
+          }
+          if (!ok) break;
+        } else {
+          tc_fence_after();
+          const int s0 = stage;
+          for (int kb = 0; kb < kS; ++kb) {  // head: half 0 only
+            int st;
+            if (!(ok = next_full(st))) break;
+            issue_half(st, kb, 0);
+            any = true;
+          }
+          if (!ok) break;
+          if (!wait_pair(&ctl->tempty[1], acc_phase ^ 1u, ctl, peer_abort, a.err, 2)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          for (int kb = 0; kb < kS; ++kb) {  // head: half 1, releasing the stages
+            const int st = (s0 + kb) % kS;
+            issue_half(st, kb, 1);
+            umma_commit_pair_both(&ctl->empty[st]);
+          }
+          for (int kb = kS; kb < nkb - kS; ++kb) {  // body: both halves per stage
+            int st;
+            if (!(ok = next_full(st))) break;
+            issue_half(st, kb, 0);
+            issue_half(st, kb, 1);
+            umma_commit_pair_both(&ctl->empty[st]);
+          }
+          if (!ok) break;
+          const int s1 = stage;
+          for (int kb = nkb - kS; kb < nkb; ++kb) {  // tail: half 0 first ...
+            int st;
+            if (!(ok = next_full(st))) break;
+            issue_half(st, kb, 0);
+          }
+          if (!ok) break;
+          umma_commit_pair_both(&ctl->tfull[0]);  // ... handed to the epilogue
+          for (int kb = nkb - kS; kb < nkb; ++kb) {
+            const int st = (s1 + kb - (nkb - kS)) % kS;
+            issue_half(st, kb, 1);
+            umma_commit_pair_both(&ctl->empty[st]);
+          }
+          umma_commit_pair_both(&ctl->tfull[1]);
+          acc_phase ^= 1u;
+          continue;
+        }
+        umma_commit_pair_both(&ctl->tfull[0]);
+        umma_commit_pair_both(&ctl->tfull[1]);
+        acc_phase ^= 1u;
+      }
+    } else {
+      for (int it = c0; ok && it < work.items; it += cstep) {
+        if (!wait_pair(&ctl->tempty[acc], acc_phase ^ 1u, ctl, peer_abort, a.err, 2)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint32_t sa = smem_u32(smem + (size_t)stage * kSB);
-        const uint64_t da = sw128_desc(sa);
+        const uint32_t d_tmem = tmem + (uint32_t)(acc * kMmaN);
+        for (int kb = 0; kb < nkb; ++kb) {
+          int st;
+          if (!(ok = next_full(st))) break;
+          const uint32_t sa = smem_u32(smem + (size_t)st * kSB);
+          const uint64_t da = sw128_desc(sa), db = sw128_desc(sa + kAHalf);
 #pragma unroll
-        for (int kk = 0; kk < kBlockK / 16; ++kk)
-#pragma unroll
-          for (int h = 0; h < NH; ++h)  // unrolled and predicated: a runtime loop here
-            if (h >= h0 && h < h1)      // measured ~7% slower
-              umma_bf16_pair(d_tmem + (uint32_t)(h * kMmaN), da + 2 * kk,
-                             sw128_desc(sa + kAHalf + h * kBHalf) + 2 * kk, idesc,
-                             (kb | kk) != 0);
-        any = true;
-        umma_commit_pair_both(&ctl->empty[stage]);
-        if (++stage == kS) { stage = 0; phase ^= 1u; }
+          for (int kk = 0; kk < kBlockK / 16; ++kk)
+            umma_bf16_pair(d_tmem, da + 2 * kk, db + 2 * kk, idesc, (kb | kk) != 0);
+          any = true;
+          umma_commit_pair_both(&ctl->empty[st]);
+        }
+        if (!ok) break;
+        umma_commit_pair_both(&ctl->tfull[acc]);
+        if (++acc == PC::kAccBufs) { acc = 0; acc_phase ^= 1u; }
       }
-      if (!ok) break;
-      umma_commit_pair_both(&ctl->tfull[acc]);
-      if (++acc == PC::kAccBufs) { acc = 0; acc_phase ^= 1u; }
     }
     if (!ok && any) {  // retire the MMAs in flight before TMEM is released
       umma_commit_pair_own(&ctl->drain);
@@ -666,37 +751,53 @@ k_ffn_tc2(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUten
     uint8_t *stage_out = smem + PC::kRing + (warp - 4) * kStageOutBytes;
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int it = c0; it < work.items; it += cstep) {
+    bool ok = true;
+    for (int it = c0; ok && it < work.items; it += cstep) {
       int sel, g, n, m;
       decode_tile(work.tile(it, sel), ppre, G, a.n_tiles, g, n, m);
-      bool ok = wait_pair(&ctl->tfull[acc], acc_phase, ctl, peer_abort, a.err, 4);
-      __syncwarp();
-      if (!__all_sync(0xffffffffu, ok)) break;
-      tc_fence_after();
       const int grow = m * kPairM + (int)rank * kTileM + ew * 32 + lane;
       const bool valid = grow < offs[g + 1] - offs[g];
       const size_t orow = (size_t)offs[g] + grow;
-      const uint32_t tbase = tmem + ((uint32_t)(ew * 32) << 16) + (uint32_t)(acc * kMmaN);
       const bool rows_full = __all_sync(0xffffffffu, valid);
       const EpiStore st{a.tma_store ? &tmO : nullptr, stage_out, rows_full,
                         (int)(orow - (size_t)lane)};
-      if (NH == 1) {  // the two warps sharing a lane quarter take half the columns each
+      if constexpr (NH == 2) {
+        // N half 0, then N half 1, each drained by all eight warps (the two warps of
+        // a lane quarter take half of its columns each) and released on its own
+        const uint32_t tbase = tmem + ((uint32_t)(ew * 32) << 16);
+        for (int h = 0; h < 2; ++h) {
+          ok = wait_pair(&ctl->tfull[h], acc_phase, ctl, peer_abort, a.err, 4);
+          __syncwarp();
+          if (!(ok = __all_sync(0xffffffffu, ok))) break;
+          tc_fence_after();
+          if (sel < 0 || sel == h) {
+            if (EPI == EPI_SWIGLU)
+              epilogue_tile<EPI>(a, tbase, g, h * kMmaN, n * kMmaN + h * (kMmaN / 2), 2 * half,
+                                 2 * half + 2, valid, orow, st);
+            else
+              epilogue_tile<EPI>(a, tbase, g, h * kMmaN, (2 * n + h) * kMmaN, 4 * half,
+                                 4 * half + 4, valid, orow, st);
+          }
+          tc_fence_before();
+          mbar_arrive_cluster(tempty0 + (uint32_t)(h * sizeof(uint64_t)));
+        }
+        acc_phase ^= 1u;
+      } else {
+        ok = wait_pair(&ctl->tfull[acc], acc_phase, ctl, peer_abort, a.err, 4);
+        __syncwarp();
+        if (!(ok = __all_sync(0xffffffffu, ok))) break;
+        tc_fence_after();
+        const uint32_t tbase = tmem + ((uint32_t)(ew * 32) << 16) + (uint32_t)(acc * kMmaN);
+        // the two warps sharing a lane quarter take half the columns each
         if (EPI == EPI_SWIGLU)
           epilogue_tile<EPI>(a, tbase, g, 0, n * (kMmaN / 2), 2 * half, 2 * half + 2, valid, orow,
                              st);
         else
           epilogue_tile<EPI>(a, tbase, g, 0, n * kMmaN, 4 * half, 4 * half + 4, valid, orow, st);
-      } else if (sel < 0 || sel == half) {  // ... or one N half (256 columns) each
-        if (EPI == EPI_SWIGLU)
-          epilogue_tile<EPI>(a, tbase, g, half * kMmaN, n * kMmaN + half * (kMmaN / 2), 0, 4,
-                             valid, orow, st);
-        else
-          epilogue_tile<EPI>(a, tbase, g, half * kMmaN, (2 * n + half) * kMmaN, 0, 8, valid,
-                             orow, st);
+        tc_fence_before();
+        mbar_arrive_cluster(tempty0 + (uint32_t)(acc * sizeof(uint64_t)));
+        if (++acc == PC::kAccBufs) { acc = 0; acc_phase ^= 1u; }
       }
-      tc_fence_before();
-      mbar_arrive_cluster(tempty0 + (uint32_t)(acc * sizeof(uint64_t)));
-      if (++acc == PC::kAccBufs) { acc = 0; acc_phase ^= 1u; }
     }
     if (a.tma_store && lane == 0) bulk_wait_all();  // this warp's output stores are done
     __syncwarp();
