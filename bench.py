@@ -626,6 +626,9 @@ def run_ours(args, wl, rank, world, local_rank):
         small = _working_set_bytes(swl) < L2_BYTES
         srep, _, _ = time_workload(swb, args.steps, args.warmup, peaks, peaks_src, local_rank,
                                    world, flush_buf if small else None)
+        srep["roofline"]["traffic"] = _traffic(swl.name)
+        if swl.n_shared and srep["roofline"]["traffic"] is not None:
+            srep["roofline"]["traffic_scope"] = "routed experts only (the shared ones not captured)"
         side[name] = srep
         del swb
         torch.cuda.empty_cache()
