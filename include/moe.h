@@ -154,8 +154,9 @@ typedef struct {
 /* Bytes of workspace every entry point needs for `cfg`. */
 moe_status_t moe_workspace_size(const moe_cfg_t *cfg, size_t *bytes);
 
-/* Zero the workspace header (the sticky device error word). Call once after
- * allocating a workspace. */
+/* Zero the workspace header (the sticky device error word, and the ticket word
+ * that the permute step's scan CTAs share; every launch leaves it at zero again).
+ * Call once after allocating a workspace. */
 moe_status_t moe_workspace_init(void *ws, size_t ws_bytes, moe_stream_t stream);
 
 /* Router + selection + gates ("GatingNetwork"/"TopKGating"/"SwitchRouter").

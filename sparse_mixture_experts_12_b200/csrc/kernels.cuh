@@ -39,6 +39,8 @@ struct ScanArgs {
   int T, k;
   float alpha;
   int32_t *sh_tbl;             // [4] or nullptr: {0, T, 0, ceil(T/kRowTile)} for the shared experts
+  unsigned *ticket;            // zero-initialised word shared by the scan's CTAs (it returns to
+                               // zero after every launch), or nullptr: one CTA does the scan
 };
 
 struct ScatterArgs {

@@ -59,7 +59,7 @@ Layout layout_for(const moe_cfg_t &c) {
   // rows of the expert-contiguous buffers: T*k (token choice) or E*C (expert choice)
   const size_t R = ec ? E * C : T * k;
   size_t sz[B_NBUF];
-  sz[B_ERR] = 2 * sizeof(int32_t);
+  sz[B_ERR] = 4 * sizeof(int32_t);  // error code, its info, the scan's ticket, spare
   sz[B_TILE_COUNTS] = E * NT * 4;
   sz[B_TILE_BASE] = E * NT * 4;
   sz[B_TILE_P] = E * NT * 4;
@@ -106,6 +106,12 @@ size_t layout_size(const Layout &L, Buf b) {
 template <typename P>
 P *at(void *ws, const Layout &L, Buf b) {
   return reinterpret_cast<P *>(static_cast<char *>(ws) + L.off[b]);
+}
+
+// The scan's ticket word: the third word of the workspace header (after the sticky
+// error code and its info), zeroed by moe_workspace_init.
+unsigned *scan_ticket(void *ws, const Layout &L) {
+  return reinterpret_cast<unsigned *>(at<int32_t>(ws, L, B_ERR) + 2);
 }
 
 bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
@@ -602,6 +608,7 @@ MOE_API moe_status_t moe_permute(const moe_cfg_t *cfg, const void *x, const int3
   int32_t *tile_counts = at<int32_t>(ws, L, B_TILE_COUNTS);
   MOE_CUDA(launch_tile_counts(topk_idx, c.n_tokens, c.top_k, c.n_experts, tile_counts, err, stream));
   ScanArgs s{};
+  s.ticket = scan_ticket(ws, L);
   s.tile_counts = tile_counts;
   s.tile_base = at<int32_t>(ws, L, B_TILE_BASE);
   s.counts = counts;
@@ -705,6 +712,7 @@ MOE_API moe_status_t moe_aux_stats(const moe_cfg_t *cfg, const float *logits,
   int32_t *tile_counts = at<int32_t>(ws, L, B_TILE_COUNTS);
   MOE_CUDA(launch_tile_counts(topk_idx, c.n_tokens, c.top_k, c.n_experts, tile_counts, err, stream));
   ScanArgs s{};
+  s.ticket = scan_ticket(ws, L);
   s.tile_counts = tile_counts;
   s.tile_base = at<int32_t>(ws, L, B_TILE_BASE);
   s.counts = at<int32_t>(ws, L, B_COUNTS);
@@ -808,6 +816,7 @@ moe_status_t forward_impl(const moe_cfg_t *cfg, const moe_weights_t *w, const vo
   // 2. scan: counts, capacity, offsets, GEMM tile table (+ aux statistics)
   MOE_TRY(sg.enter(MOE_STAGE_SCAN));
   ScanArgs s{};
+  s.ticket = scan_ticket(ws, L);
   s.tile_counts = r.tile_counts;
   s.tile_base = at<int32_t>(ws, L, B_TILE_BASE);
   s.counts = counts;
@@ -985,6 +994,7 @@ MOE_API moe_status_t moe_route_shard(const moe_cfg_t *cfg, const moe_weights_t *
   // the shard's assignments per expert before any drop (offsets etc. to scratch)
   const int NT = ceil_div(c.n_tokens, router_bm(c.n_experts));
   ScanArgs s{};
+  s.ticket = scan_ticket(ws, L);
   s.tile_counts = r.tile_counts;
   s.tile_base = at<int32_t>(ws, L, B_TILE_BASE);
   s.counts = counts;
@@ -1023,6 +1033,7 @@ MOE_API moe_status_t moe_permute_shard(const moe_cfg_t *cfg, const moe_shard_t *
   int32_t *tile_counts = at<int32_t>(ws, L, B_TILE_COUNTS);
   MOE_CUDA(launch_tile_counts(topk_idx, c.n_tokens, c.top_k, c.n_experts, tile_counts, err, stream));
   ScanArgs s{};
+  s.ticket = scan_ticket(ws, L);
   s.tile_counts = tile_counts;
   s.tile_base = at<int32_t>(ws, L, B_TILE_BASE);
   s.counts = counts;

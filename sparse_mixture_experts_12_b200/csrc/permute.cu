@@ -28,71 +28,32 @@ __device__ __forceinline__ int warp_incl_scan(int v) {
   return v;
 }
 
-constexpr int kScanThreads = 1024;
+constexpr int kScanThreads = 256;
+constexpr int kScanWarps = kScanThreads / 32;
 constexpr int kScanVPL = 8;  // tiles per lane per batch (loads issued together)
 
-// One CTA. Warp per expert: exclusive prefix of the expert's per-tile counts over
-// the token tiles (tile_counts is [E][NT], so a warp reads consecutive tiles).
-// Then one warp: counts, capacity, kept-row offsets and the 128-row tile prefix
-// over the experts. Optionally the load-balancing statistics (fixed-order sums).
+// Warp per expert, eight experts per CTA and E / 8 CTAs (one CTA looping over all
+// experts when there is no ticket word): the exclusive prefix of the expert's
+// per-tile counts over the token tiles (tile_counts is [E][NT], so a warp reads
+// consecutive tiles), its pre-drop count and (statistics) its probability sum.
+// The last CTA to finish (an atomic ticket that wraps back to zero, so nothing
+// waits) then does counts, capacity, kept-row offsets and the 128-row tile prefix
+// over the experts, and the load-balancing statistics (fixed-order sums).
 // SHARD: the tokens are one shard of a larger batch; expert e keeps at most
 // max(0, cap - pairs routed to e by the earlier shards), written to sc.cap_e.
 template <bool SHARD>
 __global__ void __launch_bounds__(kScanThreads) k_scan(ScanArgs a, ShardCaps sc) {
-  __shared__ int count_s[kMaxExperts];
-  __shared__ float P_s[kMaxExperts];
-  __shared__ float red[kScanThreads / 32];
+  __shared__ float red[kScanWarps];
+  __shared__ int last_s;
   pdl_wait();
   pdl_trigger();
   const int E = a.E, NT = a.NT;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  constexpr int nw = kScanThreads / 32;
-  if (NT <= 32 * kScanVPL) {
-    // one batch of tiles per expert: the next expert's counts and probability sums
-    // are requested before this expert's are scanned, so a warp's experts overlap
-    // their load latencies instead of paying one each
-    const bool want_p = a.aux_out != nullptr;
-    int v[kScanVPL], vn[kScanVPL];
-    float pv[kScanVPL], pn[kScanVPL];
-    auto fetch = [&](int e, int (&cv)[kScanVPL], float (&cp)[kScanVPL]) {
-#pragma unroll
-      for (int j = 0; j < kScanVPL; ++j) {
-        const int t = j * 32 + lane;
-        const bool in = e < E && t < NT;
-        cv[j] = in ? a.tile_counts[(size_t)e * NT + t] : 0;
-        cp[j] = (want_p && in) ? a.tile_p[(size_t)e * NT + t] : 0.f;
-      }
-    };
-    fetch(warp, v, pv);
-    for (int e = warp; e < E; e += nw) {
-      fetch(e + nw, vn, pn);
-      int32_t *tb = a.tile_base + (size_t)e * NT;
-      int run = 0;
-      float p = 0.f;
-#pragma unroll
-      for (int j = 0; j < kScanVPL; ++j) {
-        const int incl = warp_incl_scan(v[j]);
-        const int t = j * 32 + lane;
-        if (t < NT) tb[t] = run + incl - v[j];
-        run += __shfl_sync(0xffffffffu, incl, 31);
-        p += pv[j];
-      }
-      if (lane == 0) count_s[e] = run;
-      if (want_p) {
-        p = warp_sum(p);
-        if (lane == 0) P_s[e] = p / (float)a.T;
-      }
-#pragma unroll
-      for (int j = 0; j < kScanVPL; ++j) {
-        v[j] = vn[j];
-        pv[j] = pn[j];
-      }
-    }
-  } else {
-  for (int e = warp; e < E; e += nw) {
+  const bool want_p = a.aux_out != nullptr;
+  for (int e = blockIdx.x * kScanWarps + warp; e < E; e += gridDim.x * kScanWarps) {
     const int32_t *tc = a.tile_counts + (size_t)e * NT;
     int32_t *tb = a.tile_base + (size_t)e * NT;
-    const float *tp = a.aux_out ? a.tile_p + (size_t)e * NT : nullptr;
+    const float *tp = want_p ? a.tile_p + (size_t)e * NT : nullptr;
     int run = 0;
     float p = 0.f;  // this lane's tiles t = lane, lane + 32, ... in order
     for (int b0 = 0; b0 < NT; b0 += 32 * kScanVPL) {
@@ -114,14 +75,24 @@ __global__ void __launch_bounds__(kScanThreads) k_scan(ScanArgs a, ShardCaps sc)
         p += pv[j];
       }
     }
-    if (lane == 0) count_s[e] = run;
-    if (tp != nullptr) {
-      p = warp_sum(p);
-      if (lane == 0) P_s[e] = p / (float)a.T;
+    if (want_p) p = warp_sum(p);
+    if (lane == 0) {
+      a.counts[e] = run;
+      if (want_p) a.aux_out[3 + E + e] = p / (float)a.T;
     }
   }
+  if (gridDim.x > 1) {  // only the last CTA goes on, after every CTA's writes
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      __threadfence();
+      last_s = atomicInc(a.ticket, gridDim.x - 1) == gridDim.x - 1;
+    }
+    __syncthreads();
+    if (!last_s) return;
+    __threadfence();
+  } else {
+    __syncthreads();
   }
-  __syncthreads();
   if (warp == 0) {
     // E <= 256: eight experts per lane
     int cnt[8], kept[8], mt[8];
@@ -129,7 +100,7 @@ __global__ void __launch_bounds__(kScanThreads) k_scan(ScanArgs a, ShardCaps sc)
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
       const int e = lane * 8 + j;
-      const int c = e < E ? count_s[e] : 0;
+      const int c = e < E ? __ldcg(a.counts + e) : 0;
       cnt[j] = c;
       int cap = a.cap;
       if constexpr (SHARD) {
@@ -183,11 +154,10 @@ __global__ void __launch_bounds__(kScanThreads) k_scan(ScanArgs a, ShardCaps sc)
     const double inv_tk = 1.0 / ((double)a.T * (double)a.k);
     double fp = 0.0, bsq = 0.0;
     for (int e = lane; e < E; e += 32) {
-      const double f = (double)count_s[e] * inv_tk;
-      fp += f * (double)P_s[e];
+      const double f = (double)__ldcg(a.counts + e) * inv_tk;
+      fp += f * (double)__ldcg(a.aux_out + 3 + E + e);
       bsq += (f - 1.0 / E) * (f - 1.0 / E);
       a.aux_out[3 + e] = (float)f;
-      a.aux_out[3 + E + e] = P_s[e];
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
@@ -196,7 +166,7 @@ __global__ void __launch_bounds__(kScanThreads) k_scan(ScanArgs a, ShardCaps sc)
     }
     if (lane == 0) {
       float zs = 0.f;
-      for (int w = 0; w < nw; ++w) zs += red[w];
+      for (int w = 0; w < kScanWarps; ++w) zs += red[w];
       a.aux_out[0] = (float)((double)a.alpha * E * fp);
       a.aux_out[1] = zs / (float)a.T;
       a.aux_out[2] = (float)bsq;
@@ -219,11 +189,20 @@ __global__ void __launch_bounds__(kScatterThreads) k_scatter(ScatterArgs a, cons
   const int NC = ceil_div(bm * k, 32);
   int32_t *hist = sh;               // [NC][E]
   int32_t *prow = hist + NC * E;    // [bm*k]: in-chunk rank, then the destination row
+  int32_t *base = prow + bm * k;    // [E]: this tile's base rank in each expert
+  int32_t *first = base + E;        // [E]: the expert's first row (offsets)
+  int32_t *capv = first + E;        // [E]: the pairs the expert may keep
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int32_t *idx = a.topk_idx + (size_t)t0 * k;
   pdl_wait();
   pdl_trigger();
 
+  // the per-expert values of phase 3, requested now: they do not depend on idx
+  for (int e = tid; e < E; e += kScatterThreads) {
+    base[e] = a.tile_base[(size_t)e * NT + tile];
+    first[e] = a.offsets[e];
+    capv[e] = a.cap < 0 ? INT_MAX : (SHARD ? cap_e[e] : a.cap);
+  }
   for (int i = tid; i < NC * E; i += kScatterThreads) hist[i] = 0;
   __syncthreads();
   for (int c = warp; c < NC; c += kScatterThreads / 32) {
@@ -252,9 +231,9 @@ __global__ void __launch_bounds__(kScatterThreads) k_scatter(ScatterArgs a, cons
     if (e < 0 || e >= E) {
       report_error(a.err, MOE_DEVERR_EXPERT_INDEX, t0 * k + p);
     } else {
-      const int rank = a.tile_base[(size_t)e * NT + tile] + hist[(p / 32) * E + e] + prow[p];
-      if (a.cap < 0 || rank < (SHARD ? cap_e[e] : a.cap)) {
-        row = a.offsets[e] + rank;
+      const int rank = base[e] + hist[(p / 32) * E + e] + prow[p];
+      if (rank < capv[e]) {
+        row = first[e] + rank;
         a.perm[row] = t;
       }
     }
@@ -300,10 +279,13 @@ __global__ void __launch_bounds__(kScatterThreads) k_scatter(ScatterArgs a, cons
 
 // ------------------------------------------------------------------- combine
 // A warp per token. Each lane takes NB 16-byte vectors of the row per batch and
-// requests every kept slot's vectors (and the shared-expert row) before using
-// any, so a warp keeps NB x k loads in flight; KMAX bounds k (register budget).
-template <typename T, int KMAX, int NB>
-__global__ void __launch_bounds__(256) k_combine(CombineArgs a) {
+// requests every kept slot's vectors (and, SHARED, the shared-expert row) before
+// using any, so a warp keeps NB x k loads in flight; KMAX bounds k (register
+// budget). A token whose every slot was dropped (and that has no shared-expert
+// row) is written as zeros without loading or converting anything: in a layer
+// with tight capacity (Switch keeps 1721 of 16384 tokens) that is most of them.
+template <typename T, int KMAX, int NB, bool SHARED>
+__global__ void __launch_bounds__(256, SHARED ? 2 : (KMAX <= 2 ? 4 : 3)) k_combine(CombineArgs a) {
   constexpr int VE = Elem<T>::kPerVec;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t = blockIdx.x * 8 + warp;
@@ -330,6 +312,16 @@ __global__ void __launch_bounds__(256) k_combine(CombineArgs a) {
   const T *yp = static_cast<const T *>(a.y_perm);
   T *y = static_cast<T *>(a.y);
   const int nvec = a.d / VE;
+  if (!SHARED) {
+    bool any = false;
+#pragma unroll
+    for (int s = 0; s < KMAX; ++s) any |= row[s] >= 0;
+    if (!any) {
+      uint4 *dst = reinterpret_cast<uint4 *>(y + (size_t)t * a.d);
+      for (int v = lane; v < nvec; v += 32) dst[v] = make_uint4(0u, 0u, 0u, 0u);
+      return;
+    }
+  }
   for (int v0 = lane; v0 < nvec; v0 += 32 * NB) {
     // a dropped slot reads nothing and contributes zero
     uint4 u[KMAX][NB];
@@ -342,8 +334,8 @@ __global__ void __launch_bounds__(256) k_combine(CombineArgs a) {
                       ? __ldg(reinterpret_cast<const uint4 *>(yp + (size_t)row[s] * a.d) + v)
                       : make_uint4(0u, 0u, 0u, 0u);
       }
-    float4 sh[NB][VE / 4];
-    if (a.shared_y) {
+    float4 sh[SHARED ? NB : 1][VE / 4];
+    if (SHARED) {
 #pragma unroll
       for (int b = 0; b < NB; ++b) {
         const int v = v0 + 32 * b;
@@ -368,10 +360,10 @@ __global__ void __launch_bounds__(256) k_combine(CombineArgs a) {
 #pragma unroll
         for (int i = 0; i < VE; ++i) acc[i] = fmaf(g[s], f[i], acc[i]);
       }
-      if (a.shared_y) {
+      if (SHARED) {
 #pragma unroll
         for (int i = 0; i < VE; i += 4) {
-          const float4 q = sh[b][i / 4];
+          const float4 q = sh[SHARED ? b : 0][i / 4];
           acc[i] += q.x; acc[i + 1] += q.y; acc[i + 2] += q.z; acc[i + 3] += q.w;
         }
       }
@@ -415,12 +407,18 @@ __global__ void k_tile_table(const int32_t *offsets, int G, int max_rows, int32_
 
 }  // namespace
 
+// E / 8 CTAs with a ticket word, else one CTA over all experts
+unsigned scan_grid(const ScanArgs &a) {
+  return a.ticket != nullptr ? (unsigned)ceil_div(a.E, kScanWarps) : 1u;
+}
+
 cudaError_t launch_scan(const ScanArgs &a, cudaStream_t st) {
-  return launch_pdl(k_scan<false>, dim3(1), dim3(kScanThreads), 0, st, a, ShardCaps{});
+  return launch_pdl(k_scan<false>, dim3(scan_grid(a)), dim3(kScanThreads), 0, st, a,
+                    ShardCaps{});
 }
 
 cudaError_t launch_scan_shard(const ScanArgs &a, const ShardCaps &sc, cudaStream_t st) {
-  k_scan<true><<<1, kScanThreads, 0, st>>>(a, sc);
+  k_scan<true><<<scan_grid(a), kScanThreads, 0, st>>>(a, sc);
   return cudaGetLastError();
 }
 
@@ -431,7 +429,7 @@ cudaError_t scatter(const ScatterArgs &a, const int32_t *cap_e, cudaStream_t st)
   const int bm = router_bm(a.E);
   const int NT = ceil_div(a.T, bm);
   const int NC = ceil_div(bm * a.k, 32);
-  const size_t smem = (size_t)(NC * a.E + bm * a.k) * sizeof(int32_t);
+  const size_t smem = (size_t)(NC * a.E + bm * a.k + 3 * a.E) * sizeof(int32_t);
   return launch_pdl(k_scatter<SHARD>, dim3(NT), dim3(kScatterThreads), smem, st, a, cap_e);
 }
 }  // namespace
@@ -449,12 +447,19 @@ cudaError_t launch_combine(const CombineArgs &a, int dtype, cudaStream_t st) {
   const int grid = ceil_div(a.T, 8);
   const bool f32 = dtype == MOE_DTYPE_F32;
   const dim3 g(grid), b(256);
+  const bool sh = a.shared_y != nullptr;
   if (a.k <= 2) {
-    if (f32) return launch_pdl(k_combine<float, 2, 4>, g, b, 0, st, a);
-    return launch_pdl(k_combine<__nv_bfloat16, 2, 4>, g, b, 0, st, a);
+    if (f32)
+      return sh ? launch_pdl(k_combine<float, 2, 4, true>, g, b, 0, st, a)
+                : launch_pdl(k_combine<float, 2, 4, false>, g, b, 0, st, a);
+    return sh ? launch_pdl(k_combine<__nv_bfloat16, 2, 4, true>, g, b, 0, st, a)
+              : launch_pdl(k_combine<__nv_bfloat16, 2, 4, false>, g, b, 0, st, a);
   }
-  if (f32) return launch_pdl(k_combine<float, kMaxTopK, 1>, g, b, 0, st, a);
-  return launch_pdl(k_combine<__nv_bfloat16, kMaxTopK, 1>, g, b, 0, st, a);
+  if (f32)
+    return sh ? launch_pdl(k_combine<float, kMaxTopK, 1, true>, g, b, 0, st, a)
+              : launch_pdl(k_combine<float, kMaxTopK, 1, false>, g, b, 0, st, a);
+  return sh ? launch_pdl(k_combine<__nv_bfloat16, kMaxTopK, 1, true>, g, b, 0, st, a)
+            : launch_pdl(k_combine<__nv_bfloat16, kMaxTopK, 1, false>, g, b, 0, st, a);
 }
 
 cudaError_t launch_tile_table(const int32_t *offsets, int G, int max_rows, int32_t *mprefix,
