@@ -6,9 +6,9 @@
 // token rows on its N side (more rows are handled as further 32-row chunks), so a
 // tile costs 4 small MMAs per 64-wide K slice and the kernel is bound by reading
 // the weights. The down projection splits
-// K across CTAs when there are too few (expert, 128-row) tiles to occupy every
-// SM; the splits write fp32 partial sums that a reduction kernel adds in a fixed
-// order.
+// K across CTAs, as many splits (up to 16) as it takes to even out the tiles of
+// the persistent grid's CTAs when there are few (expert, 128-row) tiles; the
+// splits write fp32 partial sums that a reduction kernel adds in a fixed order.
 //
 // Tile = (expert g, 32-row chunk c of its rows, 128 weight rows n, K split s). Warp 0: TMA producer
 // (weight rows of W_gate [and W_up] + the expert's 32 activation rows per stage),
@@ -33,7 +33,7 @@ constexpr int kXBytes = kSwapN * kBlockK * 2;    // the token slice (4 KB)
 constexpr int kSwapStageBytes = 2 * kWBytes + kXBytes;
 constexpr int kSwapThreads = 256;
 constexpr int kSwapTmemCols = 128;               // 2 buffers x (gate 32 | up 32)
-constexpr int kMaxSplit = 8;
+constexpr int kMaxSplit = 16;
 
 enum { SW_SWIGLU = 0, SW_ACT = 1, SW_DOWN = 2 };
 enum { OUT_BF16 = 0, OUT_F32 = 1, OUT_PARTIAL = 2 };
@@ -346,8 +346,19 @@ cudaError_t launch_ffn_tc_decode(const GroupedFfnArgs &a, cudaStream_t st) {
   if (!make_map(&mx, a.h, (uint64_t)a.a_rows, (uint64_t)a.F, kSwapN)) return cudaErrorInvalidValue;
   const int nkb = ceil_div(a.F, kBlockK);
   const long long units = touched_ub * ceil_div(a.d, kSwapM);
-  int splits = (int)std::min<long long>(kMaxSplit, std::max<long long>(1, ceil_div(2 * sm_count(), (int)units)));
-  splits = std::min(splits, nkb);
+  // K splits: the fewest that bring the K slices of the busiest CTA (whole tiles
+  // over the persistent grid) to within 3 % of the best count up to kMaxSplit, so
+  // that a last, partly filled wave of tiles does not leave a few CTAs streaming
+  // alone (Mixtral T = 1: 64 weight blocks, 9 splits -> 576 tiles, 4 per CTA)
+  const long long sms = sm_count();
+  auto busiest = [&](int sp) {
+    const int kb = ceil_div(nkb, sp);
+    return (double)((units * sp + sms - 1) / sms) * kb;
+  };
+  double best = 1e300;
+  for (int sp = 1; sp <= std::min(kMaxSplit, nkb); ++sp) best = std::min(best, busiest(sp));
+  int splits = 1;
+  while (splits < std::min(kMaxSplit, nkb) && busiest(splits) > 1.03 * best) ++splits;
   const int kbps = ceil_div(nkb, splits);
   splits = ceil_div(nkb, kbps);  // every split gets at least one K slice
   const bool partial = splits > 1 && a.part != nullptr;
