@@ -43,6 +43,8 @@ import torch  # noqa: E402
 from sparse_mixture_experts_12_b200 import synth  # noqa: E402
 
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# datasheet dense peaks of a B200 (HGX), reported beside the measured denominators
+NOMINAL_PEAKS = {"hbm_gbs": 7700.0, "bf16_tflops": 2250.0}
 METRIC = "MoE-layer tokens/s"
 STAGES = ("route", "scan", "permute", "shared_ffn", "expert_ffn", "combine")
 # the workloads reported under "workloads" after the headline one (bench --workloads all)
@@ -371,6 +373,9 @@ def ffn_roofline(wl, work, ffn_ms, peaks, peaks_src):
         roof = {"bound": "hbm", "achieved": byts / (ffn_ms * 1e-3) / 1e9,
                 "peak": peaks["hbm_gbs"], "unit": "GB/s", "peak_source": f"{peaks_src} (copy)"}
     roof["frac"] = roof["achieved"] / roof["peak"]
+    nominal = NOMINAL_PEAKS["bf16_tflops" if roof["bound"] == "tensor" else "hbm_gbs"]
+    roof["nominal_peak"] = nominal
+    roof["frac_of_nominal"] = roof["achieved"] / nominal
     roof["ms_per_step"] = ffn_ms
     roof["algorithmic"] = {"flops": flops, "bytes": byts}
     return roof

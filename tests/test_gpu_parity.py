@@ -219,6 +219,9 @@ FFN_CASES = [
     ("relu_bf16_decode_ntail", synth.ACT_RELU, synth.DT_BF16, 192, 192, 2, [1, 12]),
     # still the small-batch path, with an expert spanning two 32-row chunks
     ("swiglu_bf16_decode_chunks", synth.ACT_SWIGLU, synth.DT_BF16, 256, 384, 2, [33, 20]),
+    # at most 8 rows in all (decode T = 1..4)
+    ("swiglu_bf16_decode_tiny", synth.ACT_SWIGLU, synth.DT_BF16, 256, 384, 2, [1, 1]),
+    ("swiglu_bf16_decode_tiny_k", synth.ACT_SWIGLU, synth.DT_BF16, 512, 384, 3, [1, 0, 1]),
     ("gelu_bf16_decode_chunks", synth.ACT_GELU, synth.DT_BF16, 128, 256, 2, [45, 10]),
     # 190..256 rows in all: one or two 128-row tiles per expert
     ("swiglu_bf16_medium", synth.ACT_SWIGLU, synth.DT_BF16, 256, 384, 5, [0, 1, 129, 60, 30]),
