@@ -131,6 +131,9 @@ k_ffn_swap(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUte
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  // the kernel after this one may be placed as soon as SMs free up; it waits for
+  // this grid before it reads anything this grid writes
+  pdl_trigger();
   const uint32_t tmem = ctl->tmem_base;
   const int per_expert = a.n_blocks * a.splits;
   const int total = cpre[G] * per_expert;
@@ -146,6 +149,26 @@ k_ffn_swap(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUte
     int stage = 0;
     uint32_t phase = 0, issued = 0, last_phase = 0;
     bool ok = true;
+    // The weights and the tile tables (from the routing, which has completed before
+    // the kernel ahead of this one passed its own wait) do not depend on the kernel
+    // ahead: the first stages' weight slices are requested before waiting for it.
+    // The activation rows (its output) only after the wait.
+    int early = 0;
+    for (int tile = blockIdx.x; early < kSwapStages && tile < total; tile += gridDim.x) {
+      int g, nn, ch;
+      decode_tile(tile, cpre, G, per_expert, g, nn, ch);
+      const int nb = nn / a.splits, sp = nn % a.splits;
+      const int kb0 = sp * a.kb_per_split, kb1 = min(nkb, kb0 + a.kb_per_split);
+      const int wrow = g * a.w_rows + nb * kSwapM;
+      for (int kb = kb0; kb < kb1 && early < kSwapStages; ++kb, ++early) {
+        uint8_t *sw = smem + (size_t)early * kSwapStageBytes;
+        mbar_expect_tx(&ctl->full[early], kTxBytes);
+        tma_load_2d(&tmW, &ctl->full[early], sw, kb * kBlockK, wrow);
+        if (kTwo) tma_load_2d(&tmW3, &ctl->full[early], sw + kWBytes, kb * kBlockK, wrow);
+      }
+    }
+    pdl_wait();
+    int step = 0;
     for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
       int g, nn, ch;
       decode_tile(tile, cpre, G, per_expert, g, nn, ch);
@@ -153,12 +176,21 @@ k_ffn_swap(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUte
       const int kb0 = sp * a.kb_per_split, kb1 = min(nkb, kb0 + a.kb_per_split);
       const int wrow = g * a.w_rows + nb * kSwapM;
       const int xrow = offs[g] + ch * kSwapN;
-      for (int kb = kb0; kb < kb1; ++kb) {
-        if (!wait_swap(&ctl->empty[stage], phase ^ 1u, ctl, a.err, 11)) { ok = false; break; }
+      for (int kb = kb0; kb < kb1; ++kb, ++step) {
+        // the first `early` stages are free (first use) and already carry their weight
+        // copies: they get their activation copies whatever happens, so that every
+        // copy issued completes its stage's barrier
+        if (step >= early &&
+            !wait_swap(&ctl->empty[stage], phase ^ 1u, ctl, a.err, 11)) {
+          ok = false;
+          break;
+        }
         uint8_t *sw = smem + (size_t)stage * kSwapStageBytes;
-        mbar_expect_tx(&ctl->full[stage], kTxBytes);
-        tma_load_2d(&tmW, &ctl->full[stage], sw, kb * kBlockK, wrow);
-        if (kTwo) tma_load_2d(&tmW3, &ctl->full[stage], sw + kWBytes, kb * kBlockK, wrow);
+        if (step >= early) {
+          mbar_expect_tx(&ctl->full[stage], kTxBytes);
+          tma_load_2d(&tmW, &ctl->full[stage], sw, kb * kBlockK, wrow);
+          if (kTwo) tma_load_2d(&tmW3, &ctl->full[stage], sw + kWBytes, kb * kBlockK, wrow);
+        }
         tma_load_2d(&tmX, &ctl->full[stage], sw + 2 * kWBytes, kb * kBlockK, xrow);
         issued |= 1u << stage;
         last_phase = (last_phase & ~(1u << stage)) | (phase << stage);
@@ -272,6 +304,8 @@ __global__ void __launch_bounds__(256) k_splitk_reduce(const float *__restrict__
                                                        size_t part_stride,
                                                        const int32_t *__restrict__ offsets, int G,
                                                        int N, void *out, int out_f32) {
+  pdl_wait();
+  pdl_trigger();
   const size_t n = (size_t)offsets[G] * N;
   for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
        i += (size_t)gridDim.x * blockDim.x) {
@@ -298,8 +332,8 @@ cudaError_t launch_swap(const CUtensorMap &mw, const CUtensorMap &mw3, const CUt
     attr_done[dev & 63] = true;
   }
   const int grid = (int)std::max<long long>(1, std::min<long long>(tiles_ub, sm_count()));
-  k_ffn_swap<EPI><<<grid, kSwapThreads, kSwapSmemBytes, st>>>(mw, mw3, mx, s);
-  return cudaGetLastError();
+  return launch_pdl(k_ffn_swap<EPI>, dim3(grid), dim3(kSwapThreads), kSwapSmemBytes, st, mw, mw3,
+                    mx, s);
 }
 
 }  // namespace
@@ -376,9 +410,9 @@ cudaError_t launch_ffn_tc_decode(const GroupedFfnArgs &a, cudaStream_t st) {
   s.out_mode = partial ? OUT_PARTIAL : (a.out_f32 ? OUT_F32 : OUT_BF16);
   e = launch_swap<SW_DOWN>(mw, mw, mx, s, touched_ub * s.n_blocks * splits, st);
   if (e != cudaSuccess || !partial) return e;
-  k_splitk_reduce<<<std::min(ceil_div(a.a_rows * a.d, 256), 4 * sm_count()), 256, 0, st>>>(
-      a.part, splits, s.part_stride, a.offsets, a.G, a.d, a.out, a.out_f32);
-  return cudaGetLastError();
+  return launch_pdl(k_splitk_reduce, dim3(std::min(ceil_div(a.a_rows * a.d, 256), 4 * sm_count())),
+                    dim3(256), 0, st, (const float *)a.part, splits, s.part_stride, a.offsets, a.G,
+                    a.d, a.out, a.out_f32);
 }
 
 }  // namespace moe
