@@ -263,9 +263,11 @@ k_ffn_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtens
     tmem_alloc(&ctl->tmem_base, kTmemCols);
     tmem_relinquish();
   }
-  // the set-up above overlaps the previous kernel; the tile tables, the operands
-  // and the outputs are touched only after it has completed
-  if (a.pdl_mode == PDL_WAIT) pdl_wait();
+  // The set-up above overlaps the previous kernel. So do the tile tables: they come
+  // from the routing, which completed before the kernel ahead of this one passed its
+  // own wait (or, in a standalone call, from the table kernel, which does not let
+  // this grid start early), and the first stages' weight slices. The producer waits
+  // for the kernel ahead before it requests the activation rows (its output).
   for (int i = tid; i <= G; i += kThreads1) {
     if (a.tile_mode != TILES_TAIL_ONLY) mpre[i] = a.mprefix[i];
     offs[i] = a.offsets[i];
@@ -307,32 +309,53 @@ k_ffn_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtens
     uint32_t phase = 0;
     uint32_t issued = 0, last_phase = 0;  // per-stage bit sets, for the end-of-role drain
     bool ok = true;
+    auto load_b = [&](int st, int kb, int brow) {
+      uint8_t *sb = smem + (size_t)st * kStageBytes + kABytes;
+      tma_load_2d(&tmB, &ctl->full[st], sb, kb * kBlockK, brow);
+      if (EPI == EPI_SWIGLU)
+        tma_load_2d(&tmB3, &ctl->full[st], sb + kBBytes / 2, kb * kBlockK, brow);
+    };
+    // test hook: the CTA's first stage is never loaded, so the MMA issuer's wait on it
+    // (and then the producer's wait for that stage to drain) runs out
+    auto withheld = [&](int tile, int kb) {
+      return a.withhold_load && tile == (int)blockIdx.x && kb == 0;
+    };
+    // the first stages' weight slices, before the wait for the kernel ahead
+    int early = 0;
+    for (int tile = blockIdx.x; early < kStages && tile < total; tile += gridDim.x) {
+      int g, n, m;
+      decode_tile(tile, mpre, G, a.n_tiles, g, n, m);
+      const int brow = g * a.b_rows + n * kBStep;
+      for (int kb = 0; kb < nkb && early < kStages; ++kb, ++early) {
+        if (withheld(tile, kb)) continue;
+        mbar_expect_tx(&ctl->full[early], kStageBytes);
+        load_b(early, kb, brow);
+      }
+    }
+    if (a.pdl_mode == PDL_WAIT) pdl_wait();
+    int step = 0;
     for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
       int g, n, m;
       decode_tile(tile, mpre, G, a.n_tiles, g, n, m);
       if (a.tile_mode == TILES_TAIL_ONLY) m = ceil_div(offs[g + 1] - offs[g], kTileM) - 1;
       const int arow = offs[g] + m * kTileM;
       const int brow = g * a.b_rows + n * kBStep;
-      for (int kb = 0; kb < nkb; ++kb) {
-        if (!wait_bounded(&ctl->empty[stage], phase ^ 1u, ctl, a.err, 1, true,
-                          a.wait_limit_ns)) {
+      for (int kb = 0; kb < nkb; ++kb, ++step) {
+        // the first `early` stages are free (first use) and already carry their weight
+        // copies: they get their activation copies whatever happens, so that every
+        // copy issued completes its stage's barrier
+        if (step >= early && !wait_bounded(&ctl->empty[stage], phase ^ 1u, ctl, a.err, 1,
+                                           true, a.wait_limit_ns)) {
           ok = false;
           break;
         }
-        // test hook: the CTA's first stage is never loaded, so the MMA issuer's wait
-        // on it (and then the producer's wait for that stage to drain) runs out
-        const bool withhold = a.withhold_load && tile == (int)blockIdx.x && kb == 0;
-        if (!withhold) {
+        if (!withheld(tile, kb)) {
           uint8_t *sa = smem + (size_t)stage * kStageBytes;
-          uint8_t *sb = sa + kABytes;
-          mbar_expect_tx(&ctl->full[stage], kStageBytes);
-          tma_load_2d(&tmA, &ctl->full[stage], sa, kb * kBlockK, arow);
-          if (EPI == EPI_SWIGLU) {
-            tma_load_2d(&tmB, &ctl->full[stage], sb, kb * kBlockK, brow);
-            tma_load_2d(&tmB3, &ctl->full[stage], sb + kBBytes / 2, kb * kBlockK, brow);
-          } else {
-            tma_load_2d(&tmB, &ctl->full[stage], sb, kb * kBlockK, brow);
+          if (step >= early) {
+            mbar_expect_tx(&ctl->full[stage], kStageBytes);
+            load_b(stage, kb, brow);
           }
+          tma_load_2d(&tmA, &ctl->full[stage], sa, kb * kBlockK, arow);
           issued |= 1u << stage;
           last_phase = (last_phase & ~(1u << stage)) | (phase << stage);
         }
