@@ -12,7 +12,8 @@ namespace moe {
 
 namespace {
 
-constexpr int BM = kRowTile, BN = 64, BK = 16;
+constexpr int BM = kRowTile, BN = 64, BK = 32;
+constexpr int kAPer = BM * BK / 256, kBPer = BN * BK / 256;  // slice elements per thread
 constexpr int TM = 8, TN = 4;  // per-thread micro tile; (BM/TM)*(BN/TN) = 256 threads
 
 struct SimtGemm {
@@ -71,18 +72,38 @@ __global__ void __launch_bounds__(256) k_simt_gemm(SimtGemm s) {
       acc[i][j] = 0.f;
       if (kSwiGLU) acc3[i][j] = 0.f;
     }
-  for (int k0 = 0; k0 < s.K; k0 += BK) {
-    for (int i = tid; i < BM * BK; i += 256) {
-      const int m = i / BK, kk = i % BK;
-      As[kk][m] = (m < nrows && k0 + kk < s.K) ? s.a[(size_t)(row0 + m) * s.K + k0 + kk] : 0.f;
+  // the next K slice is read from global memory into registers while this one is
+  // multiplied out of shared memory (rows of 32 consecutive K values per 32 threads)
+  float ra[kAPer], rb[kBPer], rb3[kSwiGLU ? kBPer : 1];
+  auto fetch = [&](int k0) {
+#pragma unroll
+    for (int j = 0; j < kAPer; ++j) {
+      const int i = tid + 256 * j, m = i / BK, kk = i % BK;
+      ra[j] = (m < nrows && k0 + kk < s.K) ? s.a[(size_t)(row0 + m) * s.K + k0 + kk] : 0.f;
     }
-    for (int i = tid; i < BN * BK; i += 256) {
-      const int n = i / BK, kk = i % BK;
+#pragma unroll
+    for (int j = 0; j < kBPer; ++j) {
+      const int i = tid + 256 * j, n = i / BK, kk = i % BK;
       const bool ok = n0 + n < s.N && k0 + kk < s.K;
-      Bs[kk][n] = ok ? bw[(size_t)(n0 + n) * s.K + k0 + kk] : 0.f;
-      if (kSwiGLU) B3s[kk][n] = ok ? bw3[(size_t)(n0 + n) * s.K + k0 + kk] : 0.f;
+      rb[j] = ok ? bw[(size_t)(n0 + n) * s.K + k0 + kk] : 0.f;
+      if (kSwiGLU) rb3[j] = ok ? bw3[(size_t)(n0 + n) * s.K + k0 + kk] : 0.f;
+    }
+  };
+  fetch(0);
+  for (int k0 = 0; k0 < s.K; k0 += BK) {
+#pragma unroll
+    for (int j = 0; j < kAPer; ++j) {
+      const int i = tid + 256 * j;
+      As[i % BK][i / BK] = ra[j];
+    }
+#pragma unroll
+    for (int j = 0; j < kBPer; ++j) {
+      const int i = tid + 256 * j;
+      Bs[i % BK][i / BK] = rb[j];
+      if (kSwiGLU) B3s[i % BK][i / BK] = rb3[j];
     }
     __syncthreads();
+    if (k0 + BK < s.K) fetch(k0 + BK);
 #pragma unroll
     for (int kk = 0; kk < BK; ++kk) {
       float av[TM], bv[TN], bv3[TN];
