@@ -153,11 +153,26 @@ __global__ void __launch_bounds__(kScanThreads) k_scan(ScanArgs a, ShardCaps sc)
     // fixed shuffle tree
     const double inv_tk = 1.0 / ((double)a.T * (double)a.k);
     double fp = 0.0, bsq = 0.0;
-    for (int e = lane; e < E; e += 32) {
-      const double f = (double)__ldcg(a.counts + e) * inv_tk;
-      fp += f * (double)__ldcg(a.aux_out + 3 + E + e);
-      bsq += (f - 1.0 / E) * (f - 1.0 / E);
-      a.aux_out[3 + e] = (float)f;
+    // E <= 256: the lane's (up to) eight experts' counts and probability sums are all
+    // requested before any f is stored into aux_out (a store there would keep the
+    // next loads of the same array behind it)
+    int cnt[8];
+    float pe[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int e = lane + 32 * j;
+      cnt[j] = e < E ? __ldcg(a.counts + e) : 0;
+      pe[j] = e < E ? __ldcg(a.aux_out + 3 + E + e) : 0.f;
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int e = lane + 32 * j;
+      if (e < E) {
+        const double f = (double)cnt[j] * inv_tk;
+        fp += f * (double)pe[j];
+        bsq += (f - 1.0 / E) * (f - 1.0 / E);
+        a.aux_out[3 + e] = (float)f;
+      }
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
@@ -192,12 +207,21 @@ __global__ void __launch_bounds__(kScatterThreads) k_scatter(ScatterArgs a, cons
   int32_t *base = prow + bm * k;    // [E]: this tile's base rank in each expert
   int32_t *first = base + E;        // [E]: the expert's first row (offsets)
   int32_t *capv = first + E;        // [E]: the pairs the expert may keep
+  int32_t *eidx = capv + E;         // [bm*k]: the routing indices of the tile
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  constexpr int kWarps = kScatterThreads / 32;
   const int32_t *idx = a.topk_idx + (size_t)t0 * k;
   pdl_wait();
   pdl_trigger();
 
-  // the per-expert values of phase 3, requested now: they do not depend on idx
+  // the tile's routing indices (at most two 32-pair chunks per warp: bm * k <= 512)
+  // and the per-expert values of phase 3 are all requested before the first barrier
+  int ev[2];
+#pragma unroll
+  for (int u = 0; u < 2; ++u) {
+    const int p = (warp + u * kWarps) * 32 + lane;
+    ev[u] = (p < P) ? idx[p] : -1;
+  }
   for (int e = tid; e < E; e += kScatterThreads) {
     base[e] = a.tile_base[(size_t)e * NT + tile];
     first[e] = a.offsets[e];
@@ -205,10 +229,13 @@ __global__ void __launch_bounds__(kScatterThreads) k_scatter(ScatterArgs a, cons
   }
   for (int i = tid; i < NC * E; i += kScatterThreads) hist[i] = 0;
   __syncthreads();
-  for (int c = warp; c < NC; c += kScatterThreads / 32) {
+#pragma unroll
+  for (int u = 0; u < 2; ++u) {
+    const int c = warp + u * kWarps;
+    if (c >= NC) break;
     const int p = c * 32 + lane;
-    int e = (p < P) ? idx[p] : -1;
-    if (e < 0 || e >= E) e = -1;
+    if (p < P) eidx[p] = ev[u];
+    const int e = (ev[u] < 0 || ev[u] >= E) ? -1 : ev[u];
     const unsigned peers = __match_any_sync(0xffffffffu, e);
     const int within = __popc(peers & ((1u << lane) - 1u));
     if (e >= 0 && within == 0) hist[c * E + e] = __popc(peers);
@@ -225,7 +252,7 @@ __global__ void __launch_bounds__(kScatterThreads) k_scatter(ScatterArgs a, cons
   }
   __syncthreads();
   for (int p = tid; p < P; p += kScatterThreads) {
-    const int e = idx[p];
+    const int e = eidx[p];
     const int t = t0 + p / k;
     int row = -1;
     if (e < 0 || e >= E) {
@@ -429,7 +456,8 @@ cudaError_t scatter(const ScatterArgs &a, const int32_t *cap_e, cudaStream_t st)
   const int bm = router_bm(a.E);
   const int NT = ceil_div(a.T, bm);
   const int NC = ceil_div(bm * a.k, 32);
-  const size_t smem = (size_t)(NC * a.E + bm * a.k + 3 * a.E) * sizeof(int32_t);
+  if (bm * a.k > 2 * kScatterThreads) return cudaErrorInvalidValue;  // two chunks per warp
+  const size_t smem = (size_t)(NC * a.E + 2 * bm * a.k + 3 * a.E) * sizeof(int32_t);
   return launch_pdl(k_scatter<SHARD>, dim3(NT), dim3(kScatterThreads), smem, st, a, cap_e);
 }
 }  // namespace
