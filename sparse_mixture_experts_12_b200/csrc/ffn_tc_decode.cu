@@ -16,6 +16,7 @@
 // warps 4..7: epilogue (TMEM lane = weight row, columns = tokens), writing
 // h[token][row] (coalesced across the warp's lanes) or the fp32 partials.
 #include <algorithm>
+#include <atomic>
 
 #include "tc_ptx.cuh"
 
@@ -321,15 +322,15 @@ __global__ void __launch_bounds__(256) k_splitk_reduce(const float *__restrict__
 template <int EPI>
 cudaError_t launch_swap(const CUtensorMap &mw, const CUtensorMap &mw3, const CUtensorMap &mx,
                         const SwapArgs &s, long long tiles_ub, cudaStream_t st) {
-  static bool attr_done[64] = {};
+  static std::atomic<bool> attr_done[64];  // idempotent: a racing second call sets the same value
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  if (!attr_done[dev & 63]) {
+  if (!attr_done[dev & 63].load(std::memory_order_acquire)) {
     e = cudaFuncSetAttribute(k_ffn_swap<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)kSwapSmemBytes);
     if (e != cudaSuccess) return e;
-    attr_done[dev & 63] = true;
+    attr_done[dev & 63].store(true, std::memory_order_release);
   }
   const int grid = (int)std::max<long long>(1, std::min<long long>(tiles_ub, sm_count()));
   return launch_pdl(k_ffn_swap<EPI>, dim3(grid), dim3(kSwapThreads), kSwapSmemBytes, st, mw, mw3,

@@ -7,6 +7,8 @@
 // top-k renormalised (youngju.dev ja "TopKGating"), softmax then top-1 raw
 // (SwitchRouter). Top-k is taken on the fp32 logits in every mode; equal logits
 // go to the lower expert index first.
+#include <atomic>
+
 #include "kernels.cuh"
 
 namespace moe {
@@ -338,14 +340,14 @@ k_router(RouterArgs a) {
 template <typename ET, int EPAD>
 cudaError_t launch_router_t(const RouterArgs &a, cudaStream_t st) {
   const int smem = RouterSmem<EPAD>::bytes(sizeof(ET));
-  static bool attr_done[64] = {};
+  static std::atomic<bool> attr_done[64];  // idempotent: a racing second call sets the same value
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  if (!attr_done[dev & 63]) {  // idempotent: a racing second call sets the same value
+  if (!attr_done[dev & 63].load(std::memory_order_acquire)) {
     e = cudaFuncSetAttribute(k_router<ET, EPAD>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    attr_done[dev & 63] = true;
+    attr_done[dev & 63].store(true, std::memory_order_release);
   }
   const int NT = ceil_div(a.T, RouterShape<EPAD>::BM);
   k_router<ET, EPAD><<<NT, kRouterThreads, smem, st>>>(a);
