@@ -139,6 +139,10 @@ SMALL = {
     "decode_small": MIXTRAL_PREFILL.replace(name="decode_small", T=5, d_model=256, d_ff=384),
     "deepseek_decode": DEEPSEEK_FINE.replace(name="deepseek_decode", T=20, d_model=256, d_ff=256,
                                              d_ff_shared=384),
+    # a small batch whose down projection splits K: the combine reads its partials
+    # and adds the shared experts' row
+    "deepseek_decode_split": DEEPSEEK_FINE.replace(name="deepseek_decode_split", T=20,
+                                                   d_model=128, d_ff=512, d_ff_shared=384),
     "decode_chunks": MIXTRAL_PREFILL.replace(name="decode_chunks", T=64, d_model=256, d_ff=384,
                                              n_experts=2, top_k=1),
     # SwiGLU experts with a capacity of 112 rows each
