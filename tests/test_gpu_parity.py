@@ -243,14 +243,40 @@ FFN_CASES = [
 ]
 
 
+# Capacity-limited layers (name, act, d, F, E, rows per expert, capacity): experts
+# at and below the capacity, the 128-row tiles of the single-CTA kernel split over
+# a capacity of 131-160 rows, and an expert given more rows than the capacity
+# (moe_expert_ffn takes any offsets).
+FFN_CAP_CASES = [
+    ("gelu_bf16_cap160", synth.ACT_GELU, 128, 320, 4, [5, 160, 0, 131], 160),
+    ("swiglu_bf16_cap128", synth.ACT_SWIGLU, 256, 384, 5, [0, 1, 128, 77, 40], 128),
+    ("relu_bf16_cap_over", synth.ACT_RELU, 192, 192, 3, [200, 17, 96], 96),
+    ("gelu_bf16_cap_long_k", synth.ACT_GELU, 1024, 4096, 3, [150, 3, 100], 160),
+]
+
+
 @pytest.mark.parametrize("name,act,dt,d,F,E,rows", FFN_CASES, ids=[c[0] for c in FFN_CASES])
 def test_expert_ffn_matches_oracle(name, act, dt, d, F, E, rows):
+    _expert_ffn_case(name, act, dt, d, F, E, rows)
+
+
+@pytest.mark.parametrize("name,act,d,F,E,rows,cap", FFN_CAP_CASES,
+                         ids=[c[0] for c in FFN_CAP_CASES])
+def test_expert_ffn_capacity_layers_match_oracle(name, act, d, F, E, rows, cap):
+    _expert_ffn_case(name, act, synth.DT_BF16, d, F, E, rows, cap=cap)
+
+
+def _expert_ffn_case(name, act, dt, d, F, E, rows, cap=None):
     R = int(sum(rows))
     k = 2
     T = (R + k - 1) // k + 3  # x_perm holds T*k rows; the tail rows are unused
+    # capacity floor(cf * T * k / E) == cap
+    cf = 0.0 if cap is None else (cap + 0.5) * E / (T * k)
     wl = synth.Workload(name, T=T, d_model=d, n_experts=E, top_k=k, d_ff=F, act=act,
                         gate_mode=0, dtype=dt, expert_bias=act != synth.ACT_SWIGLU,
-                        bias_std=0.3)
+                        bias_std=0.3, capacity_factor=cf)
+    if cap is not None:
+        assert O.capacity(cf, T, k, E) == cap
     inp = synth.generate(wl, seed=R)
     layer = B.MoELayer(wl, inp, DEV)
     g = torch.Generator().manual_seed(R + 1)
