@@ -109,6 +109,24 @@ cudaError_t launch_ec_combine(const void *y_perm, const int32_t *slot, const flo
                               int T, int E, int C, int d, int dtype, void *y, cudaStream_t st);
 
 cudaError_t launch_router(const RouterArgs &a, int dtype, cudaStream_t st);
+// Decode-sized batches (bf16, at most 8 tokens and 32 experts, no noise and no
+// statistics): the router and the scan's layout in one launch (route_small.cu). The
+// router arguments' tile_counts are not written: the layout comes with the routing.
+// Up to 8 tokens the one CTA beats the tensor-core router and the scan (measured:
+// decode T = 1 -5 %, T = 8 -1 % per layer call); at 32 tokens it is slower (+2.4 %).
+constexpr int kSmallRouteMaxT = 8;
+constexpr int kSmallRouteMaxE = 32;
+struct SmallRouteArgs {
+  RouterArgs r;
+  int cap;              // rows per expert kept, < 0: unlimited
+  int32_t *counts;      // [E]
+  int32_t *offsets;     // [E+1] prefix of the kept rows
+  int32_t *mprefix;     // [E+1] prefix of ceil(kept_e / kRowTile)
+  int32_t *tile_base;   // [E] the permute step's per-tile bases (one token tile: zero)
+  int32_t *sh_tbl;      // [4] or nullptr: {0, T, 0, ceil(T/kRowTile)} for the shared experts
+};
+bool small_route_supported(const RouterArgs &a);
+cudaError_t launch_route_small(const SmallRouteArgs &a, cudaStream_t st);
 // noisy top-k gating: z[i] += softplus(zn[i]) * eps[i] over n logits
 cudaError_t launch_noisy_logits(float *z, const float *zn, const float *eps, size_t n,
                                 cudaStream_t st);

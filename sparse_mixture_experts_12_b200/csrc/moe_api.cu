@@ -805,7 +805,20 @@ moe_status_t forward_impl(const moe_cfg_t *cfg, const moe_weights_t *w, const vo
   r.k = c.top_k;
   r.gate_mode = c.gate_mode;
   r.err = err;
-  if (noise != nullptr) {
+  // decode-sized batches: the router also lays out the experts (no scan kernel)
+  const bool small = noise == nullptr && sh == nullptr && c.dtype == MOE_DTYPE_BF16 &&
+                     small_route_supported(r);
+  if (small) {
+    SmallRouteArgs sr{};
+    sr.r = r;
+    sr.cap = capacity_of(c);
+    sr.counts = counts;
+    sr.offsets = offsets;
+    sr.mprefix = mprefix;
+    sr.tile_base = at<int32_t>(ws, L, B_TILE_BASE);
+    sr.sh_tbl = c.n_shared > 0 ? sh_tbl : nullptr;
+    MOE_CUDA(launch_route_small(sr, stream));
+  } else if (noise != nullptr) {
     MOE_TRY(route_noisy(c, w, x, *noise, r, logits, ws, L, stream));
   } else if (sh == nullptr) {
     MOE_CUDA(launch_router(r, c.dtype, stream));
@@ -833,7 +846,9 @@ moe_status_t forward_impl(const moe_cfg_t *cfg, const moe_weights_t *w, const vo
   s.alpha = c.aux_alpha;
   s.sh_tbl = c.n_shared > 0 ? sh_tbl : nullptr;
   ShardCaps sc{};
-  if (sh == nullptr) {
+  if (small) {
+    // laid out by the router
+  } else if (sh == nullptr) {
     MOE_CUDA(launch_scan(s, stream));
   } else {
     s.cap = capacity_for_tokens(c, sh->n_tokens_total);

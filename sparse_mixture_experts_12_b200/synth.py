@@ -145,6 +145,13 @@ SMALL = {
                                                    d_model=128, d_ff=512, d_ff_shared=384),
     "decode_chunks": MIXTRAL_PREFILL.replace(name="decode_chunks", T=64, d_model=256, d_ff=384,
                                              n_experts=2, top_k=1),
+    # decode-sized batches routed in one launch: capacity drops (cap 4 of 8 x 3
+    # pairs over 6 experts), and 32 experts with top-8, router and logit biases
+    "decode_cap": MIXTRAL_PREFILL.replace(name="decode_cap", T=8, d_model=256, d_ff=384,
+                                          n_experts=6, top_k=3, capacity_factor=1.0),
+    "decode_e32": DEEPSEEK_FINE.replace(name="decode_e32", T=8, d_model=192, d_ff=128,
+                                        n_experts=32, top_k=8, n_shared=1, d_ff_shared=128,
+                                        router_bias=True, bias_std=0.1, logit_bias_std=0.5),
     # SwiGLU experts with a capacity of 112 rows each
     "mixtral_cap": MIXTRAL_PREFILL.replace(name="mixtral_cap", T=900, d_model=256, d_ff=384,
                                            capacity_factor=0.5),

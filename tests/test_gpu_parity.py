@@ -395,15 +395,16 @@ NOISE_OFFSET = 7
 
 
 def _forward_and_compare(wl: synth.Workload, seed: int, n_sample=None, check_full_routing=True,
-                         noise_seed=None):
+                         noise_seed=None, with_aux=True):
     """noise_seed (noisy workloads): the library draws the noise for (noise_seed,
     NOISE_OFFSET) and the oracle the same counter-based draws; otherwise the noise is
-    a seeded input both sides read."""
+    a seeded input both sides read. with_aux=False: the forward without the
+    load-balancing statistics (the path of a layer that does not ask for them)."""
     inp = synth.generate(wl, seed=seed)
     layer = B.MoELayer(wl, inp, DEV)
     x = inp["x"].to(DEV)
     taps = layer.new_taps()
-    aux = layer.new_aux()
+    aux = layer.new_aux() if with_aux else None
     eps = e64 = None
     if wl.noisy and noise_seed is None:
         eps = synth.noise_draws(wl.T, wl.n_experts, seed + 99)
@@ -489,12 +490,12 @@ def _forward_and_compare(wl: synth.Workload, seed: int, n_sample=None, check_ful
     keep = np.array([t not in affected for t in sel])
     yg = y.cpu().to(torch.float64).numpy()[sel]
     err = H.max_rel_err(yg[keep], yref[keep])
-    # aux statistics (f from the forward's own routing)
-    a = aux.cpu().numpy().astype(np.float64)
-    f, Pm, auxv = O.aux_stats(r["logits"], r["idx"], E, k, wl.aux_alpha)
-    assert np.abs(a[3:3 + E] - f).max() <= len(mism) / (T * k) + 1e-7
-    assert np.allclose(a[3 + E:], Pm, rtol=1e-4, atol=1e-6)
-    assert abs(a[0] - auxv) <= 1e-4 * auxv + wl.aux_alpha * E * len(mism) / (T * k)
+    if with_aux:  # aux statistics (f from the forward's own routing)
+        a = aux.cpu().numpy().astype(np.float64)
+        f, Pm, auxv = O.aux_stats(r["logits"], r["idx"], E, k, wl.aux_alpha)
+        assert np.abs(a[3:3 + E] - f).max() <= len(mism) / (T * k) + 1e-7
+        assert np.allclose(a[3 + E:], Pm, rtol=1e-4, atol=1e-6)
+        assert abs(a[0] - auxv) <= 1e-4 * auxv + wl.aux_alpha * E * len(mism) / (T * k)
     cover = {}
     if tiles is not None:
         covered = H.tiles_covered(tiles, r["perm"], sel[keep])
@@ -560,6 +561,25 @@ def test_forward_full_size_sampled(name):
     n = None if wl.T <= 64 else 48
     # the noisy layer at full size draws its noise inside the library, as in the benchmark
     _forward_and_compare(wl, seed=0, n_sample=n, noise_seed=2024 if wl.noisy else None)
+    torch.cuda.empty_cache()
+
+
+# Decode-sized batches whose layer asks for no statistics: with at most 8 tokens
+# and 32 experts (bf16) the router also lays out the experts (counts, capacity,
+# offsets, tile table) in the same launch, the path of the benchmark's decode steps
+# at T = 1 and 8; deepseek_decode (64 experts) and T = 32 take the tensor-core
+# router and the scan.
+SMALL_BATCH = ["decode_small", "decode_cap", "decode_e32", "deepseek_decode"]
+
+
+@pytest.mark.parametrize("name", SMALL_BATCH)
+def test_forward_small_batch_without_statistics(name):
+    _forward_and_compare(synth.SMALL[name], seed=0, with_aux=False)
+
+
+@pytest.mark.parametrize("name", ["decode1", "decode8", "decode32"])
+def test_forward_decode_without_statistics(name):
+    _forward_and_compare(synth.WORKLOADS[name], seed=0, with_aux=False)
     torch.cuda.empty_cache()
 
 
