@@ -577,6 +577,29 @@ def test_forward_small_batch_without_statistics(name):
     _forward_and_compare(synth.SMALL[name], seed=0, with_aux=False)
 
 
+# edge shapes of the one-launch decode routing: one expert, k = E, 32 experts with
+# top-8, odd expert counts, a d that leaves most threads without columns, each gate
+# mode, capacity drops
+SMALL_ROUTE_EDGES = [
+    # T, E, k, d, gate mode, capacity factor
+    (1, 1, 1, 64, 0, 0.0),
+    (3, 4, 4, 128, 1, 0.0),
+    (8, 32, 8, 192, 1, 0.0),
+    (7, 17, 5, 64, 2, 0.0),
+    (8, 9, 2, 256, 0, 0.6),   # capacity 1
+    (5, 32, 1, 128, 2, 7.0),  # capacity 1
+]
+
+
+@pytest.mark.parametrize("T,E,k,d,mode,cf", SMALL_ROUTE_EDGES)
+def test_forward_small_batch_routing_edges(T, E, k, d, mode, cf):
+    wl = synth.SMALL["decode_small"].replace(name=f"edge_T{T}_E{E}_k{k}", T=T, n_experts=E,
+                                             top_k=k, d_model=d, d_ff=128, gate_mode=mode,
+                                             capacity_factor=cf, router_bias=True,
+                                             bias_std=0.1, logit_bias_std=0.3)
+    _forward_and_compare(wl, seed=T + E, with_aux=False)
+
+
 @pytest.mark.parametrize("name", ["decode1", "decode8", "decode32"])
 def test_forward_decode_without_statistics(name):
     _forward_and_compare(synth.WORKLOADS[name], seed=0, with_aux=False)
