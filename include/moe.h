@@ -27,9 +27,11 @@
  *   with programmatic stream serialisation: each may begin its set-up while the
  *   kernel before it in the stream finishes, and waits for that kernel before it
  *   reads that kernel's output or writes anything. Before that wait the expert
- *   GEMMs only read the weights and the routing tables of this call (complete by
- *   then: they come from an earlier kernel of the same call, which the kernel
- *   ahead waited for) and request their first weight slices.
+ *   GEMMs only read the weights and the routing tables of this call, and request
+ *   their first weight slices. The tables are complete by then: they come from an
+ *   earlier kernel of the same call that the kernel ahead waited for, or (the
+ *   tile table of moe_expert_ffn) from the kernel ahead itself, which does not let
+ *   its successor begin before it has completed.
  * - Layout: row-major. Weights use the nn.Linear [out_features, in_features]
  *   layout, stacked over experts. Activations, weights, x_perm, y_perm and y are
  *   stored in cfg->dtype (fp32 or bf16); biases, logits, gates are fp32; index
