@@ -333,10 +333,13 @@ def test_shared_experts_through_expert_ffn():
 
 
 # =================================================================== combine
-@pytest.mark.parametrize("dt,with_shared", [(synth.DT_BF16, False), (synth.DT_BF16, True),
-                                            (synth.DT_F32, True)])
-def test_combine_matches_oracle(dt, with_shared):
-    T, k, d = 333, 3, 128
+# k = 1 without a shared row takes the 8-tokens-per-warp kernel (T = 333 leaves a
+# last warp with 5 tokens)
+@pytest.mark.parametrize("dt,with_shared,k", [(synth.DT_BF16, False, 3), (synth.DT_BF16, True, 3),
+                                              (synth.DT_F32, True, 3), (synth.DT_BF16, False, 1),
+                                              (synth.DT_F32, False, 1), (synth.DT_BF16, True, 1)])
+def test_combine_matches_oracle(dt, with_shared, k):
+    T, d = 333, 128
     wl = synth.SMALL["mixtral_small"].replace(T=T, top_k=k, d_model=d, dtype=dt)
     cfg = B.make_cfg(wl)
     ws = _raw_ws(cfg)
