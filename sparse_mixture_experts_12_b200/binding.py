@@ -9,6 +9,7 @@ Function names follow the C ABI in ``include/moe.h``.
 from __future__ import annotations
 
 import ctypes
+import math
 import os
 from typing import Optional
 
@@ -139,6 +140,30 @@ def _check(status: int, where: str):
 
 def _ptr(t: Optional[torch.Tensor]):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def expert_rows(cfg: MoeCfg) -> int:
+    """Rows of the expert-contiguous buffers (x_perm, y_perm) the library reads and
+    writes for this configuration: T * k under token choice, E * C with
+    C = floor(cf * T / E) under expert choice (evaluated in double, as the library
+    does)."""
+    if cfg.routing == synth.ROUTING_EXPERT_CHOICE:
+        if not cfg.capacity_factor > 0:
+            return 0
+        return cfg.n_experts * math.floor(float(cfg.capacity_factor) * cfg.n_tokens /
+                                          cfg.n_experts)
+    return cfg.n_tokens * cfg.top_k
+
+
+def check_rows(t: Optional[torch.Tensor], rows: int, cols: int, name: str):
+    """The C ABI takes raw pointers and cannot see a buffer's size: a tensor with
+    fewer than the `rows` rows of `cols` elements that the library will access is
+    refused here, before anything is launched."""
+    if t is None:
+        return
+    if t.dim() != 2 or t.shape[0] < rows or t.shape[1] != cols or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous [>= {rows}, {cols}] tensor, "
+                         f"not {tuple(t.shape)}")
 
 
 def _stream():
@@ -304,18 +329,23 @@ class MoELayer:
             "moe_route_expert_choice")
 
     def permute(self, x, topk_idx, counts, offsets, perm, inv, x_perm):
+        check_rows(x_perm, expert_rows(self.cfg), self.cfg.d_model, "x_perm")
         _check(self.lib.moe_permute(ctypes.byref(self.cfg), _ptr(x), _ptr(topk_idx), _ptr(counts),
                                     _ptr(offsets), _ptr(perm), _ptr(inv), _ptr(x_perm),
                                     _ptr(self.ws), self.ws.numel(), _stream()), "moe_permute")
 
     def expert_ffn(self, x_perm, offsets, y_perm, cfg: Optional[MoeCfg] = None,
                    weights: Optional[MoeWeights] = None):
+        c = cfg or self.cfg
+        check_rows(x_perm, expert_rows(c), c.d_model, "x_perm")
+        check_rows(y_perm, expert_rows(c), c.d_model, "y_perm")
         _check(self.lib.moe_expert_ffn(ctypes.byref(cfg or self.cfg),
                                        ctypes.byref(weights or self.weights), _ptr(x_perm),
                                        _ptr(offsets), _ptr(y_perm), _ptr(self.ws),
                                        self.ws.numel(), _stream()), "moe_expert_ffn")
 
     def combine(self, y_perm, inv, topk_gate, shared_y, y):
+        check_rows(y_perm, expert_rows(self.cfg), self.cfg.d_model, "y_perm")
         _check(self.lib.moe_combine(ctypes.byref(self.cfg), _ptr(y_perm), _ptr(inv),
                                     _ptr(topk_gate), _ptr(shared_y), _ptr(y), _ptr(self.ws),
                                     self.ws.numel(), _stream()), "moe_combine")
@@ -337,6 +367,7 @@ class MoELayer:
                                         self.ws.numel(), _stream()), "moe_route_shard")
 
     def permute_shard(self, shard: MoeShard, x, topk_idx, counts, offsets, perm, inv, x_perm):
+        check_rows(x_perm, expert_rows(self.cfg), self.cfg.d_model, "x_perm")
         _check(self.lib.moe_permute_shard(ctypes.byref(self.cfg), ctypes.byref(shard), _ptr(x),
                                           _ptr(topk_idx), _ptr(counts), _ptr(offsets),
                                           _ptr(perm), _ptr(inv), _ptr(x_perm), _ptr(self.ws),

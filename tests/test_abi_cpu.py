@@ -8,6 +8,7 @@ import subprocess
 import tempfile
 
 import pytest
+import torch
 
 from sparse_mixture_experts_12_b200 import binding as B
 from sparse_mixture_experts_12_b200 import build as BUILD
@@ -196,3 +197,33 @@ def test_expert_choice_entry_points_reject_before_launching(lib):
     # moe_forward: expert choice produces no load-balancing statistics
     assert lib.moe_forward(ctypes.byref(cfg), ctypes.byref(W), good, good, good, None, ws,
                            ws_bytes, None) == 1
+
+
+# ------------------------------------------------------ buffer sizes in the binding
+def test_binding_expert_rows_follow_the_routing():
+    """x_perm / y_perm hold T*k rows under token choice and E*C under expert choice,
+    C = floor(cf*T/E) (the oracle's expert-choice capacity)."""
+    from sparse_mixture_experts_12_b200 import binding as Bd
+    from oracle import moe_oracle as Or
+    tc = synth.WORKLOADS["mixtral_prefill"]
+    assert Bd.expert_rows(Bd.make_cfg(tc)) == tc.T * tc.top_k
+    ec = synth.WORKLOADS["mixtral_ec"]
+    C = Or.expert_choice_capacity(ec.capacity_factor, ec.T, ec.n_experts)
+    assert Bd.expert_rows(Bd.make_cfg(ec)) == ec.n_experts * C == 8192
+    assert Bd.expert_rows(Bd.make_cfg(ec.replace(capacity_factor=0.0))) == 0
+
+
+def test_binding_refuses_short_expert_buffers():
+    """A tensor with fewer rows than the library will touch is refused before any
+    launch (the C ABI only sees a pointer): an expert-choice layer's x_perm sized for
+    token choice (T*k = 4096 rows instead of E*C = 8192) among them."""
+    from sparse_mixture_experts_12_b200 import binding as Bd
+    ec = synth.WORKLOADS["mixtral_ec"]
+    R, d = Bd.expert_rows(Bd.make_cfg(ec)), ec.d_model
+    Bd.check_rows(torch.empty((R, d)), R, d, "x_perm")
+    Bd.check_rows(torch.empty((R + 5, d)), R, d, "x_perm")
+    Bd.check_rows(None, R, d, "x_perm")
+    for bad in (torch.empty((ec.T * ec.top_k, d)), torch.empty((R, d + 1)),
+                torch.empty((d, R)).t(), torch.empty(R * d)):
+        with pytest.raises(ValueError):
+            Bd.check_rows(bad, R, d, "x_perm")
