@@ -259,6 +259,8 @@ __global__ void __launch_bounds__(256) k_ec_combine(const ET *__restrict__ y_per
   __shared__ float l_g[8][kMaxExperts];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t = blockIdx.x * 8 + warp;
+  pdl_wait();
+  pdl_trigger();
   if (t >= T) return;
   int n = 0;
   for (int e0 = 0; e0 < E; e0 += 32) {
@@ -275,23 +277,24 @@ __global__ void __launch_bounds__(256) k_ec_combine(const ET *__restrict__ y_per
   }
   __syncwarp();
   const int nvec = d / VE;
-  for (int v0 = lane; v0 < nvec; v0 += 64) {
-    float acc[2][VE];
+  constexpr int NB = 4;  // 16-byte vectors of a row per lane and batch
+  for (int v0 = lane; v0 < nvec; v0 += 32 * NB) {
+    float acc[NB][VE];
 #pragma unroll
-    for (int b = 0; b < 2; ++b)
+    for (int b = 0; b < NB; ++b)
 #pragma unroll
       for (int i = 0; i < VE; ++i) acc[b][i] = 0.f;
-    // two experts' rows requested together (four 16-byte loads in flight per lane),
+    // two experts' rows requested together (eight 16-byte loads in flight per lane),
     // then added in expert order
     for (int i = 0; i < n; i += 2) {
       const bool two = i + 1 < n;
-      uint4 u[2][2];
+      uint4 u[2][NB];
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         const int row = l_row[warp][two || h == 0 ? i + h : i];
         const uint4 *src = reinterpret_cast<const uint4 *>(y_perm + (size_t)row * d);
 #pragma unroll
-        for (int b = 0; b < 2; ++b)
+        for (int b = 0; b < NB; ++b)
           u[h][b] = ((h == 0 || two) && v0 + 32 * b < nvec) ? __ldg(src + v0 + 32 * b)
                                                              : make_uint4(0u, 0u, 0u, 0u);
       }
@@ -300,7 +303,7 @@ __global__ void __launch_bounds__(256) k_ec_combine(const ET *__restrict__ y_per
         if (h == 1 && !two) break;
         const float g = l_g[warp][i + h];
 #pragma unroll
-        for (int b = 0; b < 2; ++b) {
+        for (int b = 0; b < NB; ++b) {
           float f[VE];
           unpack16(u[h][b], f);
 #pragma unroll
@@ -309,7 +312,7 @@ __global__ void __launch_bounds__(256) k_ec_combine(const ET *__restrict__ y_per
       }
     }
 #pragma unroll
-    for (int b = 0; b < 2; ++b)
+    for (int b = 0; b < NB; ++b)
       if (v0 + 32 * b < nvec)
         reinterpret_cast<uint4 *>(y + (size_t)t * d)[v0 + 32 * b] = pack16(acc[b]);
   }
@@ -363,15 +366,14 @@ cudaError_t launch_ec_gather(const void *x, int T, const int32_t *ec_idx, int ro
 cudaError_t launch_ec_combine(const void *y_perm, const int32_t *slot, const float *score,
                               int T, int E, int C, int d, int dtype, void *y, cudaStream_t st) {
   if (T == 0) return cudaSuccess;
+  // programmatic dependent launch: it waits for the down projection before it reads
   if (dtype == MOE_DTYPE_F32)
-    k_ec_combine<float><<<ceil_div(T, 8), 256, 0, st>>>(static_cast<const float *>(y_perm), slot,
-                                                         score, T, E, C, d,
-                                                         static_cast<float *>(y));
-  else
-    k_ec_combine<__nv_bfloat16><<<ceil_div(T, 8), 256, 0, st>>>(
-        static_cast<const __nv_bfloat16 *>(y_perm), slot, score, T, E, C, d,
-        static_cast<__nv_bfloat16 *>(y));
-  return cudaGetLastError();
+    return launch_pdl(k_ec_combine<float>, dim3(ceil_div(T, 8)), dim3(256), 0, st,
+                      static_cast<const float *>(y_perm), slot, score, T, E, C, d,
+                      static_cast<float *>(y));
+  return launch_pdl(k_ec_combine<__nv_bfloat16>, dim3(ceil_div(T, 8)), dim3(256), 0, st,
+                    static_cast<const __nv_bfloat16 *>(y_perm), slot, score, T, E, C, d,
+                    static_cast<__nv_bfloat16 *>(y));
 }
 
 }  // namespace moe
