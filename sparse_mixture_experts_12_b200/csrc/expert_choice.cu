@@ -133,22 +133,48 @@ __global__ void __launch_bounds__(kSelThreads, 1) k_ec_select(EcArgs a, int P) {
   // ---- radix select of the C-th largest key, most significant byte first
   uint32_t prefix = 0, mask = 0;
   int remaining = C;
+  const int lane = tid & 31;
   for (int shift = 24; shift >= 0; shift -= 8) {
     for (int i = tid; i < 256; i += kSelThreads) hist[i] = 0;
     __syncthreads();
-    for (int t = tid; t < T; t += kSelThreads) {
-      const uint32_t k = key[t];
-      if ((k & mask) == prefix) atomicAdd(&hist[(k >> shift) & 0xFF], 1);
+    // warp-aggregated counts: most keys share their leading bytes, so one add per
+    // distinct bin and warp instead of one per key (integer adds: the counts do not
+    // depend on their order)
+    for (int t0 = 0; t0 < T; t0 += kSelThreads) {
+      const int t = t0 + tid;
+      const uint32_t k = t < T ? key[t] : 0u;
+      const int bin = (t < T && (k & mask) == prefix) ? (int)((k >> shift) & 0xFF) : -1;
+      const unsigned peers = __match_any_sync(0xffffffffu, bin);
+      if (bin >= 0 && lane == __ffs(peers) - 1) atomicAdd(&hist[bin], __popc(peers));
     }
     __syncthreads();
-    if (tid == 0) {
-      int above = 0, b = 255;
-      for (; b > 0; --b) {
-        if (above + hist[b] >= remaining) break;
-        above += hist[b];
+    if (tid < 32) {
+      // the highest bin b whose keys, with those of the bins above it, reach
+      // `remaining`: lane l holds bins 8l .. 8l + 7; suffix sums over the lanes
+      int c[8], lsum = 0;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        c[j] = hist[8 * lane + j];
+        lsum += c[j];
       }
-      sh_sel[0] = (uint32_t)b;
-      sh_sel[1] = (uint32_t)(remaining - above);
+      int suf = lsum;  // keys in this lane's bins and every bin above them
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_down_sync(0xffffffffu, suf, o);
+        if (lane + o < 32) suf += v;
+      }
+      int above = suf - lsum;
+      if (above < remaining && remaining <= suf) {
+        int b = 8 * lane + 7;
+#pragma unroll
+        for (int j = 7; j > 0; --j) {
+          if (above + c[j] >= remaining) break;
+          above += c[j];
+          --b;
+        }
+        sh_sel[0] = (uint32_t)b;
+        sh_sel[1] = (uint32_t)(remaining - above);
+      }
     }
     __syncthreads();
     prefix |= sh_sel[0] << shift;
