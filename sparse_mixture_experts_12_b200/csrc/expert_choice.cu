@@ -37,6 +37,8 @@ __device__ __forceinline__ uint32_t ec_key(float z) {
 __global__ void __launch_bounds__(1024) k_ec_transpose(const float *__restrict__ logits, int T,
                                                        int E, float *__restrict__ zt) {
   __shared__ float tile[32][33];
+  pdl_wait();
+  pdl_trigger();
   const int t0 = blockIdx.x * 32, e0 = blockIdx.y * 32;
   const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
   const int t = t0 + ty, e = e0 + tx;
@@ -107,6 +109,8 @@ __device__ __forceinline__ float block_sum(float v, float *sh) {
 // [P] u64 (P = C rounded up to a power of two).
 __global__ void __launch_bounds__(kSelThreads, 1) k_ec_select(EcArgs a, int P) {
   extern __shared__ __align__(16) uint8_t ec_smem[];
+  pdl_wait();
+  pdl_trigger();
   const int T = a.T, C = a.C, E = a.E;
   const int e = blockIdx.x;
   uint32_t *key = reinterpret_cast<uint32_t *>(ec_smem);
@@ -253,6 +257,8 @@ __global__ void __launch_bounds__(kSelThreads, 1) k_ec_select(EcArgs a, int P) {
 __global__ void __launch_bounds__(256) k_ec_gather(const uint8_t *__restrict__ x, int T,
                                                    const int32_t *__restrict__ idx, int rows,
                                                    int row_bytes, uint8_t *__restrict__ x_perm) {
+  pdl_wait();
+  pdl_trigger();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int r = blockIdx.x * 8 + warp;
   if (r >= rows) return;
@@ -357,8 +363,9 @@ size_t ec_select_smem_bytes(int T, int C) {
 cudaError_t launch_ec_route(const EcArgs &a, cudaStream_t st) {
   if (a.T == 0) return cudaSuccess;
   dim3 tg(ceil_div(a.T, 32), ceil_div(a.E, 32));
-  k_ec_transpose<<<tg, 1024, 0, st>>>(a.logits, a.T, a.E, a.zt);
-  cudaError_t e = cudaGetLastError();
+  // programmatic dependent launches: each kernel waits for the one before it before
+  // it touches global memory
+  cudaError_t e = launch_pdl(k_ec_transpose, tg, dim3(1024), 0, st, a.logits, a.T, a.E, a.zt);
   if (e != cudaSuccess) return e;
   int P = 1;
   while (P < a.C) P <<= 1;
@@ -376,17 +383,15 @@ cudaError_t launch_ec_route(const EcArgs &a, cudaStream_t st) {
       attr_set[dev & 63] = true;
     }
   }
-  k_ec_select<<<a.E, kSelThreads, smem, st>>>(a, P);
-  return cudaGetLastError();
+  return launch_pdl(k_ec_select, dim3(a.E), dim3(kSelThreads), smem, st, a, P);
 }
 
 cudaError_t launch_ec_gather(const void *x, int T, const int32_t *ec_idx, int rows,
                              int row_bytes, void *x_perm, cudaStream_t st) {
   if (rows == 0) return cudaSuccess;
-  k_ec_gather<<<ceil_div(rows, 8), 256, 0, st>>>(static_cast<const uint8_t *>(x), T, ec_idx,
-                                                  rows, row_bytes,
-                                                  static_cast<uint8_t *>(x_perm));
-  return cudaGetLastError();
+  return launch_pdl(k_ec_gather, dim3(ceil_div(rows, 8)), dim3(256), 0, st,
+                    static_cast<const uint8_t *>(x), T, ec_idx, rows, row_bytes,
+                    static_cast<uint8_t *>(x_perm));
 }
 
 cudaError_t launch_ec_combine(const void *y_perm, const int32_t *slot, const float *score,

@@ -404,6 +404,9 @@ __global__ void __launch_bounds__(256, SHARED ? 2 : (KMAX <= 2 ? 4 : 3)) k_combi
 // prefix from it (all zero, so nothing is computed, when the offsets are invalid).
 __global__ void k_tile_table(const int32_t *offsets, int G, int max_rows, int32_t *mprefix,
                              int32_t *err) {
+  // waits for the kernel before it, and never lets the one after it begin early: the
+  // GEMMs read mprefix before their own wait
+  pdl_wait();
   const int lane = threadIdx.x;
   int bad = G;
   for (int g = lane; g < G; g += 32) {
@@ -492,8 +495,7 @@ cudaError_t launch_combine(const CombineArgs &a, int dtype, cudaStream_t st) {
 
 cudaError_t launch_tile_table(const int32_t *offsets, int G, int max_rows, int32_t *mprefix,
                               int32_t *err, cudaStream_t st) {
-  k_tile_table<<<1, 32, 0, st>>>(offsets, G, max_rows, mprefix, err);
-  return cudaGetLastError();
+  return launch_pdl(k_tile_table, dim3(1), dim3(32), 0, st, offsets, G, max_rows, mprefix, err);
 }
 
 }  // namespace moe
